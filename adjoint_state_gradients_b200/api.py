@@ -1,0 +1,195 @@
+"""Public Python API over the C-ABI library (device tensors in, device tensors out).
+
+`Problem` owns the device buffers of one setup (model coefficients, CPML
+profiles, source / receiver indices, workspace) and runs the library's
+forward, adjoint-gradient, shot-reduction and chain-rule entry points on the
+current torch stream.  `misfit_gradient_host` is the end-to-end call on host
+arrays: it copies the inputs in, runs the whole sweep and copies the results
+out.  All arithmetic happens in the library's kernels.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import mwtm
+
+F32 = torch.float32
+
+
+def _dev(x, dtype=F32, device="cuda"):
+    if isinstance(x, torch.Tensor):
+        return x.to(device=device, dtype=dtype).contiguous()
+    return torch.as_tensor(np.ascontiguousarray(x), dtype=dtype, device=device)
+
+
+class Problem:
+    """One 2-D TM setup: grid, stencil order, time step, shots, storage mode.
+
+    src_idx [S, n_src] / rec_idx [S, n_rec] are flat cell indices y*nx + x
+    (-1 = inactive).  snapshot: "none" | "fp32" | "bf16" | "ckpt".
+    """
+
+    def __init__(self, ny, nx, order, dy, dx, dt, nt, n_pml, src_idx, rec_idx, *, vmax,
+                 snapshot="fp32", ckpt_every=64, batched=False, cq_scalar=True,
+                 grad_mask_pml=False, allow_unstable=False, check_finite=False, device="cuda"):
+        src_idx = np.asarray(src_idx, dtype=np.int64)
+        rec_idx = np.asarray(rec_idx, dtype=np.int64)
+        self.S = src_idx.shape[0]
+        self.device = device
+        self.p = mwtm.make_params(
+            ny=ny, nx=nx, order=order, n_shots=self.S, n_src=src_idx.shape[1], n_rec=rec_idx.shape[1],
+            nt=nt, dt=dt, dy=dy, dx=dx, n_pml=n_pml, model_batched=int(batched),
+            cq_is_scalar=int(cq_scalar), snap_mode=mwtm.SNAP_MODES[snapshot], ckpt_every=ckpt_every,
+            grad_mask_pml=int(grad_mask_pml), vmax=vmax, allow_unstable=int(allow_unstable),
+            check_finite=int(check_finite))
+        mwtm.check(mwtm.validate(self.p))
+        self.src_idx = _dev(src_idx if src_idx.size else np.zeros((self.S, 1), np.int64),
+                            torch.int64, device)
+        self.rec_idx = _dev(rec_idx if rec_idx.size else np.zeros((self.S, 1), np.int64),
+                            torch.int64, device)
+        self.workspace = torch.empty(mwtm.workspace_bytes(self.p) // 4 + 64, dtype=F32, device=device)
+        self.cpml = torch.empty(6 * (ny + nx), dtype=F32, device=device)
+        self.ca = self.cb = self.cq = None
+        self.state = None
+
+    # ---- model -------------------------------------------------------------
+    @property
+    def model_shape(self):
+        p = self.p
+        return (self.S, p.ny, p.nx) if p.model_batched else (p.ny, p.nx)
+
+    def set_model_eps_sigma(self, eps_r, sigma=None, mu_r=None, f0=0.0, R=1e-3):
+        """Ca, Cb, Cq from eps_r, sigma, mu_r (library kernel) and CPML profiles."""
+        d = self.device
+        eps_r = _dev(eps_r, device=d).reshape(self.model_shape)
+        sigma = None if sigma is None else _dev(sigma, device=d).reshape(self.model_shape)
+        mu_r = None if mu_r is None else _dev(mu_r, device=d).reshape(self.model_shape)
+        self.ca = torch.empty(self.model_shape, dtype=F32, device=d)
+        self.cb = torch.empty(self.model_shape, dtype=F32, device=d)
+        self.cq = torch.empty((1,) if self.p.cq_is_scalar else self.model_shape, dtype=F32, device=d)
+        mwtm.model_from_eps_sigma(self.p, eps_r, sigma, mu_r, self.ca, self.cb, self.cq)
+        mwtm.cpml_profiles(self.p, f0, R, self.cpml)
+        return self
+
+    def set_coefficients(self, ca, cb, cq, cpml):
+        d = self.device
+        self.ca = _dev(ca, device=d).reshape(self.model_shape)
+        self.cb = _dev(cb, device=d).reshape(self.model_shape)
+        self.cq = _dev(cq, device=d).reshape(-1)
+        self.cpml = _dev(cpml, device=d).reshape(-1)
+        return self
+
+    # ---- sweeps ------------------------------------------------------------
+    def new_state(self):
+        return torch.zeros(mwtm.state_floats(self.p), dtype=F32, device=self.device)
+
+    def forward(self, f, state=None, rec=None):
+        """Run nt steps; returns records [nt, S, n_rec].  `state` (flat) is in/out."""
+        p = self.p
+        f = _dev(f, device=self.device) if p.n_src > 0 else None
+        if rec is None:
+            rec = torch.empty((p.nt, self.S, max(p.n_rec, 1)), dtype=F32, device=self.device)
+        mwtm.tm_forward(p, self.ca, self.cb, self.cq, self.cpml, f, self.src_idx, self.rec_idx, state,
+                        rec if p.n_rec > 0 else None, self.workspace)
+        self._f = f
+        return rec[:, :, :p.n_rec]
+
+    def adjoint(self, res, grad_f=False, gca=None, gcb=None, adj_state=None):
+        """Adjoint sweep; returns (grad_ca_shot, grad_cb_shot, grad_f or None)."""
+        p = self.p
+        shp = (self.S, p.ny, p.nx)
+        gca = torch.zeros(shp, dtype=F32, device=self.device) if gca is None else gca
+        gcb = torch.zeros(shp, dtype=F32, device=self.device) if gcb is None else gcb
+        gf = torch.zeros((p.nt, self.S, p.n_src), dtype=F32, device=self.device) if (
+            grad_f and p.n_src > 0) else None
+        res = _dev(res, device=self.device) if p.n_rec > 0 else None
+        mwtm.tm_adjoint_grad(p, self.ca, self.cb, self.cq, self.cpml, getattr(self, "_f", None),
+                             self.src_idx, self.rec_idx, res, gca, gcb, gf, adj_state, self.workspace)
+        return gca, gcb, gf
+
+    def combine(self, g_shot, out=None, accumulate=False):
+        p = self.p
+        out = torch.empty((p.ny, p.nx), dtype=F32, device=self.device) if out is None else out
+        mwtm.combine_grad(p, g_shot, out, accumulate)
+        return out
+
+    def eps_sigma_gradient(self, gca, gcb):
+        n = gca.numel()
+        ge = torch.empty_like(gca)
+        gs = torch.empty_like(gca)
+        mwtm.grad_eps_sigma(n, self.p.dt, self.ca, self.cb, gca, gcb, ge, gs)
+        return ge, gs
+
+    def residual(self, d, d_obs, res=None, J=None):
+        res = torch.empty_like(d) if res is None else res
+        J = torch.zeros(1, dtype=torch.float64, device=self.device) if J is None else J
+        mwtm.residual(d.numel(), d, d_obs, res, J)
+        return res, J
+
+    def status(self):
+        return mwtm.sync_status(self.workspace)
+
+    def misfit_gradient(self, f, d_obs):
+        """Forward, residual, adjoint, shot sum: (J [1] f64, rec, grad_Ca, grad_Cb)."""
+        rec = self.forward(f)
+        res, J = self.residual(rec.contiguous(), d_obs)
+        gca_s, gcb_s, _ = self.adjoint(res)
+        if self.p.model_batched:
+            return J, rec, gca_s, gcb_s
+        return J, rec, self.combine(gca_s), self.combine(gcb_s)
+
+
+def unpack_state(p, flat):
+    """Split a flat state into full [S, ny, nx] arrays (memories expanded; numpy fp64)."""
+    a = flat.detach().cpu().numpy().astype(np.float64) if isinstance(flat, torch.Tensor) else flat
+    S, ny, nx, n_pml = p.n_shots, p.ny, p.nx, p.n_pml
+    Wx = ((n_pml + 1 + 3) // 4) * 4 if n_pml > 0 else 0
+    Wz = n_pml + 1 if n_pml > 0 else 0
+    SN = S * ny * nx
+    out = {"ey": a[:SN].reshape(S, ny, nx), "hx": a[SN:2 * SN].reshape(S, ny, nx),
+           "hz": a[2 * SN:3 * SN].reshape(S, ny, nx)}
+    off = 3 * SN
+    xb = S * ny * 2 * Wx
+    zb = S * 2 * Wz * nx
+    names_x = ("m_ey_x", "m_hz_x")
+    names_z = ("m_ey_z", "m_hx_z")
+    for nm in names_x:
+        full = np.zeros((S, ny, nx))
+        if Wx:
+            band = a[off:off + xb].reshape(S, ny, 2 * Wx)
+            full[:, :, :Wx] = band[:, :, :Wx]
+            full[:, :, nx - Wx:] = band[:, :, Wx:]
+        out[nm] = full
+        off += xb
+    for nm in names_z:
+        full = np.zeros((S, ny, nx))
+        if Wz:
+            band = a[off:off + zb].reshape(S, 2 * Wz, nx)
+            full[:, :Wz, :] = band[:, :Wz, :]
+            full[:, ny - Wz:, :] = band[:, Wz:, :]
+        out[nm] = full
+        off += zb
+    return out
+
+
+def misfit_gradient_host(prob: Problem, f_host, d_obs_host, eps_r_host=None, sigma_host=None,
+                         f0=0.0, pinned_out=None):
+    """End-to-end on host arrays: H2D of the inputs, the whole sweep, D2H of
+    J, records and the combined gradients.  Returns numpy arrays."""
+    dev = prob.device
+    if eps_r_host is not None:
+        prob.set_model_eps_sigma(torch.as_tensor(eps_r_host).to(dev, non_blocking=True),
+                                 None if sigma_host is None else
+                                 torch.as_tensor(sigma_host).to(dev, non_blocking=True), f0=f0)
+    f = torch.as_tensor(f_host).to(dev, non_blocking=True)
+    d_obs = torch.as_tensor(d_obs_host).to(dev, non_blocking=True)
+    J, rec, gca, gcb = prob.misfit_gradient(f, d_obs)
+    if pinned_out is None:
+        return J.cpu().numpy(), rec.cpu().numpy(), gca.cpu().numpy(), gcb.cpu().numpy()
+    outs = []
+    for t, h in zip((J, rec, gca, gcb), pinned_out):
+        h.copy_(t.reshape(h.shape), non_blocking=True)
+        outs.append(h)
+    torch.cuda.current_stream().synchronize()
+    return outs

@@ -1,0 +1,627 @@
+// C ABI of the mw_tm library (declared in include/mw_tm.h): argument checks,
+// workspace layout, the forward / adjoint time loops, checkpoint replay and
+// per-kernel event timing.  The time loops follow the page "tide-GPR 0.0.9 ...
+// tide/csrc/maxwell.cu" host drivers (forward: H, E, sources, receivers per
+// step; backward: adjoint sources, source gradient, adjoint H, adjoint E with
+// gradient, reversed in time) with the H and E kernels fused into one launch.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "mw_internal.cuh"
+
+namespace mw {
+
+static std::atomic<int64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define MW_CUDA(call)                                                                    \
+  do {                                                                                   \
+    cudaError_t e_ = (call);                                                             \
+    if (e_ != cudaSuccess)                                                               \
+      return fail(MW_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                  __FILE__, __LINE__);                                                   \
+  } while (0)
+
+// Staggered first-derivative weights (Taylor conditions on a half-integer grid).
+int stencil_weights(int order, double *c) {
+  c[0] = c[1] = c[2] = c[3] = 0.0;
+  switch (order) {
+    case 2: c[0] = 1.0; return 1;
+    case 4: c[0] = 9.0 / 8.0; c[1] = -1.0 / 24.0; return 2;
+    case 6: c[0] = 75.0 / 64.0; c[1] = -25.0 / 384.0; c[2] = 3.0 / 640.0; return 3;
+    case 8:
+      c[0] = 1225.0 / 1024.0; c[1] = -245.0 / 3072.0; c[2] = 49.0 / 5120.0;
+      c[3] = -5.0 / 7168.0;
+      return 4;
+  }
+  return 0;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Bands {
+  int Wx, Wz;
+};
+Bands bands(const mw_params *p) {
+  Bands b;
+  b.Wx = p->n_pml > 0 ? ((p->n_pml + 1 + 3) / 4) * 4 : 0;
+  b.Wz = p->n_pml > 0 ? p->n_pml + 1 : 0;
+  return b;
+}
+
+size_t state_floats(const mw_params *p) {
+  const Bands b = bands(p);
+  const size_t S = p->n_shots, ny = p->ny, nx = p->nx;
+  return S * ny * nx * 3 + S * ny * 2 * b.Wx * 2 + S * 2 * b.Wz * nx * 2;
+}
+
+int check_params(const mw_params *p, bool cfl) {
+  if (!p) return fail(MW_ERR_ARG, "params is NULL");
+  double c[4];
+  if (!stencil_weights(p->order, c)) return fail(MW_ERR_ARG, "order %d not in {2,4,6,8}", p->order);
+  if (p->ny < 1 || p->nx < 4) return fail(MW_ERR_ARG, "grid %d x %d too small", p->ny, p->nx);
+  if (p->nx % 4 != 0) return fail(MW_ERR_ARG, "nx = %d must be a multiple of 4", p->nx);
+  if (p->n_shots < 1) return fail(MW_ERR_ARG, "n_shots = %d", p->n_shots);
+  if (p->n_src < 0 || p->n_rec < 0 || p->nt < 0) return fail(MW_ERR_ARG, "negative count");
+  if (!(p->dt > 0) || !(p->dy > 0) || !(p->dx > 0) || !isfinite(p->dt) || !isfinite(p->dy) ||
+      !isfinite(p->dx))
+    return fail(MW_ERR_ARG, "dt, dy, dx must be positive and finite");
+  if (p->n_pml < 0) return fail(MW_ERR_ARG, "n_pml = %d", p->n_pml);
+  const Bands b = bands(p);
+  if (2 * b.Wx > p->nx || 2 * b.Wz > p->ny)
+    return fail(MW_ERR_ARG, "CPML band %d does not fit a %d x %d grid", p->n_pml, p->ny, p->nx);
+  if (p->snap_mode < MW_SNAP_NONE || p->snap_mode > MW_SNAP_CKPT)
+    return fail(MW_ERR_ARG, "snap_mode = %d", p->snap_mode);
+  if (p->snap_mode == MW_SNAP_CKPT && p->ckpt_every < 1)
+    return fail(MW_ERR_ARG, "ckpt_every = %d", p->ckpt_every);
+  if ((int64_t)p->ny * p->nx > ((int64_t)1 << 40)) return fail(MW_ERR_ARG, "grid too large");
+  if (cfl && !p->allow_unstable) {
+    if (!(p->vmax > 0) || !isfinite(p->vmax))
+      return fail(MW_ERR_CFL, "vmax must be positive (or set allow_unstable)");
+    const double dtmax = mw_cfl_dt(p->order, p->dy, p->dx, p->vmax);
+    if (p->dt > dtmax * (1.0 + 1e-12))
+      return fail(MW_ERR_CFL, "dt = %.6g s exceeds the stability bound %.6g s", p->dt, dtmax);
+  }
+  return MW_OK;
+}
+
+Layout layout(const mw_params *p) {
+  Layout L{};
+  const size_t SN = (size_t)p->n_shots * p->ny * p->nx;
+  L.state_bytes = state_floats(p) * sizeof(float);
+  const size_t sb = align256(L.state_bytes);
+  size_t off = 0;
+  L.flags = off; off += 256;
+  L.stA = off; off += sb;
+  L.stB = off; off += sb;
+  L.adA = L.adB = L.rpA = L.rpB = L.snap = L.seg = 0;
+  L.n_seg = 0;
+  L.snap_step_bytes = 0;
+  if (p->snap_mode != MW_SNAP_NONE) {
+    L.adA = off; off += sb;
+    L.adB = off; off += sb;
+  }
+  if (p->snap_mode == MW_SNAP_FP32 || p->snap_mode == MW_SNAP_BF16) {
+    const size_t es = p->snap_mode == MW_SNAP_FP32 ? 4 : 2;
+    L.snap_step_bytes = SN * es;
+    L.snap = off;
+    off += align256(2 * (size_t)p->nt * L.snap_step_bytes);
+  } else if (p->snap_mode == MW_SNAP_CKPT) {
+    L.n_seg = p->nt > 0 ? (p->nt + p->ckpt_every - 1) / p->ckpt_every : 0;
+    L.rpA = off; off += sb;
+    L.rpB = off; off += sb;
+    L.snap = off; off += (size_t)L.n_seg * sb;
+    L.snap_step_bytes = SN * 4;
+    L.seg = off;
+    off += align256(2 * (size_t)p->ckpt_every * L.snap_step_bytes);
+  }
+  L.total = off;
+  return L;
+}
+
+Fields fields_at(const mw_params *p, float *base) {
+  const Bands b = bands(p);
+  const size_t SN = (size_t)p->n_shots * p->ny * p->nx;
+  const size_t xb = (size_t)p->n_shots * p->ny * 2 * b.Wx;
+  const size_t zb = (size_t)p->n_shots * 2 * b.Wz * p->nx;
+  Fields f;
+  f.ey = base;
+  f.hx = base + SN;
+  f.hz = base + 2 * SN;
+  f.mxh_node = base + 3 * SN;
+  f.mxe_node = f.mxh_node + xb;
+  f.mzh_node = f.mxe_node + xb;
+  f.mze_node = f.mzh_node + zb;
+  return f;
+}
+
+// ---- launch geometry ------------------------------------------------------
+int sm_count() {
+  static int cached = -1;
+  static int cached_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (cached < 0 || dev != cached_dev) {
+    int n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+    cached = n;
+    cached_dev = dev;
+  }
+  return cached;
+}
+
+struct Launch {
+  Geom g;
+  int grid;
+};
+
+// Choose the row-chunk height so that the warps' work items fill whole waves
+// of resident warps: cost ~ waves x (rows per item + warm-up rows).
+Launch plan(const mw_params *p, bool adjoint) {
+  Launch Lc{};
+  Geom &g = Lc.g;
+  const Bands b = bands(p);
+  g.ny = p->ny;
+  g.nx = p->nx;
+  g.S = p->n_shots;
+  g.Wx = b.Wx;
+  g.Wz = b.Wz;
+  g.n_pml = p->n_pml;
+  g.grad_mask = p->grad_mask_pml ? 1 : 0;
+  g.numel = (int64_t)p->ny * p->nx;
+  g.n_strips = (p->nx + kStripCols - 1) / kStripCols;
+  const int P = p->order / 2;
+  const int warps_sm = stencil_slots_per_sm(p->order, adjoint);
+  const int64_t slots = (int64_t)sm_count() * warps_sm;
+  const int64_t cols_items = (int64_t)g.S * g.n_strips;
+  int best_nc = 1;
+  double best_cost = 1e300;
+  const int max_nc = p->ny < 4096 ? p->ny : 4096;
+  for (int nc = 1; nc <= max_nc; ++nc) {
+    const int ch = (p->ny + nc - 1) / nc;
+    if (ch < 8 && nc > 1) break;
+    const int nce = (p->ny + ch - 1) / ch;
+    const int64_t items = cols_items * nce;
+    const int64_t waves = (items + slots - 1) / slots;
+    const double cost = (double)waves * (ch + 4 * P - 2);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best_nc = nce;
+    }
+  }
+  g.chunk_h = (p->ny + best_nc - 1) / best_nc;
+  g.n_chunks = (p->ny + g.chunk_h - 1) / g.chunk_h;
+  const int64_t items = cols_items * g.n_chunks;
+  int64_t grid = (items + kWarpsPerCta - 1) / kWarpsPerCta;
+  const int64_t cap = slots / kWarpsPerCta;
+  if (grid > cap) grid = cap;
+  Lc.grid = (int)(grid > 0 ? grid : 1);
+  return Lc;
+}
+
+Coef coef_of(const mw_params *p) {
+  double c[4];
+  stencil_weights(p->order, c);
+  Coef k;
+  for (int i = 0; i < 4; ++i) {
+    k.cx[i] = (float)(c[i] / p->dx);
+    k.cy[i] = (float)(c[i] / p->dy);
+  }
+  return k;
+}
+
+Prof prof_of(const mw_params *p, const float *cpml) {
+  const size_t ny = p->ny, nx = p->nx;
+  Prof r;
+  r.ay = cpml;
+  r.ayh = cpml + ny;
+  r.by = cpml + 2 * ny;
+  r.byh = cpml + 3 * ny;
+  r.ky = cpml + 4 * ny;
+  r.kyh = cpml + 5 * ny;
+  const float *x = cpml + 6 * ny;
+  r.ax = x;
+  r.axh = x + nx;
+  r.bx = x + 2 * nx;
+  r.bxh = x + 3 * nx;
+  r.kx = x + 4 * nx;
+  r.kxh = x + 5 * nx;
+  return r;
+}
+
+// ---- per-kernel event timing ------------------------------------------------
+struct Timer {
+  std::mutex mu;
+  bool on = false;
+  std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Timer &timer() {
+  static Timer t;
+  return t;
+}
+
+template <typename F>
+cudaError_t timed(int cls, cudaStream_t st, F &&launch) {
+  Timer &T = timer();
+  if (!T.on) return launch();
+  std::lock_guard<std::mutex> lk(T.mu);
+  cudaEvent_t a = T.get(), b = T.get();
+  cudaEventRecord(a, st);
+  cudaError_t e = launch();
+  cudaEventRecord(b, st);
+  T.recs.push_back({cls, {a, b}});
+  return e;
+}
+
+int check_ptr(const void *ptr, const char *name) {
+  if (!ptr) return fail(MW_ERR_ARG, "%s is NULL", name);
+  if (((uintptr_t)ptr) % 16 != 0) return fail(MW_ERR_ARG, "%s is not 16-byte aligned", name);
+  return MW_OK;
+}
+
+}  // namespace
+}  // namespace mw
+
+using namespace mw;
+
+extern "C" {
+
+void mw_params_init(mw_params *p) {
+  if (!p) return;
+  memset(p, 0, sizeof *p);
+  p->cq_is_scalar = 1;
+  p->snap_mode = MW_SNAP_NONE;
+}
+
+size_t mw_state_floats(const mw_params *p) {
+  if (check_params(p, false) != MW_OK) return 0;
+  return state_floats(p);
+}
+
+size_t mw_workspace_bytes(const mw_params *p) {
+  if (check_params(p, false) != MW_OK) return 0;
+  return layout(p).total;
+}
+
+double mw_cfl_dt(int32_t order, double dy, double dx, double vmax) {
+  double c[4];
+  const int P = stencil_weights(order, c);
+  if (!P || !(dy > 0) || !(dx > 0) || !(vmax > 0)) return -1.0;
+  double s = 0.0;
+  for (int k = 0; k < P; ++k) s += fabs(c[k]);
+  return 1.0 / (vmax * s * sqrt(1.0 / (dx * dx) + 1.0 / (dy * dy)));
+}
+
+int mw_validate(const mw_params *p) {
+  g_err.clear();
+  return check_params(p, true);
+}
+
+const char *mw_last_error(void) { return g_err.c_str(); }
+
+int mw_model_from_eps_sigma(const mw_params *p, const float *eps_r, const float *sigma,
+                            const float *mu_r, float *ca, float *cb, float *cq, void *stream) {
+  g_err.clear();
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (!eps_r || !ca || !cb || !cq) return fail(MW_ERR_ARG, "NULL model pointer");
+  if (p->cq_is_scalar && mu_r) return fail(MW_ERR_ARG, "mu_r given but cq_is_scalar = 1");
+  const int64_t n = (int64_t)(p->model_batched ? p->n_shots : 1) * p->ny * p->nx;
+  MW_CUDA(launch_model(n, eps_r, sigma, mu_r, p->dt, ca, cb, cq, p->cq_is_scalar ? 0 : 1,
+                       (cudaStream_t)stream));
+  return MW_OK;
+}
+
+int mw_cpml_profiles(const mw_params *p, double f0, double R, float *cpml, void *stream) {
+  g_err.clear();
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (!cpml) return fail(MW_ERR_ARG, "cpml is NULL");
+  if (p->n_pml > 0 && (!(p->vmax > 0) || !(f0 >= 0) || !(R > 0 && R < 1)))
+    return fail(MW_ERR_ARG, "CPML needs vmax > 0, f0 >= 0, 0 < R < 1");
+  MW_CUDA(launch_cpml(p->ny, p->nx, p->n_pml, p->dy, p->dx, p->dt, p->vmax, f0, R, cpml,
+                      (cudaStream_t)stream));
+  return MW_OK;
+}
+
+int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const float *cq,
+                  const float *cpml, const float *f, const int64_t *src_idx,
+                  const int64_t *rec_idx, float *state, float *rec, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+  g_err.clear();
+  int rc = check_params(p, true);
+  if (rc) return rc;
+  if ((rc = check_ptr(ca, "ca")) || (rc = check_ptr(cb, "cb")) || (rc = check_ptr(cpml, "cpml")))
+    return rc;
+  if (!cq) return fail(MW_ERR_ARG, "cq is NULL");
+  if (!p->cq_is_scalar && (rc = check_ptr(cq, "cq"))) return rc;
+  if (p->n_src > 0 && (!f || !src_idx)) return fail(MW_ERR_ARG, "sources need f and src_idx");
+  if (p->n_rec > 0 && rec && !rec_idx) return fail(MW_ERR_ARG, "receivers need rec_idx");
+  if (state && (rc = check_ptr(state, "state"))) return rc;
+  if (!workspace) return fail(MW_ERR_WORKSPACE, "workspace is NULL");
+  const Layout L = layout(p);
+  if (workspace_bytes < L.total)
+    return fail(MW_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+  if (((uintptr_t)workspace) % 256 != 0) return fail(MW_ERR_WORKSPACE, "workspace not 256-aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = (char *)workspace;
+  int *flags = (int *)(ws + L.flags);
+
+  float *bufA = state ? state : (float *)(ws + L.stA);
+  float *bufB = (float *)(ws + L.stB);
+  if (!state) MW_CUDA(cudaMemsetAsync(bufA, 0, L.state_bytes, st));
+
+  StepArgs a{};
+  const Launch lc = plan(p, false);
+  a.g = lc.g;
+  a.c = coef_of(p);
+  a.pr = prof_of(p, cpml);
+  a.ca = ca;
+  a.cb = cb;
+  a.cq = cq;
+  a.cq_scalar = 0.f;
+
+  const int store = p->snap_mode == MW_SNAP_FP32 ? kStoreF32
+                    : p->snap_mode == MW_SNAP_BF16 ? kStoreBF16 : kStoreNone;
+  const int64_t SN = (int64_t)p->n_shots * p->ny * p->nx;
+  char *snap_e = ws + L.snap;
+  char *snap_c = ws + L.snap + (size_t)p->nt * L.snap_step_bytes;
+  float *cur = bufA, *nxt = bufB;
+  for (int t = 0; t < p->nt; ++t) {
+    if (p->snap_mode == MW_SNAP_CKPT && t % p->ckpt_every == 0) {
+      char *ck = ws + L.snap + (size_t)(t / p->ckpt_every) * align256(L.state_bytes);
+      MW_CUDA(cudaMemcpyAsync(ck, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
+    }
+    a.in = fields_at(p, cur);
+    a.out = fields_at(p, nxt);
+    a.snap_e = store ? snap_e + (size_t)t * L.snap_step_bytes : nullptr;
+    a.snap_c = store ? snap_c + (size_t)t * L.snap_step_bytes : nullptr;
+    MW_CUDA(timed(store ? 1 : 0, st, [&] {
+      return launch_forward(a, p->order, store, p->model_batched != 0, !p->cq_is_scalar, lc.grid,
+                            st);
+    }));
+    MW_CUDA(launch_src_rec(nxt, p->ny * (int64_t)p->nx, p->n_shots,
+                           f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
+                           p->n_src, rec_idx, p->n_rec,
+                           rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, flags, st));
+    std::swap(cur, nxt);
+  }
+  if (cur != bufA) MW_CUDA(cudaMemcpyAsync(bufA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
+  if (p->check_finite) MW_CUDA(launch_check_finite(bufA, 3 * SN, flags, st));
+  return MW_OK;
+}
+
+int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, const float *cq,
+                       const float *cpml, const float *f, const int64_t *src_idx,
+                       const int64_t *rec_idx, const float *res, float *gca, float *gcb,
+                       float *grad_f, float *adj_state, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  g_err.clear();
+  int rc = check_params(p, true);
+  if (rc) return rc;
+  if (p->snap_mode == MW_SNAP_NONE)
+    return fail(MW_ERR_ARG, "snap_mode NONE: the forward stored nothing to differentiate");
+  if ((rc = check_ptr(ca, "ca")) || (rc = check_ptr(cb, "cb")) || (rc = check_ptr(cpml, "cpml")) ||
+      (rc = check_ptr(gca, "grad_ca_shot")) || (rc = check_ptr(gcb, "grad_cb_shot")))
+    return rc;
+  if (!cq) return fail(MW_ERR_ARG, "cq is NULL");
+  if (!p->cq_is_scalar && (rc = check_ptr(cq, "cq"))) return rc;
+  if (p->n_rec > 0 && (!res || !rec_idx)) return fail(MW_ERR_ARG, "receivers need res and rec_idx");
+  if (p->n_src > 0 && grad_f && !src_idx) return fail(MW_ERR_ARG, "grad_f needs src_idx");
+  if (p->snap_mode == MW_SNAP_CKPT && p->n_src > 0 && (!f || !src_idx))
+    return fail(MW_ERR_ARG, "checkpoint replay needs f and src_idx");
+  if (adj_state && (rc = check_ptr(adj_state, "adj_state"))) return rc;
+  if (!workspace) return fail(MW_ERR_WORKSPACE, "workspace is NULL");
+  const Layout L = layout(p);
+  if (workspace_bytes < L.total)
+    return fail(MW_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+  if (((uintptr_t)workspace) % 256 != 0) return fail(MW_ERR_WORKSPACE, "workspace not 256-aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = (char *)workspace;
+  int *flags = (int *)(ws + L.flags);
+  const int64_t numel = (int64_t)p->ny * p->nx;
+  const int64_t SN = p->n_shots * numel;
+
+  float *adA = adj_state ? adj_state : (float *)(ws + L.adA);
+  float *adB = (float *)(ws + L.adB);
+  if (!adj_state) MW_CUDA(cudaMemsetAsync(adA, 0, L.state_bytes, st));
+
+  const Launch la = plan(p, true);
+  StepArgs a{};
+  a.g = la.g;
+  a.c = coef_of(p);
+  a.pr = prof_of(p, cpml);
+  a.ca = ca;
+  a.cb = cb;
+  a.cq = cq;
+  a.gca = gca;
+  a.gcb = gcb;
+  a.cq_scalar = 0.f;
+
+  float *cur = adA, *nxt = adB;
+  auto adj_step = [&](int t, const char *se, const char *sc, int bf16) -> int {
+    MW_CUDA(launch_adj_src_rec(cur, numel, p->n_shots,
+                               res ? res + (int64_t)t * p->n_shots * p->n_rec : nullptr, rec_idx,
+                               p->n_rec, src_idx, p->n_src,
+                               grad_f ? grad_f + (int64_t)t * p->n_shots * p->n_src : nullptr,
+                               flags, st));
+    a.in = fields_at(p, cur);
+    a.out = fields_at(p, nxt);
+    a.snap_e = (void *)se;
+    a.snap_c = (void *)sc;
+    MW_CUDA(timed(2, st, [&] {
+      return launch_adjoint(a, p->order, bf16, p->model_batched != 0, !p->cq_is_scalar, la.grid,
+                            st);
+    }));
+    std::swap(cur, nxt);
+    return MW_OK;
+  };
+
+  if (p->snap_mode == MW_SNAP_FP32 || p->snap_mode == MW_SNAP_BF16) {
+    const char *snap_e = ws + L.snap;
+    const char *snap_c = ws + L.snap + (size_t)p->nt * L.snap_step_bytes;
+    const int bf16 = p->snap_mode == MW_SNAP_BF16;
+    for (int t = p->nt - 1; t >= 0; --t) {
+      rc = adj_step(t, snap_e + (size_t)t * L.snap_step_bytes,
+                    snap_c + (size_t)t * L.snap_step_bytes, bf16);
+      if (rc) return rc;
+    }
+  } else {
+    // checkpoint mode: replay each segment from its checkpoint, newest first
+    const Launch lf = plan(p, false);
+    StepArgs fa = a;
+    fa.g = lf.g;
+    const int C = p->ckpt_every;
+    char *seg_e = ws + L.seg;
+    char *seg_c = ws + L.seg + (size_t)C * L.snap_step_bytes;
+    float *rA = (float *)(ws + L.rpA), *rB = (float *)(ws + L.rpB);
+    for (int k = L.n_seg - 1; k >= 0; --k) {
+      const int t0 = k * C;
+      const int t1 = (t0 + C < p->nt) ? t0 + C : p->nt;
+      MW_CUDA(cudaMemcpyAsync(rA, ws + L.snap + (size_t)k * align256(L.state_bytes),
+                              L.state_bytes, cudaMemcpyDeviceToDevice, st));
+      float *rc_ = rA, *rn = rB;
+      for (int t = t0; t < t1; ++t) {
+        fa.in = fields_at(p, rc_);
+        fa.out = fields_at(p, rn);
+        fa.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
+        fa.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
+        MW_CUDA(timed(1, st, [&] {
+          return launch_forward(fa, p->order, kStoreF32, p->model_batched != 0, !p->cq_is_scalar,
+                                lf.grid, st);
+        }));
+        MW_CUDA(launch_src_rec(rn, numel, p->n_shots,
+                               f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
+                               p->n_src, rec_idx, 0, nullptr, flags, st));
+        std::swap(rc_, rn);
+      }
+      for (int t = t1 - 1; t >= t0; --t) {
+        rc = adj_step(t, seg_e + (size_t)(t - t0) * L.snap_step_bytes,
+                      seg_c + (size_t)(t - t0) * L.snap_step_bytes, 0);
+        if (rc) return rc;
+      }
+    }
+  }
+  if (cur != adA) MW_CUDA(cudaMemcpyAsync(adA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
+  if (p->check_finite) {
+    MW_CUDA(launch_check_finite(gca, SN, flags, st));
+    MW_CUDA(launch_check_finite(gcb, SN, flags, st));
+  }
+  return MW_OK;
+}
+
+int mw_combine_grad(const mw_params *p, const float *grad_shot, float *grad, int32_t accumulate,
+                    void *stream) {
+  g_err.clear();
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (!grad_shot || !grad) return fail(MW_ERR_ARG, "NULL gradient pointer");
+  MW_CUDA(launch_combine(grad_shot, grad, p->n_shots, (int64_t)p->ny * p->nx, accumulate ? 1 : 0,
+                         (cudaStream_t)stream));
+  return MW_OK;
+}
+
+int mw_grad_eps_sigma(int64_t n, double dt, const float *ca, const float *cb, const float *gca,
+                      const float *gcb, float *ge, float *gs, void *stream) {
+  g_err.clear();
+  if (n < 0 || !(dt > 0)) return fail(MW_ERR_ARG, "n < 0 or dt <= 0");
+  if (!ca || !cb || !gca || !gcb) return fail(MW_ERR_ARG, "NULL input pointer");
+  if (n == 0 || (!ge && !gs)) return MW_OK;
+  MW_CUDA(launch_eps_sigma(n, dt, ca, cb, gca, gcb, ge, gs, (cudaStream_t)stream));
+  return MW_OK;
+}
+
+int mw_residual(int64_t n, const float *d, const float *d_obs, float *res, double *J,
+                void *stream) {
+  g_err.clear();
+  if (n < 0) return fail(MW_ERR_ARG, "n < 0");
+  if (n > 0 && (!d || !d_obs || !res)) return fail(MW_ERR_ARG, "NULL pointer");
+  if (n == 0) {
+    if (J) MW_CUDA(cudaMemsetAsync(J, 0, sizeof(double), (cudaStream_t)stream));
+    return MW_OK;
+  }
+  MW_CUDA(launch_residual(n, d, d_obs, res, J, (cudaStream_t)stream));
+  return MW_OK;
+}
+
+int mw_sync_status(void *workspace, void *stream) {
+  g_err.clear();
+  cudaStream_t st = (cudaStream_t)stream;
+  MW_CUDA(cudaStreamSynchronize(st));
+  if (!workspace) return MW_OK;
+  int h[2] = {0, 0};
+  MW_CUDA(cudaMemcpy(h, workspace, sizeof h, cudaMemcpyDeviceToHost));
+  MW_CUDA(cudaMemset(workspace, 0, sizeof h));
+  if (h[kFlagBadIndex]) return fail(MW_ERR_ARG, "a source or receiver index was out of range");
+  if (h[kFlagNonFinite]) return fail(MW_ERR_NONFINITE, "non-finite value in a field or gradient");
+  return MW_OK;
+}
+
+int64_t mw_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int mw_profile_enable(int32_t enable) {
+  Timer &T = timer();
+  std::lock_guard<std::mutex> lk(T.mu);
+  for (auto &r : T.recs) {
+    T.pool.push_back(r.second.first);
+    T.pool.push_back(r.second.second);
+  }
+  T.recs.clear();
+  T.on = enable != 0;
+  return MW_OK;
+}
+
+int mw_profile_read(int64_t *counts, double *total_ms, int32_t n_classes) {
+  g_err.clear();
+  Timer &T = timer();
+  std::lock_guard<std::mutex> lk(T.mu);
+  for (int i = 0; i < n_classes; ++i) {
+    if (counts) counts[i] = 0;
+    if (total_ms) total_ms[i] = 0.0;
+  }
+  for (auto &r : T.recs) {
+    MW_CUDA(cudaEventSynchronize(r.second.second));
+    float ms = 0.f;
+    MW_CUDA(cudaEventElapsedTime(&ms, r.second.first, r.second.second));
+    if (r.first >= 0 && r.first < n_classes) {
+      if (counts) counts[r.first] += 1;
+      if (total_ms) total_ms[r.first] += ms;
+    }
+  }
+  return MW_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,416 @@
+"""Benchmark: Gcell-updates/s of the forward + adjoint + gradient sweep of the
+2-D TM Maxwell FDTD on the 2048^2 interior (2128^2 with a 40-cell CPML band),
+order-4 stencil, 8 shots per GPU, nt = 4000, checkpoints every 64 steps with
+segment replay.  One step = one whole sweep over one batch of 8 shots:
+forward (records + checkpoints), residual and misfit, replayed adjoint with
+fused per-shot gradients, shot reduction of dJ/dCa and dJ/dCb.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  --impl reference times the fp64 CPU oracle
+(the reference arm) on a bounded sample of the same workload.  Multi-GPU runs
+(launched by torch.distributed.run) shard shots across ranks (8 per rank,
+weak scaling) and all-reduce the gradients once per step over NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+WORKLOAD = 4
+METRIC = "Gcell-updates/s (fwd; fwd+adjoint+grad) on 1 B200 and % of HBM roofline"
+UNIT = "Gcell-updates/s"
+PROFILES = os.path.join(ROOT, "profiles")
+STENCIL_SRC = os.path.join(ROOT, "adjoint_state_gradients_b200", "csrc", "mw_stencil.cu")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nt", type=int, default=None, help="override nt (profiling runs only)")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------
+# algorithmic bytes per cell-update (fixed before tuning)
+
+
+def alg_bytes(wl, S, C):
+    """Bytes per cell-update of each pass of the checkpointed sweep (fp32)."""
+    band = 2.0 * wl.n_pml / wl.nx + 2.0 * wl.n_pml / wl.ny
+    model = 8.0 / S  # Ca, Cb shared by the shots
+    fwd = 24.0 + model + 16.0 * band + 28.0 / C           # + checkpoint write
+    replay = 24.0 + model + 16.0 * band + 8.0 + 28.0 / C  # + fp32 snapshot store + ckpt read
+    adj = 24.0 + model + 16.0 * band + 8.0 + 16.0         # + snapshot read + grad RMW
+    return fwd, replay, adj
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mw_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.uuid], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.remove(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def traffic_record():
+    """DRAM bytes per adjoint launch from the committed ncu summary, if the
+    kernel source has not changed since it was taken."""
+    try:
+        with open(os.path.join(PROFILES, "adjoint_traffic.json")) as fh:
+            d = json.load(fh)
+        with open(STENCIL_SRC, "rb") as fh:
+            h = hashlib.sha256(fh.read()).hexdigest()[:16]
+        if d.get("stencil_sha") != h:
+            return None
+        return float(d["dram_bytes_per_launch_full"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------
+# CPU (oracle) baseline: bounded sample of the same workload
+
+
+def oracle_sample(nt_sample=48, C=16):
+    """Time the fp64 oracle on one shot of the workload for nt_sample steps
+    (forward with checkpoints, replay, adjoint)."""
+    import oracle
+    from adjoint_state_gradients_b200 import synth
+    inp = synth.make_inputs(WORKLOAD, n_shots=1)
+    wl = inp.wl
+    vmax = oracle.c0() / math.sqrt(inp.eps_min)
+    dt = wl.cfl_fraction * oracle.cfl_dt(wl.order, wl.h, wl.h, vmax)
+    ca, cb, cq = oracle.model(inp.eps_r, inp.sigma, None, dt)
+    py = oracle.cpml(wl.ny, wl.n_pml, wl.h, dt, vmax, wl.f0)
+    px = oracle.cpml(wl.nx, wl.n_pml, wl.h, dt, vmax, wl.f0)
+    sim = oracle.Sim(ny=wl.ny, nx=wl.nx, order=wl.order, dy=wl.h, dx=wl.h, ca=ca, cb=cb,
+                     cq=float(cq.reshape(-1)[0]), prof_y=py, prof_x=px, src_idx=inp.src_idx,
+                     rec_idx=inp.rec_idx)
+    f = inp.wavelet(dt, nt_sample)
+    res = synth.rng(7).normal(size=(nt_sample, 1, wl.n_rec))
+    t0 = time.perf_counter()
+    sim.fwd_adj_ckpt(f, res, C)
+    el = time.perf_counter() - t0
+    cells = sim.ny * sim.nx * nt_sample
+    return cells / el / 1e9, el, oracle.num_threads(), \
+        f"1 of 8 shots, first {nt_sample} of 4000 steps, checkpoint every {C}: forward + replay + adjoint"
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from adjoint_state_gradients_b200 import synth
+    wl = synth.WORKLOADS[WORKLOAD]
+    vals, els = [], []
+    for i in range(args.warmup + args.steps):
+        v, el, cores, sample = oracle_sample(nt_sample=24, C=8)
+        if i >= args.warmup:
+            vals.append(v)
+            els.append(el)
+    value = sum(vals) / len(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1000 * sum(els) / len(els), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "grid": [wl.ny, wl.nx], "order": wl.order, "nt": wl.nt,
+                   "shots_per_gpu": wl.n_shots, "snapshots": "checkpoint every 64 + replay"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from adjoint_state_gradients_b200 import api, mwtm, synth
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        args.gpus = world if world > 1 else args.gpus
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+
+    wl = synth.WORKLOADS[WORKLOAD]
+    nt = args.nt or wl.nt
+    inp = synth.make_inputs(WORKLOAD)
+    S = wl.n_shots
+    c0 = 299792458.0
+    vmax = c0 / math.sqrt(inp.eps_min)
+    dt = wl.cfl_fraction * mwtm.cfl_dt(wl.order, wl.h, wl.h, vmax)
+    C = wl.ckpt_every
+
+    prob = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
+                       vmax=vmax, snapshot="ckpt", ckpt_every=C)
+    f_host = inp.wavelet(dt, nt).astype(np.float32)
+    eps_h = inp.eps_r.astype(np.float32)
+    sig_h = inp.sigma.astype(np.float32)
+    # observed data from the perturbed model (setup, outside the timed region)
+    obs = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
+                      vmax=vmax, snapshot="none")
+    obs.set_model_eps_sigma(inp.eps_r_true.astype(np.float32), sig_h, f0=wl.f0)
+    f_dev = torch.as_tensor(f_host, device=dev)
+    d_obs = obs.forward(f_dev).clone()
+    del obs
+    torch.cuda.synchronize()
+    prob.set_model_eps_sigma(eps_h, sig_h, f0=wl.f0)
+    gca = torch.empty((wl.ny, wl.nx), device=dev)
+    gcb = torch.empty((wl.ny, wl.nx), device=dev)
+    gca_s = torch.empty((S, wl.ny, wl.nx), device=dev)
+    gcb_s = torch.empty((S, wl.ny, wl.nx), device=dev)
+    rec = torch.empty((nt, S, wl.n_rec), device=dev)
+    res = torch.empty_like(rec)
+    J = torch.zeros(1, dtype=torch.float64, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev_fwd=None):
+        prob.forward(f_dev, rec=rec)
+        if ev_fwd is not None:
+            ev_fwd.record(stream)
+        prob.residual(rec, d_obs, res=res, J=J)
+        gca_s.zero_()
+        gcb_s.zero_()
+        prob.adjoint(res, gca=gca_s, gcb=gcb_s)
+        prob.combine(gca_s, out=gca)
+        prob.combine(gcb_s, out=gcb)
+        if world > 1:
+            dist.all_reduce(gca)
+            dist.all_reduce(gcb)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc = prob.status()
+    if rc != mwtm.MW_OK:
+        raise RuntimeError(f"device status {rc}: {mwtm.last_error()}")
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    if not uuid.startswith("GPU-"):
+        uuid = "GPU-" + uuid
+    clocks = Clocks(uuid)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    mwtm.profile_enable(True)
+    n0 = mwtm.launch_count()
+    clocks.start()
+    ev0.record(stream)
+    for k in range(args.steps):
+        evs[k][0].record(stream)
+        step(ev_fwd=evs[k][1])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    n_launch = mwtm.launch_count() - n0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    counts, ms = mwtm.profile_read(3)
+    mwtm.profile_enable(False)
+    total_ms = ev0.elapsed_time(ev1)
+    fwd_ms = sum(a.elapsed_time(b) for a, b in evs)
+    t = torch.tensor([total_ms, fwd_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_ms = float(t[0]), float(t[1])
+
+    cells = wl.ny * wl.nx * nt * S * world
+    value = cells * args.steps / (total_ms / 1e3) / 1e9
+    value_fwd = cells * args.steps / (fwd_ms / 1e3) / 1e9
+    b_fwd, b_rep, b_adj = alg_bytes(wl, S, C)
+    peak, peak_kind = measured_peaks()
+    sweep_bytes = (b_fwd + b_rep + b_adj) * cells * args.steps
+    sweep_frac = sweep_bytes / (total_ms / 1e3) / 1e9 / peak / world
+    adj_launch_ms = ms[2] / max(counts[2], 1)
+    adj_bytes = b_adj * wl.ny * wl.nx * S
+    achieved = adj_bytes / (adj_launch_ms / 1e3) / 1e9
+    rep_launch_ms = ms[1] / max(counts[1], 1)
+    fwd_launch_ms = ms[0] / max(counts[0], 1)
+    traffic = traffic_record()
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda a: torch.as_tensor(a).pin_memory()
+        f_p, eps_p, sig_p = pin(f_host), pin(eps_h), pin(sig_h)
+        dobs_p = d_obs.cpu().pin_memory()
+        outs = [torch.empty(1, dtype=torch.float64).pin_memory(),
+                torch.empty((wl.ny, wl.nx)).pin_memory(), torch.empty((wl.ny, wl.nx)).pin_memory()]
+
+        def e2e_step():
+            prob.set_model_eps_sigma(eps_p.to(dev, non_blocking=True), sig_p.to(dev, non_blocking=True),
+                                     f0=wl.f0)
+            fd = f_p.to(dev, non_blocking=True)
+            do = dobs_p.to(dev, non_blocking=True)
+            prob.forward(fd, rec=rec)
+            prob.residual(rec, do, res=res, J=J)
+            gca_s.zero_()
+            gcb_s.zero_()
+            prob.adjoint(res, gca=gca_s, gcb=gcb_s)
+            prob.combine(gca_s, out=gca)
+            prob.combine(gcb_s, out=gcb)
+            if world > 1:
+                dist.all_reduce(gca)
+                dist.all_reduce(gcb)
+            for o, src in zip(outs, (J, gca, gcb)):
+                o.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        h2d = sum(x.numel() * x.element_size() for x in (f_p, eps_p, sig_p, dobs_p))
+        d2h = sum(x.numel() * x.element_size() for x in outs)
+        e2e = {"value": round(cells * args.steps / (float(e_ms[0]) / 1e3) / 1e9, 4), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, el, cores, sample = oracle_sample()
+        cpu = {"value": round(v, 6), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+               "seconds": round(el, 2)}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "grid": [wl.ny, wl.nx], "interior": wl.n_interior,
+                       "n_pml": wl.n_pml, "order": wl.order, "nt": nt, "shots_per_gpu": S,
+                       "n_rec": wl.n_rec, "snapshots": f"checkpoint every {C} steps + segment replay",
+                       "l2": "inputs larger than L2 (one state buffer is "
+                             f"{prob.p.n_shots * wl.ny * wl.nx * 12 / 1e6:.0f} MB)",
+                       "parallelism": f"shots sharded, {world} rank(s)"},
+            "value_fwd": round(value_fwd, 4),
+            "value_interior": round(value * (wl.n_interior ** 2) / (wl.ny * wl.nx), 4),
+            "hbm_frac_sweep": round(sweep_frac, 4),
+            "alg_bytes_per_cell": {"forward": round(b_fwd, 3), "replay": round(b_rep, 3),
+                                   "adjoint": round(b_adj, 3)},
+            "roofline": {"bound": "hbm", "kernel": "k_adjoint<2,false>", "achieved": round(achieved, 1),
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4),
+                         "traffic": traffic, "alg_bytes_per_launch": adj_bytes,
+                         "avg_launch_ms": round(adj_launch_ms, 4)},
+            "kernel_ms": {"forward": round(fwd_launch_ms, 4), "forward_store": round(rep_launch_ms, 4),
+                          "adjoint": round(adj_launch_ms, 4), "launches": counts},
+            "gpu_launches": int(n_launch),
+            "J": float(J.cpu()[0]),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,221 @@
+/*
+ * mw_tm.h -- C ABI of the B200 (sm_100a) 2-D TM Maxwell FDTD library:
+ * forward time stepping, exact discrete adjoint and adjoint-state model
+ * gradients, batched over shots.
+ *
+ * The method is the one stated in the header comment of the page
+ * "tide-GPR 0.0.9 ... tide/csrc/maxwell.cu" ("EXACT DISCRETE Adjoint State
+ * Method for Maxwell TM equations"):
+ *   forward   H^{n+1/2} = H^{n-1/2} -/+ Cq psi(D^h E^n)          (Hx: -, Hz: +)
+ *             E^{n+1}   = Ca E^n + Cb (psi(D_x Hz) - psi(D_z Hx))
+ *   adjoint   the same step transposed, run backwards in time
+ *   gradients dJ/dCa = sum_n E^n lambda^{n+1},  dJ/dCb = sum_n curlH^n lambda^{n+1}
+ * psi is the CPML operator of the page's H / E kernels: memory m <- b m + a d,
+ * output d / k + m.
+ *
+ * Conventions used by every entry point
+ * -------------------------------------
+ *  - Grid: ny rows (y = depth z) by nx columns (x), row-major; cell index
+ *    j = y * nx + x.  Ey at (y, x), Hx at (y + 1/2, x), Hz at (y, x + 1/2).
+ *    Every array cell of every field is updated; fields are zero outside the
+ *    array.  nx must be a multiple of 4 (rows are read as float4).
+ *  - Per-shot arrays are [S][ny][nx] float32, time series are time-major
+ *    [nt][S][n] float32 (the page's source / receiver kernels).
+ *  - Source / receiver positions are flat per-shot cell indices int64
+ *    [S][n_src] / [S][n_rec]; -1 marks an inactive entry.  Duplicate source
+ *    cells add up (applied in index order); inactive receivers record 0.
+ *  - Pointers named *_dev are device memory; *_host are host memory.  The
+ *    caller owns every buffer.  Nothing allocates device memory per call.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Compute calls are asynchronous and stream-ordered; they
+ *    return after enqueueing.  Errors found on the host return at once;
+ *    device-side status (non-finite fields) is reported by mw_sync_status.
+ *  - Return codes: MW_OK (0) or a negative MW_ERR_*; mw_last_error() gives a
+ *    thread-local message.  No entry point aborts the process.
+ *
+ * State layout (one buffer, float32, mw_state_floats() floats), used for the
+ * forward state (Ey, Hx, Hz, CPML memories) and the adjoint state (their
+ * adjoints):
+ *    [0] Ey    [S][ny][nx]
+ *    [1] Hx    [S][ny][nx]
+ *    [2] Hz    [S][ny][nx]
+ *    [3] m_ey_x  x-band memory at Hz nodes     [S][ny][2*Wx]
+ *    [4] m_hz_x  x-band memory at Ey nodes     [S][ny][2*Wx]
+ *    [5] m_ey_z  z-band memory at Hx nodes     [S][2*Wz][nx]
+ *    [6] m_hx_z  z-band memory at Ey nodes     [S][2*Wz][nx]
+ *  Wx = round_up(n_pml + 1, 4), Wz = n_pml + 1 (0 when n_pml == 0).  The
+ *  x band holds columns [0, Wx) then [nx - Wx, nx); the z band rows
+ *  [0, Wz) then [ny - Wz, ny).  CPML coefficients a and b must vanish, and
+ *  k must equal 1, outside those bands (the memories exist only there).
+ */
+#ifndef MW_TM_H
+#define MW_TM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define MW_OK 0
+#define MW_ERR_ARG (-1)         /* invalid argument, shape or index        */
+#define MW_ERR_CFL (-2)         /* dt above the stability bound             */
+#define MW_ERR_WORKSPACE (-3)   /* workspace missing or too small           */
+#define MW_ERR_CUDA (-4)        /* a CUDA runtime call failed               */
+#define MW_ERR_NONFINITE (-5)   /* NaN / Inf found in a field (device flag) */
+#define MW_ERR_UNSUPPORTED (-7) /* valid request this build does not serve  */
+
+/* forward snapshot storage for the gradient */
+#define MW_SNAP_NONE 0 /* records only; mw_tm_adjoint_grad unavailable       */
+#define MW_SNAP_FP32 1 /* Ey^n and curl^n of every step, float32, on the GPU */
+#define MW_SNAP_BF16 2 /* same, rounded to bfloat16 (round to nearest even)  */
+#define MW_SNAP_CKPT 3 /* full state every ckpt_every steps; the adjoint
+                          replays each segment into an fp32 segment buffer  */
+
+typedef struct mw_params {
+  int32_t ny, nx;        /* array size incl. the CPML band                 */
+  int32_t order;         /* stencil order: 2, 4, 6 or 8                      */
+  int32_t n_shots;       /* S                                                */
+  int32_t n_src, n_rec;  /* sources / receivers per shot (may be 0)          */
+  int32_t nt;            /* time steps of this call                          */
+  double dt, dy, dx;     /* s, m, m                                          */
+  int32_t n_pml;         /* CPML band width in cells, all four sides         */
+  int32_t model_batched; /* 0: Ca, Cb (and Cq array) [ny][nx] shared;
+                            1: [S][ny][nx] per shot                          */
+  int32_t cq_is_scalar;  /* 1: cq points to one float (mu_r constant)        */
+  int32_t snap_mode;     /* MW_SNAP_*                                        */
+  int32_t ckpt_every;    /* C for MW_SNAP_CKPT                               */
+  int32_t grad_mask_pml; /* 1: accumulate gradients only at cells outside the
+                            CPML band (the page's masking); 0: everywhere    */
+  double vmax;           /* fastest wave speed in the model, m/s (CFL check) */
+  int32_t allow_unstable;/* 1: skip the CFL check                            */
+  int32_t check_finite;  /* 1: flag NaN / Inf in the final state             */
+} mw_params;
+
+/* Fill *p with defaults (zeros, cq_is_scalar = 1, snap_mode NONE). */
+void mw_params_init(mw_params *p);
+
+/* Floats in one state buffer (layout above). 0 on invalid params. */
+size_t mw_state_floats(const mw_params *p);
+
+/* Bytes of workspace mw_tm_forward / mw_tm_adjoint_grad need for p (ping-pong
+ * state buffers, adjoint state, snapshots or checkpoints + segment buffer).
+ * The same workspace carries the forward's snapshots to the adjoint.  0 on
+ * invalid params. */
+size_t mw_workspace_bytes(const mw_params *p);
+
+/* Largest stable dt for stencil `order` and wave speed vmax:
+ * 1 / (vmax * sum_k |c_k| * sqrt(1/dx^2 + 1/dy^2)).  Negative on bad input. */
+double mw_cfl_dt(int32_t order, double dy, double dx, double vmax);
+
+/* Check p (sizes, order, band fits, CFL unless allow_unstable).  Host only. */
+int mw_validate(const mw_params *p);
+
+/* Model coefficients from relative permittivity, conductivity (S/m) and
+ * relative permeability, float32 device arrays of the model's shape
+ * ([ny][nx] or [S][ny][nx] when model_batched):
+ *   Ca = (1 - s dt / (2 eps)) / (1 + s dt / (2 eps)),  Cb = dt / (eps + s dt / 2),
+ *   Cq = dt / (mu0 mu_r),  eps = eps0 eps_r
+ * (the forms whose derivatives the page's epsilon / sigma conversion kernel
+ * uses).  Computed in fp64, stored as float32.  sigma_dev may be NULL (0);
+ * mu_r_dev may be NULL (1): then cq_dev receives one float when
+ * p->cq_is_scalar, else a full array. */
+int mw_model_from_eps_sigma(const mw_params *p, const float *eps_r_dev,
+                            const float *sigma_dev, const float *mu_r_dev,
+                            float *ca_dev, float *cb_dev, float *cq_dev,
+                            void *stream);
+
+/* CPML profiles, float32 device array of 6*(ny + nx) floats:
+ *   [ay, ayh, by, byh, ky, kyh] (ny each) then [ax, axh, bx, bxh, kx, kxh]
+ *   (nx each); "h" = half node (i + 1/2).  Quadratic damping
+ *   d = d_max s^2, d_max = -3 vmax ln(R) / (2 n_pml h), kappa = 1,
+ *   alpha = pi f0 (1 - s), b = exp(-(d + alpha) dt), a = d (b - 1) / (d + alpha),
+ *   s = distance into the band / band width.  Any profile obeying the band
+ *   rule in the layout note may be passed instead. */
+int mw_cpml_profiles(const mw_params *p, double f0, double R, float *cpml_dev,
+                     void *stream);
+
+/* Forward: nt steps of H update, E update (+ snapshot / checkpoint store),
+ * source injection f[t], receiver sampling rec[t] = Ey after injection
+ * (order of the page's forward host loop).
+ *   ca, cb     model [ny][nx] or [S][ny][nx]
+ *   cq         one float or an array shaped like ca (p->cq_is_scalar)
+ *   cpml       6*(ny+nx) profile floats (mw_cpml_profiles layout)
+ *   f          [nt][S][n_src] source amplitudes added to Ey (may be NULL if n_src == 0)
+ *   state      in/out state buffer (layout above), or NULL to start from rest
+ *              (the final state then stays in the workspace)
+ *   rec        [nt][S][n_rec] out (may be NULL)
+ *   workspace  mw_workspace_bytes(p) bytes of device memory
+ * Sources / receivers of step t use time index t of this call. */
+int mw_tm_forward(const mw_params *p, const float *ca_dev, const float *cb_dev,
+                  const float *cq_dev, const float *cpml_dev, const float *f_dev,
+                  const int64_t *src_idx_dev, const int64_t *rec_idx_dev,
+                  float *state_dev, float *rec_dev, void *workspace_dev,
+                  size_t workspace_bytes, void *stream);
+
+/* Adjoint sweep t = nt-1 .. 0 and per-shot gradients, after mw_tm_forward
+ * with the same p, model, sources and workspace (snap_mode != NONE).  Per
+ * step: lambda_E[rec] += res[t]; grad_f[t] = lambda_E[src];
+ * grad_ca_shot += Ey^t lambda_E; grad_cb_shot += curl^t lambda_E; then the
+ * transposed E and H updates, CPML band included.
+ *   res            [nt][S][n_rec] adjoint source (d - d_obs for 1/2||d - d_obs||^2)
+ *   grad_*_shot    [S][ny][nx] accumulated (+=): zero them for a fresh gradient
+ *   grad_f         [nt][S][n_src] out, or NULL
+ *   adj_state      in/out adjoint state, or NULL (start from zero)
+ * In MW_SNAP_CKPT mode the forward is replayed segment by segment from the
+ * checkpoints, which needs f and src_idx again. */
+int mw_tm_adjoint_grad(const mw_params *p, const float *ca_dev,
+                       const float *cb_dev, const float *cq_dev,
+                       const float *cpml_dev, const float *f_dev,
+                       const int64_t *src_idx_dev, const int64_t *rec_idx_dev,
+                       const float *res_dev, float *grad_ca_shot_dev,
+                       float *grad_cb_shot_dev, float *grad_f_dev,
+                       float *adj_state_dev, void *workspace_dev,
+                       size_t workspace_bytes, void *stream);
+
+/* Shot reduction (the page's combine_grad, over every cell):
+ * grad[j] (+)= sum_{s=0..S-1} grad_shot[s][j], shots summed in order in
+ * float32.  accumulate = 0 overwrites, 1 adds. */
+int mw_combine_grad(const mw_params *p, const float *grad_shot_dev,
+                    float *grad_dev, int32_t accumulate, void *stream);
+
+/* Chain rule to relative permittivity and conductivity (the page's
+ * convert_grad_ca_cb_to_eps_sigma): with dCa/deps = (1-Ca)Cb/dt,
+ * dCb/deps = -Cb^2/dt, dCa/dsigma = -(1+Ca)Cb/2, dCb/dsigma = -Cb^2/2,
+ *   grad_eps_r = eps0 (gCa dCa/deps + gCb dCb/deps),
+ *   grad_sigma = gCa dCa/dsigma + gCb dCb/dsigma.
+ * n cells; either output may be NULL. */
+int mw_grad_eps_sigma(int64_t n, double dt, const float *ca_dev,
+                      const float *cb_dev, const float *grad_ca_dev,
+                      const float *grad_cb_dev, float *grad_eps_r_dev,
+                      float *grad_sigma_dev, void *stream);
+
+/* Residual res = d - d_obs over n values and, when J_dev is not NULL, the
+ * misfit J = 1/2 sum res^2 (one double, fixed summation order). */
+int mw_residual(int64_t n, const float *d_dev, const float *d_obs_dev,
+                float *res_dev, double *J_dev, void *stream);
+
+/* Wait for `stream` and report device-side status recorded in the workspace
+ * by earlier calls (MW_ERR_NONFINITE), then clear it. */
+int mw_sync_status(void *workspace_dev, void *stream);
+
+/* Thread-local message of the last failing call ("" if none). */
+const char *mw_last_error(void);
+
+/* Per-kernel timing (CUDA events around each launch of the three stencil
+ * kernels: 0 forward, 1 forward with snapshot store, 2 adjoint).  enable = 1
+ * clears and starts recording; mw_profile_read synchronizes the recorded
+ * events and returns, per class, the launch count and total milliseconds. */
+int mw_profile_enable(int32_t enable);
+int mw_profile_read(int64_t *counts, double *total_ms, int32_t n_classes);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * entry points, all devices).  Host counter; no synchronization. */
+int64_t mw_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MW_TM_H */
