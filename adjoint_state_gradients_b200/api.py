@@ -49,6 +49,7 @@ class Problem:
         self.rec_idx = _dev(rec_idx if rec_idx.size else np.zeros((self.S, 1), np.int64),
                             torch.int64, device)
         self.workspace = torch.empty(mwtm.workspace_bytes(self.p) // 4 + 64, dtype=F32, device=device)
+        mwtm.workspace_init(self.workspace)
         self.cpml = torch.empty(6 * (ny + nx), dtype=F32, device=device)
         self.ca = self.cb = self.cq = None
         self.state = None

@@ -16,59 +16,59 @@ namespace {
 constexpr double kEps0 = 8.8541878128e-12;  // F/m (the page's EP0)
 constexpr double kMu0 = 1.25663706212e-6;   // H/m (CODATA 2018)
 
-// One block per shot.  Thread 0 applies the sources in index order (so
-// duplicate cells add up deterministically), then the block samples the
-// receivers.  Out-of-range indices set a status flag and are skipped.
-__global__ void k_src_rec(float *__restrict__ ey, int64_t numel, const float *__restrict__ f_t,
-                          const int64_t *__restrict__ src, int ns, const int64_t *__restrict__ rec,
-                          int nr, float *__restrict__ r_t, int *__restrict__ flags) {
+// Duplicate chains of a per-shot index list idx [S][n] (one block per shot):
+// lead[k] = 1 when k is the first entry with its cell, next[k] = the next
+// entry with the same cell (-1 at the end of the chain).  Inactive (-1)
+// entries are never leaders; out-of-range entries set a status flag.
+__global__ void k_dup_chains(const int64_t *__restrict__ idx, int n, int64_t numel,
+                             int *__restrict__ lead, int *__restrict__ next,
+                             int *__restrict__ flags) {
   const int s = blockIdx.x;
-  float *e = ey + (int64_t)s * numel;
-  if (threadIdx.x == 0 && f_t != nullptr) {
-    for (int k = 0; k < ns; ++k) {
-      const int64_t i = src[(int64_t)s * ns + k];
-      if (i >= 0 && i < numel) {
-        e[i] += f_t[(int64_t)s * ns + k];
-      } else if (i != -1 && flags) {
-        atomicOr(flags + kFlagBadIndex, 1);
+  const int64_t *v = idx + (int64_t)s * n;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const int64_t c = v[k];
+    const bool ok = c >= 0 && c < numel;
+    if (!ok && c != -1 && flags) atomicOr(flags + kFlagBadIndex, 1);
+    int first = ok ? 1 : 0, nx = -1;
+    for (int j = 0; j < n && ok; ++j) {
+      if (v[j] != c) continue;
+      if (j < k) first = 0;
+      if (j > k) {
+        nx = j;
+        break;
       }
     }
-  }
-  __syncthreads();
-  if (r_t != nullptr) {
-    for (int k = threadIdx.x; k < nr; k += blockDim.x) {
-      const int64_t i = rec[(int64_t)s * nr + k];
-      const bool ok = i >= 0 && i < numel;
-      if (!ok && i != -1 && flags) atomicOr(flags + kFlagBadIndex, 1);
-      r_t[(int64_t)s * nr + k] = ok ? e[i] : 0.f;
-    }
+    lead[(int64_t)s * n + k] = first;
+    next[(int64_t)s * n + k] = nx;
   }
 }
 
-// Transpose: lambda_E[rec] += res[t] (thread 0, index order), then
-// grad_f[t] = lambda_E[src].
-__global__ void k_adj_src_rec(float *__restrict__ lam, int64_t numel,
-                              const float *__restrict__ res_t, const int64_t *__restrict__ rec,
-                              int nr, const int64_t *__restrict__ src, int ns,
-                              float *__restrict__ gf_t, int *__restrict__ flags) {
+// One block per shot: add vals_t[s][k] into field cells idx_a[s][k] -- each
+// chain leader sums its duplicates in index order, so the result does not
+// depend on scheduling -- then sample the field at idx_b into out_t
+// (inactive or out-of-range entries give 0).  Forward: sources then
+// receivers; adjoint: receiver residuals then the source gradient.
+__global__ void k_inject_sample(float *__restrict__ field, int64_t numel,
+                                const float *__restrict__ vals_t, const int64_t *__restrict__ idx_a,
+                                const int *__restrict__ lead, const int *__restrict__ next, int na,
+                                const int64_t *__restrict__ idx_b, int nb,
+                                float *__restrict__ out_t) {
   const int s = blockIdx.x;
-  float *e = lam + (int64_t)s * numel;
-  if (threadIdx.x == 0 && res_t != nullptr) {
-    for (int k = 0; k < nr; ++k) {
-      const int64_t i = rec[(int64_t)s * nr + k];
-      if (i >= 0 && i < numel) {
-        e[i] += res_t[(int64_t)s * nr + k];
-      } else if (i != -1 && flags) {
-        atomicOr(flags + kFlagBadIndex, 1);
-      }
+  float *e = field + (int64_t)s * numel;
+  if (vals_t != nullptr) {
+    const int64_t base = (int64_t)s * na;
+    for (int k = threadIdx.x; k < na; k += blockDim.x) {
+      if (!lead[base + k]) continue;
+      float v = vals_t[base + k];
+      for (int j = next[base + k]; j >= 0; j = next[base + j]) v += vals_t[base + j];
+      e[idx_a[base + k]] += v;
     }
   }
   __syncthreads();
-  if (gf_t != nullptr) {
-    for (int k = threadIdx.x; k < ns; k += blockDim.x) {
-      const int64_t i = src[(int64_t)s * ns + k];
-      const bool ok = i >= 0 && i < numel;
-      gf_t[(int64_t)s * ns + k] = ok ? e[i] : 0.f;
+  if (out_t != nullptr) {
+    for (int k = threadIdx.x; k < nb; k += blockDim.x) {
+      const int64_t i = idx_b[(int64_t)s * nb + k];
+      out_t[(int64_t)s * nb + k] = (i >= 0 && i < numel) ? e[i] : 0.f;
     }
   }
 }
@@ -138,6 +138,31 @@ __global__ void k_cpml(int ny, int nx, int n_pml, double dy, double dx, double d
   }
 }
 
+// Band coefficient table from the 6*(ny+nx) profile floats (see BandTab).
+__global__ void k_band_table(const float *__restrict__ cpml, int ny, int nx, int Wx, int Wz,
+                             float *__restrict__ out) {
+  const BandTab bt{Wx, Wz};
+  const float *py = cpml, *px = cpml + 6 * (int64_t)ny;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < 6 * 2 * Wx + 6 * 2 * Wz;
+       t += gridDim.x * blockDim.x) {
+    if (t < 12 * Wx) {
+      const int k = t / (2 * Wx), j = t % (2 * Wx);
+      const int c = j < Wx ? j : nx - 2 * Wx + j;
+      // profile vector order: a, ah, b, bh, k, kh; table order a, b, 1/k, ah, bh, 1/kh
+      const int src = (k % 3) * 2 + (k >= 3 ? 1 : 0);
+      const float v = px[(int64_t)src * nx + c];
+      out[bt.x(k) + j] = (k % 3 == 2) ? 1.0f / v : v;
+    } else {
+      const int u = t - 12 * Wx;
+      const int k = u / (2 * Wz), j = u % (2 * Wz);
+      const int r = j < Wz ? j : ny - 2 * Wz + j;
+      const int src = (k % 3) * 2 + (k >= 3 ? 1 : 0);
+      const float v = py[(int64_t)src * ny + r];
+      out[bt.z(k) + j] = (k % 3 == 2) ? 1.0f / v : v;
+    }
+  }
+}
+
 __global__ void k_combine(const float *__restrict__ gs, float *__restrict__ g, int S, int64_t n,
                           int accumulate) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -197,22 +222,20 @@ int grid_for(int64_t n, int block) {
 
 }  // namespace
 
-cudaError_t launch_src_rec(float *ey, int64_t numel, int S, const float *f_t, const int64_t *src,
-                           int ns, const int64_t *rec, int nr, float *r_t, int *flags,
-                           cudaStream_t st) {
-  if ((ns == 0 || f_t == nullptr) && (nr == 0 || r_t == nullptr)) return cudaSuccess;
-  k_src_rec<<<S, 128, 0, st>>>(ey, numel, ns > 0 ? f_t : nullptr, src, ns, rec, nr,
-                              nr > 0 ? r_t : nullptr, flags);
+cudaError_t launch_dup_chains(const int64_t *idx, int S, int n, int64_t numel, int *lead,
+                              int *next, int *flags, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  k_dup_chains<<<S, 256, 0, st>>>(idx, n, numel, lead, next, flags);
   count_launches(1);
   return cudaGetLastError();
 }
 
-cudaError_t launch_adj_src_rec(float *lam, int64_t numel, int S, const float *res_t,
-                               const int64_t *rec, int nr, const int64_t *src, int ns,
-                               float *gf_t, int *flags, cudaStream_t st) {
-  if ((nr == 0 || res_t == nullptr) && (ns == 0 || gf_t == nullptr)) return cudaSuccess;
-  k_adj_src_rec<<<S, 128, 0, st>>>(lam, numel, nr > 0 ? res_t : nullptr, rec, nr, src, ns,
-                                  ns > 0 ? gf_t : nullptr, flags);
+cudaError_t launch_inject_sample(float *field, int64_t numel, int S, const float *vals_t,
+                                 const int64_t *idx_a, const int *lead, const int *next, int na,
+                                 const int64_t *idx_b, int nb, float *out_t, cudaStream_t st) {
+  if ((na == 0 || vals_t == nullptr) && (nb == 0 || out_t == nullptr)) return cudaSuccess;
+  k_inject_sample<<<S, 256, 0, st>>>(field, numel, na > 0 ? vals_t : nullptr, idx_a, lead, next,
+                                     na, idx_b, nb, nb > 0 ? out_t : nullptr);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -236,6 +259,14 @@ cudaError_t launch_cpml(int ny, int nx, int n_pml, double dy, double dx, double 
                         double f0, double R, float *out, cudaStream_t st) {
   k_cpml<<<grid_for(6LL * (ny + nx), 256), 256, 0, st>>>(ny, nx, n_pml, dy, dx, dt, vmax, f0, R,
                                                           out);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_band_table(const float *cpml, int ny, int nx, int Wx, int Wz, float *out,
+                              cudaStream_t st) {
+  if (Wx == 0 && Wz == 0) return cudaSuccess;
+  k_band_table<<<grid_for(12LL * (Wx + Wz), 256), 256, 0, st>>>(cpml, ny, nx, Wx, Wz, out);
   count_launches(1);
   return cudaGetLastError();
 }

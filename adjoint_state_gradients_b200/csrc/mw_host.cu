@@ -96,6 +96,11 @@ int check_params(const mw_params *p, bool cfl) {
     return fail(MW_ERR_ARG, "snap_mode = %d", p->snap_mode);
   if (p->snap_mode == MW_SNAP_CKPT && p->ckpt_every < 1)
     return fail(MW_ERR_ARG, "ckpt_every = %d", p->ckpt_every);
+  if (p->snap_mode == MW_SNAP_BF16 && p->nx % 8 != 0)
+    return fail(MW_ERR_ARG, "bf16 snapshots need nx %% 8 == 0 (nx = %d)", p->nx);
+  if (2 * b.Wx > 256)
+    return fail(MW_ERR_UNSUPPORTED, "n_pml = %d: a band row exceeds one TMA box (n_pml <= 123)",
+                p->n_pml);
   if ((int64_t)p->ny * p->nx > ((int64_t)1 << 40)) return fail(MW_ERR_ARG, "grid too large");
   if (cfl && !p->allow_unstable) {
     if (!(p->vmax > 0) || !isfinite(p->vmax))
@@ -114,6 +119,13 @@ Layout layout(const mw_params *p) {
   const size_t sb = align256(L.state_bytes);
   size_t off = 0;
   L.flags = off; off += 256;
+  L.chains = off;
+  off += align256(2 * sizeof(int) * (size_t)p->n_shots * (p->n_src + p->n_rec));
+  L.bandtab = off;
+  {
+    const Bands b = bands(p);
+    off += align256(sizeof(float) * (size_t)BandTab{b.Wx, b.Wz}.floats() + 16);
+  }
   L.stA = off; off += sb;
   L.stB = off; off += sb;
   L.adA = L.adB = L.rpA = L.rpB = L.snap = L.seg = 0;
@@ -157,6 +169,16 @@ Fields fields_at(const mw_params *p, float *base) {
   return f;
 }
 
+// Duplicate-chain arrays (lead, next) of the sources and receivers.
+struct Chains {
+  int *src_lead, *src_next, *rec_lead, *rec_next;
+};
+Chains chains_at(const mw_params *p, char *ws, const Layout &L) {
+  int *c = (int *)(ws + L.chains);
+  const size_t ns = (size_t)p->n_shots * p->n_src, nr = (size_t)p->n_shots * p->n_rec;
+  return Chains{c, c + ns, c + 2 * ns, c + 2 * ns + nr};
+}
+
 // ---- launch geometry ------------------------------------------------------
 int sm_count() {
   static int cached = -1;
@@ -191,27 +213,29 @@ Launch plan(const mw_params *p, bool adjoint) {
   g.n_pml = p->n_pml;
   g.grad_mask = p->grad_mask_pml ? 1 : 0;
   g.numel = (int64_t)p->ny * p->nx;
-  g.n_strips = (p->nx + kStripCols - 1) / kStripCols;
+  g.strip_cols = adjoint ? kAdjStripCols : kFwdStripCols;
+  g.n_strips = (p->nx + g.strip_cols - 1) / g.strip_cols;
   const int P = p->order / 2;
-  const int warps_sm = stencil_slots_per_sm(p->order, adjoint);
+  const int warps_sm = stencil_slots_per_sm(p->order, adjoint, b.Wx);
   const int64_t slots = (int64_t)sm_count() * warps_sm;
   const int64_t cols_items = (int64_t)g.S * g.n_strips;
-  int best_nc = 1;
+  // Items are claimed dynamically by resident warps: time ~ total iterations
+  // spread over the slots plus one item of tail; each item walks its rows
+  // plus 4P - 2 warm-up rows.
+  const int w = 4 * P - 2;
+  int best_ch = p->ny;
   double best_cost = 1e300;
-  const int max_nc = p->ny < 4096 ? p->ny : 4096;
-  for (int nc = 1; nc <= max_nc; ++nc) {
-    const int ch = (p->ny + nc - 1) / nc;
-    if (ch < 8 && nc > 1) break;
-    const int nce = (p->ny + ch - 1) / ch;
-    const int64_t items = cols_items * nce;
-    const int64_t waves = (items + slots - 1) / slots;
-    const double cost = (double)waves * (ch + 4 * P - 2);
+  for (int ch = 8; ch <= p->ny + 7; ch += (ch < 64 ? 1 : 4)) {
+    const int nc = (p->ny + ch - 1) / ch;
+    const int chh = (p->ny + nc - 1) / nc;
+    const double items = (double)cols_items * nc;
+    const double cost = items * (chh + w) / (double)slots + (chh + w);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
-      best_nc = nce;
+      best_ch = chh;
     }
   }
-  g.chunk_h = (p->ny + best_nc - 1) / best_nc;
+  g.chunk_h = best_ch;
   g.n_chunks = (p->ny + g.chunk_h - 1) / g.chunk_h;
   const int64_t items = cols_items * g.n_chunks;
   int64_t grid = (items + kWarpsPerCta - 1) / kWarpsPerCta;
@@ -249,6 +273,113 @@ Prof prof_of(const mw_params *p, const float *cpml) {
   r.kx = x + 4 * nx;
   r.kxh = x + 5 * nx;
   return r;
+}
+
+// ---- TMA tensor maps ---------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// Row-box map over a dense array [d3][d2][d1][d0] (rank 3 or 4) of float32
+// (elem 4) or bf16 (elem 2): box = (box0, 1, 1[, 1]), zero fill outside.
+int encode_rows(CUtensorMap *map, const void *base, int elem, int rank, uint64_t d0, uint64_t d1,
+                uint64_t d2, uint64_t d3, uint32_t box0) {
+  EncodeTiledFn fn = encoder();
+  if (!fn) return fail(MW_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[4] = {d0, d1, d2, d3};
+  cuuint64_t strides[3] = {d0 * elem, d0 * d1 * elem, d0 * d1 * d2 * elem};
+  cuuint32_t box[4] = {box0, 1, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MW_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): rank %d dims %llu %llu %llu box %u",
+                (int)r, rank, (unsigned long long)d0, (unsigned long long)d1,
+                (unsigned long long)d2, box0);
+  return MW_OK;
+}
+
+#define MW_TRY(x)            \
+  do {                       \
+    int rc_ = (x);           \
+    if (rc_ != MW_OK) return rc_; \
+  } while (0)
+
+int fwd_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb, FwdMaps *m) {
+  memset(m, 0, sizeof *m);
+  const Bands bd = bands(p);
+  const uint64_t nx = p->nx, ny = p->ny, S = p->n_shots, Sm = p->model_batched ? p->n_shots : 1;
+  MW_TRY(encode_rows(&m->map[kLdEy], in.ey, 4, 3, nx, ny, S, 1, 136));
+  MW_TRY(encode_rows(&m->map[kLdHz], in.hz, 4, 3, nx, ny, S, 1, 128));
+  MW_TRY(encode_rows(&m->map[kLdHx], in.hx, 4, 3, nx, ny, S, 1, 120));
+  MW_TRY(encode_rows(&m->map[kLdCa], ca, 4, 3, nx, ny, Sm, 1, 120));
+  MW_TRY(encode_rows(&m->map[kLdCb], cb, 4, 3, nx, ny, Sm, 1, 120));
+  if (bd.Wx > 0) {
+    MW_TRY(encode_rows(&m->map[kLdMxh], in.mxh_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
+    MW_TRY(encode_rows(&m->map[kLdMxe], in.mxe_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
+    MW_TRY(encode_rows(&m->map[kLdMzh], in.mzh_node, 4, 3, nx, 2 * bd.Wz, S, 1, 120));
+    MW_TRY(encode_rows(&m->map[kLdMze], in.mze_node, 4, 3, nx, 2 * bd.Wz, S, 1, 120));
+  }
+  return MW_OK;
+}
+
+int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb,
+             const float *gca, const float *gcb, const void *se, const void *sc, int snap_elem,
+             int snap_steps, AdjMaps *m) {
+  memset(m, 0, sizeof *m);
+  const Bands bd = bands(p);
+  const uint64_t nx = p->nx, ny = p->ny, S = p->n_shots, Sm = p->model_batched ? p->n_shots : 1;
+  MW_TRY(encode_rows(&m->map[kLdLam], in.ey, 4, 3, nx, ny, S, 1, 128));
+  MW_TRY(encode_rows(&m->map[kLdCbA], cb, 4, 3, nx, ny, Sm, 1, 128));
+  MW_TRY(encode_rows(&m->map[kLdLhz], in.hz, 4, 3, nx, ny, S, 1, 120));
+  MW_TRY(encode_rows(&m->map[kLdSe], se, snap_elem, 4, nx, ny, S, snap_steps, 112));
+  MW_TRY(encode_rows(&m->map[kLdSc], sc, snap_elem, 4, nx, ny, S, snap_steps, 112));
+  MW_TRY(encode_rows(&m->map[kLdGca], gca, 4, 3, nx, ny, S, 1, 112));
+  MW_TRY(encode_rows(&m->map[kLdGcb], gcb, 4, 3, nx, ny, S, 1, 112));
+  MW_TRY(encode_rows(&m->map[kLdLhx], in.hx, 4, 3, nx, ny, S, 1, 112));
+  MW_TRY(encode_rows(&m->map[kLdCaA], ca, 4, 3, nx, ny, Sm, 1, 112));
+  MW_TRY(encode_rows(&m->map[kLdLamy], in.ey, 4, 3, nx, ny, S, 1, 112));
+  if (bd.Wx > 0) {
+    MW_TRY(encode_rows(&m->map[kLdMxeA], in.mxe_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
+    MW_TRY(encode_rows(&m->map[kLdMxhA], in.mxh_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
+    MW_TRY(encode_rows(&m->map[kLdMzeA], in.mze_node, 4, 3, nx, 2 * bd.Wz, S, 1, 112));
+    MW_TRY(encode_rows(&m->map[kLdMzhA], in.mzh_node, 4, 3, nx, 2 * bd.Wz, S, 1, 112));
+  }
+  return MW_OK;
+}
+
+// Per-call set-up shared by the forward and adjoint sweeps: the CPML band
+// coefficient table and the two work-item counters.
+int stencil_prologue(const mw_params *p, const float *cpml, char *ws, const Layout &L,
+                     cudaStream_t st) {
+  const Bands b = bands(p);
+  MW_CUDA(launch_band_table(cpml, p->ny, p->nx, b.Wx, b.Wz, (float *)(ws + L.bandtab), st));
+  MW_CUDA(cudaMemsetAsync(ws + L.flags + kCtrBase * sizeof(int), 0, 2 * sizeof(int), st));
+  return MW_OK;
+}
+
+void set_layout(StepArgs &a, const mw_params *p, bool adjoint) {
+  size_t smem;
+  stencil_layout(p->order, adjoint, bands(p).Wx, &a.stage_floats, &a.band_floats, &a.warp_floats,
+                 &smem);
+  a.band_box_floats = 2 * bands(p).Wx;
 }
 
 // ---- per-kernel event timing ------------------------------------------------
@@ -357,6 +488,13 @@ int mw_cpml_profiles(const mw_params *p, double f0, double R, float *cpml, void 
   return MW_OK;
 }
 
+int mw_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+  g_err.clear();
+  if (!workspace || workspace_bytes < 256) return fail(MW_ERR_WORKSPACE, "workspace too small");
+  MW_CUDA(cudaMemsetAsync(workspace, 0, 256, (cudaStream_t)stream));
+  return MW_OK;
+}
+
 int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const float *cq,
                   const float *cpml, const float *f, const int64_t *src_idx,
                   const int64_t *rec_idx, float *state, float *rec, void *workspace,
@@ -383,6 +521,7 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   float *bufA = state ? state : (float *)(ws + L.stA);
   float *bufB = (float *)(ws + L.stB);
   if (!state) MW_CUDA(cudaMemsetAsync(bufA, 0, L.state_bytes, st));
+  if (p->nt == 0) return MW_OK;
 
   StepArgs a{};
   const Launch lc = plan(p, false);
@@ -392,11 +531,25 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   a.ca = ca;
   a.cb = cb;
   a.cq = cq;
-  a.cq_scalar = 0.f;
+  a.flags = flags;
+  a.bt = (const float *)(ws + L.bandtab);
+  set_layout(a, p, false);
+  MW_TRY(stencil_prologue(p, cpml, ws, L, st));
+  FwdMaps mA, mB;  // input buffer A / B
+  MW_TRY(fwd_maps(p, fields_at(p, bufA), ca, cb, &mA));
+  MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, &mB));
 
   const int store = p->snap_mode == MW_SNAP_FP32 ? kStoreF32
                     : p->snap_mode == MW_SNAP_BF16 ? kStoreBF16 : kStoreNone;
   const int64_t SN = (int64_t)p->n_shots * p->ny * p->nx;
+  const int64_t numel = (int64_t)p->ny * p->nx;
+  const Chains ch = chains_at(p, ws, L);
+  if (p->n_src > 0)
+    MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
+                              flags, st));
+  if (p->n_rec > 0 && rec)  // chains unused here: this validates the receiver indices
+    MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
+                              flags, st));
   char *snap_e = ws + L.snap;
   char *snap_c = ws + L.snap + (size_t)p->nt * L.snap_step_bytes;
   float *cur = bufA, *nxt = bufB;
@@ -409,14 +562,16 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
     a.out = fields_at(p, nxt);
     a.snap_e = store ? snap_e + (size_t)t * L.snap_step_bytes : nullptr;
     a.snap_c = store ? snap_c + (size_t)t * L.snap_step_bytes : nullptr;
+    const FwdMaps &m = cur == bufA ? mA : mB;
+    a.ctr_slot = t & 1;
     MW_CUDA(timed(store ? 1 : 0, st, [&] {
-      return launch_forward(a, p->order, store, p->model_batched != 0, !p->cq_is_scalar, lc.grid,
-                            st);
+      return launch_forward(m, a, p->order, store, p->model_batched != 0, !p->cq_is_scalar,
+                            lc.grid, st);
     }));
-    MW_CUDA(launch_src_rec(nxt, p->ny * (int64_t)p->nx, p->n_shots,
-                           f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
-                           p->n_src, rec_idx, p->n_rec,
-                           rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, flags, st));
+    MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots,
+                                 f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
+                                 ch.src_lead, ch.src_next, p->n_src, rec_idx, p->n_rec,
+                                 rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, st));
     std::swap(cur, nxt);
   }
   if (cur != bufA) MW_CUDA(cudaMemcpyAsync(bufA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
@@ -455,9 +610,17 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   const int64_t numel = (int64_t)p->ny * p->nx;
   const int64_t SN = p->n_shots * numel;
 
+  const Chains ch = chains_at(p, ws, L);
+  if (p->n_rec > 0)
+    MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
+                              flags, st));
+  if (p->n_src > 0 && p->snap_mode == MW_SNAP_CKPT)
+    MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
+                              flags, st));
   float *adA = adj_state ? adj_state : (float *)(ws + L.adA);
   float *adB = (float *)(ws + L.adB);
   if (!adj_state) MW_CUDA(cudaMemsetAsync(adA, 0, L.state_bytes, st));
+  if (p->nt == 0) return MW_OK;
 
   const Launch la = plan(p, true);
   StepArgs a{};
@@ -469,45 +632,56 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   a.cq = cq;
   a.gca = gca;
   a.gcb = gcb;
-  a.cq_scalar = 0.f;
+  a.flags = flags;
+  a.bt = (const float *)(ws + L.bandtab);
+  set_layout(a, p, true);
+  MW_TRY(stencil_prologue(p, cpml, ws, L, st));
+  int launch_idx = 0;  // alternates the work counter between stencil launches
+
+  // snapshot source of the adjoint: the full store, or the replay segment
+  const bool ckpt = p->snap_mode == MW_SNAP_CKPT;
+  const int bf16 = p->snap_mode == MW_SNAP_BF16;
+  const int C = ckpt ? p->ckpt_every : p->nt;
+  const char *snap_e = ckpt ? ws + L.seg : ws + L.snap;
+  const char *snap_c = snap_e + (size_t)C * L.snap_step_bytes;
+  AdjMaps mA, mB;
+  MW_TRY(adj_maps(p, fields_at(p, adA), ca, cb, gca, gcb, snap_e, snap_c, bf16 ? 2 : 4, C, &mA));
+  MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, gca, gcb, snap_e, snap_c, bf16 ? 2 : 4, C, &mB));
 
   float *cur = adA, *nxt = adB;
-  auto adj_step = [&](int t, const char *se, const char *sc, int bf16) -> int {
-    MW_CUDA(launch_adj_src_rec(cur, numel, p->n_shots,
-                               res ? res + (int64_t)t * p->n_shots * p->n_rec : nullptr, rec_idx,
-                               p->n_rec, src_idx, p->n_src,
-                               grad_f ? grad_f + (int64_t)t * p->n_shots * p->n_src : nullptr,
-                               flags, st));
+  auto adj_step = [&](int t, int slot) -> int {
+    MW_CUDA(launch_inject_sample(cur, numel, p->n_shots,
+                                 res ? res + (int64_t)t * p->n_shots * p->n_rec : nullptr,
+                                 rec_idx, ch.rec_lead, ch.rec_next, p->n_rec, src_idx, p->n_src,
+                                 grad_f ? grad_f + (int64_t)t * p->n_shots * p->n_src : nullptr,
+                                 st));
     a.in = fields_at(p, cur);
     a.out = fields_at(p, nxt);
-    a.snap_e = (void *)se;
-    a.snap_c = (void *)sc;
+    a.snap_t = slot;
+    a.ctr_slot = (launch_idx++) & 1;
+    const AdjMaps &m = cur == adA ? mA : mB;
     MW_CUDA(timed(2, st, [&] {
-      return launch_adjoint(a, p->order, bf16, p->model_batched != 0, !p->cq_is_scalar, la.grid,
-                            st);
+      return launch_adjoint(m, a, p->order, bf16, p->model_batched != 0, !p->cq_is_scalar,
+                            la.grid, st);
     }));
     std::swap(cur, nxt);
     return MW_OK;
   };
 
-  if (p->snap_mode == MW_SNAP_FP32 || p->snap_mode == MW_SNAP_BF16) {
-    const char *snap_e = ws + L.snap;
-    const char *snap_c = ws + L.snap + (size_t)p->nt * L.snap_step_bytes;
-    const int bf16 = p->snap_mode == MW_SNAP_BF16;
-    for (int t = p->nt - 1; t >= 0; --t) {
-      rc = adj_step(t, snap_e + (size_t)t * L.snap_step_bytes,
-                    snap_c + (size_t)t * L.snap_step_bytes, bf16);
-      if (rc) return rc;
-    }
+  if (!ckpt) {
+    for (int t = p->nt - 1; t >= 0; --t) MW_TRY(adj_step(t, t));
   } else {
     // checkpoint mode: replay each segment from its checkpoint, newest first
     const Launch lf = plan(p, false);
     StepArgs fa = a;
     fa.g = lf.g;
-    const int C = p->ckpt_every;
-    char *seg_e = ws + L.seg;
-    char *seg_c = ws + L.seg + (size_t)C * L.snap_step_bytes;
+    set_layout(fa, p, false);
     float *rA = (float *)(ws + L.rpA), *rB = (float *)(ws + L.rpB);
+    FwdMaps fA, fB;
+    MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, &fA));
+    MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, &fB));
+    char *seg_e = ws + L.seg;
+    char *seg_c = seg_e + (size_t)C * L.snap_step_bytes;
     for (int k = L.n_seg - 1; k >= 0; --k) {
       const int t0 = k * C;
       const int t1 = (t0 + C < p->nt) ? t0 + C : p->nt;
@@ -519,20 +693,18 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
         fa.out = fields_at(p, rn);
         fa.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
         fa.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
+        const FwdMaps &fm = rc_ == rA ? fA : fB;
+        fa.ctr_slot = (launch_idx++) & 1;
         MW_CUDA(timed(1, st, [&] {
-          return launch_forward(fa, p->order, kStoreF32, p->model_batched != 0, !p->cq_is_scalar,
-                                lf.grid, st);
+          return launch_forward(fm, fa, p->order, kStoreF32, p->model_batched != 0,
+                                !p->cq_is_scalar, lf.grid, st);
         }));
-        MW_CUDA(launch_src_rec(rn, numel, p->n_shots,
-                               f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
-                               p->n_src, rec_idx, 0, nullptr, flags, st));
+        MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
+                                     f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
+                                     ch.src_lead, ch.src_next, p->n_src, nullptr, 0, nullptr, st));
         std::swap(rc_, rn);
       }
-      for (int t = t1 - 1; t >= t0; --t) {
-        rc = adj_step(t, seg_e + (size_t)(t - t0) * L.snap_step_bytes,
-                      seg_c + (size_t)(t - t0) * L.snap_step_bytes, 0);
-        if (rc) return rc;
-      }
+      for (int t = t1 - 1; t >= t0; --t) MW_TRY(adj_step(t, t - t0));
     }
   }
   if (cur != adA) MW_CUDA(cudaMemcpyAsync(adA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
@@ -582,9 +754,10 @@ int mw_sync_status(void *workspace, void *stream) {
   cudaStream_t st = (cudaStream_t)stream;
   MW_CUDA(cudaStreamSynchronize(st));
   if (!workspace) return MW_OK;
-  int h[2] = {0, 0};
+  int h[3] = {0, 0, 0};
   MW_CUDA(cudaMemcpy(h, workspace, sizeof h, cudaMemcpyDeviceToHost));
   MW_CUDA(cudaMemset(workspace, 0, sizeof h));
+  if (h[kFlagTimeout]) return fail(MW_ERR_TIMEOUT, "a stencil kernel timed out waiting for its copies");
   if (h[kFlagBadIndex]) return fail(MW_ERR_ARG, "a source or receiver index was out of range");
   if (h[kFlagNonFinite]) return fail(MW_ERR_NONFINITE, "non-finite value in a field or gradient");
   return MW_OK;

@@ -12,6 +12,7 @@
 // shared-memory row, so each cell's state is read and written once per step.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -19,15 +20,14 @@
 
 namespace mw {
 
-constexpr int kStripCols = 128;    // columns per warp (32 lanes x float4)
+constexpr int kFwdStripCols = 120;  // forward: columns owned per warp (30 float4)
+constexpr int kAdjStripCols = 112;  // adjoint: columns owned per warp (28 float4)
 constexpr int kWarpsPerCta = 4;
-constexpr int kEySlots = 36;       // 2 left halo + 32 own + 2 right halo float4
-constexpr int kHzSlots = 34;       // 1 left halo + 32 own + 1 right halo float4
 
 struct Geom {
   int ny, nx, S;
   int Wx, Wz;         // band widths (0: no CPML band)
-  int n_strips, n_chunks, chunk_h;
+  int strip_cols, n_strips, n_chunks, chunk_h;
   int n_pml;
   int grad_mask;      // adjoint: accumulate gradients outside the band only
   int64_t numel;      // ny * nx
@@ -60,10 +60,38 @@ struct StepArgs {
   Fields in, out;
   const float *ca, *cb, *cq;
   float cq_scalar;
-  // snapshots of this step ([S][ny][nx]; float or bf16), may be null
+  // forward: snapshots of this step ([S][ny][nx]; float or bf16), may be null
   void *snap_e, *snap_c;
-  // adjoint only: per-shot gradients [S][ny][nx]
+  // adjoint only: per-shot gradients [S][ny][nx]; time index of the
+  // snapshot tensor maps
   float *gca, *gcb;
+  int snap_t;
+  int *flags;         // device status words (wait timeouts, work counters)
+  int ctr_slot;       // work counter of this launch (flags[kCtrBase + ctr_slot])
+  // CPML band coefficients (BandTab layout), float4-aligned, 1/k precomputed
+  const float *bt;
+  // shared-memory layout of one warp (floats): stage size, band slot width
+  // (padded), band row width (the TMA box, 2*Wx)
+  int stage_floats, band_floats, warp_floats, band_box_floats;
+};
+
+// TMA tensor maps of one forward launch (the input buffer set and model),
+// indexed by load slot so that lane k of a warp can issue load k.  Boxes are
+// one row high, starting at x0 - 8 (ey, 136 wide), x0 - 4 (hz, 128 wide) or
+// x0 (120 wide); x-band memories take a whole band row (2*Wx).
+enum FwdLoad { kLdEy = 0, kLdHz, kLdHx, kLdCa, kLdCb, kLdMxh, kLdMxe, kLdMzh, kLdMze, kFwdLoads };
+struct FwdMaps {
+  CUtensorMap map[kFwdLoads];
+};
+// Adjoint: lam and cb 128 wide from x0 - 8, lhz 120 from x0 - 4, the rest 112
+// from x0 (lamy: lambda_E again, for the Ca term), snapshots 4-D (x, y, shot,
+// step), x-band memories a whole band row.
+enum AdjLoad {
+  kLdLam = 0, kLdCbA, kLdLhz, kLdSe, kLdSc, kLdGca, kLdGcb, kLdLhx, kLdCaA, kLdLamy, kLdMxeA,
+  kLdMxhA, kLdMzeA, kLdMzhA, kAdjLoads
+};
+struct AdjMaps {
+  CUtensorMap map[kAdjLoads];
 };
 
 // Workspace layout (byte offsets, 256-aligned).
@@ -74,6 +102,8 @@ struct Layout {
   size_t rpA, rpB;    // replay ping-pong state buffers (checkpoint mode)
   size_t snap;        // snapshots / checkpoints
   size_t seg;         // checkpoint mode: fp32 segment snapshot buffer
+  size_t chains;      // duplicate chains of the source / receiver indices
+  size_t bandtab;     // CPML band coefficient table (BandTab)
   size_t total;
   size_t state_bytes;
   size_t snap_step_bytes;  // one step of one snapshot field ([S][ny][nx])
@@ -82,33 +112,48 @@ struct Layout {
 
 enum StoreKind { kStoreNone = 0, kStoreF32 = 1, kStoreBF16 = 2 };
 
-// device status word indices in the flags area
-enum { kFlagNonFinite = 0, kFlagBadIndex = 1 };
+// device status word indices in the flags area; kCtrBase, kCtrBase + 1: the
+// work-item counters that consecutive stencil launches alternate between
+enum { kFlagNonFinite = 0, kFlagBadIndex = 1, kFlagTimeout = 2, kCtrBase = 32 };
+
+// CPML band coefficient table (floats; Wx, Wz as in Geom): x band per band
+// column j (array column j < Wx ? j : nx - 2*Wx + j), z band per band row.
+//   [0]   a_x   [1] b_x   [2] 1/k_x     (integer nodes)
+//   [3]   a_xh  [4] b_xh  [5] 1/k_xh    (half nodes)          2*Wx each
+//   [6..11] the same along z                                  2*Wz each
+struct BandTab {
+  int Wx, Wz;
+  __host__ __device__ int x(int k) const { return k * 2 * Wx; }
+  __host__ __device__ int z(int k) const { return 12 * Wx + k * 2 * Wz; }
+  __host__ __device__ int floats() const { return 12 * Wx + 12 * Wz; }
+};
 
 // count of kernel launches made by the library (mw_host.cu)
 void count_launches(int n);
 
 // stencil launchers (mw_stencil.cu); return a cudaError_t
-cudaError_t launch_forward(const StepArgs &a, int order, int store, bool batched,
-                           bool cq_array, int grid, cudaStream_t st);
-cudaError_t launch_adjoint(const StepArgs &a, int order, int snap_bf16,
-                           bool batched, bool cq_array, int grid,
-                           cudaStream_t st);
-int stencil_slots_per_sm(int order, bool adjoint);
+cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int store,
+                           bool batched, bool cq_array, int grid, cudaStream_t st);
+cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int snap_bf16,
+                           bool batched, bool cq_array, int grid, cudaStream_t st);
+// shared-memory layout (floats per stage / per warp) and dynamic smem bytes
+void stencil_layout(int order, bool adjoint, int Wx, int *stage_floats, int *band_floats,
+                    int *warp_floats, size_t *smem_bytes);
+int stencil_slots_per_sm(int order, bool adjoint, int Wx);
 
 // small kernels (mw_aux.cu)
-cudaError_t launch_src_rec(float *ey, int64_t numel, int S, const float *f_t,
-                           const int64_t *src, int ns, const int64_t *rec,
-                           int nr, float *r_t, int *flags, cudaStream_t st);
-cudaError_t launch_adj_src_rec(float *lam, int64_t numel, int S,
-                               const float *res_t, const int64_t *rec, int nr,
-                               const int64_t *src, int ns, float *gf_t,
-                               int *flags, cudaStream_t st);
+cudaError_t launch_dup_chains(const int64_t *idx, int S, int n, int64_t numel, int *lead,
+                              int *next, int *flags, cudaStream_t st);
+cudaError_t launch_inject_sample(float *field, int64_t numel, int S, const float *vals_t,
+                                 const int64_t *idx_a, const int *lead, const int *next, int na,
+                                 const int64_t *idx_b, int nb, float *out_t, cudaStream_t st);
 cudaError_t launch_check_finite(const float *x, int64_t n, int *flags,
                                 cudaStream_t st);
 cudaError_t launch_model(int64_t n, const float *eps_r, const float *sigma,
                          const float *mu_r, double dt, float *ca, float *cb,
                          float *cq, int cq_full, cudaStream_t st);
+cudaError_t launch_band_table(const float *cpml, int ny, int nx, int Wx, int Wz, float *out,
+                              cudaStream_t st);
 cudaError_t launch_cpml(int ny, int nx, int n_pml, double dy, double dx,
                         double dt, double vmax, double f0, double R, float *out,
                         cudaStream_t st);

@@ -19,6 +19,7 @@ MW_ERR_CFL = -2
 MW_ERR_WORKSPACE = -3
 MW_ERR_CUDA = -4
 MW_ERR_NONFINITE = -5
+MW_ERR_TIMEOUT = -6
 MW_ERR_UNSUPPORTED = -7
 
 SNAP_NONE, SNAP_FP32, SNAP_BF16, SNAP_CKPT = 0, 1, 2, 3
@@ -69,6 +70,7 @@ SIGNATURES = [
     ("mw_profile_read", ctypes.c_int, [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double),
                                        ctypes.c_int32]),
     ("mw_launch_count", ctypes.c_int64, []),
+    ("mw_workspace_init", ctypes.c_int, [_VP, ctypes.c_size_t, _VP]),
 ]
 
 
@@ -156,6 +158,11 @@ def model_from_eps_sigma(p, eps_r, sigma, mu_r, ca, cb, cq, stream=None):
 
 def cpml_profiles(p, f0, R, cpml, stream=None):
     return check(lib().mw_cpml_profiles(ctypes.byref(p), f0, R, ptr(cpml), stream_ptr(stream)))
+
+
+def workspace_init(workspace, stream=None):
+    return check(lib().mw_workspace_init(ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         stream_ptr(stream)))
 
 
 def tm_forward(p, ca, cb, cq, cpml, f, src_idx, rec_idx, state, rec, workspace, stream=None):

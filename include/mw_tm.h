@@ -18,7 +18,9 @@
  *  - Grid: ny rows (y = depth z) by nx columns (x), row-major; cell index
  *    j = y * nx + x.  Ey at (y, x), Hx at (y + 1/2, x), Hz at (y, x + 1/2).
  *    Every array cell of every field is updated; fields are zero outside the
- *    array.  nx must be a multiple of 4 (rows are read as float4).
+ *    array.  nx must be a multiple of 4 (rows are read as float4; a multiple
+ *    of 8 with bf16 snapshots) and n_pml at most 123 (a CPML band row is one
+ *    TMA box of at most 256 floats).
  *  - Per-shot arrays are [S][ny][nx] float32, time series are time-major
  *    [nt][S][n] float32 (the page's source / receiver kernels).
  *  - Source / receiver positions are flat per-shot cell indices int64
@@ -65,6 +67,8 @@ extern "C" {
 #define MW_ERR_WORKSPACE (-3)   /* workspace missing or too small           */
 #define MW_ERR_CUDA (-4)        /* a CUDA runtime call failed               */
 #define MW_ERR_NONFINITE (-5)   /* NaN / Inf found in a field (device flag) */
+#define MW_ERR_TIMEOUT (-6)     /* a kernel gave up waiting for its own copies
+                                   (device flag; results of that call invalid) */
 #define MW_ERR_UNSUPPORTED (-7) /* valid request this build does not serve  */
 
 /* forward snapshot storage for the gradient */
@@ -137,6 +141,11 @@ int mw_model_from_eps_sigma(const mw_params *p, const float *eps_r_dev,
 int mw_cpml_profiles(const mw_params *p, double f0, double R, float *cpml_dev,
                      void *stream);
 
+/* Prepare a workspace for first use: zero its status words (the first 256
+ * bytes).  Call once after allocating it; mw_sync_status clears them again
+ * after reporting. */
+int mw_workspace_init(void *workspace_dev, size_t workspace_bytes, void *stream);
+
 /* Forward: nt steps of H update, E update (+ snapshot / checkpoint store),
  * source injection f[t], receiver sampling rec[t] = Ey after injection
  * (order of the page's forward host loop).
@@ -147,7 +156,8 @@ int mw_cpml_profiles(const mw_params *p, double f0, double R, float *cpml_dev,
  *   state      in/out state buffer (layout above), or NULL to start from rest
  *              (the final state then stays in the workspace)
  *   rec        [nt][S][n_rec] out (may be NULL)
- *   workspace  mw_workspace_bytes(p) bytes of device memory
+ *   workspace  mw_workspace_bytes(p) bytes of device memory, 256-byte
+ *              aligned, prepared once with mw_workspace_init
  * Sources / receivers of step t use time index t of this call. */
 int mw_tm_forward(const mw_params *p, const float *ca_dev, const float *cb_dev,
                   const float *cq_dev, const float *cpml_dev, const float *f_dev,

@@ -1,0 +1,67 @@
+"""The C-ABI library loads without a GPU and exports every entry point that
+include/mw_tm.h declares; host-only entry points behave as documented."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from adjoint_state_gradients_b200 import build, mwtm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mw_tm.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(mw_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_path_entry_points():
+    names = declared_functions()
+    for n in ("mw_tm_forward", "mw_tm_adjoint_grad", "mw_combine_grad", "mw_workspace_bytes",
+              "mw_last_error", "mw_grad_eps_sigma", "mw_model_from_eps_sigma"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(build.build())
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_declared_symbol():
+    bound = {name for name, _, _ in mwtm.SIGNATURES}
+    missing = [n for n in declared_functions() if n not in bound]
+    assert not missing, missing
+
+
+def test_host_only_entry_points():
+    p = mwtm.make_params(ny=84, nx=84, order=2, n_shots=1, n_src=1, n_rec=32, nt=300, dt=4.7e-11,
+                         dy=0.02, dx=0.02, n_pml=10, snap_mode=mwtm.SNAP_FP32, vmax=1.5e8)
+    assert mwtm.validate(p) == mwtm.MW_OK
+    # state: 3 fields + 2 x-band (Wx = 12) + 2 z-band (Wz = 11) memories
+    assert mwtm.state_floats(p) == 3 * 84 * 84 + 2 * 84 * 24 + 2 * 22 * 84
+    ws = mwtm.workspace_bytes(p)
+    assert ws >= 2 * 300 * 84 * 84 * 4
+    bad = mwtm.make_params(ny=84, nx=82, order=2, n_shots=1, nt=1, dt=1e-12, dy=0.02, dx=0.02,
+                           vmax=1.5e8)
+    assert mwtm.validate(bad) == mwtm.MW_ERR_ARG
+    assert "multiple of 4" in mwtm.last_error()
+    big_pml = mwtm.make_params(ny=600, nx=600, order=2, n_shots=1, nt=1, dt=1e-12, dy=0.02,
+                               dx=0.02, n_pml=130, vmax=1.5e8)
+    assert mwtm.validate(big_pml) == mwtm.MW_ERR_UNSUPPORTED
+    assert mwtm.workspace_bytes(p) == ws
+
+
+@pytest.mark.parametrize("order,s", [(2, 1.0), (4, 7 / 6), (6, 1.2416666666666667),
+                                     (8, 1.2863095238095237)])
+def test_cfl_dt_matches_oracle(order, s):
+    import oracle
+    for h, v in ((0.02, 1.5e8), (0.01, 2.9e8)):
+        assert mwtm.cfl_dt(order, h, h, v) == pytest.approx(oracle.cfl_dt(order, h, h, v), rel=1e-15)
+        assert mwtm.cfl_dt(order, h, h, v) == pytest.approx(1 / (v * s * (2 / h ** 2) ** 0.5), rel=1e-12)
