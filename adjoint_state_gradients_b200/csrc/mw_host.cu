@@ -797,4 +797,132 @@ int mw_profile_read(int64_t *counts, double *total_ms, int32_t n_classes) {
   return MW_OK;
 }
 
+// ---- forward without allocations -------------------------------------------
+// The scratch of mw_tm_forward_noalloc: status words | duplicate chains | CPML
+// band table | the second state buffer of the ping-pong.  Host code must not
+// use the symbol itself (it is a host-side stand-in); it takes the device
+// address from cudaGetSymbolAddress, once per device.
+}  // extern "C"
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MW_NOALLOC_SCRATCH_BYTES];
+
+namespace mw {
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[64];
+
+int noalloc_scratch(char **out) {
+  int dev = 0;
+  MW_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MW_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(MW_ERR_CUDA, "cudaGetSymbolAddress of the built-in scratch failed: %s",
+                  cudaGetErrorString(e));
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = (char *)g_noalloc_addr[dev];
+  return MW_OK;
+}
+}  // namespace
+}  // namespace mw
+
+extern "C" {
+
+int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, const float *cq,
+                          const float *cpml, const float *f, const int64_t *src_idx,
+                          const int64_t *rec_idx, float *state, float *rec, void *stream) {
+  g_err.clear();
+  int rc = check_params(p, true);
+  if (rc) return rc;
+  if (p->snap_mode != MW_SNAP_NONE)
+    return fail(MW_ERR_ARG, "the scratch-free forward keeps no snapshots: snap_mode must be NONE");
+  if ((rc = check_ptr(ca, "ca")) || (rc = check_ptr(cb, "cb")) || (rc = check_ptr(cpml, "cpml")) ||
+      (rc = check_ptr(state, "state")))
+    return rc;
+  if (!cq) return fail(MW_ERR_ARG, "cq is NULL");
+  if (!p->cq_is_scalar && (rc = check_ptr(cq, "cq"))) return rc;
+  if (p->n_src > 0 && (!f || !src_idx)) return fail(MW_ERR_ARG, "sources need f and src_idx");
+  if (p->n_rec > 0 && rec && !rec_idx) return fail(MW_ERR_ARG, "receivers need rec_idx");
+
+  // layout inside the built-in scratch; reject what does not fit
+  const Bands bd = bands(p);
+  Layout L{};
+  L.flags = 0;
+  L.chains = 256;
+  L.bandtab = L.chains + align256(2 * sizeof(int) * (size_t)p->n_shots * (p->n_src + p->n_rec));
+  L.state_bytes = state_floats(p) * sizeof(float);
+  const size_t off_state =
+      L.bandtab + align256(sizeof(float) * (size_t)BandTab{bd.Wx, bd.Wz}.floats() + 16);
+  const size_t need = off_state + align256(L.state_bytes);
+  if (need > MW_NOALLOC_SCRATCH_BYTES)
+    return fail(MW_ERR_WORKSPACE,
+                "this problem needs %zu bytes of scratch but the built-in scratch holds %zu; "
+                "use mw_tm_forward with a caller-provided workspace",
+                need, (size_t)MW_NOALLOC_SCRATCH_BYTES);
+  char *ws = nullptr;
+  MW_TRY(noalloc_scratch(&ws));
+  cudaStream_t st = (cudaStream_t)stream;
+  int *flags = (int *)(ws + L.flags);
+  // the array keeps the previous call's contents: clear the status words
+  // (the band table, chains and state buffer are fully rewritten below)
+  MW_CUDA(cudaMemsetAsync(ws, 0, 256, st));
+
+  float *bufA = state;
+  float *bufB = (float *)(ws + off_state);
+  if (p->nt > 0) {
+    StepArgs a{};
+    const Launch lc = plan(p, false);
+    a.g = lc.g;
+    a.c = coef_of(p);
+    a.pr = prof_of(p, cpml);
+    a.ca = ca;
+    a.cb = cb;
+    a.cq = cq;
+    a.flags = flags;
+    a.bt = (const float *)(ws + L.bandtab);
+    set_layout(a, p, false);
+    MW_TRY(stencil_prologue(p, cpml, ws, L, st));
+    FwdMaps mA, mB;
+    MW_TRY(fwd_maps(p, fields_at(p, bufA), ca, cb, &mA));
+    MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, &mB));
+    const int64_t numel = (int64_t)p->ny * p->nx;
+    const Chains ch = chains_at(p, ws, L);
+    if (p->n_src > 0)
+      MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
+                                flags, st));
+    if (p->n_rec > 0 && rec)
+      MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
+                                flags, st));
+    float *cur = bufA, *nxt = bufB;
+    for (int t = 0; t < p->nt; ++t) {
+      a.in = fields_at(p, cur);
+      a.out = fields_at(p, nxt);
+      a.ctr_slot = t & 1;
+      MW_CUDA(launch_forward(cur == bufA ? mA : mB, a, p->order, kStoreNone,
+                             p->model_batched != 0, !p->cq_is_scalar, lc.grid, st));
+      MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots,
+                                   f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
+                                   ch.src_lead, ch.src_next, p->n_src, rec_idx, p->n_rec,
+                                   rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, st));
+      std::swap(cur, nxt);
+    }
+    if (cur != bufA)
+      MW_CUDA(cudaMemcpyAsync(bufA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
+    if (p->check_finite)
+      MW_CUDA(launch_check_finite(bufA, 3 * (int64_t)p->n_shots * numel, flags, st));
+  }
+  // wait for this call's work and report its device status
+  MW_CUDA(cudaStreamSynchronize(st));
+  int h[3] = {0, 0, 0};
+  MW_CUDA(cudaMemcpy(h, ws, sizeof h, cudaMemcpyDeviceToHost));
+  if (h[kFlagTimeout]) return fail(MW_ERR_TIMEOUT, "a stencil kernel timed out waiting for its copies");
+  if (h[kFlagBadIndex]) return fail(MW_ERR_ARG, "a source or receiver index was out of range");
+  if (h[kFlagNonFinite]) return fail(MW_ERR_NONFINITE, "non-finite value in the final state");
+  return MW_OK;
+}
+
 }  // extern "C"

@@ -71,7 +71,10 @@ SIGNATURES = [
                                        ctypes.c_int32]),
     ("mw_launch_count", ctypes.c_int64, []),
     ("mw_workspace_init", ctypes.c_int, [_VP, ctypes.c_size_t, _VP]),
+    ("mw_tm_forward_noalloc", ctypes.c_int, [_P, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
 ]
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def lib_path() -> str:
@@ -169,6 +172,13 @@ def tm_forward(p, ca, cb, cq, cpml, f, src_idx, rec_idx, state, rec, workspace, 
     return check(lib().mw_tm_forward(ctypes.byref(p), ptr(ca), ptr(cb), ptr(cq), ptr(cpml), ptr(f),
                                      ptr(src_idx), ptr(rec_idx), ptr(state), ptr(rec), ptr(workspace),
                                      workspace.numel() * workspace.element_size(), stream_ptr(stream)))
+
+
+def tm_forward_noalloc(p, ca, cb, cq, cpml, f, src_idx, rec_idx, state, rec, stream=None) -> int:
+    """Scratch-free forward (records only); returns the status code."""
+    return lib().mw_tm_forward_noalloc(ctypes.byref(p), ptr(ca), ptr(cb), ptr(cq), ptr(cpml), ptr(f),
+                                       ptr(src_idx), ptr(rec_idx), ptr(state), ptr(rec),
+                                       stream_ptr(stream))
 
 
 def tm_adjoint_grad(p, ca, cb, cq, cpml, f, src_idx, rec_idx, res, gca_shot, gcb_shot, grad_f,

@@ -165,6 +165,36 @@ int mw_tm_forward(const mw_params *p, const float *ca_dev, const float *cb_dev,
                   float *state_dev, float *rec_dev, void *workspace_dev,
                   size_t workspace_bytes, void *stream);
 
+/* Forward sweep that allocates nothing and needs no workspace (this entry
+ * point has no counterpart on the reference pages; it exists for callers that
+ * cannot allocate device memory, for instance a library embedded in an
+ * application whose device memory all belongs to another allocator, or a
+ * service that may allocate only at start-up).  Same arguments and results
+ * as mw_tm_forward with snap_mode MW_SNAP_NONE (records only), except:
+ *   - `state` is required (in/out; zero it for a run from rest);
+ *   - the scratch it needs (status words, duplicate chains, CPML band table,
+ *     the second ping-pong state buffer) lives in one array of
+ *     MW_NOALLOC_SCRATCH_BYTES bytes that the library defines in device
+ *     memory; every GPU that loads the library holds that array until the
+ *     process exits.  A problem needing more than that is rejected with
+ *     MW_ERR_WORKSPACE before any work is queued;
+ *   - the call waits for its work on `stream` to finish and returns the
+ *     device status of this call (MW_ERR_ARG for an out-of-range index,
+ *     MW_ERR_TIMEOUT, MW_ERR_NONFINITE with check_finite), so no
+ *     mw_sync_status call is needed;
+ *   - the first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture;
+ *   - every call shares the one array: calls that overlap on the GPU (other
+ *     threads, other streams) race and corrupt each other's results. */
+#define MW_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+int mw_tm_forward_noalloc(const mw_params *p, const float *ca_dev,
+                          const float *cb_dev, const float *cq_dev,
+                          const float *cpml_dev, const float *f_dev,
+                          const int64_t *src_idx_dev,
+                          const int64_t *rec_idx_dev, float *state_dev,
+                          float *rec_dev, void *stream);
+
 /* Adjoint sweep t = nt-1 .. 0 and per-shot gradients, after mw_tm_forward
  * with the same p, model, sources and workspace (snap_mode != NONE).  Per
  * step: lambda_E[rec] += res[t]; grad_f[t] = lambda_E[src];
