@@ -59,6 +59,12 @@ int stencil_weights(int order, double *c) {
   return 0;
 }
 
+#define MW_TRY(x)                 \
+  do {                            \
+    int rc_ = (x);                \
+    if (rc_ != MW_OK) return rc_; \
+  } while (0)
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Bands {
@@ -216,7 +222,7 @@ Launch plan(const mw_params *p, bool adjoint) {
   g.strip_cols = adjoint ? kAdjStripCols : kFwdStripCols;
   g.n_strips = (p->nx + g.strip_cols - 1) / g.strip_cols;
   const int P = p->order / 2;
-  const int warps_sm = stencil_slots_per_sm(p->order, adjoint, b.Wx);
+  const int warps_sm = stencil_slots_per_sm(p->order, adjoint, b.Wx, !p->cq_is_scalar);
   const int64_t slots = (int64_t)sm_count() * warps_sm;
   const int64_t cols_items = (int64_t)g.S * g.n_strips;
   // Items are claimed dynamically by resident warps: time ~ total iterations
@@ -238,8 +244,9 @@ Launch plan(const mw_params *p, bool adjoint) {
   g.chunk_h = best_ch;
   g.n_chunks = (p->ny + g.chunk_h - 1) / g.chunk_h;
   const int64_t items = cols_items * g.n_chunks;
-  int64_t grid = (items + kWarpsPerCta - 1) / kWarpsPerCta;
-  const int64_t cap = slots / kWarpsPerCta;
+  const int wpc = adjoint ? kAdjWarpsPerCta : kWarpsPerCta;
+  int64_t grid = (items + wpc - 1) / wpc;
+  const int64_t cap = slots / wpc;
   if (grid > cap) grid = cap;
   Lc.grid = (int)(grid > 0 ? grid : 1);
   return Lc;
@@ -295,15 +302,19 @@ EncodeTiledFn encoder() {
   return fn;
 }
 
-// Row-box map over a dense array [d3][d2][d1][d0] (rank 3 or 4) of float32
-// (elem 4) or bf16 (elem 2): box = (box0, 1, 1[, 1]), zero fill outside.
+// Row-box map over an array [d3][d2][d1][d0] (rank 3 or 4) of float32 (elem
+// 4) or bf16 (elem 2) with dense strides, or with the given outermost stride
+// (bytes, rank 4 only; 0 = dense): box = (box0, 1, 1[, box3]), zero fill
+// outside.
 int encode_rows(CUtensorMap *map, const void *base, int elem, int rank, uint64_t d0, uint64_t d1,
-                uint64_t d2, uint64_t d3, uint32_t box0) {
+                uint64_t d2, uint64_t d3, uint32_t box0, uint32_t box3 = 1,
+                uint64_t stride3 = 0) {
   EncodeTiledFn fn = encoder();
   if (!fn) return fail(MW_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[4] = {d0, d1, d2, d3};
-  cuuint64_t strides[3] = {d0 * elem, d0 * d1 * elem, d0 * d1 * d2 * elem};
-  cuuint32_t box[4] = {box0, 1, 1, 1};
+  cuuint64_t strides[3] = {d0 * elem, d0 * d1 * elem,
+                           stride3 ? stride3 : d0 * d1 * d2 * elem};
+  cuuint32_t box[4] = {box0, 1, 1, box3};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                   (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
@@ -316,51 +327,124 @@ int encode_rows(CUtensorMap *map, const void *base, int elem, int rank, uint64_t
   return MW_OK;
 }
 
-#define MW_TRY(x)            \
-  do {                       \
-    int rc_ = (x);           \
-    if (rc_ != MW_OK) return rc_; \
-  } while (0)
+// Map of rank 2..5 with explicit strides (bytes, rank - 1 of them) and box;
+// zero fill outside.
+int encode_map(CUtensorMap *map, const void *base, int elem, int rank, const uint64_t *dims,
+               const uint64_t *strides, const uint32_t *box) {
+  EncodeTiledFn fn = encoder();
+  if (!fn) return fail(MW_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], e[5];
+  for (int k = 0; k < rank; ++k) {
+    d[k] = dims[k];
+    b[k] = box[k];
+    e[k] = 1;
+    if (k + 1 < rank) st[k] = strides[k];
+  }
+  CUresult r = fn(map, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  (cuuint32_t)rank, const_cast<void *>(base), d, st, b, e,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MW_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): rank %d dims %llu %llu box %u",
+                (int)r, rank, (unsigned long long)dims[0], (unsigned long long)dims[1], box[0]);
+  return MW_OK;
+}
 
-int fwd_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb, FwdMaps *m) {
+// Two same-shaped arrays are fetched as one pair box when they are distinct,
+// non-overlapping and their distance TMA can express as a stride.
+struct Pairing {
+  bool pair, swap;
+  uint64_t stride;
+};
+Pairing pairing(const void *x, const void *y, uint64_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(x), b = reinterpret_cast<uintptr_t>(y);
+  Pairing r{false, false, 0};
+  const uint64_t d = a < b ? b - a : a - b;
+  if (d >= bytes && d % 16 == 0 && d < ((uint64_t)1 << 40)) {
+    r.pair = true;
+    r.swap = b < a;
+    r.stride = d;
+  }
+  return r;
+}
+typedef Pairing MdPair;
+MdPair md_pairing(const mw_params *p, const float *ca, const float *cb) {
+  const uint64_t Sm = p->model_batched ? p->n_shots : 1;
+  return pairing(ca, cb, Sm * (uint64_t)p->ny * p->nx * sizeof(float));
+}
+Pairing gg_pairing(const mw_params *p, const float *gca, const float *gcb) {
+  return pairing(gca, gcb, (uint64_t)p->n_shots * p->ny * p->nx * sizeof(float));
+}
+
+int fwd_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb,
+             const float *cq, FwdMaps *m) {
   memset(m, 0, sizeof *m);
   const Bands bd = bands(p);
   const uint64_t nx = p->nx, ny = p->ny, S = p->n_shots, Sm = p->model_batched ? p->n_shots : 1;
-  MW_TRY(encode_rows(&m->map[kLdEy], in.ey, 4, 3, nx, ny, S, 1, 136));
-  MW_TRY(encode_rows(&m->map[kLdHz], in.hz, 4, 3, nx, ny, S, 1, 128));
-  MW_TRY(encode_rows(&m->map[kLdHx], in.hx, 4, 3, nx, ny, S, 1, 120));
-  MW_TRY(encode_rows(&m->map[kLdCa], ca, 4, 3, nx, ny, Sm, 1, 120));
-  MW_TRY(encode_rows(&m->map[kLdCb], cb, 4, 3, nx, ny, Sm, 1, 120));
+  const uint64_t field = (uint64_t)(in.hz - in.ey) * sizeof(float);
+  MW_TRY(encode_rows(&m->map[kMapEH], in.ey, 4, 4, nx, ny, S, 2, 136, 2, field));
+  MW_TRY(encode_rows(&m->map[kMapHX], in.hx, 4, 3, nx, ny, S, 1, 120));
+  const MdPair md = md_pairing(p, ca, cb);
+  if (md.pair) {
+    MW_TRY(encode_rows(&m->map[kMapMD], md.swap ? cb : ca, 4, 4, nx, ny, Sm, 2, 120, 2,
+                       md.stride));
+  } else {
+    MW_TRY(encode_rows(&m->map[kMapMD], ca, 4, 3, nx, ny, Sm, 1, 120));
+    MW_TRY(encode_rows(&m->map[kMapCB], cb, 4, 3, nx, ny, Sm, 1, 120));
+  }
+  if (!p->cq_is_scalar) MW_TRY(encode_rows(&m->map[kMapCQ], cq, 4, 3, nx, ny, Sm, 1, 128));
   if (bd.Wx > 0) {
-    MW_TRY(encode_rows(&m->map[kLdMxh], in.mxh_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
-    MW_TRY(encode_rows(&m->map[kLdMxe], in.mxe_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
-    MW_TRY(encode_rows(&m->map[kLdMzh], in.mzh_node, 4, 3, nx, 2 * bd.Wz, S, 1, 120));
-    MW_TRY(encode_rows(&m->map[kLdMze], in.mze_node, 4, 3, nx, 2 * bd.Wz, S, 1, 120));
+    MW_TRY(encode_rows(&m->map[kMapMXH], in.mxh_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
+    MW_TRY(encode_rows(&m->map[kMapMXE], in.mxe_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
+    MW_TRY(encode_rows(&m->map[kMapMZH], in.mzh_node, 4, 3, nx, 2 * bd.Wz, S, 1, 120));
+    MW_TRY(encode_rows(&m->map[kMapMZE], in.mze_node, 4, 3, nx, 2 * bd.Wz, S, 1, 120));
   }
   return MW_OK;
 }
 
 int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb,
-             const float *gca, const float *gcb, const void *se, const void *sc, int snap_elem,
-             int snap_steps, AdjMaps *m) {
+             const float *cq, const float *gca, const float *gcb, const void *se, const void *sc,
+             int snap_elem, int snap_steps, AdjMaps *m) {
   memset(m, 0, sizeof *m);
   const Bands bd = bands(p);
   const uint64_t nx = p->nx, ny = p->ny, S = p->n_shots, Sm = p->model_batched ? p->n_shots : 1;
-  MW_TRY(encode_rows(&m->map[kLdLam], in.ey, 4, 3, nx, ny, S, 1, 128));
-  MW_TRY(encode_rows(&m->map[kLdCbA], cb, 4, 3, nx, ny, Sm, 1, 128));
-  MW_TRY(encode_rows(&m->map[kLdLhz], in.hz, 4, 3, nx, ny, S, 1, 120));
-  MW_TRY(encode_rows(&m->map[kLdSe], se, snap_elem, 4, nx, ny, S, snap_steps, 112));
-  MW_TRY(encode_rows(&m->map[kLdSc], sc, snap_elem, 4, nx, ny, S, snap_steps, 112));
-  MW_TRY(encode_rows(&m->map[kLdGca], gca, 4, 3, nx, ny, S, 1, 112));
-  MW_TRY(encode_rows(&m->map[kLdGcb], gcb, 4, 3, nx, ny, S, 1, 112));
-  MW_TRY(encode_rows(&m->map[kLdLhx], in.hx, 4, 3, nx, ny, S, 1, 112));
-  MW_TRY(encode_rows(&m->map[kLdCaA], ca, 4, 3, nx, ny, Sm, 1, 112));
-  MW_TRY(encode_rows(&m->map[kLdLamy], in.ey, 4, 3, nx, ny, S, 1, 112));
+  MW_TRY(encode_rows(&m->map[kAMapEH], in.ey, 4, 4, nx, ny, S, 2, 128, 2,
+                     (uint64_t)(in.hz - in.ey) * sizeof(float)));
+  const MdPair md = md_pairing(p, ca, cb);
+  if (md.pair) {
+    MW_TRY(encode_rows(&m->map[kAMapMD], md.swap ? cb : ca, 4, 4, nx, ny, Sm, 2, 128, 2,
+                       md.stride));
+  } else {
+    MW_TRY(encode_rows(&m->map[kAMapMD], ca, 4, 3, nx, ny, Sm, 1, 128));
+    MW_TRY(encode_rows(&m->map[kAMapCB], cb, 4, 3, nx, ny, Sm, 1, 128));
+  }
+  MW_TRY(encode_rows(&m->map[kAMapHX], in.hx, 4, 3, nx, ny, S, 1, 112));
+  {
+    // (x, y, shot, step, field): the curl snapshots follow the E snapshots
+    const uint64_t e = (uint64_t)snap_elem;
+    const uint64_t dims[5] = {nx, ny, S, (uint64_t)snap_steps, 2};
+    const uint64_t strides[4] = {nx * e, nx * ny * e, nx * ny * S * e,
+                                 (uint64_t)((const char *)sc - (const char *)se)};
+    const uint32_t box[5] = {112, 1, 1, 1, 2};
+    if ((const char *)sc <= (const char *)se)
+      return fail(MW_ERR_ARG, "internal: snapshot fields out of order");
+    MW_TRY(encode_map(&m->map[kAMapSS], se, snap_elem, 5, dims, strides, box));
+  }
+  const Pairing gg = gg_pairing(p, gca, gcb);
+  if (gg.pair) {
+    MW_TRY(encode_rows(&m->map[kAMapGG], gg.swap ? gcb : gca, 4, 4, nx, ny, S, 2, 112, 2,
+                       gg.stride));
+  } else {
+    MW_TRY(encode_rows(&m->map[kAMapGG], gca, 4, 3, nx, ny, S, 1, 112));
+    MW_TRY(encode_rows(&m->map[kAMapGB], gcb, 4, 3, nx, ny, S, 1, 112));
+  }
+  if (!p->cq_is_scalar) MW_TRY(encode_rows(&m->map[kAMapCQ], cq, 4, 3, nx, ny, Sm, 1, 128));
   if (bd.Wx > 0) {
-    MW_TRY(encode_rows(&m->map[kLdMxeA], in.mxe_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
-    MW_TRY(encode_rows(&m->map[kLdMxhA], in.mxh_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
-    MW_TRY(encode_rows(&m->map[kLdMzeA], in.mze_node, 4, 3, nx, 2 * bd.Wz, S, 1, 112));
-    MW_TRY(encode_rows(&m->map[kLdMzhA], in.mzh_node, 4, 3, nx, 2 * bd.Wz, S, 1, 112));
+    MW_TRY(encode_rows(&m->map[kAMapMX], in.mxh_node, 4, 4, 2 * bd.Wx, ny, S, 2, 2 * bd.Wx, 2,
+                       (uint64_t)(in.mxe_node - in.mxh_node) * sizeof(float)));
+    MW_TRY(encode_rows(&m->map[kAMapMZE], in.mze_node, 4, 3, nx, 2 * bd.Wz, S, 1, 112));
+    MW_TRY(encode_rows(&m->map[kAMapMZH], in.mzh_node, 4, 3, nx, 2 * bd.Wz, S, 1, 112));
   }
   return MW_OK;
 }
@@ -377,9 +461,23 @@ int stencil_prologue(const mw_params *p, const float *cpml, char *ws, const Layo
 
 void set_layout(StepArgs &a, const mw_params *p, bool adjoint) {
   size_t smem;
-  stencil_layout(p->order, adjoint, bands(p).Wx, &a.stage_floats, &a.band_floats, &a.warp_floats,
-                 &smem);
-  a.band_box_floats = 2 * bands(p).Wx;
+  if (adjoint) {
+    // needs a.ca / a.cb and a.gca / a.gcb (pair fetches)
+    adjoint_layout(p->order, bands(p).Wx, !p->cq_is_scalar, p->snap_mode == MW_SNAP_BF16, &a,
+                   &smem);
+    const MdPair md = md_pairing(p, a.ca, a.cb);
+    a.md_pair = md.pair ? 1 : 0;
+    a.md_swap = md.swap ? 1 : 0;
+    const Pairing gg = gg_pairing(p, a.gca, a.gcb);
+    a.gg_pair = gg.pair ? 1 : 0;
+    a.gg_swap = gg.swap ? 1 : 0;
+  } else {
+    // forward: needs a.ca / a.cb (the Ca / Cb pair fetch)
+    forward_layout(p->order, bands(p).Wx, !p->cq_is_scalar, &a, &smem);
+    const MdPair md = md_pairing(p, a.ca, a.cb);
+    a.md_pair = md.pair ? 1 : 0;
+    a.md_swap = md.swap ? 1 : 0;
+  }
 }
 
 // ---- per-kernel event timing ------------------------------------------------
@@ -536,8 +634,8 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   set_layout(a, p, false);
   MW_TRY(stencil_prologue(p, cpml, ws, L, st));
   FwdMaps mA, mB;  // input buffer A / B
-  MW_TRY(fwd_maps(p, fields_at(p, bufA), ca, cb, &mA));
-  MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, &mB));
+  MW_TRY(fwd_maps(p, fields_at(p, bufA), ca, cb, cq, &mA));
+  MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, cq, &mB));
 
   const int store = p->snap_mode == MW_SNAP_FP32 ? kStoreF32
                     : p->snap_mode == MW_SNAP_BF16 ? kStoreBF16 : kStoreNone;
@@ -645,8 +743,8 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   const char *snap_e = ckpt ? ws + L.seg : ws + L.snap;
   const char *snap_c = snap_e + (size_t)C * L.snap_step_bytes;
   AdjMaps mA, mB;
-  MW_TRY(adj_maps(p, fields_at(p, adA), ca, cb, gca, gcb, snap_e, snap_c, bf16 ? 2 : 4, C, &mA));
-  MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, gca, gcb, snap_e, snap_c, bf16 ? 2 : 4, C, &mB));
+  MW_TRY(adj_maps(p, fields_at(p, adA), ca, cb, cq, gca, gcb, snap_e, snap_c, bf16 ? 2 : 4, C, &mA));
+  MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, cq, gca, gcb, snap_e, snap_c, bf16 ? 2 : 4, C, &mB));
 
   float *cur = adA, *nxt = adB;
   auto adj_step = [&](int t, int slot) -> int {
@@ -678,8 +776,8 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     set_layout(fa, p, false);
     float *rA = (float *)(ws + L.rpA), *rB = (float *)(ws + L.rpB);
     FwdMaps fA, fB;
-    MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, &fA));
-    MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, &fB));
+    MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, cq, &fA));
+    MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, cq, &fB));
     char *seg_e = ws + L.seg;
     char *seg_c = seg_e + (size_t)C * L.snap_step_bytes;
     for (int k = L.n_seg - 1; k >= 0; --k) {
@@ -887,8 +985,8 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
     set_layout(a, p, false);
     MW_TRY(stencil_prologue(p, cpml, ws, L, st));
     FwdMaps mA, mB;
-    MW_TRY(fwd_maps(p, fields_at(p, bufA), ca, cb, &mA));
-    MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, &mB));
+    MW_TRY(fwd_maps(p, fields_at(p, bufA), ca, cb, cq, &mA));
+    MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, cq, &mB));
     const int64_t numel = (int64_t)p->ny * p->nx;
     const Chains ch = chains_at(p, ws, L);
     if (p->n_src > 0)

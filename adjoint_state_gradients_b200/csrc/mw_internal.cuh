@@ -6,10 +6,11 @@
 //   z-band mem   [S][2*Wz][nx]         rows    [0,Wz) then [ny-Wz,ny)
 //   model        [ny][nx] or [S][ny][nx]
 //   snapshots    [n][S][ny][nx]        float32 or bf16
-// Stencil kernels are "marching strips": one warp owns a 128-column strip of
-// one shot over a chunk of rows and walks down it, keeping the y-direction
-// stencil operands in registers and the x-direction ones in a per-warp
-// shared-memory row, so each cell's state is read and written once per step.
+// Stencil kernels are "marching strips": one warp owns a 120- (forward) or
+// 112-column (adjoint) strip of one shot over a chunk of rows and walks down
+// it, keeping the y-direction stencil operands in registers and the
+// x-direction ones in per-warp shared-memory rows, so each cell's state is
+// read and written once per step.
 #pragma once
 
 #include <cuda.h>
@@ -22,7 +23,8 @@ namespace mw {
 
 constexpr int kFwdStripCols = 120;  // forward: columns owned per warp (30 float4)
 constexpr int kAdjStripCols = 112;  // adjoint: columns owned per warp (28 float4)
-constexpr int kWarpsPerCta = 4;
+constexpr int kWarpsPerCta = 4;    // forward CTA: 4 warps
+constexpr int kAdjWarpsPerCta = 5; // adjoint CTA: 5 warps
 
 struct Geom {
   int ny, nx, S;
@@ -53,6 +55,11 @@ struct Fields {
   float *mze_node;  // z-band memory at the E nodes
 };
 
+// Forward stage slots placed by the host (float offsets within a stage).
+enum { kFoCqH = 0, kFoCqX, kFoMzh, kFoMze, kFoMxh, kFoMxe, kFoCount };
+// Adjoint stage slots placed by the host.
+enum { kAoCqR = 0, kAoCqH, kAoMx, kAoMze, kAoMzh, kAoCount };
+
 struct StepArgs {
   Geom g;
   Coef c;
@@ -73,25 +80,51 @@ struct StepArgs {
   // shared-memory layout of one warp (floats): stage size, band slot width
   // (padded), band row width (the TMA box, 2*Wx)
   int stage_floats, band_floats, warp_floats, band_box_floats;
+  // forward only: optional stage slots (kFo*), Ca / Cb pair fetch and order
+  int fo[kFoCount];
+  int md_pair, md_swap;
+  // adjoint only: optional stage slots (kAo*), gCa / gCb pair fetch and order
+  int ao[kAoCount];
+  int gg_pair, gg_swap;
 };
 
-// TMA tensor maps of one forward launch (the input buffer set and model),
-// indexed by load slot so that lane k of a warp can issue load k.  Boxes are
-// one row high, starting at x0 - 8 (ey, 136 wide), x0 - 4 (hz, 128 wide) or
-// x0 (120 wide); x-band memories take a whole band row (2*Wx).
-enum FwdLoad { kLdEy = 0, kLdHz, kLdHx, kLdCa, kLdCb, kLdMxh, kLdMxe, kLdMzh, kLdMze, kFwdLoads };
-struct FwdMaps {
-  CUtensorMap map[kFwdLoads];
+// TMA tensor maps of one forward launch (the input buffer set and model).
+// Boxes are one row high:
+//   kMapEH  Ey and Hz of one row as one 4-D box (x, y, shot, field) with the
+//           field stride Hz - Ey: 136 wide from x0 - 8, 2 fields
+//   kMapHX  Hx, 120 wide from x0
+//   kMapMD  Ca and Cb as one pair box (x, y, shot, field; field stride
+//           |Cb - Ca|, the lower address first) when md_pair, else Ca alone
+//           with kMapCB beside it; 120 wide from x0
+//   kMapCQ  Cq when it is an array: 128 wide from x0 - 4
+//   kMapMXH / kMapMXE  x-band memories, a whole band row (2*Wx)
+//   kMapMZH / kMapMZE  z-band memories, 120 wide from x0
+enum FwdMap {
+  kMapEH = 0, kMapHX, kMapMD, kMapCB, kMapCQ, kMapMXH, kMapMXE, kMapMZH, kMapMZE, kFwdMaps
 };
-// Adjoint: lam and cb 128 wide from x0 - 8, lhz 120 from x0 - 4, the rest 112
-// from x0 (lamy: lambda_E again, for the Ca term), snapshots 4-D (x, y, shot,
-// step), x-band memories a whole band row.
-enum AdjLoad {
-  kLdLam = 0, kLdCbA, kLdLhz, kLdSe, kLdSc, kLdGca, kLdGcb, kLdLhx, kLdCaA, kLdLamy, kLdMxeA,
-  kLdMxhA, kLdMzeA, kLdMzhA, kAdjLoads
+struct FwdMaps {
+  CUtensorMap map[kFwdMaps];
+};
+// TMA tensor maps of one adjoint launch.  Boxes are one row high:
+//   kAMapEH  lambda_E and lambda_Hz of one row as one 4-D box (field stride
+//            lambda_Hz - lambda_E): 128 wide from x0 - 8, 2 fields
+//   kAMapMD  Ca and Cb of one row as one pair box when md_pair (else Ca, with
+//            kAMapCB beside it): 128 wide from x0 - 8
+//   kAMapHX  lambda_Hx, 112 wide from x0
+//   kAMapSS  the E and curl snapshots as one 5-D box (x, y, shot, step,
+//            field): 112 wide from x0
+//   kAMapGG  the per-shot gradients gCa, gCb as one pair box when gg_pair
+//            (else gCa, with kAMapGB beside it): 112 wide from x0
+//   kAMapCQ  Cq when it is an array: 128 wide from x0 - 8
+//   kAMapMX  the x-band memories at the H and E nodes (adjacent arrays) as
+//            one pair box of whole band rows
+//   kAMapMZE / kAMapMZH  z-band memories, 112 wide from x0
+enum AdjMap {
+  kAMapEH = 0, kAMapMD, kAMapCB, kAMapHX, kAMapSS, kAMapGG, kAMapGB, kAMapCQ, kAMapMX,
+  kAMapMZE, kAMapMZH, kAdjMaps
 };
 struct AdjMaps {
-  CUtensorMap map[kAdjLoads];
+  CUtensorMap map[kAdjMaps];
 };
 
 // Workspace layout (byte offsets, 256-aligned).
@@ -136,10 +169,11 @@ cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int s
                            bool batched, bool cq_array, int grid, cudaStream_t st);
 cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int snap_bf16,
                            bool batched, bool cq_array, int grid, cudaStream_t st);
-// shared-memory layout (floats per stage / per warp) and dynamic smem bytes
-void stencil_layout(int order, bool adjoint, int Wx, int *stage_floats, int *band_floats,
-                    int *warp_floats, size_t *smem_bytes);
-int stencil_slots_per_sm(int order, bool adjoint, int Wx);
+// forward / adjoint: the full stage layout (optional slots for a Cq array and
+// bands)
+void forward_layout(int order, int Wx, bool cq_array, StepArgs *a, size_t *smem_bytes);
+void adjoint_layout(int order, int Wx, bool cq_array, bool bf16, StepArgs *a, size_t *smem_bytes);
+int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array);
 
 // small kernels (mw_aux.cu)
 cudaError_t launch_dup_chains(const int64_t *idx, int S, int n, int64_t numel, int *lead,

@@ -24,14 +24,16 @@
 // x0 - 4 + 4l (forward) or x0 - 8 + 4l (adjoint), so the halo columns the
 // x-stencils need are computed in the same SIMD pass as the owned ones.
 // Input rows arrive by TMA (cp.async.bulk.tensor, one-row boxes, zero fill
-// outside the array; lane k issues load k) into a ring of L+1 shared-memory
-// stages, L rows ahead of the row being computed, each tracked by an
-// mbarrier with a bounded wait.  The y-stencil operands (Ey rows for Hx, Hx
-// rows for the E update) live in register queues; the x-stencil operands
-// come from the staged row and from a ring of 2P computed Hz rows.  States
-// are ping-ponged between two buffers so halo recompute never races with a
-// neighbour's writes.  CPML memories exist only in the bands and are fetched
-// only where a row or strip lies in one.
+// outside the array) into a ring of L+1 shared-memory stages, L rows ahead
+// of the row being computed, each tracked by an mbarrier with a bounded
+// wait.  Lane 0 issues all of a row's loads; fields that share a row and a
+// column range come as one multi-field box (Ey with Hz, Ca with Cb, the two
+// snapshots, the two gradients).  The y-stencil operands live in register
+// queues; the x-stencil operands come from the staged row and from a ring of
+// 2P computed rows.  States are ping-ponged between two buffers so halo
+// recompute never races with a neighbour's writes.  Items whose walk touches
+// neither a CPML band nor the array's side edges take a lean path with no
+// band code; CPML memories exist only in the bands.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -46,11 +48,15 @@ constexpr uint32_t kWaitPolls = 1u << 22;  // ~0.5 s of polling, then give up
 constexpr unsigned kFull = 0xffffffffu;
 
 // Stage layouts (float offsets, 128-byte aligned slots).
-constexpr int kF_EY = 0, kF_HZ = 160, kF_HX = 288, kF_CA = 416, kF_CB = 544, kF_MZH = 672,
-              kF_MZE = 800, kF_BAND = 928;
-constexpr int kA_LAM = 0, kA_CB = 128, kA_LHZ = 256, kA_SE = 384, kA_SC = 512, kA_GCA = 640,
-              kA_GCB = 768, kA_LHX = 896, kA_CA = 1024, kA_LAMY = 1152, kA_MZE = 1280,
-              kA_MZH = 1408, kA_BAND = 1536;
+// forward: Ey and Hz of row r (one pair box), Hx of row r - P, Ca / Cb of
+// row r - 2P + 1 (one pair box); optional slots follow at host-given offsets
+constexpr int kF_EY = 0, kF_HZ = 136, kF_HX = 288, kF_MD = 416, kF_FIXED = 672;
+static_assert(kF_MD + 128 + 120 <= kF_FIXED, "Ca / Cb slots overflow");
+// adjoint: lambda_E and lambda_Hz of row r (one pair box), Ca / Cb of row r
+// (one pair box), lambda_Hx of row r - P, the two snapshots of row r (one
+// box), the per-shot gradients of row r (one pair box); optional slots follow
+constexpr int kA_EH = 0, kA_MD = 256, kA_HX = 512, kA_SS = 640, kA_GG = 896, kA_FIXED = 1152;
+static_assert(kA_GG + 128 + 112 <= kA_FIXED, "gradient slots overflow");
 constexpr int kFRing = 128;  // forward Hz ring row: 32 float4
 constexpr int kAPx = 128;    // adjoint px row: 32 float4
 constexpr int kARing = 120;  // adjoint qx ring row: 30 float4
@@ -58,6 +64,7 @@ constexpr int kARing = 120;  // adjoint qx ring row: 30 float4
 template <int L>
 struct Stages {
   static_assert(kWarpsPerCta * (L + 1) * 8 <= 128, "barrier area too small");
+  static_assert(kAdjWarpsPerCta * (L + 1) * 8 <= 128, "barrier area too small");
 };
 
 struct F4 {
@@ -65,10 +72,6 @@ struct F4 {
 };
 
 __device__ __forceinline__ F4 zero4() { return F4{{0.f, 0.f, 0.f, 0.f}}; }
-__device__ __forceinline__ F4 lds4(const float *p) {
-  float4 t = *reinterpret_cast<const float4 *>(p);
-  return F4{{t.x, t.y, t.z, t.w}};
-}
 __device__ __forceinline__ F4 ld4(const float *p) {
   float4 t = __ldg(reinterpret_cast<const float4 *>(p));
   return F4{{t.x, t.y, t.z, t.w}};
@@ -77,69 +80,16 @@ __device__ __forceinline__ F4 splat4(float x) { return F4{{x, x, x, x}}; }
 __device__ __forceinline__ void st4(float *p, const F4 &a) {
   *reinterpret_cast<float4 *>(p) = make_float4(a.v[0], a.v[1], a.v[2], a.v[3]);
 }
-__device__ __forceinline__ void win12(const float *p, float w[12]) {
-  const float4 *q = reinterpret_cast<const float4 *>(p);
-  float4 a = q[0], b = q[1], c = q[2];
-  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-  w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-  w[8] = c.x; w[9] = c.y; w[10] = c.z; w[11] = c.w;
-}
 
 // ---- TMA / mbarrier primitives (PTX) ---------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
 }
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait for phase `parity` of a stage barrier, called by all 32 lanes:
-// every lane polls (acquire) and the warp votes, so the outcome is uniform.
-// Returns false after the poll limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t k = 0; k < kWaitPolls; ++k) {
-    if (__all_sync(kFull, mbar_test(bar, parity))) return true;
-    if (k >= 32) __nanosleep(100);
-  }
-  return false;
-}
-__device__ __forceinline__ void tma3(float *dst, const CUtensorMap *map, int c0, int c1, int c2,
-                                     uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tma4(float *dst, const CUtensorMap *map, int c0, int c1, int c2,
-                                     int c3, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
-      "r"(smem_u32(bar))
-      : "memory");
 }
 
 // Snapshot row store (4 consecutive cells), float32 or bf16 (RNE).
@@ -154,20 +104,6 @@ __device__ __forceinline__ void snap_store(void *row, const F4 &v) {
     pk.x = *reinterpret_cast<uint32_t *>(&lo);
     pk.y = *reinterpret_cast<uint32_t *>(&hi);
     *reinterpret_cast<uint2 *>(row) = pk;
-  }
-}
-// Staged snapshot values of own float4 o (float32 or bf16 in smem).
-template <bool BF16>
-__device__ __forceinline__ F4 snap_lds(const float *stage_row, int o) {
-  if constexpr (!BF16) {
-    return lds4(stage_row + 4 * o);
-  } else {
-    uint2 pk = *reinterpret_cast<const uint2 *>(
-        reinterpret_cast<const __nv_bfloat16 *>(stage_row) + 4 * o);
-    __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162 *>(&pk.x);
-    __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162 *>(&pk.y);
-    float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
-    return F4{{a.x, a.y, b.x, b.y}};
   }
 }
 
@@ -213,27 +149,13 @@ struct Ring {
   }
 };
 
-// Rows a walk iteration touches: r (new Ey / lambda row), rh = r - P (H row
-// updated in the z direction), y = r - 2P + 1 (E row updated).
-template <int P>
-struct Rows {
-  int r, rh, y;
-  bool own_r, hx_need, hx_in, e_row;
-  __device__ __forceinline__ Rows(int r0, int i, int ya, int yb, int ny) {
-    r = r0 + i;
-    rh = r - P;
-    y = r - 2 * P + 1;
-    own_r = r >= ya && r < yb;
-    hx_need = rh >= ya - P && rh <= yb + P - 2;
-    hx_in = hx_need && rh >= 0 && rh < ny;
-    e_row = y >= ya && y < yb;
-  }
-};
 
 // Strip / chunk of one work item.
 struct Item {
   int s, sm, x0, ya, yb, r0, n_it;
-  bool xb;  // the strip (with its halo) touches an x band
+  int hx_lo, hx_hi;  // iterations whose H row r - P lies in the array and is needed
+  bool xb;    // the strip (with its halo) touches an x band
+  bool edge;  // the walk touches a band or the array's side edges
 };
 
 template <int P>
@@ -248,101 +170,373 @@ __device__ __forceinline__ bool make_item(const Geom &g, int item, bool batched,
   it.yb = min(g.ny, it.ya + g.chunk_h);
   it.r0 = it.ya - (2 * P - 1);
   it.n_it = (it.yb - it.ya) + 4 * P - 2;
-  it.xb = g.Wx > 0 && (it.x0 - 8 < g.Wx || it.x0 + g.strip_cols + 8 > g.nx - g.Wx);
+  const bool near_x = it.x0 - 8 < g.Wx || it.x0 + g.strip_cols + 8 > g.nx - g.Wx;
+  it.xb = g.Wx > 0 && near_x;
+  it.edge = near_x || (g.Wz > 0 && (it.r0 < g.Wz || it.r0 + it.n_it > g.ny - g.Wz));
+  it.hx_lo = max(it.ya - P, 0) - (it.r0 - P);
+  it.hx_hi = min(it.yb + P - 2, g.ny - 1) - (it.r0 - P);
   return it.ya < it.yb;
 }
 
 // ---------------------------------------------------------------------------
 // forward
 
-// Issue the TMA loads of walk iteration i into stage `st`: lane k issues load
-// k (FwdLoad order; the per-lane operands are chosen with selects, not
-// branches), lane 0 posts the expected byte count first.
-template <int P>
-__device__ __forceinline__ void fwd_issue(const FwdMaps &m, const Geom &g, const Item &it, int i,
-                                          float *st, uint64_t *bar, int band_slot, int band_box,
-                                          int lane) {
-  const Rows<P> R(it.r0, i, it.ya, it.yb, g.ny);
-  const int zh = R.hx_in ? zband_row(R.rh, g.ny, g.Wz) : -1;
-  const int ze = R.e_row ? zband_row(R.y, g.ny, g.Wz) : -1;
-  const bool l_ey = lane == kLdEy, l_hz = lane == kLdHz, l_hx = lane == kLdHx;
-  const bool l_ca = lane == kLdCa, l_cb = lane == kLdCb, l_mxh = lane == kLdMxh;
-  const bool l_mxe = lane == kLdMxe, l_mzh = lane == kLdMzh, l_mze = lane == kLdMze;
-  const bool act = l_ey | (l_hz & R.own_r) | (l_hx & R.hx_in) | ((l_ca | l_cb) & R.e_row) |
-                   (l_mxh & R.own_r & it.xb) | (l_mxe & R.e_row & it.xb) | (l_mzh & (zh >= 0)) |
-                   (l_mze & (ze >= 0));
-  const int c0 = l_ey ? it.x0 - 8 : l_hz ? it.x0 - 4 : (l_mxh | l_mxe) ? 0 : it.x0;
-  const int c1 = l_hx ? R.rh : (l_ca | l_cb | l_mxe) ? R.y : l_mzh ? zh : l_mze ? ze : R.r;
-  const int c2 = (l_ca | l_cb) ? it.sm : it.s;
-  const int off = l_ey ? kF_EY : l_hz ? kF_HZ : l_hx ? kF_HX : l_ca ? kF_CA : l_cb ? kF_CB
-                : l_mzh ? kF_MZH : l_mze ? kF_MZE : l_mxh ? kF_BAND : kF_BAND + band_slot;
-  const uint32_t bytes = l_ey ? 136 * 4 : l_hz ? 128 * 4 : (l_mxh | l_mxe) ? band_box : 120 * 4;
-  const uint32_t total = __reduce_add_sync(kFull, act ? bytes : 0u);
-  if (lane == 0) mbar_expect_tx(bar, total);
-  __syncwarp();
-  if (act) {
-    fence_proxy_async();
-    tma3(st + off, &m.map[lane < kFwdLoads ? lane : 0], c0, c1, c2, bar);
+// Shared-memory access by 32-bit shared-window address.
+__device__ __forceinline__ F4 lds4s(uint32_t addr) {
+  F4 r;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(r.v[0]), "=f"(r.v[1]), "=f"(r.v[2]), "=f"(r.v[3])
+               : "r"(addr)
+               : "memory");
+  return r;
+}
+__device__ __forceinline__ void sts4s(uint32_t addr, const F4 &v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.v[0]), "f"(v.v[1]),
+               "f"(v.v[2]), "f"(v.v[3])
+               : "memory");
+}
+__device__ __forceinline__ void win12s(uint32_t addr, float w[12]) {
+  const F4 a = lds4s(addr), b = lds4s(addr + 16), c = lds4s(addr + 32);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    w[q] = a.v[q];
+    w[q + 4] = b.v[q];
+    w[q + 8] = c.v[q];
+  }
+}
+__device__ __forceinline__ void expect_tx_s(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_test_s(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded, warp-uniform wait (all 32 lanes poll and vote); false after the
+// poll limit.
+__device__ __forceinline__ bool mbar_wait_s(uint32_t bar, uint32_t parity) {
+  for (uint32_t k = 0; k < kWaitPolls; ++k) {
+    if (__all_sync(kFull, mbar_test_s(bar, parity))) return true;
+    if (k >= 32) __nanosleep(100);
+  }
+  return false;
+}
+__device__ __forceinline__ void tma3s(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                      uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma4s(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                      int c3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+
+// One warp's shared memory: stage barriers, the stage ring, the Hz ring.
+struct FwdWarp {
+  uint32_t bars, stage0, hring;
+  uint32_t stage_bytes;
+  uint32_t ca_o, cb_o;  // byte offsets of the Ca / Cb rows in a stage
+  int lane;
+  Ring ring;
+};
+
+// Issue the loads of walk iteration i into stage `st` (lane 0 only): the
+// rows are r (Ey, Hz; Cq), r - P (Hx; Cq, z-band memory of Hx) and
+// y = r - 2P + 1 (Ca, Cb; band memories of E); the x-band memory of Hz is
+// that of row r.  Rows outside the array read as zeros.
+template <int P, bool BAND>
+__device__ __forceinline__ void fwd_issue(const FwdMaps &m, const StepArgs &a, const Item &it,
+                                          int i, uint32_t st, uint32_t bar, int cq_arr) {
+  const int r = it.r0 + i;
+  const bool hx_in = i >= it.hx_lo && i <= it.hx_hi;
+  const bool e_row = (unsigned)(i - (4 * P - 2)) < (unsigned)(it.yb - it.ya);
+  uint32_t bytes = 2 * 136 * 4;
+  if (hx_in) bytes += 120 * 4;
+  if (e_row) bytes += 2 * 120 * 4;
+  if (cq_arr) bytes += hx_in ? 2 * 128 * 4 : 128 * 4;
+  int zh = -1, ze = -1;
+  if constexpr (BAND) {
+    if (hx_in) zh = zband_row(r - P, a.g.ny, a.g.Wz);
+    if (e_row) ze = zband_row(r - 2 * P + 1, a.g.ny, a.g.Wz);
+    if (zh >= 0) bytes += 120 * 4;
+    if (ze >= 0) bytes += 120 * 4;
+    if (it.xb) bytes += (uint32_t)a.band_box_floats * 4 * (e_row ? 2 : 1);
+  }
+  expect_tx_s(bar, bytes);
+  fence_proxy_async();
+  tma4s(st + kF_EY * 4, &m.map[kMapEH], it.x0 - 8, r, it.s, 0, bar);
+  if (hx_in) tma3s(st + kF_HX * 4, &m.map[kMapHX], it.x0, r - P, it.s, bar);
+  if (e_row) {
+    if (a.md_pair) {
+      tma4s(st + kF_MD * 4, &m.map[kMapMD], it.x0, r - 2 * P + 1, it.sm, 0, bar);
+    } else {
+      tma3s(st + kF_MD * 4, &m.map[kMapMD], it.x0, r - 2 * P + 1, it.sm, bar);
+      tma3s(st + (kF_MD + 128) * 4, &m.map[kMapCB], it.x0, r - 2 * P + 1, it.sm, bar);
+    }
+  }
+  if (cq_arr) {
+    tma3s(st + a.fo[kFoCqH] * 4, &m.map[kMapCQ], it.x0 - 4, r, it.sm, bar);
+    if (hx_in) tma3s(st + a.fo[kFoCqX] * 4, &m.map[kMapCQ], it.x0 - 4, r - P, it.sm, bar);
+  }
+  if constexpr (BAND) {
+    if (zh >= 0) tma3s(st + a.fo[kFoMzh] * 4, &m.map[kMapMZH], it.x0, zh, it.s, bar);
+    if (ze >= 0) tma3s(st + a.fo[kFoMze] * 4, &m.map[kMapMZE], it.x0, ze, it.s, bar);
+    if (it.xb) {
+      tma3s(st + a.fo[kFoMxh] * 4, &m.map[kMapMXH], 0, r, it.s, bar);
+      if (e_row) tma3s(st + a.fo[kFoMxe] * 4, &m.map[kMapMXE], 0, r - 2 * P + 1, it.s, bar);
+    }
   }
 }
 
-// Forward H update of one Hz float4 (half nodes c..c+3, +1/2) on row r;
-// band_col >= 0: the float4 lies in the x band (memory row `mband`, table
-// entries at band column band_col).
-template <int P>
-__device__ __forceinline__ F4 hz_float4(const StepArgs &a, const BandTab &T, const float *ewin,
-                                        const F4 &hz_old, const F4 &cq, int band_col,
-                                        const float *mband, F4 &m_new) {
-  float w[12];
-  win12(ewin, w);
-  F4 out;
-  if (band_col < 0) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) out.v[q] = fmaf(cq.v[q], d_half<P>(w, q, a.c.cx), hz_old.v[q]);
-  } else {
-    m_new = lds4(mband + band_col);
-    const F4 ah = ld4(a.bt + T.x(3) + band_col), bh = ld4(a.bt + T.x(4) + band_col);
-    const F4 rk = ld4(a.bt + T.x(5) + band_col);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float d = d_half<P>(w, q, a.c.cx);
-      m_new.v[q] = fmaf(bh.v[q], m_new.v[q], ah.v[q] * d);
-      out.v[q] = fmaf(cq.v[q], fmaf(d, rk.v[q], m_new.v[q]), hz_old.v[q]);
+// Give up after a wait timed out: flag it, let the copies in flight land.
+template <int L>
+__device__ __noinline__ void give_up_s(int *flags, uint32_t bars, Ring ring, int i, int n_it,
+                                       int lane) {
+  if (lane == 0) atomicOr(flags + kFlagTimeout, 1);
+  for (int j = i; j < n_it && j <= i + L; ++j) {
+    mbar_wait_s(bars + 8 * ring.slot, ring.phase);
+    ring.next(L + 1);
+  }
+}
+
+// Walk one item.  Every phase (Hz of row r, Hx of row r - P, E of row
+// y = r - 2P + 1) is computed on every iteration and only the stores are
+// predicated on the row ranges; BAND adds the CPML recursions and the
+// array-edge masks that interior items do not need.
+template <int P, int STORE, int L, bool BAND>
+__device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, const Item &it,
+                                         FwdWarp &w, int cq_arr, float cqs) {
+  constexpr int NQ = 2 * P;
+  constexpr int NS = L + 1;
+  const int lane = w.lane;
+  const int nx = a.g.nx;
+  const int c = it.x0 - 4 + 4 * lane;
+  const bool c_ok = !BAND || (c >= 0 && c < nx);
+  const bool own_lane = lane >= 1 && lane <= 30;
+  const bool own = own_lane && c_ok;
+  const int wl = own_lane ? lane : 1;  // window base for the E update
+  const int rows = it.yb - it.ya;
+  const int64_t pb = (int64_t)it.s * a.g.numel + c;
+  float *const hz_o = a.out.hz + pb;
+  float *const hx_o = a.out.hx + pb;
+  float *const ey_o = a.out.ey + pb;
+  int ro = it.r0 * nx;  // r * nx of the running iteration
+  // CPML band state of this lane / item
+  const BandTab T{a.g.Wx, a.g.Wz};
+  const int bcol = BAND ? xband_col(c, nx, a.g.Wx) : -1;
+  const int64_t xbw = BAND ? (int64_t)it.s * a.g.ny * 2 * a.g.Wx + bcol : 0;
+  const int64_t zbw = BAND ? (int64_t)it.s * 2 * a.g.Wz * nx + c : 0;
+
+  {
+    Ring pr = w.ring;
+    for (int j = 0; j < L && j < it.n_it; ++j) {
+      if (lane == 0)
+        fwd_issue<P, BAND>(m, a, it, j, w.stage0 + pr.slot * w.stage_bytes, w.bars + 8 * pr.slot,
+                           cq_arr);
+      pr.next(NS);
     }
   }
-  return out;
+  F4 eq[NQ], hq[NQ];
+#pragma unroll
+  for (int k = 0; k < NQ; ++k) eq[k] = hq[k] = zero4();
+
+  for (int i0 = 0; i0 < it.n_it; i0 += NQ) {
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+      const int i = i0 + u;
+      if (i < it.n_it) {
+        if (i + L < it.n_it && lane == 0) {
+          const int ps = w.ring.slot == 0 ? NS - 1 : w.ring.slot - 1;
+          fwd_issue<P, BAND>(m, a, it, i + L, w.stage0 + ps * w.stage_bytes, w.bars + 8 * ps,
+                             cq_arr);
+        }
+        if (!mbar_wait_s(w.bars + 8 * w.ring.slot, w.ring.phase)) {
+          give_up_s<L>(a.flags, w.bars, w.ring, i, it.n_it, lane);
+          return false;
+        }
+        const uint32_t st = w.stage0 + w.ring.slot * w.stage_bytes;
+        const bool own_r = (unsigned)(i - (2 * P - 1)) < (unsigned)rows;
+        const bool hx_own = (unsigned)(i - (3 * P - 1)) < (unsigned)rows;  // r - P in [ya, yb)
+        const bool e_row = (unsigned)(i - (4 * P - 2)) < (unsigned)rows;
+        const bool hx_in = i >= it.hx_lo && i <= it.hx_hi;
+
+        // ---- Hz, row r: every lane, float4 at column c
+        {
+          float wv[12];
+          win12s(st + kF_EY * 4 + 16 * lane, wv);
+          eq[u] = F4{{wv[4], wv[5], wv[6], wv[7]}};
+          const F4 hz_old = lds4s(st + (kF_HZ + 4) * 4 + 16 * lane);
+          const F4 cq = cq_arr ? lds4s(st + a.fo[kFoCqH] * 4 + 16 * lane) : splat4(cqs);
+          F4 hn;
+          if (!BAND || bcol < 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) hn.v[q] = fmaf(cq.v[q], d_half<P>(wv, q, a.c.cx), hz_old.v[q]);
+          } else {
+            F4 mn = lds4s(st + (a.fo[kFoMxh] + bcol) * 4);
+            const F4 ah = ld4(a.bt + T.x(3) + bcol), bh = ld4(a.bt + T.x(4) + bcol);
+            const F4 rk = ld4(a.bt + T.x(5) + bcol);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float d = d_half<P>(wv, q, a.c.cx);
+              mn.v[q] = fmaf(bh.v[q], mn.v[q], ah.v[q] * d);
+              hn.v[q] = fmaf(cq.v[q], fmaf(d, rk.v[q], mn.v[q]), hz_old.v[q]);
+            }
+            if (own && own_r) st4(a.out.mxh_node + xbw + (int64_t)(it.r0 + i) * 2 * a.g.Wx, mn);
+          }
+          sts4s(w.hring + u * kFRing * 4 + 16 * lane, c_ok ? hn : zero4());
+          if (own && own_r) st4(hz_o + ro, hn);
+        }
+
+        // ---- Hx, row r - P (z-stencil from the Ey queue)
+        {
+          const F4 hx_old = lds4s(st + (kF_HX - 4) * 4 + 16 * lane);
+          const F4 cq = cq_arr ? lds4s(st + a.fo[kFoCqX] * 4 + 16 * lane) : splat4(cqs);
+          F4 d;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float s = 0.f;
+#pragma unroll
+            for (int k = 1; k <= P; ++k)
+              s = fmaf(a.c.cy[k - 1],
+                       eq[(u - P + k + NQ) % NQ].v[q] - eq[(u - P - k + 1 + 2 * NQ) % NQ].v[q], s);
+            d.v[q] = s;
+          }
+          if constexpr (BAND) {
+            const int zr = hx_in ? zband_row(it.r0 + i - P, a.g.ny, a.g.Wz) : -1;
+            if (zr >= 0) {
+              F4 mz = lds4s(st + (a.fo[kFoMzh] - 4) * 4 + 16 * lane);
+              const float ayh = __ldg(a.bt + T.z(3) + zr), byh = __ldg(a.bt + T.z(4) + zr);
+              const float rkyh = __ldg(a.bt + T.z(5) + zr);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mz.v[q] = fmaf(byh, mz.v[q], ayh * d.v[q]);
+                d.v[q] = fmaf(d.v[q], rkyh, mz.v[q]);
+              }
+              if (own && hx_own) st4(a.out.mzh_node + zbw + (int64_t)zr * nx, mz);
+            }
+          }
+          F4 hn;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) hn.v[q] = fmaf(-cq.v[q], d.v[q], hx_old.v[q]);
+          hq[u] = hx_in ? hn : zero4();
+          if (own && hx_own) st4(hx_o + (ro - P * nx), hn);
+        }
+
+        // ---- E, row y = r - 2P + 1
+        {
+          float wv[12];
+          win12s(w.hring + ((u + 1) % NQ) * kFRing * 4 + 16 * wl - 16, wv);
+          const F4 ca4 = lds4s(st + w.ca_o + 16 * lane - 16);
+          const F4 cb4 = lds4s(st + w.cb_o + 16 * lane - 16);
+          const F4 &e_old = eq[(u + 1) % NQ];
+          F4 cx, cz;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            cx.v[q] = d_int<P>(wv, q, a.c.cx);
+            float s = 0.f;
+#pragma unroll
+            for (int k = 1; k <= P; ++k)
+              s = fmaf(a.c.cy[k - 1], hq[(u + P + k) % NQ].v[q] - hq[(u + 1 + P - k) % NQ].v[q], s);
+            cz.v[q] = s;
+          }
+          if constexpr (BAND) {
+            const int y = it.r0 + i - 2 * P + 1;
+            if (bcol >= 0) {
+              F4 mx = lds4s(st + (a.fo[kFoMxe] + bcol) * 4);
+              const F4 ax = ld4(a.bt + T.x(0) + bcol), bx = ld4(a.bt + T.x(1) + bcol);
+              const F4 rk = ld4(a.bt + T.x(2) + bcol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mx.v[q] = fmaf(bx.v[q], mx.v[q], ax.v[q] * cx.v[q]);
+                cx.v[q] = fmaf(cx.v[q], rk.v[q], mx.v[q]);
+              }
+              if (own && e_row) st4(a.out.mxe_node + xbw + (int64_t)y * 2 * a.g.Wx, mx);
+            }
+            const int zr = e_row ? zband_row(y, a.g.ny, a.g.Wz) : -1;
+            if (zr >= 0) {
+              F4 mz = lds4s(st + (a.fo[kFoMze] - 4) * 4 + 16 * lane);
+              const float ay = __ldg(a.bt + T.z(0) + zr), by = __ldg(a.bt + T.z(1) + zr);
+              const float rky = __ldg(a.bt + T.z(2) + zr);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mz.v[q] = fmaf(by, mz.v[q], ay * cz.v[q]);
+                cz.v[q] = fmaf(cz.v[q], rky, mz.v[q]);
+              }
+              if (own) st4(a.out.mze_node + zbw + (int64_t)zr * nx, mz);
+            }
+          }
+          F4 curl, en;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            curl.v[q] = cx.v[q] - cz.v[q];
+            en.v[q] = fmaf(ca4.v[q], e_old.v[q], cb4.v[q] * curl.v[q]);
+          }
+          if (own && e_row) {
+            const int off = ro - (2 * P - 1) * nx;
+            if constexpr (STORE == kStoreF32) {
+              snap_store<STORE>(reinterpret_cast<float *>(a.snap_e) + pb + off, e_old);
+              snap_store<STORE>(reinterpret_cast<float *>(a.snap_c) + pb + off, curl);
+            } else if constexpr (STORE == kStoreBF16) {
+              snap_store<STORE>(reinterpret_cast<__nv_bfloat16 *>(a.snap_e) + pb + off, e_old);
+              snap_store<STORE>(reinterpret_cast<__nv_bfloat16 *>(a.snap_c) + pb + off, curl);
+            }
+            st4(ey_o + off, en);
+          }
+        }
+        __syncwarp();
+        w.ring.next(NS);
+        ro += nx;
+      }
+    }
+  }
+  return true;
 }
 
 template <int P, int STORE, int L>
 __global__ void __launch_bounds__(128) k_forward(const __grid_constant__ FwdMaps m,
                                                  const StepArgs a, const int batched,
                                                  const int cq_arr) {
-  constexpr int NQ = 2 * P;
   constexpr int NS = L + 1;
   (void)sizeof(Stages<L>);
-  extern __shared__ float smem_raw[];
-  float *smem = reinterpret_cast<float *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  extern __shared__ __align__(128) float smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 127u) & ~127u;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem) + warp * NS;
-  float *wb = smem + 32 + warp * a.warp_floats;
-  float *hs = wb + NS * a.stage_floats;  // Hz ring: NQ rows of 32 float4
-  const int band_slot = a.band_floats, band_box = a.band_box_floats * 4;
+  FwdWarp w;
+  w.lane = lane;
+  w.bars = base + warp * NS * 8;
+  w.stage_bytes = (uint32_t)a.stage_floats * 4;
+  w.stage0 = base + 128 + warp * a.warp_floats * 4;
+  w.hring = w.stage0 + NS * w.stage_bytes;  // Hz ring: 2P rows of 32 float4
+  // pair box: [Ca][Cb] (or [Cb][Ca] when Cb lies first), 120 floats each;
+  // two boxes: Ca at kF_MD, Cb at kF_MD + 128 (every box starts 128-aligned)
+  w.ca_o = (kF_MD + (a.md_pair && a.md_swap ? 120 : 0)) * 4;
+  w.cb_o = (kF_MD + (a.md_pair ? (a.md_swap ? 0 : 120) : 128)) * 4;
+  w.ring = Ring{0, 0u};
   const Geom &g = a.g;
-  const int nx = g.nx, ny = g.ny;
   const int n_items = g.S * g.n_strips * g.n_chunks;
   if (__any_sync(kFull, *reinterpret_cast<volatile int *>(a.flags + kFlagTimeout) != 0)) return;
   if (lane == 0) {
-    for (int k = 0; k < NS; ++k) mbar_init(&bars[k], 1);
+    for (int k = 0; k < NS; ++k)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(w.bars + 8 * k), "r"(1)
+                   : "memory");
     fence_mbar_init();
   }
   __syncwarp();
   const float cqs = cq_arr ? 0.f : __ldg(a.cq);
-  const bool own_lane = lane >= 1 && lane <= 30;
-  const int wl = own_lane ? lane : 1;  // window base for the E update
-  const BandTab T{g.Wx, g.Wz};
-  Ring ring{0, 0u};
   // work items are claimed dynamically; the counter of the next launch is
   // reset here (the previous launch that used it has completed)
   int *ctr = a.flags + kCtrBase + a.ctr_slot;
@@ -355,240 +549,373 @@ __global__ void __launch_bounds__(128) k_forward(const __grid_constant__ FwdMaps
     if (item >= n_items) break;
     Item it;
     if (!make_item<P>(g, item, batched != 0, it)) continue;
-    // this lane's column: Hz float4 at c; owned cells (lanes 1..30) also at c
-    const int c = it.x0 - 4 + 4 * lane;
-    const bool c_ok = c >= 0 && c < nx;
-    const bool own = own_lane && c_ok;
-    const int bcol = xband_col(c, nx, g.Wx);
-    const int64_t sb = (int64_t)it.s * g.numel + c;  // + row * nx
-    const int64_t mb = (int64_t)it.sm * g.numel + c;
-    const int64_t xbw = (int64_t)it.s * ny * 2 * g.Wx + bcol;
-    const int64_t zbw = (int64_t)it.s * 2 * g.Wz * nx + c;
-    {
-      Ring pr = ring;
-      for (int j = 0; j < L && j < it.n_it; ++j) {
-        fwd_issue<P>(m, g, it, j, wb + pr.slot * a.stage_floats, &bars[pr.slot], band_slot,
-                     band_box, lane);
-        pr.next(NS);
-      }
-    }
-    F4 eq[NQ], hq[NQ];
-#pragma unroll
-    for (int k = 0; k < NQ; ++k) eq[k] = hq[k] = zero4();
-
-    for (int i0 = 0; i0 < it.n_it; i0 += NQ) {
-#pragma unroll
-      for (int u = 0; u < NQ; ++u) {
-        const int i = i0 + u;
-        if (i < it.n_it) {
-          if (i + L < it.n_it) {
-            const int ps = ring.slot == 0 ? NS - 1 : ring.slot - 1;
-            fwd_issue<P>(m, g, it, i + L, wb + ps * a.stage_floats, &bars[ps], band_slot,
-                         band_box, lane);
-          }
-          const float *st = wb + ring.slot * a.stage_floats;
-          if (!mbar_wait(&bars[ring.slot], ring.phase)) {
-            // give up: flag it, let the copies in flight land, leave
-            if (lane == 0) atomicOr(a.flags + kFlagTimeout, 1);
-            Ring dr = ring;
-            for (int j = i; j < it.n_it && j <= i + L; ++j) {
-              mbar_wait(&bars[dr.slot], dr.phase);
-              dr.next(NS);
-            }
-            return;
-          }
-          const Rows<P> R(it.r0, i, it.ya, it.yb, ny);
-          const float *sey = st + kF_EY;
-          eq[u] = lds4(sey + 4 * lane + 4);
-
-          // ---- Hz update, row r: every lane, float4 at column c
-          if (R.own_r) {
-            const F4 cq = cq_arr ? (c_ok ? ld4(a.cq + mb + (int64_t)R.r * nx) : zero4()) : splat4(cqs);
-            F4 mn;
-            F4 hn = hz_float4<P>(a, T, sey + 4 * lane, lds4(st + kF_HZ + 4 * lane), cq, bcol,
-                                 st + kF_BAND, mn);
-            st4(hs + u * kFRing + 4 * lane, c_ok ? hn : zero4());
-            if (own) {
-              st4(a.out.hz + sb + (int64_t)R.r * nx, hn);
-              if (bcol >= 0) st4(a.out.mxh_node + xbw + (int64_t)R.r * 2 * g.Wx, mn);
-            }
-          }
-
-          // ---- Hx update, row rh (owned lanes; z-stencil from the Ey queue)
-          if (R.hx_need) {
-            F4 hn = zero4();
-            if (R.hx_in) {
-              const F4 hx_old = lds4(st + kF_HX + 4 * lane - 4);
-              const F4 cq = cq_arr ? (own ? ld4(a.cq + mb + (int64_t)R.rh * nx) : zero4()) : splat4(cqs);
-              const int zr = zband_row(R.rh, ny, g.Wz);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                float d = 0.f;
-#pragma unroll
-                for (int k = 1; k <= P; ++k)
-                  d = fmaf(a.c.cy[k - 1],
-                           eq[(u - P + k + NQ) % NQ].v[q] - eq[(u - P - k + 1 + 2 * NQ) % NQ].v[q],
-                           d);
-                hn.v[q] = d;
-              }
-              if (zr >= 0) {
-                F4 mz = lds4(st + kF_MZH + 4 * lane - 4);
-                const float ayh = __ldg(a.bt + T.z(3) + zr), byh = __ldg(a.bt + T.z(4) + zr);
-                const float rkyh = __ldg(a.bt + T.z(5) + zr);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  mz.v[q] = fmaf(byh, mz.v[q], ayh * hn.v[q]);
-                  hn.v[q] = fmaf(hn.v[q], rkyh, mz.v[q]);
-                }
-                if (own && R.rh >= it.ya && R.rh < it.yb)
-                  st4(a.out.mzh_node + zbw + (int64_t)zr * nx, mz);
-              }
-#pragma unroll
-              for (int q = 0; q < 4; ++q) hn.v[q] = fmaf(-cq.v[q], hn.v[q], hx_old.v[q]);
-              if (own && R.rh >= it.ya && R.rh < it.yb) st4(a.out.hx + sb + (int64_t)R.rh * nx, hn);
-            }
-            hq[u] = hn;
-          }
-
-          // ---- E update, row y (owned lanes)
-          if (R.e_row && own) {
-            float w[12];
-            win12(hs + ((u + 1) % NQ) * kFRing + 4 * wl - 4, w);
-            const F4 ca4 = lds4(st + kF_CA + 4 * lane - 4);
-            const F4 cb4 = lds4(st + kF_CB + 4 * lane - 4);
-            const F4 &e_old = eq[(u + 1) % NQ];
-            const int zr = zband_row(R.y, ny, g.Wz);
-            F4 cx, cz;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              cx.v[q] = d_int<P>(w, q, a.c.cx);
-              float d = 0.f;
-#pragma unroll
-              for (int k = 1; k <= P; ++k)
-                d = fmaf(a.c.cy[k - 1], hq[(u + P + k) % NQ].v[q] - hq[(u + 1 + P - k) % NQ].v[q],
-                         d);
-              cz.v[q] = d;
-            }
-            if (bcol >= 0) {
-              F4 mx = lds4(st + kF_BAND + band_slot + bcol);
-              const F4 ax = ld4(a.bt + T.x(0) + bcol), bx = ld4(a.bt + T.x(1) + bcol);
-              const F4 rk = ld4(a.bt + T.x(2) + bcol);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                mx.v[q] = fmaf(bx.v[q], mx.v[q], ax.v[q] * cx.v[q]);
-                cx.v[q] = fmaf(cx.v[q], rk.v[q], mx.v[q]);
-              }
-              st4(a.out.mxe_node + xbw + (int64_t)R.y * 2 * g.Wx, mx);
-            }
-            if (zr >= 0) {
-              F4 mz = lds4(st + kF_MZE + 4 * lane - 4);
-              const float ay = __ldg(a.bt + T.z(0) + zr), by = __ldg(a.bt + T.z(1) + zr);
-              const float rky = __ldg(a.bt + T.z(2) + zr);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                mz.v[q] = fmaf(by, mz.v[q], ay * cz.v[q]);
-                cz.v[q] = fmaf(cz.v[q], rky, mz.v[q]);
-              }
-              st4(a.out.mze_node + zbw + (int64_t)zr * nx, mz);
-            }
-            F4 curl, en;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              curl.v[q] = cx.v[q] - cz.v[q];
-              en.v[q] = fmaf(ca4.v[q], e_old.v[q], cb4.v[q] * curl.v[q]);
-            }
-            const int64_t off = sb + (int64_t)R.y * nx;
-            if constexpr (STORE == kStoreF32) {
-              snap_store<STORE>(reinterpret_cast<float *>(a.snap_e) + off, e_old);
-              snap_store<STORE>(reinterpret_cast<float *>(a.snap_c) + off, curl);
-            } else if constexpr (STORE == kStoreBF16) {
-              snap_store<STORE>(reinterpret_cast<__nv_bfloat16 *>(a.snap_e) + off, e_old);
-              snap_store<STORE>(reinterpret_cast<__nv_bfloat16 *>(a.snap_c) + off, curl);
-            }
-            st4(a.out.ey + off, en);
-          }
-          __syncwarp();
-          ring.next(NS);
-        }
-      }
-    }
+    const bool ok = it.edge ? fwd_walk<P, STORE, L, true>(m, a, it, w, cq_arr, cqs)
+                            : fwd_walk<P, STORE, L, false>(m, a, it, w, cq_arr, cqs);
+    if (!ok) return;
   }
 }
 
 // ---------------------------------------------------------------------------
 // adjoint
 
-template <int P, bool BF16>
-__device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, const Geom &g,
-                                          const Item &it, int i, float *st, uint64_t *bar,
-                                          int band_slot, int band_box, int lane) {
-  const Rows<P> R(it.r0, i, it.ya, it.yb, g.ny);
-  const int ze = zband_row(R.r, g.ny, g.Wz);
-  const int zh = R.hx_in ? zband_row(R.rh, g.ny, g.Wz) : -1;
-  constexpr uint32_t snap_bytes = BF16 ? 112 * 2 : 112 * 4;
-  const bool l_lam = lane == kLdLam, l_cb = lane == kLdCbA, l_lhz = lane == kLdLhz;
-  const bool l_se = lane == kLdSe, l_sc = lane == kLdSc, l_gca = lane == kLdGca;
-  const bool l_gcb = lane == kLdGcb, l_lhx = lane == kLdLhx, l_ca = lane == kLdCaA;
-  const bool l_lamy = lane == kLdLamy, l_mxe = lane == kLdMxeA, l_mxh = lane == kLdMxhA;
-  const bool l_mze = lane == kLdMzeA, l_mzh = lane == kLdMzhA;
-  const bool l_own = l_lhz | l_se | l_sc | l_gca | l_gcb;
-  const bool act = l_lam | l_cb | (l_own & R.own_r) | (l_lhx & R.hx_in) | ((l_ca | l_lamy) & R.e_row) |
-                   ((l_mxe | l_mxh) & R.own_r & it.xb) | (l_mze & (ze >= 0)) | (l_mzh & (zh >= 0));
-  const int c0 = (l_lam | l_cb) ? it.x0 - 8 : l_lhz ? it.x0 - 4 : (l_mxe | l_mxh) ? 0 : it.x0;
-  const int c1 = l_lhx ? R.rh : (l_ca | l_lamy) ? R.y : l_mze ? ze : l_mzh ? zh : R.r;
-  const int c2 = (l_cb | l_ca) ? it.sm : it.s;
-  const int off = l_lam ? kA_LAM : l_cb ? kA_CB : l_lhz ? kA_LHZ : l_se ? kA_SE : l_sc ? kA_SC
-                : l_gca ? kA_GCA : l_gcb ? kA_GCB : l_lhx ? kA_LHX : l_ca ? kA_CA
-                : l_lamy ? kA_LAMY : l_mze ? kA_MZE : l_mzh ? kA_MZH : l_mxe ? kA_BAND
-                : kA_BAND + band_slot;
-  const uint32_t bytes = (l_lam | l_cb) ? 128 * 4 : l_lhz ? 120 * 4 : (l_se | l_sc) ? snap_bytes
-                       : (l_mxe | l_mxh) ? band_box : 112 * 4;
-  const uint32_t total = __reduce_add_sync(kFull, act ? bytes : 0u);
-  if (lane == 0) mbar_expect_tx(bar, total);
-  __syncwarp();
-  if (act) {
-    fence_proxy_async();
-    const CUtensorMap *map = &m.map[lane < kAdjLoads ? lane : 0];
-    if (l_se | l_sc)
-      tma4(st + off, map, c0, c1, c2, a.snap_t, bar);
-    else
-      tma3(st + off, map, c0, c1, c2, bar);
+__device__ __forceinline__ void tma5s(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                      int c3, int c4, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+      "r"(bar)
+      : "memory");
+}
+// Staged snapshot float4 (4 cells) at byte address addr: float32 or bf16.
+template <bool BF16>
+__device__ __forceinline__ F4 snap_lds_s(uint32_t addr) {
+  if constexpr (!BF16) {
+    return lds4s(addr);
+  } else {
+    uint32_t lo, hi;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi) : "r"(addr) : "memory");
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&lo);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&hi);
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return F4{{fa.x, fa.y, fb.x, fb.y}};
   }
 }
 
-template <int P, bool BF16, int L>
-__global__ void __launch_bounds__(128) k_adjoint(const __grid_constant__ AdjMaps m,
-                                                 const StepArgs a, const int batched,
-                                                 const int cq_arr) {
+struct AdjWarp {
+  uint32_t bars, stage0, prow, qring;
+  uint32_t stage_bytes;
+  uint32_t ca_o, cb_o, gca_o, gcb_o;  // byte offsets within a stage
+  int lane;
+  Ring ring;
+};
+
+// Issue the loads of walk iteration i (lane 0 only): row r = r0 + i for
+// lambda_E / lambda_Hz, Ca / Cb, Cq, the snapshots, the gradients and the
+// band memories of the E nodes and (x band) H nodes; row r - P for
+// lambda_Hx, its Cq and its z-band memory.  Rows outside the array read as
+// zeros.
+template <int P, bool BF16, bool BAND>
+__device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, const Item &it,
+                                          int i, uint32_t st, uint32_t bar, int cq_arr) {
+  const int r = it.r0 + i;
+  const bool own_r = (unsigned)(i - (2 * P - 1)) < (unsigned)(it.yb - it.ya);
+  const bool hx_in = i >= it.hx_lo && i <= it.hx_hi;
+  constexpr uint32_t snap_bytes = BF16 ? 2 * 112 * 2 : 2 * 112 * 4;
+  uint32_t bytes = 2 * 128 * 4 + 2 * 128 * 4;
+  if (hx_in) bytes += 112 * 4;
+  if (own_r) bytes += snap_bytes + 2 * 112 * 4;
+  if (cq_arr) bytes += hx_in ? 2 * 128 * 4 : 128 * 4;
+  int ze = -1, zh = -1;
+  if constexpr (BAND) {
+    ze = zband_row(r, a.g.ny, a.g.Wz);
+    if (hx_in) zh = zband_row(r - P, a.g.ny, a.g.Wz);
+    if (ze >= 0) bytes += 112 * 4;
+    if (zh >= 0) bytes += 112 * 4;
+    if (own_r && it.xb) bytes += 2 * (uint32_t)a.band_box_floats * 4;
+  }
+  expect_tx_s(bar, bytes);
+  fence_proxy_async();
+  tma4s(st + kA_EH * 4, &m.map[kAMapEH], it.x0 - 8, r, it.s, 0, bar);
+  if (a.md_pair) {
+    tma4s(st + kA_MD * 4, &m.map[kAMapMD], it.x0 - 8, r, it.sm, 0, bar);
+  } else {
+    tma3s(st + kA_MD * 4, &m.map[kAMapMD], it.x0 - 8, r, it.sm, bar);
+    tma3s(st + (kA_MD + 128) * 4, &m.map[kAMapCB], it.x0 - 8, r, it.sm, bar);
+  }
+  if (hx_in) tma3s(st + kA_HX * 4, &m.map[kAMapHX], it.x0, r - P, it.s, bar);
+  if (own_r) {
+    tma5s(st + kA_SS * 4, &m.map[kAMapSS], it.x0, r, it.s, a.snap_t, 0, bar);
+    if (a.gg_pair) {
+      tma4s(st + kA_GG * 4, &m.map[kAMapGG], it.x0, r, it.s, 0, bar);
+    } else {
+      tma3s(st + kA_GG * 4, &m.map[kAMapGG], it.x0, r, it.s, bar);
+      tma3s(st + (kA_GG + 128) * 4, &m.map[kAMapGB], it.x0, r, it.s, bar);
+    }
+  }
+  if (cq_arr) {
+    tma3s(st + a.ao[kAoCqR] * 4, &m.map[kAMapCQ], it.x0 - 8, r, it.sm, bar);
+    if (hx_in) tma3s(st + a.ao[kAoCqH] * 4, &m.map[kAMapCQ], it.x0 - 8, r - P, it.sm, bar);
+  }
+  if constexpr (BAND) {
+    if (ze >= 0) tma3s(st + a.ao[kAoMze] * 4, &m.map[kAMapMZE], it.x0, ze, it.s, bar);
+    if (zh >= 0) tma3s(st + a.ao[kAoMzh] * 4, &m.map[kAMapMZH], it.x0, zh, it.s, bar);
+    if (own_r && it.xb) tma4s(st + a.ao[kAoMx] * 4, &m.map[kAMapMX], 0, r, it.s, 0, bar);
+  }
+}
+
+// Walk one item of the adjoint.  Per iteration (row r = r0 + i):
+//   g = Cb lam, Ca lam (queued for the E update of this row), pz (every
+//   row, queued for the z-stencil); on owned rows the gradients, px and then
+//   lamHz and qx; lamHx and qz of row r - P; lamE of row r - 2P + 1.
+// Lanes: 0..31 hold the float4 at x0 - 8 + 4 lane (g, px, pz; lanes 2..29
+// own theirs), lanes 0..29 the qx float4 at x0 - 4 + 4 lane.
+template <int P, bool BF16, int L, bool BAND>
+__device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, const Item &it,
+                                         AdjWarp &w, int cq_arr, float cqs) {
   constexpr int NQ = 2 * P;
   constexpr int NS = L + 1;
+  const int lane = w.lane;
+  const int nx = a.g.nx, ny = a.g.ny;
+  const bool own_lane = lane >= 2 && lane <= 29;  // owned float4 o = lane - 2
+  const bool q_lane = lane <= 29;
+  const int wq = q_lane ? lane : 0;        // px window base (lanes 30, 31 idle)
+  const int wo = own_lane ? lane - 2 : 0;  // qx window base of the E update
+  const int pc = it.x0 - 8 + 4 * lane;
+  const int qc = it.x0 - 4 + 4 * lane;
+  const bool pc_ok = !BAND || (pc >= 0 && pc < nx);
+  const bool qc_ok = q_lane && (!BAND || (qc >= 0 && qc < nx));
+  const bool own = own_lane && pc_ok;
+  const bool q_own = lane >= 1 && lane <= 28 && qc_ok;
+  const int rows = it.yb - it.ya;
+  const int64_t sp = (int64_t)it.s * a.g.numel + pc;
+  float *const hz_o = a.out.hz + (sp + 4);
+  float *const hx_o = a.out.hx + sp;
+  float *const ey_o = a.out.ey + sp;
+  float *const gca_o = a.gca + sp;
+  float *const gcb_o = a.gcb + sp;
+  int ro = it.r0 * nx;
+  const BandTab T{a.g.Wx, a.g.Wz};
+  const int pb = BAND ? xband_col(pc, nx, a.g.Wx) : -1;
+  const int qb = BAND && q_lane ? xband_col(qc, nx, a.g.Wx) : -1;
+  const int64_t xw = BAND ? (int64_t)it.s * ny * 2 * a.g.Wx : 0;
+  const int64_t zbw = BAND ? (int64_t)it.s * 2 * a.g.Wz * nx + pc : 0;
+  bool colmask[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    colmask[q] = !BAND || !a.g.grad_mask || (pc + q >= a.g.n_pml && pc + q < nx - a.g.n_pml);
+
+  {
+    Ring pr = w.ring;
+    for (int j = 0; j < L && j < it.n_it; ++j) {
+      if (lane == 0)
+        adj_issue<P, BF16, BAND>(m, a, it, j, w.stage0 + pr.slot * w.stage_bytes,
+                                 w.bars + 8 * pr.slot, cq_arr);
+      pr.next(NS);
+    }
+  }
+  F4 pq[NQ], qq[NQ], cl[NQ];
+#pragma unroll
+  for (int k = 0; k < NQ; ++k) pq[k] = qq[k] = cl[k] = zero4();
+
+  for (int i0 = 0; i0 < it.n_it; i0 += NQ) {
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+      const int i = i0 + u;
+      if (i < it.n_it) {
+        if (i + L < it.n_it && lane == 0) {
+          const int ps = w.ring.slot == 0 ? NS - 1 : w.ring.slot - 1;
+          adj_issue<P, BF16, BAND>(m, a, it, i + L, w.stage0 + ps * w.stage_bytes,
+                                   w.bars + 8 * ps, cq_arr);
+        }
+        if (!mbar_wait_s(w.bars + 8 * w.ring.slot, w.ring.phase)) {
+          give_up_s<L>(a.flags, w.bars, w.ring, i, it.n_it, lane);
+          return false;
+        }
+        const uint32_t st = w.stage0 + w.ring.slot * w.stage_bytes;
+        const int r = it.r0 + i;
+        const bool own_r = (unsigned)(i - (2 * P - 1)) < (unsigned)rows;
+        const bool hx_own = (unsigned)(i - (3 * P - 1)) < (unsigned)rows;  // r - P in [ya, yb)
+        const bool e_row = (unsigned)(i - (4 * P - 2)) < (unsigned)rows;
+        const bool hx_in = i >= it.hx_lo && i <= it.hx_hi;
+
+        const F4 lam = lds4s(st + kA_EH * 4 + 16 * lane);
+        const F4 cbv = lds4s(st + w.cb_o + 16 * lane);
+        const F4 cav = lds4s(st + w.ca_o + 16 * lane);
+        F4 gv;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gv.v[q] = cbv.v[q] * lam.v[q];
+          cl[u].v[q] = cav.v[q] * lam.v[q];
+        }
+        // ---- pz at E nodes (every row; owned lanes matter)
+        {
+          F4 pz;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) pz.v[q] = -gv.v[q];
+          if constexpr (BAND) {
+            const int zr = zband_row(r, ny, a.g.Wz);
+            if (zr >= 0) {
+              F4 M = lds4s(st + (a.ao[kAoMze] - 8) * 4 + 16 * lane);
+              const float ay = __ldg(a.bt + T.z(0) + zr), by = __ldg(a.bt + T.z(1) + zr);
+              const float rky = __ldg(a.bt + T.z(2) + zr);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                M.v[q] -= gv.v[q];
+                pz.v[q] = fmaf(ay, M.v[q], -gv.v[q] * rky);
+                M.v[q] *= by;
+              }
+              if (own && own_r) st4(a.out.mze_node + zbw + (int64_t)zr * nx, M);
+            }
+          }
+          pq[u] = pz;
+        }
+        // ---- owned rows: gradients (lam = lambda_E^{t+1}) and px
+        if (own_r) {
+          if (own) {
+            const uint32_t sbase = st + kA_SS * 4;
+            constexpr uint32_t sfield = BF16 ? 112 * 2 : 112 * 4;
+            constexpr uint32_t sstep = BF16 ? 8 : 16;
+            const F4 se = snap_lds_s<BF16>(sbase + sstep * wo);
+            const F4 sc = snap_lds_s<BF16>(sbase + sfield + sstep * wo);
+            F4 gca = lds4s(st + w.gca_o + 16 * wo), gcb = lds4s(st + w.gcb_o + 16 * wo);
+            const bool rowmask = !BAND || !a.g.grad_mask || (r >= a.g.n_pml && r < ny - a.g.n_pml);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (rowmask && colmask[q]) {
+                gca.v[q] = fmaf(se.v[q], lam.v[q], gca.v[q]);
+                gcb.v[q] = fmaf(sc.v[q], lam.v[q], gcb.v[q]);
+              }
+            }
+            st4(gca_o + ro, gca);
+            st4(gcb_o + ro, gcb);
+          }
+          F4 px = gv;
+          if constexpr (BAND) {
+            if (pb >= 0) {
+              F4 M = lds4s(st + (a.ao[kAoMx] + a.band_box_floats + pb) * 4);
+              const F4 ax = ld4(a.bt + T.x(0) + pb), bx = ld4(a.bt + T.x(1) + pb);
+              const F4 rk = ld4(a.bt + T.x(2) + pb);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                M.v[q] += gv.v[q];
+                px.v[q] = fmaf(ax.v[q], M.v[q], gv.v[q] * rk.v[q]);
+                M.v[q] *= bx.v[q];
+              }
+              if (own) st4(a.out.mxe_node + xw + (int64_t)r * 2 * a.g.Wx + pb, M);
+            }
+          }
+          sts4s(w.prow + 16 * lane, pc_ok ? px : zero4());
+        }
+        __syncwarp();
+
+        // ---- owned rows: lamHz and qx (lanes 0..29)
+        if (own_r) {
+          float wv[12];
+          win12s(w.prow + 16 * wq, wv);
+          const F4 lhz_old = lds4s(st + (kA_EH + 128 + 4) * 4 + 16 * wq);
+          const F4 cq = cq_arr ? lds4s(st + (a.ao[kAoCqR] + 4) * 4 + 16 * wq) : splat4(cqs);
+          F4 lhz, v;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            lhz.v[q] = lhz_old.v[q] - d_half<P>(wv, q, a.c.cx);
+            v.v[q] = cq.v[q] * lhz.v[q];
+          }
+          if (q_own) st4(hz_o + ro, lhz);
+          if constexpr (BAND) {
+            if (qb >= 0) {
+              F4 M = lds4s(st + (a.ao[kAoMx] + qb) * 4);
+              const F4 ah = ld4(a.bt + T.x(3) + qb), bh = ld4(a.bt + T.x(4) + qb);
+              const F4 rk = ld4(a.bt + T.x(5) + qb);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                M.v[q] += v.v[q];
+                const float vq = v.v[q];
+                v.v[q] = fmaf(ah.v[q], M.v[q], vq * rk.v[q]);
+                M.v[q] *= bh.v[q];
+              }
+              if (q_own) st4(a.out.mxh_node + xw + (int64_t)r * 2 * a.g.Wx + qb, M);
+            }
+          }
+          if (q_lane) sts4s(w.qring + u * kARing * 4 + 16 * lane, qc_ok ? v : zero4());
+        }
+
+        // ---- lamHx and qz of row r - P (owned lanes)
+        {
+          const F4 lhx = lds4s(st + (kA_HX - 8) * 4 + 16 * lane);
+          const F4 cq = cq_arr ? lds4s(st + a.ao[kAoCqH] * 4 + 16 * lane) : splat4(cqs);
+          F4 lh, qz;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float d = 0.f;
+#pragma unroll
+            for (int k = 1; k <= P; ++k)
+              d = fmaf(a.c.cy[k - 1],
+                       pq[(u - P + k + NQ) % NQ].v[q] - pq[(u - P - k + 1 + 2 * NQ) % NQ].v[q], d);
+            lh.v[q] = lhx.v[q] - d;
+            qz.v[q] = -cq.v[q] * lh.v[q];
+          }
+          if (own && hx_own) st4(hx_o + (ro - P * nx), lh);
+          if constexpr (BAND) {
+            const int zr = hx_in ? zband_row(r - P, ny, a.g.Wz) : -1;
+            if (zr >= 0) {
+              F4 M = lds4s(st + (a.ao[kAoMzh] - 8) * 4 + 16 * lane);
+              const float ayh = __ldg(a.bt + T.z(3) + zr), byh = __ldg(a.bt + T.z(4) + zr);
+              const float rkyh = __ldg(a.bt + T.z(5) + zr);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float vq = qz.v[q];
+                M.v[q] += vq;
+                qz.v[q] = fmaf(ayh, M.v[q], vq * rkyh);
+                M.v[q] *= byh;
+              }
+              if (own && hx_own) st4(a.out.mzh_node + zbw + (int64_t)zr * nx, M);
+            }
+          }
+          qq[u] = hx_in ? qz : zero4();
+        }
+
+        // ---- lamE of row r - 2P + 1 (owned lanes)
+        if (e_row) {
+          float wv[12];
+          win12s(w.qring + ((u + 1) % NQ) * kARing * 4 + 16 * wo, wv);
+          F4 en;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float dz = 0.f;
+#pragma unroll
+            for (int k = 1; k <= P; ++k)
+              dz = fmaf(a.c.cy[k - 1], qq[(u + P + k) % NQ].v[q] - qq[(u + 1 + P - k) % NQ].v[q],
+                        dz);
+            en.v[q] = cl[(u + 1) % NQ].v[q] - d_int<P>(wv, q, a.c.cx) - dz;
+          }
+          if (own) st4(ey_o + (ro - (2 * P - 1) * nx), en);
+        }
+        __syncwarp();
+        w.ring.next(NS);
+        ro += nx;
+      }
+    }
+  }
+  return true;
+}
+
+template <int P, bool BF16, int L>
+__global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_constant__ AdjMaps m,
+                                                                  const StepArgs a,
+                                                                  const int batched,
+                                                                  const int cq_arr) {
+  constexpr int NS = L + 1;
   (void)sizeof(Stages<L>);
-  extern __shared__ float smem_raw[];
-  float *smem = reinterpret_cast<float *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+  extern __shared__ __align__(128) float smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 127u) & ~127u;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem) + warp * NS;
-  float *wb = smem + 32 + warp * a.warp_floats;
-  float *prow = wb + NS * a.stage_floats;  // px row: 32 float4
-  float *hs = prow + kAPx;                 // qx ring: NQ rows of 30 float4
-  const int band_slot = a.band_floats, band_box = a.band_box_floats * 4;
+  AdjWarp w;
+  w.lane = lane;
+  w.bars = base + warp * NS * 8;
+  w.stage_bytes = (uint32_t)a.stage_floats * 4;
+  w.stage0 = base + 128 + warp * a.warp_floats * 4;
+  w.prow = w.stage0 + NS * w.stage_bytes;  // px row: 32 float4
+  w.qring = w.prow + kAPx * 4;             // qx ring: 2P rows of 30 float4
+  // pair boxes: [Ca][Cb] / [gCa][gCb], or the other order when the second
+  // array lies first; single boxes at 128-float slots
+  w.ca_o = (kA_MD + (a.md_pair && a.md_swap ? 128 : 0)) * 4;
+  w.cb_o = (kA_MD + (a.md_pair && a.md_swap ? 0 : 128)) * 4;
+  w.gca_o = (kA_GG + (a.gg_pair && a.gg_swap ? 112 : 0)) * 4;
+  w.gcb_o = (kA_GG + (a.gg_pair ? (a.gg_swap ? 0 : 112) : 128)) * 4;
+  w.ring = Ring{0, 0u};
   const Geom &g = a.g;
-  const int nx = g.nx, ny = g.ny;
   const int n_items = g.S * g.n_strips * g.n_chunks;
   if (__any_sync(kFull, *reinterpret_cast<volatile int *>(a.flags + kFlagTimeout) != 0)) return;
   if (lane == 0) {
-    for (int k = 0; k < NS; ++k) mbar_init(&bars[k], 1);
+    for (int k = 0; k < NS; ++k)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(w.bars + 8 * k), "r"(1)
+                   : "memory");
     fence_mbar_init();
   }
   __syncwarp();
   const float cqs = cq_arr ? 0.f : __ldg(a.cq);
-  const bool own_lane = lane >= 2 && lane <= 29;   // owned float4 o = lane - 2
-  const bool q_lane = lane <= 29;                  // qx float4 at column x0 - 4 + 4 lane
-  const int wq = q_lane ? lane : 0;                // px window base (lanes 30, 31 idle)
-  const int wo = own_lane ? lane - 2 : 0;          // qx window base of the E update
-  const BandTab T{g.Wx, g.Wz};
-  Ring ring{0, 0u};
   int *ctr = a.flags + kCtrBase + a.ctr_slot;
   if (blockIdx.x == 0 && threadIdx.x == 0) a.flags[kCtrBase + (a.ctr_slot ^ 1)] = 0;
 
@@ -599,209 +926,9 @@ __global__ void __launch_bounds__(128) k_adjoint(const __grid_constant__ AdjMaps
     if (item >= n_items) break;
     Item it;
     if (!make_item<P>(g, item, batched != 0, it)) continue;
-    const int pc = it.x0 - 8 + 4 * lane;  // px / own float4 column
-    const int qc = it.x0 - 4 + 4 * lane;  // qx float4 column
-    const bool pc_ok = pc >= 0 && pc < nx;
-    const bool qc_ok = q_lane && qc >= 0 && qc < nx;
-    const bool own = own_lane && pc_ok;
-    const bool q_own = lane >= 1 && lane <= 28 && qc_ok;  // qx float4 inside the strip
-    const int pb = xband_col(pc, nx, g.Wx);
-    const int qb = q_lane ? xband_col(qc, nx, g.Wx) : -1;
-    const int64_t sbp = (int64_t)it.s * g.numel + pc;
-    const int64_t sbq = (int64_t)it.s * g.numel + qc;
-    const int64_t mbp = (int64_t)it.sm * g.numel + pc;
-    const int64_t mbq = (int64_t)it.sm * g.numel + qc;
-    const int64_t xw = (int64_t)it.s * ny * 2 * g.Wx;
-    const int64_t zbw = (int64_t)it.s * 2 * g.Wz * nx + pc;
-    bool colmask[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      colmask[q] = !g.grad_mask || (pc + q >= g.n_pml && pc + q < nx - g.n_pml);
-    {
-      Ring pr = ring;
-      for (int j = 0; j < L && j < it.n_it; ++j) {
-        adj_issue<P, BF16>(m, a, g, it, j, wb + pr.slot * a.stage_floats, &bars[pr.slot],
-                           band_slot, band_box, lane);
-        pr.next(NS);
-      }
-    }
-    F4 pq[NQ], qq[NQ];
-#pragma unroll
-    for (int k = 0; k < NQ; ++k) pq[k] = qq[k] = zero4();
-
-    for (int i0 = 0; i0 < it.n_it; i0 += NQ) {
-#pragma unroll
-      for (int u = 0; u < NQ; ++u) {
-        const int i = i0 + u;
-        if (i < it.n_it) {
-          if (i + L < it.n_it) {
-            const int ps = ring.slot == 0 ? NS - 1 : ring.slot - 1;
-            adj_issue<P, BF16>(m, a, g, it, i + L, wb + ps * a.stage_floats, &bars[ps],
-                               band_slot, band_box, lane);
-          }
-          const float *st = wb + ring.slot * a.stage_floats;
-          if (!mbar_wait(&bars[ring.slot], ring.phase)) {
-            if (lane == 0) atomicOr(a.flags + kFlagTimeout, 1);
-            Ring dr = ring;
-            for (int j = i; j < it.n_it && j <= i + L; ++j) {
-              mbar_wait(&bars[dr.slot], dr.phase);
-              dr.next(NS);
-            }
-            return;
-          }
-          const Rows<P> R(it.r0, i, it.ya, it.yb, ny);
-          const F4 lam = lds4(st + kA_LAM + 4 * lane);
-          const F4 cbv = lds4(st + kA_CB + 4 * lane);
-          F4 gv;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) gv.v[q] = cbv.v[q] * lam.v[q];
-
-          // ---- gradients (lam = lambda_E^{t+1}) and px: own rows
-          if (R.own_r) {
-            const int64_t roff = (int64_t)R.r * nx;
-            if (own) {
-              const F4 se = snap_lds<BF16>(st + kA_SE, wo);
-              const F4 sc = snap_lds<BF16>(st + kA_SC, wo);
-              F4 gca = lds4(st + kA_GCA + 4 * wo), gcb = lds4(st + kA_GCB + 4 * wo);
-              const bool rowmask = !g.grad_mask || (R.r >= g.n_pml && R.r < ny - g.n_pml);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                if (rowmask && colmask[q]) {
-                  gca.v[q] = fmaf(se.v[q], lam.v[q], gca.v[q]);
-                  gcb.v[q] = fmaf(sc.v[q], lam.v[q], gcb.v[q]);
-                }
-              }
-              st4(a.gca + sbp + roff, gca);
-              st4(a.gcb + sbp + roff, gcb);
-            }
-            F4 px = gv;
-            if (pb >= 0) {
-              F4 M = lds4(st + kA_BAND + pb);
-              const F4 ax = ld4(a.bt + T.x(0) + pb), bx = ld4(a.bt + T.x(1) + pb);
-              const F4 rk = ld4(a.bt + T.x(2) + pb);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                M.v[q] += gv.v[q];
-                px.v[q] = fmaf(ax.v[q], M.v[q], gv.v[q] * rk.v[q]);
-                M.v[q] *= bx.v[q];
-              }
-              if (own) st4(a.out.mxe_node + xw + (int64_t)R.r * 2 * g.Wx + pb, M);
-            }
-            st4(prow + 4 * lane, pc_ok ? px : zero4());
-          }
-          // ---- pz (queue) at E nodes, every row of the walk (owned lanes)
-          {
-            F4 pz;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) pz.v[q] = -gv.v[q];
-            const int zr = zband_row(R.r, ny, g.Wz);
-            if (zr >= 0) {
-              F4 M = lds4(st + kA_MZE + 4 * wo);
-              const float ay = __ldg(a.bt + T.z(0) + zr), by = __ldg(a.bt + T.z(1) + zr);
-              const float rky = __ldg(a.bt + T.z(2) + zr);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                M.v[q] -= gv.v[q];
-                pz.v[q] = fmaf(ay, M.v[q], -gv.v[q] * rky);
-                M.v[q] *= by;
-              }
-              if (own && R.own_r) st4(a.out.mze_node + zbw + (int64_t)zr * nx, M);
-            }
-            pq[u] = pz;
-          }
-          __syncwarp();
-
-          // ---- lamHz, qx at row r (lanes 0..29)
-          if (R.own_r) {
-            const int64_t roff = (int64_t)R.r * nx;
-            float w[12];
-            win12(prow + 4 * wq, w);
-            const F4 lhz_old = lds4(st + kA_LHZ + 4 * wq);
-            const F4 cq = cq_arr ? (qc_ok ? ld4(a.cq + mbq + roff) : zero4()) : splat4(cqs);
-            F4 lhz, v;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              lhz.v[q] = lhz_old.v[q] - d_half<P>(w, q, a.c.cx);
-              v.v[q] = cq.v[q] * lhz.v[q];
-            }
-            if (q_own) st4(a.out.hz + sbq + roff, lhz);
-            if (qb >= 0) {
-              F4 M = lds4(st + kA_BAND + band_slot + qb);
-              const F4 ah = ld4(a.bt + T.x(3) + qb), bh = ld4(a.bt + T.x(4) + qb);
-              const F4 rk = ld4(a.bt + T.x(5) + qb);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                M.v[q] += v.v[q];
-                const float vq = v.v[q];
-                v.v[q] = fmaf(ah.v[q], M.v[q], vq * rk.v[q]);
-                M.v[q] *= bh.v[q];
-              }
-              if (q_own) st4(a.out.mxh_node + xw + (int64_t)R.r * 2 * g.Wx + qb, M);
-            }
-            if (q_lane) st4(hs + u * kARing + 4 * lane, qc_ok ? v : zero4());
-          }
-
-          // ---- lamHx, qz at row rh (owned lanes)
-          if (R.hx_need) {
-            F4 qz = zero4();
-            if (R.hx_in) {
-              const bool own_h = own && R.rh >= it.ya && R.rh < it.yb;
-              const F4 lhx = lds4(st + kA_LHX + 4 * wo);
-              const F4 cq = cq_arr ? (own ? ld4(a.cq + mbp + (int64_t)R.rh * nx) : zero4()) : splat4(cqs);
-              F4 lh;
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                float d = 0.f;
-#pragma unroll
-                for (int k = 1; k <= P; ++k)
-                  d = fmaf(a.c.cy[k - 1],
-                           pq[(u - P + k + NQ) % NQ].v[q] - pq[(u - P - k + 1 + 2 * NQ) % NQ].v[q],
-                           d);
-                lh.v[q] = lhx.v[q] - d;
-                qz.v[q] = -cq.v[q] * lh.v[q];
-              }
-              if (own_h) st4(a.out.hx + sbp + (int64_t)R.rh * nx, lh);
-              const int zr = zband_row(R.rh, ny, g.Wz);
-              if (zr >= 0) {
-                F4 M = lds4(st + kA_MZH + 4 * wo);
-                const float ayh = __ldg(a.bt + T.z(3) + zr), byh = __ldg(a.bt + T.z(4) + zr);
-                const float rkyh = __ldg(a.bt + T.z(5) + zr);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const float v = qz.v[q];
-                  M.v[q] += v;
-                  qz.v[q] = fmaf(ayh, M.v[q], v * rkyh);
-                  M.v[q] *= byh;
-                }
-                if (own_h) st4(a.out.mzh_node + zbw + (int64_t)zr * nx, M);
-              }
-            }
-            qq[u] = qz;
-          }
-
-          // ---- lamE at row y (owned lanes)
-          if (R.e_row && own) {
-            float w[12];
-            win12(hs + ((u + 1) % NQ) * kARing + 4 * wo, w);
-            const F4 ca4 = lds4(st + kA_CA + 4 * wo);
-            const F4 lam_y = lds4(st + kA_LAMY + 4 * wo);
-            F4 en;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float dz = 0.f;
-#pragma unroll
-              for (int k = 1; k <= P; ++k)
-                dz = fmaf(a.c.cy[k - 1], qq[(u + P + k) % NQ].v[q] - qq[(u + 1 + P - k) % NQ].v[q],
-                          dz);
-              en.v[q] = ca4.v[q] * lam_y.v[q] - d_int<P>(w, q, a.c.cx) - dz;
-            }
-            st4(a.out.ey + sbp + (int64_t)R.y * nx, en);
-          }
-          __syncwarp();
-          ring.next(NS);
-        }
-      }
-    }
+    const bool ok = it.edge ? adj_walk<P, BF16, L, true>(m, a, it, w, cq_arr, cqs)
+                            : adj_walk<P, BF16, L, false>(m, a, it, w, cq_arr, cqs);
+    if (!ok) return;
   }
 }
 
@@ -810,17 +937,60 @@ __global__ void __launch_bounds__(128) k_adjoint(const __grid_constant__ AdjMaps
 constexpr int kFwdL = 1;  // forward lookahead (rows in flight)
 constexpr int kAdjL = 1;  // adjoint lookahead
 
+// Forward stage: the fixed slots, then a Cq array's rows r and r - P, then
+// the z-band memory rows and the two x-band memory rows, each only if used.
 template <int P>
-void layout_t(bool adjoint, int Wx, int *stage_floats, int *band_floats, int *warp_floats,
-              size_t *smem) {
+void fwd_layout_t(int Wx, bool cq_arr, StepArgs *a, size_t *smem) {
   const int bw = Wx > 0 ? ((2 * Wx + 31) / 32) * 32 : 0;
-  const int sf = (adjoint ? kA_BAND : kF_BAND) + 2 * bw;
-  int wf = adjoint ? (kAdjL + 1) * sf + kAPx + 2 * P * kARing : (kFwdL + 1) * sf + 2 * P * kFRing;
+  int o = kF_FIXED;
+  for (int k = 0; k < kFoCount; ++k) a->fo[k] = 0;
+  if (cq_arr) {
+    a->fo[kFoCqH] = o;
+    a->fo[kFoCqX] = o + 128;
+    o += 256;
+  }
+  if (Wx > 0) {
+    a->fo[kFoMzh] = o;
+    a->fo[kFoMze] = o + 128;
+    a->fo[kFoMxh] = o + 256;
+    a->fo[kFoMxe] = o + 256 + bw;
+    o += 256 + 2 * bw;
+  }
+  int wf = (kFwdL + 1) * o + 2 * P * kFRing;
   wf = ((wf + 31) / 32) * 32;
-  *stage_floats = sf;
-  *band_floats = bw;
-  *warp_floats = wf;
+  a->stage_floats = o;
+  a->band_floats = bw;
+  a->warp_floats = wf;
+  a->band_box_floats = 2 * Wx;
   *smem = (size_t)(32 + kWarpsPerCta * wf) * sizeof(float) + 128;
+}
+
+// Adjoint stage: the fixed slots, then a Cq array's rows r and r - P, then
+// the x-band memory pair row and the two z-band memory rows, each only if
+// used.  The warp area adds the px row and the qx ring.
+template <int P>
+void adj_layout_t(int Wx, bool cq_arr, StepArgs *a, size_t *smem) {
+  int o = kA_FIXED;
+  for (int k = 0; k < kAoCount; ++k) a->ao[k] = 0;
+  if (cq_arr) {
+    a->ao[kAoCqR] = o;
+    a->ao[kAoCqH] = o + 128;
+    o += 256;
+  }
+  if (Wx > 0) {
+    a->ao[kAoMx] = o;
+    o += ((4 * Wx + 31) / 32) * 32;
+    a->ao[kAoMze] = o;
+    a->ao[kAoMzh] = o + 128;
+    o += 256;
+  }
+  int wf = (kAdjL + 1) * o + kAPx + 2 * P * kARing;
+  wf = ((wf + 31) / 32) * 32;
+  a->stage_floats = o;
+  a->band_floats = 0;
+  a->warp_floats = wf;
+  a->band_box_floats = 2 * Wx;
+  *smem = (size_t)(32 + kAdjWarpsPerCta * wf) * sizeof(float) + 128;
 }
 
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per
@@ -849,9 +1019,7 @@ std::atomic<uint64_t> &adj_smem_flag() {
 template <int P, int STORE>
 cudaError_t fwd_t(const FwdMaps &m, const StepArgs &a, bool batched, bool cq_arr, int grid,
                   cudaStream_t st) {
-  int sf, bw, wf;
-  size_t smem;
-  layout_t<P>(false, a.g.Wx, &sf, &bw, &wf, &smem);
+  const size_t smem = (size_t)(32 + kWarpsPerCta * a.warp_floats) * sizeof(float) + 128;
   allow_big_smem(k_forward<P, STORE, kFwdL>, fwd_smem_flag<P, STORE>());
   k_forward<P, STORE, kFwdL><<<grid, 128, smem, st>>>(m, a, batched ? 1 : 0, cq_arr ? 1 : 0);
   count_launches(1);
@@ -860,11 +1028,10 @@ cudaError_t fwd_t(const FwdMaps &m, const StepArgs &a, bool batched, bool cq_arr
 template <int P, bool BF16>
 cudaError_t adj_t(const AdjMaps &m, const StepArgs &a, bool batched, bool cq_arr, int grid,
                   cudaStream_t st) {
-  int sf, bw, wf;
-  size_t smem;
-  layout_t<P>(true, a.g.Wx, &sf, &bw, &wf, &smem);
+  const size_t smem = (size_t)(32 + kAdjWarpsPerCta * a.warp_floats) * sizeof(float) + 128;
   allow_big_smem(k_adjoint<P, BF16, kAdjL>, adj_smem_flag<P, BF16>());
-  k_adjoint<P, BF16, kAdjL><<<grid, 128, smem, st>>>(m, a, batched ? 1 : 0, cq_arr ? 1 : 0);
+  k_adjoint<P, BF16, kAdjL><<<grid, 32 * kAdjWarpsPerCta, smem, st>>>(m, a, batched ? 1 : 0,
+                                                                       cq_arr ? 1 : 0);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -881,21 +1048,27 @@ cudaError_t fwd_store(const FwdMaps &m, const StepArgs &a, int store, bool batch
 }
 
 template <typename K>
-int occupancy(K kern, size_t smem, std::atomic<uint64_t> &flag) {
+int occupancy(K kern, int threads, size_t smem, std::atomic<uint64_t> &flag) {
   allow_big_smem(kern, flag);
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 128, smem) != cudaSuccess) return 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess)
+    return 1;
   return n > 0 ? n : 1;
 }
 
 template <int P>
-int slots_t(bool adjoint, int Wx) {
-  int sf, bw, wf;
+int slots_t(bool adjoint, int Wx, bool cq_arr) {
   size_t smem;
-  layout_t<P>(adjoint, Wx, &sf, &bw, &wf, &smem);
-  return (adjoint ? occupancy(k_adjoint<P, false, kAdjL>, smem, adj_smem_flag<P, false>())
-                  : occupancy(k_forward<P, kStoreF32, kFwdL>, smem,
-                              fwd_smem_flag<P, kStoreF32>())) *
+  StepArgs a{};
+  if (adjoint) {
+    adj_layout_t<P>(Wx, cq_arr, &a, &smem);
+    return occupancy(k_adjoint<P, false, kAdjL>, 32 * kAdjWarpsPerCta, smem,
+                     adj_smem_flag<P, false>()) *
+           kAdjWarpsPerCta;
+  }
+  fwd_layout_t<P>(Wx, cq_arr, &a, &smem);
+  return occupancy(k_forward<P, kStoreF32, kFwdL>, 32 * kWarpsPerCta, smem,
+                   fwd_smem_flag<P, kStoreF32>()) *
          kWarpsPerCta;
 }
 
@@ -928,21 +1101,31 @@ cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int s
   return cudaErrorInvalidValue;
 }
 
-void stencil_layout(int order, bool adjoint, int Wx, int *sf, int *bw, int *wf, size_t *smem) {
+int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array) {
   switch (order) {
-    case 2: layout_t<1>(adjoint, Wx, sf, bw, wf, smem); return;
-    case 4: layout_t<2>(adjoint, Wx, sf, bw, wf, smem); return;
-    case 6: layout_t<3>(adjoint, Wx, sf, bw, wf, smem); return;
-    default: layout_t<4>(adjoint, Wx, sf, bw, wf, smem); return;
+    case 2: return slots_t<1>(adjoint, Wx, cq_array);
+    case 4: return slots_t<2>(adjoint, Wx, cq_array);
+    case 6: return slots_t<3>(adjoint, Wx, cq_array);
+    default: return slots_t<4>(adjoint, Wx, cq_array);
   }
 }
 
-int stencil_slots_per_sm(int order, bool adjoint, int Wx) {
+void adjoint_layout(int order, int Wx, bool cq_array, bool bf16, StepArgs *a, size_t *smem) {
+  (void)bf16;  // the snapshot slot is sized for float32 either way
   switch (order) {
-    case 2: return slots_t<1>(adjoint, Wx);
-    case 4: return slots_t<2>(adjoint, Wx);
-    case 6: return slots_t<3>(adjoint, Wx);
-    default: return slots_t<4>(adjoint, Wx);
+    case 2: adj_layout_t<1>(Wx, cq_array, a, smem); return;
+    case 4: adj_layout_t<2>(Wx, cq_array, a, smem); return;
+    case 6: adj_layout_t<3>(Wx, cq_array, a, smem); return;
+    default: adj_layout_t<4>(Wx, cq_array, a, smem); return;
+  }
+}
+
+void forward_layout(int order, int Wx, bool cq_array, StepArgs *a, size_t *smem) {
+  switch (order) {
+    case 2: fwd_layout_t<1>(Wx, cq_array, a, smem); return;
+    case 4: fwd_layout_t<2>(Wx, cq_array, a, smem); return;
+    case 6: fwd_layout_t<3>(Wx, cq_array, a, smem); return;
+    default: fwd_layout_t<4>(Wx, cq_array, a, smem); return;
   }
 }
 

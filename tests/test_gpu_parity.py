@@ -68,6 +68,84 @@ def test_small_forward_adjoint_parity(order, ny, nx, S, n_pml, batched, cq_array
     assert prob.status() == mwtm.MW_OK
 
 
+@pytest.mark.parametrize("placement", ["ca_then_cb", "cb_then_ca", "same_array"])
+def test_model_array_placement(placement):
+    """Ca and Cb reach the forward stencil as one two-row box when their
+    distance in memory allows it (in either order) and as two boxes otherwise
+    (here: both arguments are the same array).  Records and states must match
+    the oracle in every placement."""
+    ny, nx, S, n_pml, nt = 64, 264, 2, 6, 50
+    sim, dt, _ = small_sim(515, ny, nx, S, 2, 5, 4, n_pml, round_f32=True, sigma_max=0.02)
+    if placement == "same_array":
+        # Ca = Cb = 1 with Cq scaled by max(Cb): a lossless medium inside the
+        # stability bound (the scheme couples Cb and Cq only through their product)
+        one = np.ones_like(sim.ca)
+        sim = oracle.Sim(ny=ny, nx=nx, order=4, dy=sim.dy, dx=sim.dx, ca=one, cb=one,
+                         cq=float(np.float32(sim.cq[0] * sim.cb.max())), prof_y=sim.prof_y,
+                         prof_x=sim.prof_x, src_idx=sim.src_idx, rec_idx=sim.rec_idx)
+    g = synth.rng(51)
+    f = f32(g.normal(size=(nt, S, 2)))
+    fw = sim.forward(f, snapshots=False)
+    prob = problem_from_sim(sim, nt, dt, n_pml, snapshot="none")
+    ca = torch.as_tensor(sim.ca, dtype=torch.float32, device="cuda")
+    cb = torch.as_tensor(sim.cb, dtype=torch.float32, device="cuda")
+    if placement == "same_array":
+        prob.ca = prob.cb = ca
+    else:
+        buf = torch.empty((2, ny, nx), dtype=torch.float32, device="cuda")
+        first, second = (0, 1) if placement == "ca_then_cb" else (1, 0)
+        buf[first] = ca
+        buf[second] = cb
+        prob.ca, prob.cb = buf[first], buf[second]
+    state = prob.new_state()
+    rec = run_forward(prob, f, state=state)
+    assert rel_l2(rec, fw["rec"]) <= REC_TOL
+    st = api.unpack_state(prob.p, state)
+    for i, nm in enumerate(oracle.FIELDS):
+        assert rel_l2(st[nm], fw["state"][i]) <= REC_TOL, nm
+    assert prob.status() == mwtm.MW_OK
+
+
+@pytest.mark.parametrize("placement", ["first_then_second", "second_then_first", "same_model"])
+def test_adjoint_array_placement(placement):
+    """The adjoint fetches Ca / Cb and the per-shot gradients gCa / gCb as
+    pair boxes when their distance allows it (either order) and as single
+    boxes otherwise (Ca and Cb given as one array).  Gradients must match the
+    oracle in every placement."""
+    ny, nx, S, n_pml, nt = 60, 240, 2, 5, 40
+    sim, dt, _ = small_sim(616, ny, nx, S, 2, 5, 4, n_pml, round_f32=True, sigma_max=0.02)
+    if placement == "same_model":
+        one = np.ones_like(sim.ca)
+        sim = oracle.Sim(ny=ny, nx=nx, order=4, dy=sim.dy, dx=sim.dx, ca=one, cb=one,
+                         cq=float(np.float32(sim.cq[0] * sim.cb.max())), prof_y=sim.prof_y,
+                         prof_x=sim.prof_x, src_idx=sim.src_idx, rec_idx=sim.rec_idx)
+    g = synth.rng(61)
+    f = f32(g.normal(size=(nt, S, 2)))
+    res = f32(g.normal(size=(nt, S, 5)))
+    fw, adj = _oracle_pair(sim, f, res)
+    prob = problem_from_sim(sim, nt, dt, n_pml)
+    ca = torch.as_tensor(sim.ca, dtype=torch.float32, device="cuda")
+    cb = torch.as_tensor(sim.cb, dtype=torch.float32, device="cuda")
+    gbuf = torch.zeros((2, S, ny, nx), dtype=torch.float32, device="cuda")
+    if placement == "same_model":
+        prob.ca = prob.cb = ca
+        gca, gcb = gbuf[0], gbuf[1]
+    else:
+        mbuf = torch.empty((2, ny, nx), dtype=torch.float32, device="cuda")
+        k = (0, 1) if placement == "first_then_second" else (1, 0)
+        mbuf[k[0]] = ca
+        mbuf[k[1]] = cb
+        prob.ca, prob.cb = mbuf[k[0]], mbuf[k[1]]
+        gca, gcb = gbuf[k[0]], gbuf[k[1]]
+    rec = run_forward(prob, f)
+    assert rel_l2(rec, fw["rec"]) <= REC_TOL
+    prob.adjoint(torch.as_tensor(np.asarray(res, dtype=np.float32)).cuda(), gca=gca, gcb=gcb)
+    torch.cuda.synchronize()
+    assert rel_l2(gca.cpu().numpy().astype(np.float64), adj["gca"]) <= GRAD_TOL
+    assert rel_l2(gcb.cpu().numpy().astype(np.float64), adj["gcb"]) <= GRAD_TOL
+    assert prob.status() == mwtm.MW_OK
+
+
 @pytest.mark.parametrize("nt", [0, 1, 2, 3, 64, 65])
 def test_step_counts_and_checkpoint_partial_segments(nt):
     sim, dt, _ = small_sim(300 + nt, 40, 48, 2, 1, 3, 4, 5, round_f32=True)
