@@ -205,6 +205,52 @@ struct Launch {
   int grid;
 };
 
+// Interior rectangle of the item grid (the same edge rule as the kernels'
+// make_item): strip x0 with its 8-column halo clear of the x bands and the
+// array's sides; chunk [ya, yb) whose walk rows ya - 2P + 1 .. yb + 2P - 2
+// stay clear of the z bands.  Checked to give a bijection of the items.
+void interior_rect(Geom &g, int P) {
+  auto strip_edge = [&](int k) {
+    const int x0 = k * g.strip_cols;
+    return x0 - 8 < g.Wx || x0 + g.strip_cols + 8 > g.nx - g.Wx;
+  };
+  auto chunk_edge = [&](int k) {
+    const int ya = k * g.chunk_h;
+    const int yb = ya + g.chunk_h < g.ny ? ya + g.chunk_h : g.ny;
+    return g.Wz > 0 && (ya - (2 * P - 1) < g.Wz || yb + 2 * P - 1 > g.ny - g.Wz);
+  };
+  int a = 0, b = g.n_strips;
+  while (a < b && strip_edge(a)) ++a;
+  while (b > a && strip_edge(b - 1)) --b;
+  int c = 0, d = g.n_chunks;
+  while (c < d && chunk_edge(c)) ++c;
+  while (d > c && chunk_edge(d - 1)) --d;
+  for (int k = a; k < b; ++k)
+    if (strip_edge(k)) a = b;  // not a single run: no interior rectangle
+  for (int k = c; k < d; ++k)
+    if (chunk_edge(k)) c = d;
+  g.is_lo = a;
+  g.is_hi = b;
+  g.ic_lo = c;
+  g.ic_hi = d;
+  // the claim order must visit every (shot, strip, chunk) once
+  const int64_t n = (int64_t)g.S * g.n_strips * g.n_chunks;
+  std::vector<unsigned char> seen((size_t)n, 0);
+  bool ok = true;
+  for (int64_t i = 0; i < n && ok; ++i) {
+    int s, st, ch;
+    item_coords(g, (int)i, &s, &st, &ch);
+    if (s < 0 || s >= g.S || st < 0 || st >= g.n_strips || ch < 0 || ch >= g.n_chunks) {
+      ok = false;
+      break;
+    }
+    unsigned char &f = seen[((size_t)ch * g.n_strips + st) * g.S + s];
+    if (f) ok = false;
+    f = 1;
+  }
+  if (!ok) g.is_lo = g.is_hi = g.ic_lo = g.ic_hi = 0;
+}
+
 // Choose the row-chunk height so that the warps' work items fill whole waves
 // of resident warps: cost ~ waves x (rows per item + warm-up rows).
 Launch plan(const mw_params *p, bool adjoint) {
@@ -243,6 +289,7 @@ Launch plan(const mw_params *p, bool adjoint) {
   }
   g.chunk_h = best_ch;
   g.n_chunks = (p->ny + g.chunk_h - 1) / g.chunk_h;
+  interior_rect(g, P);
   const int64_t items = cols_items * g.n_chunks;
   const int wpc = adjoint ? kAdjWarpsPerCta : kWarpsPerCta;
   int64_t grid = (items + wpc - 1) / wpc;

@@ -30,6 +30,9 @@ struct Geom {
   int ny, nx, S;
   int Wx, Wz;         // band widths (0: no CPML band)
   int strip_cols, n_strips, n_chunks, chunk_h;
+  // strips [is_lo, is_hi) and chunks [ic_lo, ic_hi) form the interior
+  // rectangle (items whose walk touches no band and no array edge)
+  int is_lo, is_hi, ic_lo, ic_hi;
   int n_pml;
   int grad_mask;      // adjoint: accumulate gradients outside the band only
   int64_t numel;      // ny * nx
@@ -126,6 +129,38 @@ enum AdjMap {
 struct AdjMaps {
   CUtensorMap map[kAdjMaps];
 };
+
+// Claim order of the work items: items touching a band or an array edge
+// first, then the interior rectangle; the shot index runs fastest, then the
+// strip, then the chunk.  A bijection of [0, S * n_strips * n_chunks).
+__host__ __device__ inline void item_coords(const Geom &g, int item, int *s, int *strip,
+                                            int *chunk) {
+  const int ns = g.n_strips, nc = g.n_chunks;
+  const int n_is = g.is_hi > g.is_lo ? g.is_hi - g.is_lo : 0;
+  const int n_ic = g.ic_hi > g.ic_lo ? g.ic_hi - g.ic_lo : 0;
+  const int n_int = g.S * n_is * n_ic;
+  const int n_band = g.S * ns * nc - n_int;
+  *s = item % g.S;
+  if (item < n_band) {
+    const int jj = item / g.S;
+    const int n_ec = nc - n_ic;  // chunks touching a z edge: all their strips
+    if (jj < n_ec * ns) {
+      const int ci = jj / ns;
+      *strip = jj % ns;
+      *chunk = ci < g.ic_lo ? ci : g.ic_hi + (ci - g.ic_lo);
+    } else {  // interior chunks: only the edge strips
+      const int k = jj - n_ec * ns;
+      const int n_es = ns - n_is;
+      const int e = k % n_es;
+      *chunk = g.ic_lo + k / n_es;
+      *strip = e < g.is_lo ? e : g.is_hi + (e - g.is_lo);
+    }
+  } else {
+    const int jj = (item - n_band) / g.S;
+    *strip = g.is_lo + jj % n_is;
+    *chunk = g.ic_lo + jj / n_is;
+  }
+}
 
 // Workspace layout (byte offsets, 256-aligned).
 struct Layout {

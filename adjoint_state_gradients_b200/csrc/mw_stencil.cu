@@ -160,10 +160,8 @@ struct Item {
 
 template <int P>
 __device__ __forceinline__ bool make_item(const Geom &g, int item, bool batched, Item &it) {
-  it.s = item % g.S;
-  const int rest = item / g.S;
-  const int strip = rest % g.n_strips;
-  const int chunk = rest / g.n_strips;
+  int strip, chunk;
+  item_coords(g, item, &it.s, &strip, &chunk);
   it.sm = batched ? it.s : 0;
   it.x0 = strip * g.strip_cols;
   it.ya = chunk * g.chunk_h;
