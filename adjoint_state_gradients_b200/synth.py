@@ -143,8 +143,14 @@ class Inputs:
         return np.ascontiguousarray(np.broadcast_to(w[:, None, None], (nt, S, ns)))
 
 
-def make_inputs(number: int, n_shots: int | None = None) -> Inputs:
-    """Inputs of workload `number` (1..5).  n_shots < S keeps the first shots."""
+def make_inputs(number: int, n_shots: int | None = None, survey_shots: int | None = None,
+                first_shot: int = 0) -> Inputs:
+    """Inputs of workload `number` (1..5).  n_shots < S keeps the first shots.
+
+    Workload 4 only: `survey_shots` spreads that many sources evenly over the
+    interior (default: the workload's 8) and the inputs hold shots
+    first_shot .. first_shot + n_shots - 1 of that survey, so that ranks of a
+    multi-GPU run each simulate their own block of one larger survey."""
     wl = WORKLOADS[number]
     S = wl.n_shots if n_shots is None else n_shots
     n, p = wl.n, wl.n_pml
@@ -179,7 +185,10 @@ def make_inputs(number: int, n_shots: int | None = None) -> Inputs:
         eps = smooth_field(g, (n, n), 16.0, 3.0, 20.0)
         sig = np.zeros((n, n))
         eps_true = eps + gaussian_blob((n, n), 1.0, N / 10.0)
-        src_cols = [[128 + 256 * k] for k in range(8)]
+        n_survey = wl.n_shots if survey_shots is None else survey_shots
+        if first_shot < 0 or first_shot + S > n_survey:
+            raise ValueError("shot block outside the survey")
+        src_cols = [[int((k + 0.5) * N / n_survey)] for k in range(first_shot, first_shot + S)]
         rec_cols = 4 * np.arange(512) + 2
     elif number == 5:
         eps = np.empty((S, n, n))

@@ -212,7 +212,7 @@ def main():
     import torch
     import torch.distributed as dist
 
-    from adjoint_state_gradients_b200 import api, mwtm, synth
+    from adjoint_state_gradients_b200 import api, mwtm, shard, synth
 
     rank, world, local = dist_env()
     if world != args.gpus:
@@ -226,8 +226,11 @@ def main():
 
     wl = synth.WORKLOADS[WORKLOAD]
     nt = args.nt or wl.nt
-    inp = synth.make_inputs(WORKLOAD)
     S = wl.n_shots
+    # weak scaling: every rank simulates its own block of S shots of one
+    # survey of S * world shots (sources spread over the interior)
+    lo, hi = shard.shot_block(S * world, rank, world)
+    inp = synth.make_inputs(WORKLOAD, n_shots=hi - lo, survey_shots=S * world, first_shot=lo)
     c0 = 299792458.0
     vmax = c0 / math.sqrt(inp.eps_min)
     dt = wl.cfl_fraction * mwtm.cfl_dt(wl.order, wl.h, wl.h, vmax)
@@ -266,9 +269,7 @@ def main():
         prob.adjoint(res, gca=gca_s, gcb=gcb_s)
         prob.combine(gca_s, out=gca)
         prob.combine(gcb_s, out=gcb)
-        if world > 1:
-            dist.all_reduce(gca)
-            dist.all_reduce(gcb)
+        shard.sum_over_ranks_(gca, gcb)
 
     for _ in range(args.warmup):
         step()
@@ -304,10 +305,8 @@ def main():
     mwtm.profile_enable(False)
     total_ms = ev0.elapsed_time(ev1)
     fwd_ms = sum(a.elapsed_time(b) for a, b in evs)
-    t = torch.tensor([total_ms, fwd_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_ms = float(t[0]), float(t[1])
+    total_ms = shard.max_over_ranks(total_ms, dev)
+    fwd_ms = shard.max_over_ranks(fwd_ms, dev)
 
     cells = wl.ny * wl.nx * nt * S * world
     value = cells * args.steps / (total_ms / 1e3) / 1e9
@@ -344,9 +343,7 @@ def main():
             prob.adjoint(res, gca=gca_s, gcb=gcb_s)
             prob.combine(gca_s, out=gca)
             prob.combine(gcb_s, out=gcb)
-            if world > 1:
-                dist.all_reduce(gca)
-                dist.all_reduce(gcb)
+            shard.sum_over_ranks_(gca, gcb)
             for o, src in zip(outs, (J, gca, gcb)):
                 o.copy_(src, non_blocking=True)
 
@@ -360,12 +357,10 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_ms = shard.max_over_ranks(a.elapsed_time(b), dev)
         h2d = sum(x.numel() * x.element_size() for x in (f_p, eps_p, sig_p, dobs_p))
         d2h = sum(x.numel() * x.element_size() for x in outs)
-        e2e = {"value": round(cells * args.steps / (float(e_ms[0]) / 1e3) / 1e9, 4), "unit": UNIT,
+        e2e = {"value": round(cells * args.steps / (e_ms / 1e3) / 1e9, 4), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     cpu = None

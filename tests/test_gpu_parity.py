@@ -14,7 +14,7 @@ import torch
 
 import oracle
 from adjoint_state_gradients_b200 import api, mwtm, synth
-from tests._cases import rel_l2, small_sim, workload_sim
+from tests._cases import oracle_sim, rel_l2, small_sim, workload_sim
 from tests._gpu import f32, problem_from_sim, run_adjoint, run_forward
 
 pytestmark = pytest.mark.gpu
@@ -318,6 +318,87 @@ def test_workload5_batched_records():
     prob = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot="none")
     rec = run_forward(prob, f)
     assert rel_l2(rec, fw["rec"]) <= REC_TOL
+
+
+# ----------------------------------------------------------------------------
+# full shot batches in the launch configuration the benchmark times; shots
+# are independent, so the oracle checks sampled shots one by one
+
+
+def _subset_sim(inp, sel, dt, batched=False):
+    wl = inp.wl
+    vmax = oracle.c0() / np.sqrt(inp.eps_min)
+    eps = inp.eps_r[sel] if batched else inp.eps_r
+    sig = inp.sigma[sel] if batched else inp.sigma
+    return oracle_sim(eps, sig, inp.src_idx[sel], inp.rec_idx[sel], wl.order, wl.h, dt, wl.n_pml,
+                      wl.f0, vmax=vmax, round_f32=True)
+
+
+def test_workload4_all_shots_sampled():
+    """2128x2128 order 4, all 8 shots, checkpoints every 64 steps (the
+    benchmark's launch plan), nt 137 = two full segments + a partial one;
+    records and per-shot gradients of shots 0 and 7 against the oracle."""
+    nt, sel = 137, [0, 7]
+    sim, inp, dt, f = workload_sim(4, n_shots=8, nt=nt)
+    g = synth.rng(404)
+    res = f32(g.normal(size=(nt, 8, inp.wl.n_rec)))
+    prob = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot="ckpt", ckpt_every=64)
+    rec = run_forward(prob, f)
+    gca, gcb, gf = run_adjoint(prob, res)
+    assert prob.status() == mwtm.MW_OK
+    del prob
+    sub = _subset_sim(inp, sel, dt)
+    ck = sub.fwd_adj_ckpt(f[:, sel], res[:, sel], 64)
+    assert rel_l2(rec[:, sel], ck["rec"]) <= REC_TOL
+    assert rel_l2(gca[sel], ck["gca"]) <= GRAD_TOL
+    assert rel_l2(gcb[sel], ck["gcb"]) <= GRAD_TOL
+    assert rel_l2(gf[:, sel], ck["grad_f"]) <= GRAD_TOL
+
+
+def test_workload5_all_shots_sampled():
+    """552x552 order 8, all 256 shots with per-shot models, records only,
+    nt 300; shots 0, 131 and 255 against the oracle."""
+    nt, sel = 300, [0, 131, 255]
+    inp = synth.make_inputs(5)
+    wl = inp.wl
+    vmax = oracle.c0() / np.sqrt(inp.eps_min)
+    dt = wl.cfl_fraction * oracle.cfl_dt(wl.order, wl.h, wl.h, vmax)
+    f = f32(inp.wavelet(dt, nt))
+    sim = oracle_sim(inp.eps_r, inp.sigma, inp.src_idx, inp.rec_idx, wl.order, wl.h, dt, wl.n_pml,
+                     wl.f0, vmax=vmax, round_f32=True)
+    prob = problem_from_sim(sim, nt, dt, wl.n_pml, snapshot="none")
+    rec = run_forward(prob, f)
+    assert prob.status() == mwtm.MW_OK
+    del prob
+    sub = _subset_sim(inp, sel, dt, batched=True)
+    fw = sub.forward(f[:, sel])
+    assert rel_l2(rec[:, sel], fw["rec"]) <= REC_TOL
+
+
+def test_workload3_all_shots_sampled_bf16():
+    """1064x1064 order 8, all 16 shots, nt 150: fp32-storage gradients of
+    shots 0 and 15 against the oracle, and the bf16-storage gradient error
+    against fp32 storage on every shot (reported, <= 2e-2)."""
+    nt, sel = 150, [0, 15]
+    sim, inp, dt, f = workload_sim(3, n_shots=16, nt=nt)
+    g = synth.rng(303)
+    res = f32(g.normal(size=(nt, 16, inp.wl.n_rec)))
+    p32 = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot="fp32")
+    rec = run_forward(p32, f)
+    gca32, gcb32, _ = run_adjoint(p32, res)
+    del p32
+    p16 = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot="bf16")
+    run_forward(p16, f)
+    gca16, gcb16, _ = run_adjoint(p16, res)
+    del p16
+    sub = _subset_sim(inp, sel, dt)
+    ck = sub.fwd_adj_ckpt(f[:, sel], res[:, sel], 32)
+    assert rel_l2(rec[:, sel], ck["rec"]) <= REC_TOL
+    assert rel_l2(gca32[sel], ck["gca"]) <= GRAD_TOL
+    assert rel_l2(gcb32[sel], ck["gcb"]) <= GRAD_TOL
+    e_ca, e_cb = rel_l2(gca16, gca32), rel_l2(gcb16, gcb32)
+    print(f"bf16-snapshot gradient error vs fp32 storage (16 shots): Ca {e_ca:.3e} Cb {e_cb:.3e}")
+    assert e_ca <= 2e-2 and e_cb <= 2e-2
 
 
 # ----------------------------------------------------------------------------
