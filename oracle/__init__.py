@@ -84,6 +84,10 @@ def lib():
         L.orc_residual.argtypes = [ctypes.c_int64, _D, _D, _D]
         L.orc_residual.restype = ctypes.c_double
         L.orc_num_threads.restype = ctypes.c_int
+        _U8 = ctypes.POINTER(ctypes.c_uint8)
+        L.orc_quant_bf16.argtypes = [ctypes.c_int64, _D, _D]
+        L.orc_fp8_encode.argtypes = [ctypes.c_int64, _D, _U8]
+        L.orc_fp8_decode.argtypes = [ctypes.c_int64, _U8, _D]
         _lib = L
     return _lib
 
@@ -152,6 +156,38 @@ def combine(g_shot):
     g = np.empty(g_shot.shape[1:])
     lib().orc_combine(S, g.size, _p(g_shot.reshape(S, -1)), _p(g.reshape(-1)))
     return g
+
+
+def quant_bf16(x):
+    """Snapshot storage in bfloat16: x rounded to fp32, then to bf16
+    (nearest, ties to even); returned as fp64 values."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    lib().orc_quant_bf16(x.size, _p(x.reshape(-1)), _p(out.reshape(-1)))
+    return out
+
+
+def fp8_encode(x):
+    """E4M3 codes (uint8) of x rounded to fp32: nearest, ties to even,
+    saturating to +-448."""
+    x = _f64(x)
+    codes = np.empty(x.shape, dtype=np.uint8)
+    lib().orc_fp8_encode(x.size, _p(x.reshape(-1)),
+                         codes.reshape(-1).ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return codes
+
+
+def fp8_decode(codes):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape, dtype=np.float64)
+    lib().orc_fp8_decode(codes.size, codes.reshape(-1).ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                         _p(out.reshape(-1)))
+    return out
+
+
+def quant_fp8(x):
+    """Snapshot storage in FP8 E4M3: decode(encode(x))."""
+    return fp8_decode(fp8_encode(x))
 
 
 def residual(d, d_obs):

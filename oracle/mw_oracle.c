@@ -26,7 +26,10 @@
  *     included (the page's adjoint kernels apply the forward-form recursion
  *     at the other node; the sibling PR "DeepWave-KAUST/sweep #125" documents
  *     that defect class);
- *   - CPML profile: quadratic d, kappa = 1, linear alpha, R = 1e-3.
+ *   - CPML profile: quadratic d, kappa = 1, linear alpha, R = 1e-3;
+ *   - snapshot storage in bfloat16 or FP8 E4M3 rounds the fp32 value to
+ *     nearest, ties to even, E4M3 saturating to +-448 (orc_quant_bf16,
+ *     orc_fp8_encode; pinned to the format definitions and to torch's casts).
  *
  * Layout: row-major [shot][y][x], y = depth (z), x = columns, cell index
  * j = y*nx + x.  Hx lives at (y+1/2, x), Hz at (y, x+1/2), Ey at (y, x).
@@ -516,6 +519,88 @@ double orc_residual(int64_t n, const double *d, const double *d_obs,
     J += 0.5 * r * r;
   }
   return J;
+}
+
+/* ---- snapshot storage formats ----------------------------------------------
+ * The page stores the snapshots E^n, curl^n rounded to a narrower format
+ * (forward_kernel_e_with_storage_bf16 / _fp8 and the matching backward
+ * kernels' loads; the helpers "FP8 E4M3 (1 sign, 4 exponent, 3 mantissa)"
+ * with saturation to the largest finite value).  The GPU computes in fp32,
+ * so the stored value is the fp32 value rounded to the format; the oracle
+ * rounds its fp64 value to fp32 first, then to the format.  Both encoders
+ * below are written from the format definitions:
+ *   bfloat16: the top 16 bits of an fp32, round to nearest, ties to even;
+ *   E4M3: sign, 4-bit exponent (bias 7), 3-bit mantissa; subnormals
+ *     m * 2^-9 (exponent field 0); normals (1 + m/8) 2^(e-7); the code
+ *     S.1111.111 is NaN, so the largest finite value is 448 (S.1111.110);
+ *     round to nearest, ties to even, saturating to +-448.
+ */
+static double fp32_round(double x) { return (double)(float)x; }
+
+/* bfloat16 rounding of n values (fp64 in, fp64 out holding bf16 values). */
+void orc_quant_bf16(int64_t n, const double *in, double *out) {
+  for (int64_t i = 0; i < n; ++i) {
+    float f = (float)in[i];
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) {
+      u |= 0x00400000u;  /* NaN stays NaN */
+    } else {
+      const uint32_t lsb = (u >> 16) & 1u;
+      u += 0x7fffu + lsb;
+    }
+    u &= 0xffff0000u;
+    memcpy(&f, &u, 4);
+    out[i] = (double)f;
+  }
+}
+
+/* E4M3 code of one finite value a >= 0 (already an fp32 value). */
+static unsigned fp8_code_abs(double a) {
+  if (a >= 448.0) return 0x7eu;
+  if (a == 0.0) return 0u;
+  int e2;
+  frexp(a, &e2);     /* a = m 2^e2, m in [0.5, 1): floor(log2 a) = e2 - 1 */
+  int E = e2 - 1;
+  if (E < -6) E = -6; /* subnormal range: quantum 2^-9 like the first binade */
+  const double quantum = ldexp(1.0, E - 3);
+  const double q = rint(a / quantum); /* exact quotient; ties to even */
+  /* codes are contiguous across binades: ((E + 7) << 3) + (q - 8), and for
+   * the subnormal binade (E = -6) code = q (0..8) */
+  long code = (long)((E + 7) * 8) + (long)q - 8;
+  if (E == -6) code = (long)q;
+  if (code > 0x7e) code = 0x7e;
+  return (unsigned)code;
+}
+
+/* E4M3 codes of n values (rounded to fp32 first). */
+void orc_fp8_encode(int64_t n, const double *in, uint8_t *codes) {
+  for (int64_t i = 0; i < n; ++i) {
+    const double x = fp32_round(in[i]);
+    if (x != x) {
+      codes[i] = 0x7f;
+      continue;
+    }
+    const unsigned sign = (x < 0.0 || (x == 0.0 && signbit(x))) ? 0x80u : 0u;
+    codes[i] = (uint8_t)(sign | fp8_code_abs(fabs(x)));
+  }
+}
+
+/* Values of n E4M3 codes. */
+void orc_fp8_decode(int64_t n, const uint8_t *codes, double *out) {
+  for (int64_t i = 0; i < n; ++i) {
+    const unsigned c = codes[i];
+    const unsigned e = (c >> 3) & 0xfu, m = c & 7u;
+    double v;
+    if (e == 15 && m == 7) {
+      v = NAN;
+    } else if (e == 0) {
+      v = ldexp((double)m, -9);
+    } else {
+      v = ldexp(1.0 + m / 8.0, (int)e - 7);
+    }
+    out[i] = (c & 0x80u) ? -v : v;
+  }
 }
 
 int orc_num_threads(void) {

@@ -14,6 +14,7 @@ from fractions import Fraction
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from adjoint_state_gradients_b200 import synth
@@ -586,3 +587,58 @@ def test_workload_configs_are_stable_and_shaped():
     inp = synth.make_inputs(4, n_shots=1)
     dt = 0.6 * oracle.cfl_dt(4, 0.02, 0.02, oracle.c0() / math.sqrt(inp.eps_min))
     assert dt == pytest.approx(4.20e-11, rel=0.01)
+
+
+# ----------------------------------------------------------------------------
+# snapshot storage formats (bfloat16, FP8 E4M3 with saturation)
+
+
+def test_fp8_e4m3_code_table_follows_the_format_definition():
+    """1 sign, 4 exponent (bias 7), 3 mantissa bits; exponent field 0 holds
+    subnormals m * 2^-9; S.1111.111 is NaN, so 448 is the largest value."""
+    codes = np.arange(256, dtype=np.uint8)
+    v = oracle.fp8_decode(codes)
+    assert v[0x00] == 0.0 and v[0x01] == 2.0 ** -9 and v[0x07] == 7 * 2.0 ** -9
+    assert v[0x08] == 2.0 ** -6 and v[0x38] == 1.0 and v[0x39] == 1.125
+    assert v[0x7E] == 448.0 and np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    assert np.all(v[0x80:0xFF] == -v[0x00:0x7F])
+    pos = v[:0x7F]
+    assert np.all(np.diff(pos) > 0)
+    # encoding a representable value gives its code back
+    assert np.all(oracle.fp8_encode(pos) == codes[:0x7F])
+    assert np.all(oracle.fp8_encode(-pos[1:]) == codes[0x81:0xFF])
+
+
+def test_fp8_e4m3_rounds_to_nearest_even_and_saturates():
+    v = oracle.fp8_decode(np.arange(0x7F, dtype=np.uint8))
+    mid = (v[:-1] + v[1:]) / 2          # exact ties between neighbouring codes
+    got = oracle.fp8_encode(mid)
+    lo = np.arange(0x7E)
+    want = np.where(lo % 2 == 0, lo, lo + 1)  # the even code wins a tie
+    assert np.all(got == want)
+    # just off the tie goes to the nearer code
+    assert np.all(oracle.fp8_encode(mid * (1 - 1e-6)) == lo)
+    assert np.all(oracle.fp8_encode(mid * (1 + 1e-6)) == lo + 1)
+    # saturation to the largest finite value, both signs
+    assert list(oracle.fp8_encode(np.array([448.0, 464.0, 1e6, -1e30]))) == [0x7E, 0x7E, 0x7E, 0xFE]
+    # underflow: half the smallest subnormal is a tie to zero (even)
+    assert list(oracle.fp8_encode(np.array([2.0 ** -10, 1.5 * 2.0 ** -10, 1e-30]))) == [0, 1, 0]
+
+
+def test_bf16_rounds_to_nearest_even():
+    one = 1.0
+    x = np.array([one + 2.0 ** -8, one + 3 * 2.0 ** -8, one + 2.0 ** -8 + 2.0 ** -20, -(one + 2.0 ** -8)])
+    assert list(oracle.quant_bf16(x)) == [1.0, 1.0 + 2.0 ** -6, 1.0 + 2.0 ** -7, -1.0]
+    # the value is first rounded to fp32
+    assert oracle.quant_bf16(np.array([1.0 + 2.0 ** -30]))[0] == 1.0
+
+
+def test_storage_formats_match_torch_casts():
+    """Against an independent implementation: torch's float32 -> bfloat16 and
+    float32 -> float8_e4m3fn casts (both nearest-even) inside the range."""
+    g = np.random.default_rng(5)
+    x = g.normal(size=50000) * 10.0 ** g.uniform(-5, 2.6, size=50000)
+    x = x[np.abs(x) < 448].astype(np.float32).astype(np.float64)
+    t = torch.tensor(x, dtype=torch.float32)
+    assert np.array_equal(oracle.quant_fp8(x), t.to(torch.float8_e4m3fn).double().numpy())
+    assert np.array_equal(oracle.quant_bf16(x), t.to(torch.bfloat16).double().numpy())
