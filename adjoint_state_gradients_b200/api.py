@@ -27,7 +27,7 @@ class Problem:
     """One 2-D TM setup: grid, stencil order, time step, shots, storage mode.
 
     src_idx [S, n_src] / rec_idx [S, n_rec] are flat cell indices y*nx + x
-    (-1 = inactive).  snapshot: "none" | "fp32" | "bf16" | "ckpt".
+    (-1 = inactive).  snapshot: "none" | "fp32" | "bf16" | "fp8" | "ckpt".
     """
 
     def __init__(self, ny, nx, order, dy, dx, dt, nt, n_pml, src_idx, rec_idx, *, vmax,

@@ -98,12 +98,10 @@ int check_params(const mw_params *p, bool cfl) {
   const Bands b = bands(p);
   if (2 * b.Wx > p->nx || 2 * b.Wz > p->ny)
     return fail(MW_ERR_ARG, "CPML band %d does not fit a %d x %d grid", p->n_pml, p->ny, p->nx);
-  if (p->snap_mode < MW_SNAP_NONE || p->snap_mode > MW_SNAP_CKPT)
+  if (p->snap_mode < MW_SNAP_NONE || p->snap_mode > MW_SNAP_FP8)
     return fail(MW_ERR_ARG, "snap_mode = %d", p->snap_mode);
   if (p->snap_mode == MW_SNAP_CKPT && p->ckpt_every < 1)
     return fail(MW_ERR_ARG, "ckpt_every = %d", p->ckpt_every);
-  if (p->snap_mode == MW_SNAP_BF16 && p->nx % 8 != 0)
-    return fail(MW_ERR_ARG, "bf16 snapshots need nx %% 8 == 0 (nx = %d)", p->nx);
   if (2 * b.Wx > 256)
     return fail(MW_ERR_UNSUPPORTED, "n_pml = %d: a band row exceeds one TMA box (n_pml <= 123)",
                 p->n_pml);
@@ -116,6 +114,17 @@ int check_params(const mw_params *p, bool cfl) {
       return fail(MW_ERR_CFL, "dt = %.6g s exceeds the stability bound %.6g s", p->dt, dtmax);
   }
   return MW_OK;
+}
+
+// bytes per stored snapshot value of a full-storage mode
+size_t snap_elem_bytes(int snap_mode) {
+  return snap_mode == MW_SNAP_BF16 ? 2 : snap_mode == MW_SNAP_FP8 ? 1 : 4;
+}
+// store kind of the forward (full-storage modes) / load kind of the adjoint
+int snap_store_kind(int snap_mode) {
+  return snap_mode == MW_SNAP_FP32 ? kStoreF32
+         : snap_mode == MW_SNAP_BF16 ? kStoreBF16
+         : snap_mode == MW_SNAP_FP8 ? kStoreFP8 : kStoreNone;
 }
 
 Layout layout(const mw_params *p) {
@@ -137,13 +146,17 @@ Layout layout(const mw_params *p) {
   L.adA = L.adB = L.rpA = L.rpB = L.snap = L.seg = 0;
   L.n_seg = 0;
   L.snap_step_bytes = 0;
+  L.snap_pitch = p->nx;
   if (p->snap_mode != MW_SNAP_NONE) {
     L.adA = off; off += sb;
     L.adB = off; off += sb;
   }
-  if (p->snap_mode == MW_SNAP_FP32 || p->snap_mode == MW_SNAP_BF16) {
-    const size_t es = p->snap_mode == MW_SNAP_FP32 ? 4 : 2;
-    L.snap_step_bytes = SN * es;
+  if (p->snap_mode == MW_SNAP_FP32 || p->snap_mode == MW_SNAP_BF16 ||
+      p->snap_mode == MW_SNAP_FP8) {
+    const size_t es = snap_elem_bytes(p->snap_mode);
+    const size_t per_row = 16 / es;  // elements per 16 bytes
+    L.snap_pitch = (int)(((size_t)p->nx + per_row - 1) / per_row * per_row);
+    L.snap_step_bytes = (size_t)p->n_shots * p->ny * L.snap_pitch * es;
     L.snap = off;
     off += align256(2 * (size_t)p->nt * L.snap_step_bytes);
   } else if (p->snap_mode == MW_SNAP_CKPT) {
@@ -151,6 +164,7 @@ Layout layout(const mw_params *p) {
     L.rpA = off; off += sb;
     L.rpB = off; off += sb;
     L.snap = off; off += (size_t)L.n_seg * sb;
+    L.snap_pitch = p->nx;
     L.snap_step_bytes = SN * 4;
     L.seg = off;
     off += align256(2 * (size_t)p->ckpt_every * L.snap_step_bytes);
@@ -349,6 +363,12 @@ EncodeTiledFn encoder() {
   return fn;
 }
 
+// TMA element type of a 4-, 2- or 1-byte element (float32, bf16, E4M3 bytes)
+CUtensorMapDataType elem_type(int elem) {
+  return elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+         : elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+}
+
 // Row-box map over an array [d3][d2][d1][d0] (rank 3 or 4) of float32 (elem
 // 4) or bf16 (elem 2) with dense strides, or with the given outermost stride
 // (bytes, rank 4 only; 0 = dense): box = (box0, 1, 1[, box3]), zero fill
@@ -363,8 +383,8 @@ int encode_rows(CUtensorMap *map, const void *base, int elem, int rank, uint64_t
                            stride3 ? stride3 : d0 * d1 * d2 * elem};
   cuuint32_t box[4] = {box0, 1, 1, box3};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                  (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, estr,
+  CUresult r = fn(map, elem_type(elem), (cuuint32_t)rank, const_cast<void *>(base), dims, strides,
+                  box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
@@ -388,8 +408,7 @@ int encode_map(CUtensorMap *map, const void *base, int elem, int rank, const uin
     e[k] = 1;
     if (k + 1 < rank) st[k] = strides[k];
   }
-  CUresult r = fn(map, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                  (cuuint32_t)rank, const_cast<void *>(base), d, st, b, e,
+  CUresult r = fn(map, elem_type(elem), (cuuint32_t)rank, const_cast<void *>(base), d, st, b, e,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
@@ -452,7 +471,7 @@ int fwd_maps(const mw_params *p, const Fields &in, const float *ca, const float 
 
 int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb,
              const float *cq, const float *gca, const float *gcb, const void *se, const void *sc,
-             int snap_elem, int snap_steps, AdjMaps *m) {
+             int snap_elem, int snap_steps, int snap_pitch, AdjMaps *m) {
   memset(m, 0, sizeof *m);
   const Bands bd = bands(p);
   const uint64_t nx = p->nx, ny = p->ny, S = p->n_shots, Sm = p->model_batched ? p->n_shots : 1;
@@ -471,7 +490,8 @@ int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float 
     // (x, y, shot, step, field): the curl snapshots follow the E snapshots
     const uint64_t e = (uint64_t)snap_elem;
     const uint64_t dims[5] = {nx, ny, S, (uint64_t)snap_steps, 2};
-    const uint64_t strides[4] = {nx * e, nx * ny * e, nx * ny * S * e,
+    const uint64_t pitch = (uint64_t)snap_pitch;
+    const uint64_t strides[4] = {pitch * e, pitch * ny * e, pitch * ny * S * e,
                                  (uint64_t)((const char *)sc - (const char *)se)};
     const uint32_t box[5] = {112, 1, 1, 1, 2};
     if ((const char *)sc <= (const char *)se)
@@ -510,8 +530,7 @@ void set_layout(StepArgs &a, const mw_params *p, bool adjoint) {
   size_t smem;
   if (adjoint) {
     // needs a.ca / a.cb and a.gca / a.gcb (pair fetches)
-    adjoint_layout(p->order, bands(p).Wx, !p->cq_is_scalar, p->snap_mode == MW_SNAP_BF16, &a,
-                   &smem);
+    adjoint_layout(p->order, bands(p).Wx, !p->cq_is_scalar, false, &a, &smem);
     const MdPair md = md_pairing(p, a.ca, a.cb);
     a.md_pair = md.pair ? 1 : 0;
     a.md_swap = md.swap ? 1 : 0;
@@ -679,13 +698,13 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   a.flags = flags;
   a.bt = (const float *)(ws + L.bandtab);
   set_layout(a, p, false);
+  a.snap_pitch = L.snap_pitch;
   MW_TRY(stencil_prologue(p, cpml, ws, L, st));
   FwdMaps mA, mB;  // input buffer A / B
   MW_TRY(fwd_maps(p, fields_at(p, bufA), ca, cb, cq, &mA));
   MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, cq, &mB));
 
-  const int store = p->snap_mode == MW_SNAP_FP32 ? kStoreF32
-                    : p->snap_mode == MW_SNAP_BF16 ? kStoreBF16 : kStoreNone;
+  const int store = snap_store_kind(p->snap_mode);
   const int64_t SN = (int64_t)p->n_shots * p->ny * p->nx;
   const int64_t numel = (int64_t)p->ny * p->nx;
   const Chains ch = chains_at(p, ws, L);
@@ -785,13 +804,15 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
 
   // snapshot source of the adjoint: the full store, or the replay segment
   const bool ckpt = p->snap_mode == MW_SNAP_CKPT;
-  const int bf16 = p->snap_mode == MW_SNAP_BF16;
+  // snapshots the adjoint reads: the full store, or the fp32 replay segment
+  const int snap = ckpt ? kStoreF32 : snap_store_kind(p->snap_mode);
+  const int snap_elem = ckpt ? 4 : (int)snap_elem_bytes(p->snap_mode);
   const int C = ckpt ? p->ckpt_every : p->nt;
   const char *snap_e = ckpt ? ws + L.seg : ws + L.snap;
   const char *snap_c = snap_e + (size_t)C * L.snap_step_bytes;
   AdjMaps mA, mB;
-  MW_TRY(adj_maps(p, fields_at(p, adA), ca, cb, cq, gca, gcb, snap_e, snap_c, bf16 ? 2 : 4, C, &mA));
-  MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, cq, gca, gcb, snap_e, snap_c, bf16 ? 2 : 4, C, &mB));
+  MW_TRY(adj_maps(p, fields_at(p, adA), ca, cb, cq, gca, gcb, snap_e, snap_c, snap_elem, C, L.snap_pitch, &mA));
+  MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, cq, gca, gcb, snap_e, snap_c, snap_elem, C, L.snap_pitch, &mB));
 
   float *cur = adA, *nxt = adB;
   auto adj_step = [&](int t, int slot) -> int {
@@ -806,7 +827,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     a.ctr_slot = (launch_idx++) & 1;
     const AdjMaps &m = cur == adA ? mA : mB;
     MW_CUDA(timed(2, st, [&] {
-      return launch_adjoint(m, a, p->order, bf16, p->model_batched != 0, !p->cq_is_scalar,
+      return launch_adjoint(m, a, p->order, snap, p->model_batched != 0, !p->cq_is_scalar,
                             la.grid, st);
     }));
     std::swap(cur, nxt);
@@ -821,6 +842,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     StepArgs fa = a;
     fa.g = lf.g;
     set_layout(fa, p, false);
+    fa.snap_pitch = p->nx;  // the fp32 segment
     float *rA = (float *)(ws + L.rpA), *rB = (float *)(ws + L.rpB);
     FwdMaps fA, fB;
     MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, cq, &fA));
@@ -919,6 +941,22 @@ int mw_profile_enable(int32_t enable) {
   }
   T.recs.clear();
   T.on = enable != 0;
+  return MW_OK;
+}
+
+int mw_snapshot_encode(int32_t snap_mode, int64_t n, const float *x_dev, void *out_dev,
+                       void *stream) {
+  g_err.clear();
+  if (snap_mode != MW_SNAP_BF16 && snap_mode != MW_SNAP_FP8)
+    return fail(MW_ERR_ARG, "snap_mode %d has no narrow storage format", snap_mode);
+  if (n < 0 || n % 4 != 0) return fail(MW_ERR_ARG, "n = %lld must be a multiple of 4", (long long)n);
+  if (n == 0) return MW_OK;
+  if (!x_dev || !out_dev) return fail(MW_ERR_ARG, "NULL pointer");
+  const uintptr_t ax = (uintptr_t)x_dev, ao = (uintptr_t)out_dev;
+  if (ax % 16 != 0 || ao % (snap_mode == MW_SNAP_BF16 ? 8 : 4) != 0)
+    return fail(MW_ERR_ARG, "misaligned pointer");
+  MW_CUDA(launch_snap_encode(snap_store_kind(snap_mode), n, x_dev, out_dev,
+                             (cudaStream_t)stream));
   return MW_OK;
 }
 

@@ -5,7 +5,8 @@
 //   x-band mem   [S][ny][2*Wx]         columns [0,Wx) then [nx-Wx,nx)
 //   z-band mem   [S][2*Wz][nx]         rows    [0,Wz) then [ny-Wz,ny)
 //   model        [ny][nx] or [S][ny][nx]
-//   snapshots    [n][S][ny][nx]        float32 or bf16
+//   snapshots    [2][n][S][ny][pitch]  float32, bf16 or E4M3 (rows padded
+//                                      to 16 bytes)
 // Stencil kernels are "marching strips": one warp owns a 120- (forward) or
 // 112-column (adjoint) strip of one shot over a chunk of rows and walks down
 // it, keeping the y-direction stencil operands in registers and the
@@ -70,8 +71,10 @@ struct StepArgs {
   Fields in, out;
   const float *ca, *cb, *cq;
   float cq_scalar;
-  // forward: snapshots of this step ([S][ny][nx]; float or bf16), may be null
+  // forward: snapshots of this step ([S][ny][snap_pitch]; float32, bf16 or
+  // E4M3 bytes), may be null
   void *snap_e, *snap_c;
+  int snap_pitch;     // snapshot row pitch in elements (>= nx, 16-byte rows)
   // adjoint only: per-shot gradients [S][ny][nx]; time index of the
   // snapshot tensor maps
   float *gca, *gcb;
@@ -174,11 +177,12 @@ struct Layout {
   size_t bandtab;     // CPML band coefficient table (BandTab)
   size_t total;
   size_t state_bytes;
-  size_t snap_step_bytes;  // one step of one snapshot field ([S][ny][nx])
+  size_t snap_step_bytes;  // one step of one snapshot field ([S][ny][snap_pitch])
+  int snap_pitch;          // snapshot row pitch (elements): rows start 16-byte aligned
   int n_seg;
 };
 
-enum StoreKind { kStoreNone = 0, kStoreF32 = 1, kStoreBF16 = 2 };
+enum StoreKind { kStoreNone = 0, kStoreF32 = 1, kStoreBF16 = 2, kStoreFP8 = 3 };
 
 // device status word indices in the flags area; kCtrBase, kCtrBase + 1: the
 // work-item counters that consecutive stencil launches alternate between
@@ -202,8 +206,12 @@ void count_launches(int n);
 // stencil launchers (mw_stencil.cu); return a cudaError_t
 cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int store,
                            bool batched, bool cq_array, int grid, cudaStream_t st);
-cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int snap_bf16,
+// snap: the snapshot storage (kStoreF32, kStoreBF16 or kStoreFP8)
+cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int snap,
                            bool batched, bool cq_array, int grid, cudaStream_t st);
+// snapshot storage encoding of n floats (n % 4 == 0) with the forward's
+// conversion (kStoreBF16 or kStoreFP8)
+cudaError_t launch_snap_encode(int store, int64_t n, const float *x, void *out, cudaStream_t st);
 // forward / adjoint: the full stage layout (optional slots for a Cq array and
 // bands)
 void forward_layout(int order, int Wx, bool cq_array, StepArgs *a, size_t *smem_bytes);

@@ -36,6 +36,8 @@
 // band code; CPML memories exist only in the bands.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <atomic>
 
@@ -92,18 +94,26 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Snapshot row store (4 consecutive cells), float32 or bf16 (RNE).
+// Snapshot row store (4 consecutive cells at element `elem` of `base`):
+// float32, bfloat16 (nearest even) or FP8 E4M3 (nearest even, saturating to
+// the largest finite value, no scaling: the maxwell.cu page's fp8 storage).
 template <int STORE>
-__device__ __forceinline__ void snap_store(void *row, const F4 &v) {
+__device__ __forceinline__ void snap_store(void *base, int64_t elem, const F4 &v) {
   if constexpr (STORE == kStoreF32) {
-    st4(reinterpret_cast<float *>(row), v);
+    st4(reinterpret_cast<float *>(base) + elem, v);
   } else if constexpr (STORE == kStoreBF16) {
     __nv_bfloat162 lo = __floats2bfloat162_rn(v.v[0], v.v[1]);
     __nv_bfloat162 hi = __floats2bfloat162_rn(v.v[2], v.v[3]);
     uint2 pk;
     pk.x = *reinterpret_cast<uint32_t *>(&lo);
     pk.y = *reinterpret_cast<uint32_t *>(&hi);
-    *reinterpret_cast<uint2 *>(row) = pk;
+    *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(base) + elem) = pk;
+  } else if constexpr (STORE == kStoreFP8) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v.v[0], v.v[1]), __NV_SATFINITE,
+                                                 __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v.v[2], v.v[3]), __NV_SATFINITE,
+                                                 __NV_E4M3);
+    *reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(base) + elem) = lo | (hi << 16);
   }
 }
 
@@ -484,12 +494,10 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
           }
           if (own && e_row) {
             const int off = ro - (2 * P - 1) * nx;
-            if constexpr (STORE == kStoreF32) {
-              snap_store<STORE>(reinterpret_cast<float *>(a.snap_e) + pb + off, e_old);
-              snap_store<STORE>(reinterpret_cast<float *>(a.snap_c) + pb + off, curl);
-            } else if constexpr (STORE == kStoreBF16) {
-              snap_store<STORE>(reinterpret_cast<__nv_bfloat16 *>(a.snap_e) + pb + off, e_old);
-              snap_store<STORE>(reinterpret_cast<__nv_bfloat16 *>(a.snap_c) + pb + off, curl);
+            if constexpr (STORE != kStoreNone) {
+              const int64_t so = ((int64_t)it.s * a.g.ny + (it.r0 + i - 2 * P + 1)) * a.snap_pitch + c;
+              snap_store<STORE>(a.snap_e, so, e_old);
+              snap_store<STORE>(a.snap_c, so, curl);
             }
             st4(ey_o + off, en);
           }
@@ -565,17 +573,25 @@ __device__ __forceinline__ void tma5s(uint32_t dst, const CUtensorMap *map, int 
       "r"(bar)
       : "memory");
 }
-// Staged snapshot float4 (4 cells) at byte address addr: float32 or bf16.
-template <bool BF16>
+// Staged snapshot float4 (4 cells) at byte address addr: float32, bf16 or
+// FP8 E4M3 (SNAP = kStoreF32 / kStoreBF16 / kStoreFP8).
+template <int SNAP>
 __device__ __forceinline__ F4 snap_lds_s(uint32_t addr) {
-  if constexpr (!BF16) {
+  if constexpr (SNAP == kStoreF32) {
     return lds4s(addr);
-  } else {
+  } else if constexpr (SNAP == kStoreBF16) {
     uint32_t lo, hi;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi) : "r"(addr) : "memory");
     __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&lo);
     __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&hi);
     const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return F4{{fa.x, fa.y, fb.x, fb.y}};
+  } else {
+    uint32_t w;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(addr) : "memory");
+    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xffffu), __NV_E4M3);
+    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+    const float2 fa = __half22float2(__half2(lo)), fb = __half22float2(__half2(hi));
     return F4{{fa.x, fa.y, fb.x, fb.y}};
   }
 }
@@ -593,13 +609,14 @@ struct AdjWarp {
 // band memories of the E nodes and (x band) H nodes; row r - P for
 // lambda_Hx, its Cq and its z-band memory.  Rows outside the array read as
 // zeros.
-template <int P, bool BF16, bool BAND>
+template <int P, int SNAP, bool BAND>
 __device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, const Item &it,
                                           int i, uint32_t st, uint32_t bar, int cq_arr) {
   const int r = it.r0 + i;
   const bool own_r = (unsigned)(i - (2 * P - 1)) < (unsigned)(it.yb - it.ya);
   const bool hx_in = i >= it.hx_lo && i <= it.hx_hi;
-  constexpr uint32_t snap_bytes = BF16 ? 2 * 112 * 2 : 2 * 112 * 4;
+  constexpr uint32_t snap_elem = SNAP == kStoreF32 ? 4 : SNAP == kStoreBF16 ? 2 : 1;
+  constexpr uint32_t snap_bytes = 2 * 112 * snap_elem;
   uint32_t bytes = 2 * 128 * 4 + 2 * 128 * 4;
   if (hx_in) bytes += 112 * 4;
   if (own_r) bytes += snap_bytes + 2 * 112 * 4;
@@ -648,7 +665,7 @@ __device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, c
 //   lamHz and qx; lamHx and qz of row r - P; lamE of row r - 2P + 1.
 // Lanes: 0..31 hold the float4 at x0 - 8 + 4 lane (g, px, pz; lanes 2..29
 // own theirs), lanes 0..29 the qx float4 at x0 - 4 + 4 lane.
-template <int P, bool BF16, int L, bool BAND>
+template <int P, int SNAP, int L, bool BAND>
 __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, const Item &it,
                                          AdjWarp &w, int cq_arr, float cqs) {
   constexpr int NQ = 2 * P;
@@ -687,7 +704,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
     Ring pr = w.ring;
     for (int j = 0; j < L && j < it.n_it; ++j) {
       if (lane == 0)
-        adj_issue<P, BF16, BAND>(m, a, it, j, w.stage0 + pr.slot * w.stage_bytes,
+        adj_issue<P, SNAP, BAND>(m, a, it, j, w.stage0 + pr.slot * w.stage_bytes,
                                  w.bars + 8 * pr.slot, cq_arr);
       pr.next(NS);
     }
@@ -703,7 +720,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
       if (i < it.n_it) {
         if (i + L < it.n_it && lane == 0) {
           const int ps = w.ring.slot == 0 ? NS - 1 : w.ring.slot - 1;
-          adj_issue<P, BF16, BAND>(m, a, it, i + L, w.stage0 + ps * w.stage_bytes,
+          adj_issue<P, SNAP, BAND>(m, a, it, i + L, w.stage0 + ps * w.stage_bytes,
                                    w.bars + 8 * ps, cq_arr);
         }
         if (!mbar_wait_s(w.bars + 8 * w.ring.slot, w.ring.phase)) {
@@ -752,10 +769,10 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
         if (own_r) {
           if (own) {
             const uint32_t sbase = st + kA_SS * 4;
-            constexpr uint32_t sfield = BF16 ? 112 * 2 : 112 * 4;
-            constexpr uint32_t sstep = BF16 ? 8 : 16;
-            const F4 se = snap_lds_s<BF16>(sbase + sstep * wo);
-            const F4 sc = snap_lds_s<BF16>(sbase + sfield + sstep * wo);
+            constexpr uint32_t selem = SNAP == kStoreF32 ? 4 : SNAP == kStoreBF16 ? 2 : 1;
+            constexpr uint32_t sfield = 112 * selem, sstep = 4 * selem;
+            const F4 se = snap_lds_s<SNAP>(sbase + sstep * wo);
+            const F4 sc = snap_lds_s<SNAP>(sbase + sfield + sstep * wo);
             F4 gca = lds4s(st + w.gca_o + 16 * wo), gcb = lds4s(st + w.gcb_o + 16 * wo);
             const bool rowmask = !BAND || !a.g.grad_mask || (r >= a.g.n_pml && r < ny - a.g.n_pml);
 #pragma unroll
@@ -878,7 +895,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
   return true;
 }
 
-template <int P, bool BF16, int L>
+template <int P, int SNAP, int L>
 __global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_constant__ AdjMaps m,
                                                                   const StepArgs a,
                                                                   const int batched,
@@ -924,8 +941,8 @@ __global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_c
     if (item >= n_items) break;
     Item it;
     if (!make_item<P>(g, item, batched != 0, it)) continue;
-    const bool ok = it.edge ? adj_walk<P, BF16, L, true>(m, a, it, w, cq_arr, cqs)
-                            : adj_walk<P, BF16, L, false>(m, a, it, w, cq_arr, cqs);
+    const bool ok = it.edge ? adj_walk<P, SNAP, L, true>(m, a, it, w, cq_arr, cqs)
+                            : adj_walk<P, SNAP, L, false>(m, a, it, w, cq_arr, cqs);
     if (!ok) return;
   }
 }
@@ -1008,7 +1025,7 @@ std::atomic<uint64_t> &fwd_smem_flag() {
   static std::atomic<uint64_t> f{0};
   return f;
 }
-template <int P, bool BF16>
+template <int P, int SNAP>
 std::atomic<uint64_t> &adj_smem_flag() {
   static std::atomic<uint64_t> f{0};
   return f;
@@ -1023,12 +1040,12 @@ cudaError_t fwd_t(const FwdMaps &m, const StepArgs &a, bool batched, bool cq_arr
   count_launches(1);
   return cudaGetLastError();
 }
-template <int P, bool BF16>
+template <int P, int SNAP>
 cudaError_t adj_t(const AdjMaps &m, const StepArgs &a, bool batched, bool cq_arr, int grid,
                   cudaStream_t st) {
   const size_t smem = (size_t)(32 + kAdjWarpsPerCta * a.warp_floats) * sizeof(float) + 128;
-  allow_big_smem(k_adjoint<P, BF16, kAdjL>, adj_smem_flag<P, BF16>());
-  k_adjoint<P, BF16, kAdjL><<<grid, 32 * kAdjWarpsPerCta, smem, st>>>(m, a, batched ? 1 : 0,
+  allow_big_smem(k_adjoint<P, SNAP, kAdjL>, adj_smem_flag<P, SNAP>());
+  k_adjoint<P, SNAP, kAdjL><<<grid, 32 * kAdjWarpsPerCta, smem, st>>>(m, a, batched ? 1 : 0,
                                                                        cq_arr ? 1 : 0);
   count_launches(1);
   return cudaGetLastError();
@@ -1041,8 +1058,28 @@ cudaError_t fwd_store(const FwdMaps &m, const StepArgs &a, int store, bool batch
     case kStoreNone: return fwd_t<P, kStoreNone>(m, a, batched, cq_arr, grid, st);
     case kStoreF32: return fwd_t<P, kStoreF32>(m, a, batched, cq_arr, grid, st);
     case kStoreBF16: return fwd_t<P, kStoreBF16>(m, a, batched, cq_arr, grid, st);
+    case kStoreFP8: return fwd_t<P, kStoreFP8>(m, a, batched, cq_arr, grid, st);
   }
   return cudaErrorInvalidValue;
+}
+
+template <int P>
+cudaError_t adj_snap(const AdjMaps &m, const StepArgs &a, int snap, bool batched, bool cq_arr,
+                     int grid, cudaStream_t st) {
+  switch (snap) {
+    case kStoreF32: return adj_t<P, kStoreF32>(m, a, batched, cq_arr, grid, st);
+    case kStoreBF16: return adj_t<P, kStoreBF16>(m, a, batched, cq_arr, grid, st);
+    case kStoreFP8: return adj_t<P, kStoreFP8>(m, a, batched, cq_arr, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// Snapshot encoding of n floats with the forward's store conversion.
+template <int STORE>
+__global__ void k_snap_encode(const float *__restrict__ x, void *out, int64_t n4) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x)
+    snap_store<STORE>(out, 4 * i, ld4(x + 4 * i));
 }
 
 template <typename K>
@@ -1060,8 +1097,8 @@ int slots_t(bool adjoint, int Wx, bool cq_arr) {
   StepArgs a{};
   if (adjoint) {
     adj_layout_t<P>(Wx, cq_arr, &a, &smem);
-    return occupancy(k_adjoint<P, false, kAdjL>, 32 * kAdjWarpsPerCta, smem,
-                     adj_smem_flag<P, false>()) *
+    return occupancy(k_adjoint<P, kStoreF32, kAdjL>, 32 * kAdjWarpsPerCta, smem,
+                     adj_smem_flag<P, kStoreF32>()) *
            kAdjWarpsPerCta;
   }
   fwd_layout_t<P>(Wx, cq_arr, &a, &smem);
@@ -1083,20 +1120,29 @@ cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int s
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int snap_bf16,
+cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int snap,
                            bool batched, bool cq_array, int grid, cudaStream_t st) {
-  const bool b = snap_bf16 != 0;
   switch (order) {
-    case 2: return b ? adj_t<1, true>(m, a, batched, cq_array, grid, st)
-                     : adj_t<1, false>(m, a, batched, cq_array, grid, st);
-    case 4: return b ? adj_t<2, true>(m, a, batched, cq_array, grid, st)
-                     : adj_t<2, false>(m, a, batched, cq_array, grid, st);
-    case 6: return b ? adj_t<3, true>(m, a, batched, cq_array, grid, st)
-                     : adj_t<3, false>(m, a, batched, cq_array, grid, st);
-    case 8: return b ? adj_t<4, true>(m, a, batched, cq_array, grid, st)
-                     : adj_t<4, false>(m, a, batched, cq_array, grid, st);
+    case 2: return adj_snap<1>(m, a, snap, batched, cq_array, grid, st);
+    case 4: return adj_snap<2>(m, a, snap, batched, cq_array, grid, st);
+    case 6: return adj_snap<3>(m, a, snap, batched, cq_array, grid, st);
+    case 8: return adj_snap<4>(m, a, snap, batched, cq_array, grid, st);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_snap_encode(int store, int64_t n, const float *x, void *out, cudaStream_t st) {
+  const int64_t n4 = n / 4;
+  if (n4 == 0) return cudaSuccess;
+  const int grid = (int)(n4 < 148 * 32 * 256 ? (n4 + 255) / 256 : 148 * 32);
+  if (store == kStoreBF16)
+    k_snap_encode<kStoreBF16><<<grid, 256, 0, st>>>(x, out, n4);
+  else if (store == kStoreFP8)
+    k_snap_encode<kStoreFP8><<<grid, 256, 0, st>>>(x, out, n4);
+  else
+    return cudaErrorInvalidValue;
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array) {

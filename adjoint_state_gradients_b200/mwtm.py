@@ -22,8 +22,9 @@ MW_ERR_NONFINITE = -5
 MW_ERR_TIMEOUT = -6
 MW_ERR_UNSUPPORTED = -7
 
-SNAP_NONE, SNAP_FP32, SNAP_BF16, SNAP_CKPT = 0, 1, 2, 3
-SNAP_MODES = {"none": SNAP_NONE, "fp32": SNAP_FP32, "bf16": SNAP_BF16, "ckpt": SNAP_CKPT}
+SNAP_NONE, SNAP_FP32, SNAP_BF16, SNAP_CKPT, SNAP_FP8 = 0, 1, 2, 3, 4
+SNAP_MODES = {"none": SNAP_NONE, "fp32": SNAP_FP32, "bf16": SNAP_BF16, "ckpt": SNAP_CKPT,
+              "fp8": SNAP_FP8}
 
 
 class Params(ctypes.Structure):
@@ -70,6 +71,8 @@ SIGNATURES = [
     ("mw_profile_read", ctypes.c_int, [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double),
                                        ctypes.c_int32]),
     ("mw_launch_count", ctypes.c_int64, []),
+    ("mw_snapshot_encode", ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p]),
     ("mw_workspace_init", ctypes.c_int, [_VP, ctypes.c_size_t, _VP]),
     ("mw_tm_forward_noalloc", ctypes.c_int, [_P, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
 ]
@@ -221,3 +224,10 @@ def profile_read(n_classes: int = 3):
     ms = (ctypes.c_double * n_classes)()
     check(lib().mw_profile_read(counts, ms, n_classes))
     return list(counts), list(ms)
+
+
+def snapshot_encode(snap_mode, x, out, stream=None):
+    """Round float32 `x` to the storage format of snap_mode (SNAP_BF16 or
+    SNAP_FP8) into `out` (2 or 1 bytes per value) on the device."""
+    return check(lib().mw_snapshot_encode(int(snap_mode), x.numel(), ptr(x), ptr(out),
+                                          stream_ptr(stream)))

@@ -77,6 +77,10 @@ extern "C" {
 #define MW_SNAP_BF16 2 /* same, rounded to bfloat16 (round to nearest even)  */
 #define MW_SNAP_CKPT 3 /* full state every ckpt_every steps; the adjoint
                           replays each segment into an fp32 segment buffer  */
+#define MW_SNAP_FP8 4  /* Ey^n and curl^n rounded to FP8 E4M3 (nearest even,
+                          saturating to +-448, no scaling), as the
+                          maxwell.cu page's forward_kernel_e_with_storage_fp8
+                          stores them                                        */
 
 typedef struct mw_params {
   int32_t ny, nx;        /* array size incl. the CPML band                 */
@@ -254,6 +258,18 @@ int mw_profile_read(int64_t *counts, double *total_ms, int32_t n_classes);
 /* Number of CUDA kernels this library has launched in this process (all
  * entry points, all devices).  Host counter; no synchronization. */
 int64_t mw_launch_count(void);
+
+/* Snapshot storage encoding (page: maxwell.cu, the bf16 / "FP8 E4M3"
+ * storage helpers used by forward_kernel_e_with_storage_bf16 / _fp8).
+ * Rounds n float32 values x_dev[0..n) to the storage format of snap_mode
+ * (MW_SNAP_BF16: bfloat16, 2 bytes each; MW_SNAP_FP8: E4M3, 1 byte each)
+ * into out_dev, with the same device conversion the forward kernel applies
+ * when it stores snapshots.  n % 4 == 0; x_dev 16-byte aligned, out_dev
+ * 8-byte (bf16) or 4-byte (fp8) aligned; device pointers owned by the
+ * caller.  Asynchronous on `stream`.  MW_ERR_ARG for another snap_mode, a
+ * bad n or misaligned pointers. */
+int mw_snapshot_encode(int32_t snap_mode, int64_t n, const float *x_dev, void *out_dev,
+                       void *stream);
 
 #ifdef __cplusplus
 }

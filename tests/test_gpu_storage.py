@@ -1,0 +1,114 @@
+"""Narrow snapshot storage on the GPU (bfloat16, FP8 E4M3) against the oracle.
+
+(1) The conversion the forward kernel applies when it stores a snapshot,
+called through mw_snapshot_encode, gives bit for bit the oracle's encoding
+(nearest even; E4M3 saturating to +-448) on random values across the whole
+range, every E4M3 tie, bf16 ties, saturation and underflow.
+(2) The gradients of a run with bf16 or fp8 snapshots match the oracle's
+adjoint fed the same rounding of its own snapshots (within the fp32 gradient
+tolerance: the two sides round values that differ by fp32 rounding, so a code
+can flip only where a value sits on a rounding boundary).
+(3) The storage error itself, against fp32 storage, is reported.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from adjoint_state_gradients_b200 import mwtm, synth
+from tests._cases import rel_l2, small_sim
+from tests._gpu import f32, problem_from_sim, run_adjoint, run_forward
+
+pytestmark = pytest.mark.gpu
+
+GRAD_TOL = 1e-4
+REC_TOL = 1e-5
+
+
+def _test_values():
+    g = np.random.default_rng(17)
+    x = g.normal(size=200000) * 10.0 ** g.uniform(-6, 3.5, size=200000)
+    v = oracle.fp8_decode(np.arange(0x7F, dtype=np.uint8))
+    ties = (v[:-1] + v[1:]) / 2
+    bf = 1.0 + np.arange(0, 256) * 2.0 ** -8  # every other one a bf16 tie
+    extra = np.array([0.0, -0.0, 448.0, 464.0, 500.0, 1e9, -1e9, 2.0 ** -10, 3 * 2.0 ** -11,
+                      1e-30, -1e-30])
+    x = np.concatenate([x, ties, -ties, bf, -bf, extra])
+    x = x[: len(x) // 4 * 4].astype(np.float32)
+    return x
+
+
+def test_fp8_encoding_matches_oracle_bitwise():
+    x = _test_values()
+    xd = torch.as_tensor(x).cuda()
+    out = torch.empty(x.size, dtype=torch.uint8, device="cuda")
+    mwtm.snapshot_encode(mwtm.SNAP_FP8, xd, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    want = oracle.fp8_encode(x.astype(np.float64))
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, [(float(x[i]), int(got[i]), int(want[i])) for i in bad[:10]]
+
+
+def test_bf16_encoding_matches_oracle_bitwise():
+    x = _test_values()
+    x = x[np.abs(x) < 1e30]
+    x = x[: len(x) // 4 * 4]
+    xd = torch.as_tensor(x).cuda()
+    out = torch.empty(x.size, dtype=torch.bfloat16, device="cuda")
+    mwtm.snapshot_encode(mwtm.SNAP_BF16, xd, out)
+    torch.cuda.synchronize()
+    got = out.double().cpu().numpy()
+    want = oracle.quant_bf16(x.astype(np.float64))
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("mode,order,batched,nx", [("fp8", 4, False, 160), ("bf16", 4, False, 160),
+                                                   ("fp8", 8, True, 160), ("bf16", 2, False, 160),
+                                                   ("fp8", 4, False, 148), ("bf16", 6, False, 148)])
+def test_narrow_snapshot_gradients_match_oracle(mode, order, batched, nx):
+    """nx = 148: snapshot rows are padded to 16 bytes (148 is no multiple of
+    16 or 8), so the stored rows have a pitch larger than nx."""
+    ny, S = 64, 2
+    sim, dt, _ = small_sim(700 + order, ny, nx, S, 2, 6, order, 6, round_f32=True,
+                           sigma_max=0.02, batched=batched)
+    nt = 60
+    g = synth.rng(70 + order)
+    f = f32(g.normal(size=(nt, S, 2)))
+    res = f32(g.normal(size=(nt, S, 6)))
+    fw = sim.forward(f, snapshots=True)
+    quant = oracle.quant_fp8 if mode == "fp8" else oracle.quant_bf16
+    adj = sim.adjoint(res, quant(fw["snap_ey"]), quant(fw["snap_curl"]))
+    prob = problem_from_sim(sim, nt, dt, 6, snapshot=mode)
+    rec = run_forward(prob, f)
+    assert rel_l2(rec, fw["rec"]) <= REC_TOL
+    gca, gcb, gf = run_adjoint(prob, res)
+    assert rel_l2(gca, adj["gca"]) <= GRAD_TOL
+    assert rel_l2(gcb, adj["gcb"]) <= GRAD_TOL
+    assert rel_l2(gf, adj["grad_f"]) <= GRAD_TOL
+    assert prob.status() == mwtm.MW_OK
+
+
+def test_narrow_storage_error_against_fp32_workload2():
+    """296x296 order 4, 4 shots, nt 1000: gradient error of bf16 and fp8
+    storage against fp32 storage on the GPU (reported; the fp8 format is the
+    page's unscaled E4M3, so small field values underflow)."""
+    from tests._cases import workload_sim
+    nt = 1000
+    sim, inp, dt, f = workload_sim(2, n_shots=4, nt=nt)
+    g = synth.rng(22)
+    res = f32(g.normal(size=(nt, 4, inp.wl.n_rec)))
+    out = {}
+    for mode in ("fp32", "bf16", "fp8"):
+        prob = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot=mode)
+        run_forward(prob, f)
+        out[mode] = run_adjoint(prob, res)[:2]
+        del prob
+    for mode in ("bf16", "fp8"):
+        e_ca = rel_l2(out[mode][0], out["fp32"][0])
+        e_cb = rel_l2(out[mode][1], out["fp32"][1])
+        print(f"{mode} snapshot gradient error vs fp32 storage: Ca {e_ca:.3e} Cb {e_cb:.3e}")
+        assert np.isfinite(e_ca) and np.isfinite(e_cb)
+    assert rel_l2(out["bf16"][0], out["fp32"][0]) <= 2e-2
