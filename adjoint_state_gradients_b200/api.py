@@ -28,11 +28,14 @@ class Problem:
 
     src_idx [S, n_src] / rec_idx [S, n_rec] are flat cell indices y*nx + x
     (-1 = inactive).  snapshot: "none" | "fp32" | "bf16" | "fp8" | "ckpt".
+    snapshot_host: keep the fp32 / bf16 / fp8 snapshots in page-locked host
+    memory (staged through a 3-step device ring) instead of the workspace.
     """
 
     def __init__(self, ny, nx, order, dy, dx, dt, nt, n_pml, src_idx, rec_idx, *, vmax,
                  snapshot="fp32", ckpt_every=64, batched=False, cq_scalar=True,
-                 grad_mask_pml=False, allow_unstable=False, check_finite=False, device="cuda"):
+                 grad_mask_pml=False, allow_unstable=False, check_finite=False, device="cuda",
+                 snapshot_host=False):
         src_idx = np.asarray(src_idx, dtype=np.int64)
         rec_idx = np.asarray(rec_idx, dtype=np.int64)
         self.S = src_idx.shape[0]
@@ -42,8 +45,13 @@ class Problem:
             nt=nt, dt=dt, dy=dy, dx=dx, n_pml=n_pml, model_batched=int(batched),
             cq_is_scalar=int(cq_scalar), snap_mode=mwtm.SNAP_MODES[snapshot], ckpt_every=ckpt_every,
             grad_mask_pml=int(grad_mask_pml), vmax=vmax, allow_unstable=int(allow_unstable),
-            check_finite=int(check_finite))
+            check_finite=int(check_finite), snap_host=int(bool(snapshot_host)))
         mwtm.check(mwtm.validate(self.p))
+        self.host_snapshots = None
+        if snapshot_host:
+            n = mwtm.snap_host_bytes(self.p)
+            self.host_snapshots = torch.empty(max(n, 1), dtype=torch.uint8, pin_memory=True)
+            self.p.snap_host_ptr = self.host_snapshots.data_ptr()
         self.src_idx = _dev(src_idx if src_idx.size else np.zeros((self.S, 1), np.int64),
                             torch.int64, device)
         self.rec_idx = _dev(rec_idx if rec_idx.size else np.zeros((self.S, 1), np.int64),
@@ -116,6 +124,11 @@ class Problem:
         return out
 
     def eps_sigma_gradient(self, gca, gcb):
+        """Chain rule to (eps_r, sigma), cell by cell: gca / gcb shaped like the
+        model (the shot sum for a shared model, per-shot gradients for a
+        batched one)."""
+        if gca.numel() != self.ca.numel() or gcb.numel() != self.ca.numel():
+            raise ValueError(f"gradients of {gca.numel()} cells for a model of {self.ca.numel()}")
         n = gca.numel()
         ge = torch.empty_like(gca)
         gs = torch.empty_like(gca)

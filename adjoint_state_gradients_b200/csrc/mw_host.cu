@@ -100,6 +100,9 @@ int check_params(const mw_params *p, bool cfl) {
     return fail(MW_ERR_ARG, "CPML band %d does not fit a %d x %d grid", p->n_pml, p->ny, p->nx);
   if (p->snap_mode < MW_SNAP_NONE || p->snap_mode > MW_SNAP_FP8)
     return fail(MW_ERR_ARG, "snap_mode = %d", p->snap_mode);
+  if (p->snap_host && p->snap_mode != MW_SNAP_FP32 && p->snap_mode != MW_SNAP_BF16 &&
+      p->snap_mode != MW_SNAP_FP8)
+    return fail(MW_ERR_ARG, "snap_host needs snap_mode FP32, BF16 or FP8 (got %d)", p->snap_mode);
   if (p->snap_mode == MW_SNAP_CKPT && p->ckpt_every < 1)
     return fail(MW_ERR_ARG, "ckpt_every = %d", p->ckpt_every);
   if (2 * b.Wx > 256)
@@ -115,6 +118,9 @@ int check_params(const mw_params *p, bool cfl) {
   }
   return MW_OK;
 }
+
+// device ring slots of the pinned-host snapshot store
+constexpr int kHostRing = 3;
 
 // bytes per stored snapshot value of a full-storage mode
 size_t snap_elem_bytes(int snap_mode) {
@@ -158,7 +164,10 @@ Layout layout(const mw_params *p) {
     L.snap_pitch = (int)(((size_t)p->nx + per_row - 1) / per_row * per_row);
     L.snap_step_bytes = (size_t)p->n_shots * p->ny * L.snap_pitch * es;
     L.snap = off;
-    off += align256(2 * (size_t)p->nt * L.snap_step_bytes);
+    // device copy of every step, or with snap_host a ring of kHostRing steps
+    // ([2][kHostRing] step slots) that the host copies pass through
+    const size_t steps = p->snap_host ? (size_t)kHostRing : (size_t)p->nt;
+    off += align256(2 * steps * L.snap_step_bytes);
   } else if (p->snap_mode == MW_SNAP_CKPT) {
     L.n_seg = p->nt > 0 ? (p->nt + p->ckpt_every - 1) / p->ckpt_every : 0;
     L.rpA = off; off += sb;
@@ -188,6 +197,45 @@ Fields fields_at(const mw_params *p, float *base) {
   f.mze_node = f.mzh_node + zb;
   return f;
 }
+
+// Pinned-host snapshot store: the caller's page-locked buffer holds step t
+// as [E block][curl block] at 2 t step_bytes; a ring of kHostRing device
+// slots per field stages the copies, which run on a stream of their own and
+// are ordered with the compute stream by events.
+int check_host_snap(const mw_params *p) {
+  if (!p->snap_host) return MW_OK;
+  if (!p->snap_host_ptr) return fail(MW_ERR_ARG, "snap_host_ptr is NULL");
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p->snap_host_ptr) != cudaSuccess ||
+      at.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return fail(MW_ERR_ARG, "snap_host_ptr is not page-locked host memory");
+  }
+  return MW_OK;
+}
+struct HostCopies {
+  cudaStream_t cs = nullptr;
+  cudaEvent_t filled[kHostRing] = {}, freed[kHostRing] = {}, start = nullptr;
+  int init() {
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess)
+      return fail(MW_ERR_CUDA, "cannot create the snapshot copy stream");
+    for (int k = 0; k < kHostRing; ++k)
+      if (cudaEventCreateWithFlags(&filled[k], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&freed[k], cudaEventDisableTiming) != cudaSuccess)
+        return fail(MW_ERR_CUDA, "cannot create snapshot copy events");
+    if (cudaEventCreateWithFlags(&start, cudaEventDisableTiming) != cudaSuccess)
+      return fail(MW_ERR_CUDA, "cannot create snapshot copy events");
+    return MW_OK;
+  }
+  ~HostCopies() {  // resources are released once the queued work completes
+    for (int k = 0; k < kHostRing; ++k) {
+      if (filled[k]) cudaEventDestroy(filled[k]);
+      if (freed[k]) cudaEventDestroy(freed[k]);
+    }
+    if (start) cudaEventDestroy(start);
+    if (cs) cudaStreamDestroy(cs);
+  }
+};
 
 // Duplicate-chain arrays (lead, next) of the sources and receivers.
 struct Chains {
@@ -606,6 +654,11 @@ size_t mw_state_floats(const mw_params *p) {
   return state_floats(p);
 }
 
+size_t mw_snap_host_bytes(const mw_params *p) {
+  if (check_params(p, false) != MW_OK || !p->snap_host) return 0;
+  return 2 * (size_t)p->nt * layout(p).snap_step_bytes;
+}
+
 size_t mw_workspace_bytes(const mw_params *p) {
   if (check_params(p, false) != MW_OK) return 0;
   return layout(p).total;
@@ -666,6 +719,7 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   g_err.clear();
   int rc = check_params(p, true);
   if (rc) return rc;
+  if ((rc = check_host_snap(p))) return rc;
   if ((rc = check_ptr(ca, "ca")) || (rc = check_ptr(cb, "cb")) || (rc = check_ptr(cpml, "cpml")))
     return rc;
   if (!cq) return fail(MW_ERR_ARG, "cq is NULL");
@@ -714,30 +768,50 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   if (p->n_rec > 0 && rec)  // chains unused here: this validates the receiver indices
     MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
                               flags, st));
+  const bool host = p->snap_host != 0;
+  const size_t ring_steps = host ? (size_t)kHostRing : (size_t)p->nt;
   char *snap_e = ws + L.snap;
-  char *snap_c = ws + L.snap + (size_t)p->nt * L.snap_step_bytes;
+  char *snap_c = ws + L.snap + ring_steps * L.snap_step_bytes;
+  HostCopies hc;
+  if (host) MW_TRY(hc.init());
+  char *hbuf = (char *)p->snap_host_ptr;
   float *cur = bufA, *nxt = bufB;
   for (int t = 0; t < p->nt; ++t) {
     if (p->snap_mode == MW_SNAP_CKPT && t % p->ckpt_every == 0) {
       char *ck = ws + L.snap + (size_t)(t / p->ckpt_every) * align256(L.state_bytes);
       MW_CUDA(cudaMemcpyAsync(ck, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
     }
+    const int slot = host ? t % kHostRing : t;
+    // the slot's previous step must have reached the host
+    if (host && t >= kHostRing) MW_CUDA(cudaStreamWaitEvent(st, hc.freed[slot], 0));
     a.in = fields_at(p, cur);
     a.out = fields_at(p, nxt);
-    a.snap_e = store ? snap_e + (size_t)t * L.snap_step_bytes : nullptr;
-    a.snap_c = store ? snap_c + (size_t)t * L.snap_step_bytes : nullptr;
+    a.snap_e = store ? snap_e + (size_t)slot * L.snap_step_bytes : nullptr;
+    a.snap_c = store ? snap_c + (size_t)slot * L.snap_step_bytes : nullptr;
     const FwdMaps &m = cur == bufA ? mA : mB;
     a.ctr_slot = t & 1;
     MW_CUDA(timed(store ? 1 : 0, st, [&] {
       return launch_forward(m, a, p->order, store, p->model_batched != 0, !p->cq_is_scalar,
                             lc.grid, st);
     }));
+    if (host) {  // step t: ring slot -> host, on the copy stream
+      MW_CUDA(cudaEventRecord(hc.filled[slot], st));
+      MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.filled[slot], 0));
+      char *h = hbuf + 2 * (size_t)t * L.snap_step_bytes;
+      MW_CUDA(cudaMemcpyAsync(h, a.snap_e, L.snap_step_bytes, cudaMemcpyDeviceToHost, hc.cs));
+      MW_CUDA(cudaMemcpyAsync(h + L.snap_step_bytes, a.snap_c, L.snap_step_bytes,
+                              cudaMemcpyDeviceToHost, hc.cs));
+      MW_CUDA(cudaEventRecord(hc.freed[slot], hc.cs));
+    }
     MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots,
                                  f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
                                  ch.src_lead, ch.src_next, p->n_src, rec_idx, p->n_rec,
                                  rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, st));
     std::swap(cur, nxt);
   }
+  if (host)  // the call's stream completes only after every copy reached the host
+    for (int k = 0; k < kHostRing && k < p->nt; ++k)
+      MW_CUDA(cudaStreamWaitEvent(st, hc.freed[(p->nt - 1 - k) % kHostRing], 0));
   if (cur != bufA) MW_CUDA(cudaMemcpyAsync(bufA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
   if (p->check_finite) MW_CUDA(launch_check_finite(bufA, 3 * SN, flags, st));
   return MW_OK;
@@ -751,6 +825,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   g_err.clear();
   int rc = check_params(p, true);
   if (rc) return rc;
+  if ((rc = check_host_snap(p))) return rc;
   if (p->snap_mode == MW_SNAP_NONE)
     return fail(MW_ERR_ARG, "snap_mode NONE: the forward stored nothing to differentiate");
   if ((rc = check_ptr(ca, "ca")) || (rc = check_ptr(cb, "cb")) || (rc = check_ptr(cpml, "cpml")) ||
@@ -807,7 +882,8 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   // snapshots the adjoint reads: the full store, or the fp32 replay segment
   const int snap = ckpt ? kStoreF32 : snap_store_kind(p->snap_mode);
   const int snap_elem = ckpt ? 4 : (int)snap_elem_bytes(p->snap_mode);
-  const int C = ckpt ? p->ckpt_every : p->nt;
+  const bool host = p->snap_host != 0;
+  const int C = ckpt ? p->ckpt_every : host ? kHostRing : p->nt;
   const char *snap_e = ckpt ? ws + L.seg : ws + L.snap;
   const char *snap_c = snap_e + (size_t)C * L.snap_step_bytes;
   AdjMaps mA, mB;
@@ -834,7 +910,35 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     return MW_OK;
   };
 
-  if (!ckpt) {
+  if (host) {
+    // pinned-host snapshots: prefetch step t into ring slot t % kHostRing on
+    // the copy stream, kHostRing steps ahead of the adjoint that reads it
+    HostCopies hc;
+    MW_TRY(hc.init());
+    MW_CUDA(cudaEventRecord(hc.start, st));
+    MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.start, 0));
+    const char *hbuf = (const char *)p->snap_host_ptr;
+    auto fetch = [&](int t) -> int {
+      const int slot = t % kHostRing;
+      if (t + kHostRing <= p->nt - 1) MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.freed[slot], 0));
+      const char *h = hbuf + 2 * (size_t)t * L.snap_step_bytes;
+      MW_CUDA(cudaMemcpyAsync((void *)(snap_e + (size_t)slot * L.snap_step_bytes), h,
+                              L.snap_step_bytes, cudaMemcpyHostToDevice, hc.cs));
+      MW_CUDA(cudaMemcpyAsync((void *)(snap_c + (size_t)slot * L.snap_step_bytes),
+                              h + L.snap_step_bytes, L.snap_step_bytes, cudaMemcpyHostToDevice,
+                              hc.cs));
+      MW_CUDA(cudaEventRecord(hc.filled[slot], hc.cs));
+      return MW_OK;
+    };
+    for (int t = p->nt - 1; t >= 0 && t >= p->nt - kHostRing; --t) MW_TRY(fetch(t));
+    for (int t = p->nt - 1; t >= 0; --t) {
+      const int slot = t % kHostRing;
+      MW_CUDA(cudaStreamWaitEvent(st, hc.filled[slot], 0));
+      MW_TRY(adj_step(t, slot));
+      MW_CUDA(cudaEventRecord(hc.freed[slot], st));
+      if (t - kHostRing >= 0) MW_TRY(fetch(t - kHostRing));
+    }
+  } else if (!ckpt) {
     for (int t = p->nt - 1; t >= 0; --t) MW_TRY(adj_step(t, t));
   } else {
     // checkpoint mode: replay each segment from its checkpoint, newest first

@@ -35,7 +35,8 @@ class Params(ctypes.Structure):
                 ("cq_is_scalar", ctypes.c_int32), ("snap_mode", ctypes.c_int32),
                 ("ckpt_every", ctypes.c_int32), ("grad_mask_pml", ctypes.c_int32),
                 ("vmax", ctypes.c_double), ("allow_unstable", ctypes.c_int32),
-                ("check_finite", ctypes.c_int32)]
+                ("check_finite", ctypes.c_int32), ("snap_host", ctypes.c_int32),
+                ("snap_host_ptr", ctypes.c_void_p)]
 
 
 class MWError(RuntimeError):
@@ -52,6 +53,7 @@ _P = ctypes.POINTER(Params)
 SIGNATURES = [
     ("mw_params_init", None, [_P]),
     ("mw_state_floats", ctypes.c_size_t, [_P]),
+    ("mw_snap_host_bytes", ctypes.c_size_t, [_P]),
     ("mw_workspace_bytes", ctypes.c_size_t, [_P]),
     ("mw_cfl_dt", ctypes.c_double, [ctypes.c_int32, ctypes.c_double, ctypes.c_double, ctypes.c_double]),
     ("mw_validate", ctypes.c_int, [_P]),
@@ -140,6 +142,11 @@ def state_floats(p: Params) -> int:
     if n == 0:
         raise MWError(MW_ERR_ARG, last_error())
     return n
+
+
+def snap_host_bytes(p: Params) -> int:
+    """Pinned host bytes of the snapshots when p.snap_host = 1."""
+    return lib().mw_snap_host_bytes(ctypes.byref(p))
 
 
 def workspace_bytes(p: Params) -> int:

@@ -100,10 +100,23 @@ typedef struct mw_params {
   double vmax;           /* fastest wave speed in the model, m/s (CFL check) */
   int32_t allow_unstable;/* 1: skip the CFL check                            */
   int32_t check_finite;  /* 1: flag NaN / Inf in the final state             */
+  int32_t snap_host;     /* 1 (with MW_SNAP_FP32 / BF16 / FP8): keep the
+                            snapshots in pinned host memory (snap_host_ptr,
+                            mw_snap_host_bytes(p) bytes, caller-owned) and
+                            stage them through a 3-step ring in the
+                            workspace, copied on a stream of the library's
+                            own (the page's CPU snapshot storage with its
+                            ring of device buffers and prefetch)           */
+  void *snap_host_ptr;   /* page-locked host buffer for snap_host = 1        */
 } mw_params;
 
 /* Fill *p with defaults (zeros, cq_is_scalar = 1, snap_mode NONE). */
 void mw_params_init(mw_params *p);
+
+/* Bytes of pinned host memory the snapshots of p take when p->snap_host = 1
+ * (both fields of every step; rows padded to 16 bytes).  0 otherwise or on
+ * invalid params. */
+size_t mw_snap_host_bytes(const mw_params *p);
 
 /* Floats in one state buffer (layout above). 0 on invalid params. */
 size_t mw_state_floats(const mw_params *p);

@@ -375,6 +375,38 @@ def test_workload5_all_shots_sampled():
     assert rel_l2(rec[:, sel], fw["rec"]) <= REC_TOL
 
 
+def test_workload5_per_shot_model_gradients_sampled():
+    """Per-shot models (552x552 order 8, all 256 shots): the adjoint keeps one
+    gradient per shot and the chain rule runs per shot (no shot sum).
+    Checkpoints every 64 steps, nt 130; shots 0 and 255 against the oracle."""
+    nt, sel = 130, [0, 255]
+    inp = synth.make_inputs(5)
+    wl = inp.wl
+    vmax = oracle.c0() / np.sqrt(inp.eps_min)
+    dt = wl.cfl_fraction * oracle.cfl_dt(wl.order, wl.h, wl.h, vmax)
+    f = f32(inp.wavelet(dt, nt))
+    g = synth.rng(505)
+    res = f32(g.normal(size=(nt, wl.n_shots, wl.n_rec)))
+    sim = oracle_sim(inp.eps_r, inp.sigma, inp.src_idx, inp.rec_idx, wl.order, wl.h, dt, wl.n_pml,
+                     wl.f0, vmax=vmax, round_f32=True)
+    prob = problem_from_sim(sim, nt, dt, wl.n_pml, snapshot="ckpt", ckpt_every=64)
+    run_forward(prob, f)
+    gca_t, gcb_t, _ = prob.adjoint(torch.as_tensor(res, dtype=torch.float32).cuda())
+    ge_t, gs_t = prob.eps_sigma_gradient(gca_t, gcb_t)
+    torch.cuda.synchronize()
+    assert prob.status() == mwtm.MW_OK
+    gca, gcb = gca_t.cpu().numpy(), gcb_t.cpu().numpy()
+    ge, gs = ge_t.cpu().numpy(), gs_t.cpu().numpy()
+    del prob, gca_t, gcb_t, ge_t, gs_t
+    sub = _subset_sim(inp, sel, dt, batched=True)
+    ck = sub.fwd_adj_ckpt(f[:, sel], res[:, sel], 64)
+    assert rel_l2(gca[sel], ck["gca"]) <= GRAD_TOL
+    assert rel_l2(gcb[sel], ck["gcb"]) <= GRAD_TOL
+    ge_o, gs_o = oracle.eps_sigma_grad(sub.ca, sub.cb, dt, ck["gca"], ck["gcb"])
+    assert rel_l2(ge[sel], ge_o) <= GRAD_TOL
+    assert rel_l2(gs[sel], gs_o) <= GRAD_TOL
+
+
 def test_workload3_all_shots_sampled_bf16():
     """1064x1064 order 8, all 16 shots, nt 150: fp32-storage gradients of
     shots 0 and 15 against the oracle, and the bf16-storage gradient error
