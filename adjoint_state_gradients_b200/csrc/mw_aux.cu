@@ -55,6 +55,10 @@ __global__ void k_inject_sample(float *__restrict__ field, int64_t numel,
                                 float *__restrict__ out_t) {
   const int s = blockIdx.x;
   float *e = field + (int64_t)s * numel;
+  // programmatic dependent launch (no-ops without the launch attribute):
+  // let the next stencil launch begin, then wait for the previous one
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (vals_t != nullptr) {
     const int64_t base = (int64_t)s * na;
     for (int k = threadIdx.x; k < na; k += blockDim.x) {
@@ -234,8 +238,10 @@ cudaError_t launch_inject_sample(float *field, int64_t numel, int S, const float
                                  const int64_t *idx_a, const int *lead, const int *next, int na,
                                  const int64_t *idx_b, int nb, float *out_t, cudaStream_t st) {
   if ((na == 0 || vals_t == nullptr) && (nb == 0 || out_t == nullptr)) return cudaSuccess;
-  k_inject_sample<<<S, 256, 0, st>>>(field, numel, na > 0 ? vals_t : nullptr, idx_a, lead, next,
-                                     na, idx_b, nb, nb > 0 ? out_t : nullptr);
+  const cudaError_t e = launch_dependent(k_inject_sample, S, 256, 0, st, field, numel,
+                                         na > 0 ? vals_t : nullptr, idx_a, lead, next, na, idx_b,
+                                         nb, nb > 0 ? out_t : nullptr);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }

@@ -18,6 +18,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/mw_tm.h"
 
 namespace mw {
@@ -202,6 +204,25 @@ struct BandTab {
 
 // count of kernel launches made by the library (mw_host.cu)
 void count_launches(int n);
+
+// Launch with programmatic stream serialization: the kernel may begin
+// launching while the previous kernel in the stream finishes; it must wait
+// (griddepcontrol.wait) before reading that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), int grid, int block, size_t smem,
+                             cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // stencil launchers (mw_stencil.cu); return a cudaError_t
 cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int store,

@@ -90,6 +90,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// Programmatic dependent launch: let the next kernel in the stream start
+// launching (its blocks then wait in grid_dep_wait), and wait for the
+// previous kernel's completion and memory before touching its results.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -320,10 +330,11 @@ __device__ __noinline__ void give_up_s(int *flags, uint32_t bars, Ring ring, int
   }
 }
 
-// Walk one item.  Every phase (Hz of row r, Hx of row r - P, E of row
-// y = r - 2P + 1) is computed on every iteration and only the stores are
-// predicated on the row ranges; BAND adds the CPML recursions and the
-// array-edge masks that interior items do not need.
+// Walk one item.  Per iteration: Hz of row r (owned rows), Hx of row r - P
+// (every row, queued for the E update's z-stencil), E of row y = r - 2P + 1
+// (owned rows); the row-range tests are warp-uniform, the per-lane ones only
+// predicate stores.  BAND adds the CPML recursions and the array-edge masks
+// that interior items do not need.
 template <int P, int STORE, int L, bool BAND>
 __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, const Item &it,
                                          FwdWarp &w, int cq_arr, float cqs) {
@@ -381,11 +392,23 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
         const bool e_row = (unsigned)(i - (4 * P - 2)) < (unsigned)rows;
         const bool hx_in = i >= it.hx_lo && i <= it.hx_hi;
 
-        // ---- Hz, row r: every lane, float4 at column c
-        {
+        // Ey of row r at this lane's column: the z-stencil queue (every row)
+        eq[u] = lds4s(st + (kF_EY + 4) * 4 + 16 * lane);
+
+        // ---- Hz, row r: every lane, float4 at column c (owned rows only; the
+        // E update reads the Hz of its own row)
+        if (own_r) {
           float wv[12];
-          win12s(st + kF_EY * 4 + 16 * lane, wv);
-          eq[u] = F4{{wv[4], wv[5], wv[6], wv[7]}};
+          {
+            const F4 lo = lds4s(st + kF_EY * 4 + 16 * lane);
+            const F4 hi = lds4s(st + (kF_EY + 8) * 4 + 16 * lane);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              wv[q] = lo.v[q];
+              wv[q + 4] = eq[u].v[q];
+              wv[q + 8] = hi.v[q];
+            }
+          }
           const F4 hz_old = lds4s(st + (kF_HZ + 4) * 4 + 16 * lane);
           const F4 cq = cq_arr ? lds4s(st + a.fo[kFoCqH] * 4 + 16 * lane) : splat4(cqs);
           F4 hn;
@@ -444,7 +467,7 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
         }
 
         // ---- E, row y = r - 2P + 1
-        {
+        if (e_row) {
           float wv[12];
           win12s(w.hring + ((u + 1) % NQ) * kFRing * 4 + 16 * wl - 16, wv);
           const F4 ca4 = lds4s(st + w.ca_o + 16 * lane - 16);
@@ -534,7 +557,7 @@ __global__ void __launch_bounds__(128) k_forward(const __grid_constant__ FwdMaps
   w.ring = Ring{0, 0u};
   const Geom &g = a.g;
   const int n_items = g.S * g.n_strips * g.n_chunks;
-  if (__any_sync(kFull, *reinterpret_cast<volatile int *>(a.flags + kFlagTimeout) != 0)) return;
+  grid_dep_launch();
   if (lane == 0) {
     for (int k = 0; k < NS; ++k)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(w.bars + 8 * k), "r"(1)
@@ -542,6 +565,8 @@ __global__ void __launch_bounds__(128) k_forward(const __grid_constant__ FwdMaps
     fence_mbar_init();
   }
   __syncwarp();
+  grid_dep_wait();  // everything below reads what earlier kernels wrote
+  if (__any_sync(kFull, *reinterpret_cast<volatile int *>(a.flags + kFlagTimeout) != 0)) return;
   const float cqs = cq_arr ? 0.f : __ldg(a.cq);
   // work items are claimed dynamically; the counter of the next launch is
   // reset here (the previous launch that used it has completed)
@@ -922,7 +947,7 @@ __global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_c
   w.ring = Ring{0, 0u};
   const Geom &g = a.g;
   const int n_items = g.S * g.n_strips * g.n_chunks;
-  if (__any_sync(kFull, *reinterpret_cast<volatile int *>(a.flags + kFlagTimeout) != 0)) return;
+  grid_dep_launch();
   if (lane == 0) {
     for (int k = 0; k < NS; ++k)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(w.bars + 8 * k), "r"(1)
@@ -930,6 +955,8 @@ __global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_c
     fence_mbar_init();
   }
   __syncwarp();
+  grid_dep_wait();  // everything below reads what earlier kernels wrote
+  if (__any_sync(kFull, *reinterpret_cast<volatile int *>(a.flags + kFlagTimeout) != 0)) return;
   const float cqs = cq_arr ? 0.f : __ldg(a.cq);
   int *ctr = a.flags + kCtrBase + a.ctr_slot;
   if (blockIdx.x == 0 && threadIdx.x == 0) a.flags[kCtrBase + (a.ctr_slot ^ 1)] = 0;
@@ -1036,7 +1063,9 @@ cudaError_t fwd_t(const FwdMaps &m, const StepArgs &a, bool batched, bool cq_arr
                   cudaStream_t st) {
   const size_t smem = (size_t)(32 + kWarpsPerCta * a.warp_floats) * sizeof(float) + 128;
   allow_big_smem(k_forward<P, STORE, kFwdL>, fwd_smem_flag<P, STORE>());
-  k_forward<P, STORE, kFwdL><<<grid, 128, smem, st>>>(m, a, batched ? 1 : 0, cq_arr ? 1 : 0);
+  const cudaError_t e = launch_dependent(k_forward<P, STORE, kFwdL>, grid, 128, smem, st, m, a,
+                                         batched ? 1 : 0, cq_arr ? 1 : 0);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }
@@ -1045,8 +1074,9 @@ cudaError_t adj_t(const AdjMaps &m, const StepArgs &a, bool batched, bool cq_arr
                   cudaStream_t st) {
   const size_t smem = (size_t)(32 + kAdjWarpsPerCta * a.warp_floats) * sizeof(float) + 128;
   allow_big_smem(k_adjoint<P, SNAP, kAdjL>, adj_smem_flag<P, SNAP>());
-  k_adjoint<P, SNAP, kAdjL><<<grid, 32 * kAdjWarpsPerCta, smem, st>>>(m, a, batched ? 1 : 0,
-                                                                       cq_arr ? 1 : 0);
+  const cudaError_t e = launch_dependent(k_adjoint<P, SNAP, kAdjL>, grid, 32 * kAdjWarpsPerCta,
+                                         smem, st, m, a, batched ? 1 : 0, cq_arr ? 1 : 0);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }
