@@ -372,25 +372,6 @@ Coef coef_of(const mw_params *p) {
   return k;
 }
 
-Prof prof_of(const mw_params *p, const float *cpml) {
-  const size_t ny = p->ny, nx = p->nx;
-  Prof r;
-  r.ay = cpml;
-  r.ayh = cpml + ny;
-  r.by = cpml + 2 * ny;
-  r.byh = cpml + 3 * ny;
-  r.ky = cpml + 4 * ny;
-  r.kyh = cpml + 5 * ny;
-  const float *x = cpml + 6 * ny;
-  r.ax = x;
-  r.axh = x + nx;
-  r.bx = x + 2 * nx;
-  r.bxh = x + 3 * nx;
-  r.kx = x + 4 * nx;
-  r.kxh = x + 5 * nx;
-  return r;
-}
-
 // ---- TMA tensor maps ---------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -745,7 +726,6 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   const Launch lc = plan(p, false);
   a.g = lc.g;
   a.c = coef_of(p);
-  a.pr = prof_of(p, cpml);
   a.ca = ca;
   a.cb = cb;
   a.cq = cq;
@@ -865,7 +845,6 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   StepArgs a{};
   a.g = la.g;
   a.c = coef_of(p);
-  a.pr = prof_of(p, cpml);
   a.ca = ca;
   a.cb = cb;
   a.cq = cq;
@@ -1165,7 +1144,6 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
     const Launch lc = plan(p, false);
     a.g = lc.g;
     a.c = coef_of(p);
-    a.pr = prof_of(p, cpml);
     a.ca = ca;
     a.cb = cb;
     a.cq = cq;

@@ -46,12 +46,6 @@ struct Coef {
   float cx[4], cy[4];
 };
 
-// CPML profiles (device): y axis then x axis; "h" = half node.
-struct Prof {
-  const float *ay, *ayh, *by, *byh, *ky, *kyh;
-  const float *ax, *axh, *bx, *bxh, *kx, *kxh;
-};
-
 // One state buffer (forward fields or their adjoints).
 struct Fields {
   float *ey, *hx, *hz;
@@ -69,7 +63,6 @@ enum { kAoCqR = 0, kAoCqH, kAoMx, kAoMze, kAoMzh, kAoCount };
 struct StepArgs {
   Geom g;
   Coef c;
-  Prof pr;
   Fields in, out;
   const float *ca, *cb, *cq;
   float cq_scalar;
@@ -85,9 +78,9 @@ struct StepArgs {
   int ctr_slot;       // work counter of this launch (flags[kCtrBase + ctr_slot])
   // CPML band coefficients (BandTab layout), float4-aligned, 1/k precomputed
   const float *bt;
-  // shared-memory layout of one warp (floats): stage size, band slot width
-  // (padded), band row width (the TMA box, 2*Wx)
-  int stage_floats, band_floats, warp_floats, band_box_floats;
+  // shared-memory layout of one warp (floats): stage size, warp area, band
+  // row width (the x-band memory TMA box, 2*Wx)
+  int stage_floats, warp_floats, band_box_floats;
   // forward only: optional stage slots (kFo*), Ca / Cb pair fetch and order
   int fo[kFoCount];
   int md_pair, md_swap;

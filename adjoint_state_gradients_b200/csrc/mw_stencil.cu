@@ -1001,7 +1001,6 @@ void fwd_layout_t(int Wx, bool cq_arr, StepArgs *a, size_t *smem) {
   int wf = (kFwdL + 1) * o + 2 * P * kFRing;
   wf = ((wf + 31) / 32) * 32;
   a->stage_floats = o;
-  a->band_floats = bw;
   a->warp_floats = wf;
   a->band_box_floats = 2 * Wx;
   *smem = (size_t)(32 + kWarpsPerCta * wf) * sizeof(float) + 128;
@@ -1029,7 +1028,6 @@ void adj_layout_t(int Wx, bool cq_arr, StepArgs *a, size_t *smem) {
   int wf = (kAdjL + 1) * o + kAPx + 2 * P * kARing;
   wf = ((wf + 31) / 32) * 32;
   a->stage_floats = o;
-  a->band_floats = 0;
   a->warp_floats = wf;
   a->band_box_floats = 2 * Wx;
   *smem = (size_t)(32 + kAdjWarpsPerCta * wf) * sizeof(float) + 128;
