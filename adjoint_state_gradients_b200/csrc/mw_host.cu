@@ -277,8 +277,8 @@ void interior_rect(Geom &g, int P) {
     return x0 - 8 < g.Wx || x0 + g.strip_cols + 8 > g.nx - g.Wx;
   };
   auto chunk_edge = [&](int k) {
-    const int ya = k * g.chunk_h;
-    const int yb = ya + g.chunk_h < g.ny ? ya + g.chunk_h : g.ny;
+    int ya, yb;
+    chunk_rows(g, k, &ya, &yb);
     return g.Wz > 0 && (ya - (2 * P - 1) < g.Wz || yb + 2 * P - 1 > g.ny - g.Wz);
   };
   int a = 0, b = g.n_strips;
@@ -333,24 +333,54 @@ Launch plan(const mw_params *p, bool adjoint) {
   const int warps_sm = stencil_slots_per_sm(p->order, adjoint, b.Wx, !p->cq_is_scalar);
   const int64_t slots = (int64_t)sm_count() * warps_sm;
   const int64_t cols_items = (int64_t)g.S * g.n_strips;
-  // Items are claimed dynamically by resident warps: time ~ total iterations
-  // spread over the slots plus one item of tail; each item walks its rows
-  // plus 4P - 2 warm-up rows.
+  // Items are claimed dynamically by resident warps.  Each item walks its
+  // rows plus 4P - 2 warm-up rows.  Model: the claimed work spread over the
+  // slots, plus the duration of the items claimed last (the tail); with n1
+  // long chunks of H1 rows first and short chunks of H2 rows after them, the
+  // last long items must also end in time:
+  //   cost = max(W / slots + (H2 + w), W_long / slots + (H1 + w)).
   const int w = 4 * P - 2;
-  int best_ch = p->ny;
+  const double cols = (double)cols_items, sl = (double)slots;
+  int best_h1 = p->ny, best_h2 = p->ny, best_n1 = 1;
   double best_cost = 1e300;
-  for (int ch = 8; ch <= p->ny + 7; ch += (ch < 64 ? 1 : 4)) {
-    const int nc = (p->ny + ch - 1) / ch;
-    const int chh = (p->ny + nc - 1) / nc;
-    const double items = (double)cols_items * nc;
-    const double cost = items * (chh + w) / (double)slots + (chh + w);
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best_ch = chh;
+  for (int h1 = 8; h1 <= p->ny + 7; h1 += (h1 < 64 ? 1 : 4)) {
+    const int n1_max = (p->ny + h1 - 1) / h1;
+    for (int n1 = 1; n1 <= n1_max; ++n1) {
+      const int rest = p->ny - n1 * h1;
+      const double wl = cols * n1 * (h1 + w);
+      if (rest <= 0) {  // long chunks only (the last one ragged)
+        const double cost = wl / sl + (h1 + w);
+        if (cost < best_cost - 1e-9) {
+          best_cost = cost;
+          best_h1 = h1;
+          best_h2 = h1;
+          best_n1 = n1;
+        }
+        continue;
+      }
+      const int h2_max = h1 - 1 < 64 ? h1 - 1 : 64;
+      for (int h2 = 4; h2 <= h2_max; ++h2) {
+        const int n2 = (rest + h2 - 1) / h2;
+        const double W = wl + cols * n2 * (h2 + w);
+        const double a = W / sl + (h2 + w), b = wl / sl + (h1 + w);
+        const double cost = a > b ? a : b;
+        if (cost < best_cost - 1e-9) {
+          best_cost = cost;
+          best_h1 = h1;
+          best_h2 = h2;
+          best_n1 = n1;
+        }
+      }
     }
   }
-  g.chunk_h = best_ch;
-  g.n_chunks = (p->ny + g.chunk_h - 1) / g.chunk_h;
+  g.chunk_h = best_h1;
+  g.chunk_h2 = best_h2;
+  g.n_big = best_n1;
+  {
+    const int rest = p->ny - best_n1 * best_h1;
+    g.n_chunks = rest > 0 ? best_n1 + (rest + best_h2 - 1) / best_h2 : (p->ny + best_h1 - 1) / best_h1;
+    if (rest <= 0) g.n_big = g.n_chunks;
+  }
   interior_rect(g, P);
   const int64_t items = cols_items * g.n_chunks;
   const int wpc = adjoint ? kAdjWarpsPerCta : kWarpsPerCta;

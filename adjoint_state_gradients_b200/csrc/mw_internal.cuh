@@ -32,7 +32,10 @@ constexpr int kAdjWarpsPerCta = 5; // adjoint CTA: 5 warps
 struct Geom {
   int ny, nx, S;
   int Wx, Wz;         // band widths (0: no CPML band)
-  int strip_cols, n_strips, n_chunks, chunk_h;
+  int strip_cols, n_strips, n_chunks;
+  // row chunks: n_big chunks of chunk_h rows, then chunks of chunk_h2 rows
+  // (the last one ragged); the short chunks are claimed last
+  int chunk_h, chunk_h2, n_big;
   // strips [is_lo, is_hi) and chunks [ic_lo, ic_hi) form the interior
   // rectangle (items whose walk touches no band and no array edge)
   int is_lo, is_hi, ic_lo, ic_hi;
@@ -127,6 +130,15 @@ enum AdjMap {
 struct AdjMaps {
   CUtensorMap map[kAdjMaps];
 };
+
+// Rows [ya, yb) of row chunk k.
+__host__ __device__ inline void chunk_rows(const Geom &g, int k, int *ya, int *yb) {
+  const bool big = k < g.n_big;
+  const int a = big ? k * g.chunk_h : g.n_big * g.chunk_h + (k - g.n_big) * g.chunk_h2;
+  const int h = big ? g.chunk_h : g.chunk_h2;
+  *ya = a;
+  *yb = a + h < g.ny ? a + h : g.ny;
+}
 
 // Claim order of the work items: items touching a band or an array edge
 // first, then the interior rectangle; the shot index runs fastest, then the

@@ -184,8 +184,7 @@ __device__ __forceinline__ bool make_item(const Geom &g, int item, bool batched,
   item_coords(g, item, &it.s, &strip, &chunk);
   it.sm = batched ? it.s : 0;
   it.x0 = strip * g.strip_cols;
-  it.ya = chunk * g.chunk_h;
-  it.yb = min(g.ny, it.ya + g.chunk_h);
+  chunk_rows(g, chunk, &it.ya, &it.yb);
   it.r0 = it.ya - (2 * P - 1);
   it.n_it = (it.yb - it.ya) + 4 * P - 2;
   const bool near_x = it.x0 - 8 < g.Wx || it.x0 + g.strip_cols + 8 > g.nx - g.Wx;
