@@ -1057,6 +1057,14 @@ int mw_profile_enable(int32_t enable) {
   return MW_OK;
 }
 
+int mw_selftest_wait_timeout(void *workspace, void *stream) {
+  g_err.clear();
+  if (!workspace) return fail(MW_ERR_WORKSPACE, "workspace is NULL");
+  if (((uintptr_t)workspace) % 256 != 0) return fail(MW_ERR_WORKSPACE, "workspace not 256-aligned");
+  MW_CUDA(launch_wait_selftest((int *)workspace, (cudaStream_t)stream));
+  return MW_OK;
+}
+
 int mw_snapshot_encode(int32_t snap_mode, int64_t n, const float *x_dev, void *out_dev,
                        void *stream) {
   g_err.clear();

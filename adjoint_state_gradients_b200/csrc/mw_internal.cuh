@@ -238,6 +238,8 @@ cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int s
 // snapshot storage encoding of n floats (n % 4 == 0) with the forward's
 // conversion (kStoreBF16 or kStoreFP8)
 cudaError_t launch_snap_encode(int store, int64_t n, const float *x, void *out, cudaStream_t st);
+// a stage wait that nothing completes (bounded; sets the timeout flag)
+cudaError_t launch_wait_selftest(int *flags, cudaStream_t st);
 // forward / adjoint: the full stage layout (optional slots for a Cq array and
 // bands)
 void forward_layout(int order, int Wx, bool cq_array, StepArgs *a, size_t *smem_bytes);

@@ -1101,6 +1101,22 @@ cudaError_t adj_snap(const AdjMaps &m, const StepArgs &a, int snap, bool batched
   return cudaErrorInvalidValue;
 }
 
+// A stage wait that nothing completes: one expected-byte count that no copy
+// ever delivers.  Exercises the bounded wait every stencil kernel uses and
+// the timeout report, without a fault and with no copy in flight.
+__global__ void k_wait_selftest(int *flags) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b), "r"(1) : "memory");
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) expect_tx_s(b, 16);
+  __syncwarp();
+  if (!mbar_wait_s(b, 0) && threadIdx.x == 0) atomicOr(flags + kFlagTimeout, 1);
+}
+
 // Snapshot encoding of n floats with the forward's store conversion.
 template <int STORE>
 __global__ void k_snap_encode(const float *__restrict__ x, void *out, int64_t n4) {
@@ -1156,6 +1172,12 @@ cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int s
     case 8: return adj_snap<4>(m, a, snap, batched, cq_array, grid, st);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_wait_selftest(int *flags, cudaStream_t st) {
+  k_wait_selftest<<<1, 32, 0, st>>>(flags);
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_snap_encode(int store, int64_t n, const float *x, void *out, cudaStream_t st) {

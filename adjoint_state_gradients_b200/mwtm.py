@@ -73,6 +73,7 @@ SIGNATURES = [
     ("mw_profile_read", ctypes.c_int, [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double),
                                        ctypes.c_int32]),
     ("mw_launch_count", ctypes.c_int64, []),
+    ("mw_selftest_wait_timeout", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     ("mw_snapshot_encode", ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p,
                                           ctypes.c_void_p, ctypes.c_void_p]),
     ("mw_workspace_init", ctypes.c_int, [_VP, ctypes.c_size_t, _VP]),
@@ -238,3 +239,8 @@ def snapshot_encode(snap_mode, x, out, stream=None):
     SNAP_FP8) into `out` (2 or 1 bytes per value) on the device."""
     return check(lib().mw_snapshot_encode(int(snap_mode), x.numel(), ptr(x), ptr(out),
                                           stream_ptr(stream)))
+
+
+def selftest_wait_timeout(workspace, stream=None):
+    """Run the bounded-wait self-test kernel on `workspace` (see mw_tm.h)."""
+    return check(lib().mw_selftest_wait_timeout(ptr(workspace), stream_ptr(stream)))

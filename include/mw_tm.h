@@ -272,6 +272,16 @@ int mw_profile_read(int64_t *counts, double *total_ms, int32_t n_classes);
  * entry points, all devices).  Host counter; no synchronization. */
 int64_t mw_launch_count(void);
 
+/* Failure-detection self-test (no counterpart on the pages): launches one
+ * kernel whose stage wait nothing completes (an expected byte count no copy
+ * delivers).  The wait gives up after its bounded poll count (about half a
+ * second), records the timeout in the workspace's status words and returns,
+ * exactly as a stencil kernel does when one of its copies never lands.  The
+ * next mw_sync_status reports MW_ERR_TIMEOUT and clears it; until then the
+ * stencil kernels launched on this workspace return at once.  No copy is in
+ * flight when the kernel ends and the context stays usable. */
+int mw_selftest_wait_timeout(void *workspace_dev, void *stream);
+
 /* Snapshot storage encoding (page: maxwell.cu, the bf16 / "FP8 E4M3"
  * storage helpers used by forward_kernel_e_with_storage_bf16 / _fp8).
  * Rounds n float32 values x_dev[0..n) to the storage format of snap_mode
