@@ -31,7 +31,17 @@ WORKLOAD = 4
 METRIC = "Gcell-updates/s (fwd; fwd+adjoint+grad) on 1 B200 and % of HBM roofline"
 UNIT = "Gcell-updates/s"
 PROFILES = os.path.join(ROOT, "profiles")
-STENCIL_SRC = os.path.join(ROOT, "adjoint_state_gradients_b200", "csrc", "mw_stencil.cu")
+# the stencil kernels' source: the recorded ncu traffic is valid for it only
+STENCIL_SRCS = [os.path.join(ROOT, "adjoint_state_gradients_b200", "csrc", f)
+                for f in ("mw_device.cuh", "mw_stencil.cu")]
+
+
+def stencil_sha() -> str:
+    h = hashlib.sha256()
+    for path in STENCIL_SRCS:
+        with open(path, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def parse():
@@ -136,9 +146,7 @@ def traffic_record():
     try:
         with open(os.path.join(PROFILES, "adjoint_traffic.json")) as fh:
             d = json.load(fh)
-        with open(STENCIL_SRC, "rb") as fh:
-            h = hashlib.sha256(fh.read()).hexdigest()[:16]
-        if d.get("stencil_sha") != h:
+        if d.get("stencil_sha") != stencil_sha():
             return None
         return float(d["dram_bytes_per_launch_full"])
     except Exception:
