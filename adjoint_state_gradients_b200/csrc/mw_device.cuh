@@ -172,5 +172,47 @@ __device__ __forceinline__ F4 snap_lds_s(uint32_t addr) {
   }
 }
 
+// Predicated forms (no branch around them): the store or copy happens only
+// where p holds; the address may be anything where it does not.
+__device__ __forceinline__ void st4p(bool p, float *ptr, const F4 &v) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n"
+      " @q st.global.v4.f32 [%1], {%2, %3, %4, %5};\n}\n" ::"r"((int)p),
+      "l"(ptr), "f"(v.v[0]), "f"(v.v[1]), "f"(v.v[2]), "f"(v.v[3])
+      : "memory");
+}
+__device__ __forceinline__ void sts4p(bool p, uint32_t addr, const F4 &v) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n"
+      " @q st.shared.v4.f32 [%1], {%2, %3, %4, %5};\n}\n" ::"r"((int)p),
+      "r"(addr), "f"(v.v[0]), "f"(v.v[1]), "f"(v.v[2]), "f"(v.v[3])
+      : "memory");
+}
+// Snapshot row store (4 cells) where p holds.
+template <int STORE>
+__device__ __forceinline__ void snap_store_p(bool p, void *base, int64_t elem, const F4 &v) {
+  if constexpr (STORE == kStoreF32) {
+    st4p(p, reinterpret_cast<float *>(base) + elem, v);
+  } else if constexpr (STORE == kStoreBF16) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(v.v[0], v.v[1]);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(v.v[2], v.v[3]);
+    const uint32_t a = *reinterpret_cast<uint32_t *>(&lo), b = *reinterpret_cast<uint32_t *>(&hi);
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n @q st.global.v2.u32 [%1], {%2, %3};\n}\n" ::"r"(
+            (int)p),
+        "l"(reinterpret_cast<__nv_bfloat16 *>(base) + elem), "r"(a), "r"(b)
+        : "memory");
+  } else if constexpr (STORE == kStoreFP8) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v.v[0], v.v[1]), __NV_SATFINITE,
+                                                 __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v.v[2], v.v[3]), __NV_SATFINITE,
+                                                 __NV_E4M3);
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n @q st.global.u32 [%1], %2;\n}\n" ::"r"((int)p),
+        "l"(reinterpret_cast<uint8_t *>(base) + elem), "r"(lo | (hi << 16))
+        : "memory");
+  }
+}
+
 }  // namespace dev
 }  // namespace mw

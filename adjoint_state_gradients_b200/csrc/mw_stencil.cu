@@ -302,10 +302,10 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
               mn.v[q] = fmaf(bh.v[q], mn.v[q], ah.v[q] * d);
               hn.v[q] = fmaf(cq.v[q], fmaf(d, rk.v[q], mn.v[q]), hz_old.v[q]);
             }
-            if (own && own_r) st4(a.out.mxh_node + xbw + (int64_t)(it.r0 + i) * 2 * a.g.Wx, mn);
+            st4p(own, a.out.mxh_node + xbw + (int64_t)(it.r0 + i) * 2 * a.g.Wx, mn);
           }
           sts4s(w.hring + u * kFRing * 4 + 16 * lane, c_ok ? hn : zero4());
-          if (own && own_r) st4(hz_o + ro, hn);
+          st4p(own, hz_o + ro, hn);
         }
 
         // ---- Hx, row r - P (z-stencil from the Ey queue)
@@ -333,14 +333,14 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
                 mz.v[q] = fmaf(byh, mz.v[q], ayh * d.v[q]);
                 d.v[q] = fmaf(d.v[q], rkyh, mz.v[q]);
               }
-              if (own && hx_own) st4(a.out.mzh_node + zbw + (int64_t)zr * nx, mz);
+              st4p(own && hx_own, a.out.mzh_node + zbw + (int64_t)zr * nx, mz);
             }
           }
           F4 hn;
 #pragma unroll
           for (int q = 0; q < 4; ++q) hn.v[q] = fmaf(-cq.v[q], d.v[q], hx_old.v[q]);
           hq[u] = hx_in ? hn : zero4();
-          if (own && hx_own) st4(hx_o + (ro - P * nx), hn);
+          st4p(own && hx_own, hx_o + (ro - P * nx), hn);
         }
 
         // ---- E, row y = r - 2P + 1
@@ -371,7 +371,7 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
                 mx.v[q] = fmaf(bx.v[q], mx.v[q], ax.v[q] * cx.v[q]);
                 cx.v[q] = fmaf(cx.v[q], rk.v[q], mx.v[q]);
               }
-              if (own && e_row) st4(a.out.mxe_node + xbw + (int64_t)y * 2 * a.g.Wx, mx);
+              st4p(own, a.out.mxe_node + xbw + (int64_t)y * 2 * a.g.Wx, mx);
             }
             const int zr = e_row ? zband_row(y, a.g.ny, a.g.Wz) : -1;
             if (zr >= 0) {
@@ -383,7 +383,7 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
                 mz.v[q] = fmaf(by, mz.v[q], ay * cz.v[q]);
                 cz.v[q] = fmaf(cz.v[q], rky, mz.v[q]);
               }
-              if (own) st4(a.out.mze_node + zbw + (int64_t)zr * nx, mz);
+              st4p(own, a.out.mze_node + zbw + (int64_t)zr * nx, mz);
             }
           }
           F4 curl, en;
@@ -392,14 +392,14 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
             curl.v[q] = cx.v[q] - cz.v[q];
             en.v[q] = fmaf(ca4.v[q], e_old.v[q], cb4.v[q] * curl.v[q]);
           }
-          if (own && e_row) {
+          {
             const int off = ro - (2 * P - 1) * nx;
             if constexpr (STORE != kStoreNone) {
               const int64_t so = ((int64_t)it.s * a.g.ny + (it.r0 + i - 2 * P + 1)) * a.snap_pitch + c;
-              snap_store<STORE>(a.snap_e, so, e_old);
-              snap_store<STORE>(a.snap_c, so, curl);
+              snap_store_p<STORE>(own, a.snap_e, so, e_old);
+              snap_store_p<STORE>(own, a.snap_c, so, curl);
             }
-            st4(ey_o + off, en);
+            st4p(own, ey_o + off, en);
           }
         }
         __syncwarp();
@@ -412,7 +412,7 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
 }
 
 template <int P, int STORE, int L>
-__global__ void __launch_bounds__(128) k_forward(const __grid_constant__ FwdMaps m,
+__global__ void __launch_bounds__(128, P <= 3 ? 5 : 4) k_forward(const __grid_constant__ FwdMaps m,
                                                  const StepArgs a, const int batched,
                                                  const int cq_arr) {
   constexpr int NS = L + 1;
@@ -630,14 +630,14 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
                 pz.v[q] = fmaf(ay, M.v[q], -gv.v[q] * rky);
                 M.v[q] *= by;
               }
-              if (own && own_r) st4(a.out.mze_node + zbw + (int64_t)zr * nx, M);
+              st4p(own && own_r, a.out.mze_node + zbw + (int64_t)zr * nx, M);
             }
           }
           pq[u] = pz;
         }
         // ---- owned rows: gradients (lam = lambda_E^{t+1}) and px
         if (own_r) {
-          if (own) {
+          {  // every lane computes (in-bounds staged reads); owned lanes store
             const uint32_t sbase = st + kA_SS * 4;
             constexpr uint32_t selem = SNAP == kStoreF32 ? 4 : SNAP == kStoreBF16 ? 2 : 1;
             constexpr uint32_t sfield = 112 * selem, sstep = 4 * selem;
@@ -652,8 +652,8 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
                 gcb.v[q] = fmaf(sc.v[q], lam.v[q], gcb.v[q]);
               }
             }
-            st4(gca_o + ro, gca);
-            st4(gcb_o + ro, gcb);
+            st4p(own, gca_o + ro, gca);
+            st4p(own, gcb_o + ro, gcb);
           }
           F4 px = gv;
           if constexpr (BAND) {
@@ -667,7 +667,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
                 px.v[q] = fmaf(ax.v[q], M.v[q], gv.v[q] * rk.v[q]);
                 M.v[q] *= bx.v[q];
               }
-              if (own) st4(a.out.mxe_node + xw + (int64_t)r * 2 * a.g.Wx + pb, M);
+              st4p(own, a.out.mxe_node + xw + (int64_t)r * 2 * a.g.Wx + pb, M);
             }
           }
           sts4s(w.prow + 16 * lane, pc_ok ? px : zero4());
@@ -686,7 +686,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
             lhz.v[q] = lhz_old.v[q] - d_half<P>(wv, q, a.c.cx);
             v.v[q] = cq.v[q] * lhz.v[q];
           }
-          if (q_own) st4(hz_o + ro, lhz);
+          st4p(q_own, hz_o + ro, lhz);
           if constexpr (BAND) {
             if (qb >= 0) {
               F4 M = lds4s(st + (a.ao[kAoMx] + qb) * 4);
@@ -699,10 +699,10 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
                 v.v[q] = fmaf(ah.v[q], M.v[q], vq * rk.v[q]);
                 M.v[q] *= bh.v[q];
               }
-              if (q_own) st4(a.out.mxh_node + xw + (int64_t)r * 2 * a.g.Wx + qb, M);
+              st4p(q_own, a.out.mxh_node + xw + (int64_t)r * 2 * a.g.Wx + qb, M);
             }
           }
-          if (q_lane) sts4s(w.qring + u * kARing * 4 + 16 * lane, qc_ok ? v : zero4());
+          sts4p(q_lane, w.qring + u * kARing * 4 + 16 * lane, qc_ok ? v : zero4());
         }
 
         // ---- lamHx and qz of row r - P (owned lanes)
@@ -720,7 +720,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
             lh.v[q] = lhx.v[q] - d;
             qz.v[q] = -cq.v[q] * lh.v[q];
           }
-          if (own && hx_own) st4(hx_o + (ro - P * nx), lh);
+          st4p(own && hx_own, hx_o + (ro - P * nx), lh);
           if constexpr (BAND) {
             const int zr = hx_in ? zband_row(r - P, ny, a.g.Wz) : -1;
             if (zr >= 0) {
@@ -734,7 +734,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
                 qz.v[q] = fmaf(ayh, M.v[q], vq * rkyh);
                 M.v[q] *= byh;
               }
-              if (own && hx_own) st4(a.out.mzh_node + zbw + (int64_t)zr * nx, M);
+              st4p(own && hx_own, a.out.mzh_node + zbw + (int64_t)zr * nx, M);
             }
           }
           qq[u] = hx_in ? qz : zero4();
@@ -754,7 +754,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
                         dz);
             en.v[q] = cl[(u + 1) % NQ].v[q] - d_int<P>(wv, q, a.c.cx) - dz;
           }
-          if (own) st4(ey_o + (ro - (2 * P - 1) * nx), en);
+          st4p(own, ey_o + (ro - (2 * P - 1) * nx), en);
         }
         __syncwarp();
         w.ring.next(NS);
