@@ -5,7 +5,11 @@ segment replay.  One step = one whole sweep over one batch of 8 shots:
 forward (records + checkpoints), residual and misfit, replayed adjoint with
 fused per-shot gradients, shot reduction of dJ/dCa and dJ/dCb.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload 1..5]
+
+--workload picks another of the five workloads (default 4, the headline):
+1 and 2 store fp32 snapshots, 3 bf16 snapshots, 5 times the forward alone
+(records of 256 shots with per-shot models).
 
 Prints one JSON line (rank 0).  --impl reference times the fp64 CPU oracle
 (the reference arm) on a bounded sample of the same workload.  Multi-GPU runs
@@ -53,6 +57,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--nt", type=int, default=None, help="override nt (profiling runs only)")
+    ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5],
+                    help="workload to time (default: the 2048^2 order-4 checkpointed sweep)")
     return ap.parse_args()
 
 
@@ -67,14 +73,37 @@ def dist_env():
 # algorithmic bytes per cell-update (fixed before tuning)
 
 
-def alg_bytes(wl, S, C):
-    """Bytes per cell-update of each pass of the checkpointed sweep (fp32)."""
-    band = 2.0 * wl.n_pml / wl.nx + 2.0 * wl.n_pml / wl.ny
-    model = 8.0 / S  # Ca, Cb shared by the shots
-    fwd = 24.0 + model + 16.0 * band + 28.0 / C           # + checkpoint write
-    replay = 24.0 + model + 16.0 * band + 8.0 + 28.0 / C  # + fp32 snapshot store + ckpt read
-    adj = 24.0 + model + 16.0 * band + 8.0 + 16.0         # + snapshot read + grad RMW
-    return fwd, replay, adj
+def alg_bytes(wl, S):
+    """Bytes per cell-update of each pass of the workload's sweep (fp32 fields):
+    state read + write 24 B, Ca and Cb (shared by the shots unless the model is
+    batched), the CPML band memories, snapshot write / read (8, 4 or 2 B), the
+    per-shot gradient read-modify-write 16 B, checkpoint copies 28 / C B."""
+    band = 16.0 * (2.0 * wl.n_pml / wl.nx + 2.0 * wl.n_pml / wl.ny)
+    model = 8.0 if wl.batched else 8.0 / S
+    base = 24.0 + model + band
+    if wl.snapshot == "ckpt":
+        C = wl.ckpt_every
+        return {"forward": base + 28.0 / C, "replay": base + 8.0 + 28.0 / C,
+                "adjoint": base + 8.0 + 16.0}
+    if wl.snapshot == "none":
+        return {"forward": base}
+    sb = {"fp32": 8.0, "bf16": 4.0, "fp8": 2.0}[wl.snapshot]
+    return {"forward": base + sb, "adjoint": base + sb + 16.0}
+
+
+# the library's per-launch timing classes: 0 forward, 1 forward with snapshot
+# store, 2 adjoint; which class each pass of a sweep uses
+def pass_classes(wl):
+    if wl.snapshot == "ckpt":
+        return {"forward": 0, "replay": 1, "adjoint": 2}
+    if wl.snapshot == "none":
+        return {"forward": 0}
+    return {"forward": 1, "adjoint": 2}
+
+
+def sample_steps(wl, target_cell_updates):
+    """Steps of a one-shot oracle sample worth about target_cell_updates."""
+    return int(max(16, min(wl.nt, target_cell_updates // (wl.ny * wl.nx))))
 
 
 # ----------------------------------------------------------------------------
@@ -157,12 +186,13 @@ def traffic_record():
 # CPU (oracle) baseline: bounded sample of the same workload
 
 
-def oracle_sample(nt_sample=48, C=16):
-    """Time the fp64 oracle on one shot of the workload for nt_sample steps
-    (forward with checkpoints, replay, adjoint)."""
+def oracle_sample(number, nt_sample):
+    """Time the fp64 oracle on one shot of workload `number` for nt_sample
+    steps of its sweep (checkpointed forward + replay + adjoint, forward with
+    snapshots + adjoint, or the forward alone)."""
     import oracle
     from adjoint_state_gradients_b200 import synth
-    inp = synth.make_inputs(WORKLOAD, n_shots=1)
+    inp = synth.make_inputs(number, n_shots=1)
     wl = inp.wl
     vmax = oracle.c0() / math.sqrt(inp.eps_min)
     dt = wl.cfl_fraction * oracle.cfl_dt(wl.order, wl.h, wl.h, vmax)
@@ -175,11 +205,28 @@ def oracle_sample(nt_sample=48, C=16):
     f = inp.wavelet(dt, nt_sample)
     res = synth.rng(7).normal(size=(nt_sample, 1, wl.n_rec))
     t0 = time.perf_counter()
-    sim.fwd_adj_ckpt(f, res, C)
+    if wl.snapshot == "ckpt":
+        sim.fwd_adj_ckpt(f, res, wl.ckpt_every)
+        what = f"checkpoint every {wl.ckpt_every}: forward + replay + adjoint"
+    elif wl.snapshot == "none":
+        sim.forward(f)
+        what = "forward, records only"
+    else:
+        fw = sim.forward(f, snapshots=True)
+        sim.adjoint(res, fw["snap_ey"], fw["snap_curl"])
+        what = "forward with snapshots + adjoint"
     el = time.perf_counter() - t0
     cells = sim.ny * sim.nx * nt_sample
     return cells / el / 1e9, el, oracle.num_threads(), \
-        f"1 of 8 shots, first {nt_sample} of 4000 steps, checkpoint every {C}: forward + replay + adjoint"
+        f"1 of {wl.n_shots} shots, first {nt_sample} of {wl.nt} steps, {what}"
+
+
+def snapshot_desc(wl):
+    if wl.snapshot == "ckpt":
+        return f"checkpoint every {wl.ckpt_every} steps + segment replay"
+    if wl.snapshot == "none":
+        return "none (records only, forward throughput)"
+    return f"every step, {wl.snapshot}, on the GPU"
 
 
 def run_reference(args):
@@ -187,10 +234,10 @@ def run_reference(args):
     if rank != 0:
         return
     from adjoint_state_gradients_b200 import synth
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = synth.WORKLOADS[args.workload]
     vals, els = [], []
     for i in range(args.warmup + args.steps):
-        v, el, cores, sample = oracle_sample(nt_sample=24, C=8)
+        v, el, cores, sample = oracle_sample(args.workload, sample_steps(wl, 0.3e9))
         if i >= args.warmup:
             vals.append(v)
             els.append(el)
@@ -201,7 +248,7 @@ def run_reference(args):
         "ms_per_step": round(1000 * sum(els) / len(els), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "grid": [wl.ny, wl.nx], "order": wl.order, "nt": wl.nt,
-                   "shots_per_gpu": wl.n_shots, "snapshots": "checkpoint every 64 + replay"},
+                   "shots_per_gpu": wl.n_shots, "snapshots": snapshot_desc(wl)},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -232,36 +279,42 @@ def main():
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
 
-    wl = synth.WORKLOADS[WORKLOAD]
+    number = args.workload
+    wl = synth.WORKLOADS[number]
     nt = args.nt or wl.nt
     S = wl.n_shots
+    grad = wl.snapshot != "none"   # workload 5 times the forward alone
     # weak scaling: every rank simulates its own block of S shots of one
     # survey of S * world shots (sources spread over the interior)
     lo, hi = shard.shot_block(S * world, rank, world)
-    inp = synth.make_inputs(WORKLOAD, n_shots=hi - lo, survey_shots=S * world, first_shot=lo)
+    if number == 4:
+        inp = synth.make_inputs(number, n_shots=hi - lo, survey_shots=S * world, first_shot=lo)
+    else:  # the other workloads' shots are the same set on every rank
+        inp = synth.make_inputs(number)
     c0 = 299792458.0
     vmax = c0 / math.sqrt(inp.eps_min)
     dt = wl.cfl_fraction * mwtm.cfl_dt(wl.order, wl.h, wl.h, vmax)
     C = wl.ckpt_every
 
     prob = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
-                       vmax=vmax, snapshot="ckpt", ckpt_every=C)
+                       vmax=vmax, snapshot=wl.snapshot, ckpt_every=max(C, 1), batched=wl.batched)
     f_host = inp.wavelet(dt, nt).astype(np.float32)
     eps_h = inp.eps_r.astype(np.float32)
     sig_h = inp.sigma.astype(np.float32)
     # observed data from the perturbed model (setup, outside the timed region)
     obs = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
-                      vmax=vmax, snapshot="none")
+                      vmax=vmax, snapshot="none", batched=wl.batched)
     obs.set_model_eps_sigma(inp.eps_r_true.astype(np.float32), sig_h, f0=wl.f0)
     f_dev = torch.as_tensor(f_host, device=dev)
     d_obs = obs.forward(f_dev).clone()
     del obs
     torch.cuda.synchronize()
     prob.set_model_eps_sigma(eps_h, sig_h, f0=wl.f0)
-    gca = torch.empty((wl.ny, wl.nx), device=dev)
-    gcb = torch.empty((wl.ny, wl.nx), device=dev)
-    gca_s = torch.empty((S, wl.ny, wl.nx), device=dev)
-    gcb_s = torch.empty((S, wl.ny, wl.nx), device=dev)
+    gshape = (wl.ny, wl.nx) if grad else (1,)
+    gca = torch.empty(gshape, device=dev)
+    gcb = torch.empty(gshape, device=dev)
+    gca_s = torch.empty((S, wl.ny, wl.nx) if grad else (1,), device=dev)
+    gcb_s = torch.empty((S, wl.ny, wl.nx) if grad else (1,), device=dev)
     rec = torch.empty((nt, S, wl.n_rec), device=dev)
     res = torch.empty_like(rec)
     J = torch.zeros(1, dtype=torch.float64, device=dev)
@@ -272,6 +325,8 @@ def main():
         if ev_fwd is not None:
             ev_fwd.record(stream)
         prob.residual(rec, d_obs, res=res, J=J)
+        if not grad:
+            return
         gca_s.zero_()
         gcb_s.zero_()
         prob.adjoint(res, gca=gca_s, gcb=gcb_s)
@@ -330,16 +385,22 @@ def main():
     cells = wl.ny * wl.nx * nt * S * world
     value = cells * args.steps / (total_ms / 1e3) / 1e9
     value_fwd = cells * args.steps / (fwd_ms / 1e3) / 1e9
-    b_fwd, b_rep, b_adj = alg_bytes(wl, S, C)
+    passes = alg_bytes(wl, S)
+    classes = pass_classes(wl)
     peak, peak_kind = measured_peaks()
-    sweep_bytes = (b_fwd + b_rep + b_adj) * cells * args.steps
+    sweep_bytes = sum(passes.values()) * cells * args.steps
     sweep_frac = sweep_bytes / (total_ms / 1e3) / 1e9 / peak / world
-    adj_launch_ms = ms[2] / max(counts[2], 1)
-    adj_bytes = b_adj * wl.ny * wl.nx * S
-    achieved = adj_bytes / (adj_launch_ms / 1e3) / 1e9
-    rep_launch_ms = ms[1] / max(counts[1], 1)
-    fwd_launch_ms = ms[0] / max(counts[0], 1)
-    traffic = traffic_record()
+    launch_ms = {k: ms[c] / max(counts[c], 1) for k, c in classes.items()}
+    top = "adjoint" if grad else "forward"   # the dominant kernel
+    top_launch_ms = launch_ms[top]
+    top_bytes = passes[top] * wl.ny * wl.nx * S
+    achieved = top_bytes / (top_launch_ms / 1e3) / 1e9
+    # the recorded ncu traffic is that of the 8-shot order-4 adjoint launch
+    traffic = traffic_record() if number == WORKLOAD else None
+    kname = {("adjoint", "fp32"): "kStoreF32", ("adjoint", "ckpt"): "kStoreF32",
+             ("adjoint", "bf16"): "kStoreBF16", ("adjoint", "fp8"): "kStoreFP8"}
+    kernel_name = (f"k_adjoint<{wl.order // 2}, {kname[(top, wl.snapshot)]}, 1>" if grad
+                   else f"k_forward<{wl.order // 2}, kStoreNone, 1>")
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -348,7 +409,10 @@ def main():
         f_p, eps_p, sig_p = pin(f_host), pin(eps_h), pin(sig_h)
         dobs_p = d_obs.cpu().pin_memory()
         outs = [torch.empty(1, dtype=torch.float64).pin_memory(),
-                torch.empty((wl.ny, wl.nx)).pin_memory(), torch.empty((wl.ny, wl.nx)).pin_memory()]
+                torch.empty(gshape).pin_memory(), torch.empty(gshape).pin_memory()]
+        if not grad:  # records-only workload: the result is the records
+            outs = [torch.empty(1, dtype=torch.float64).pin_memory(),
+                    torch.empty(rec.shape).pin_memory()]
 
         def e2e_step():
             prob.set_model_eps_sigma(eps_p.to(dev, non_blocking=True), sig_p.to(dev, non_blocking=True),
@@ -357,13 +421,14 @@ def main():
             do = dobs_p.to(dev, non_blocking=True)
             prob.forward(fd, rec=rec)
             prob.residual(rec, do, res=res, J=J)
-            gca_s.zero_()
-            gcb_s.zero_()
-            prob.adjoint(res, gca=gca_s, gcb=gcb_s)
-            prob.combine(gca_s, out=gca)
-            prob.combine(gcb_s, out=gcb)
-            shard.sum_over_ranks_(gca, gcb)
-            for o, src in zip(outs, (J, gca, gcb)):
+            if grad:
+                gca_s.zero_()
+                gcb_s.zero_()
+                prob.adjoint(res, gca=gca_s, gcb=gcb_s)
+                prob.combine(gca_s, out=gca)
+                prob.combine(gcb_s, out=gcb)
+                shard.sum_over_ranks_(gca, gcb)
+            for o, src in zip(outs, (J, gca, gcb) if grad else (J, rec)):
                 o.copy_(src, non_blocking=True)
 
         e2e_step()
@@ -384,7 +449,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, el, cores, sample = oracle_sample()
+        v, el, cores, sample = oracle_sample(number, sample_steps(wl, 1.2e9))
         cpu = {"value": round(v, 6), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
                "seconds": round(el, 2)}
 
@@ -398,24 +463,23 @@ def main():
             "data": "synthetic",
             "config": {"workload": wl.name, "grid": [wl.ny, wl.nx], "interior": wl.n_interior,
                        "n_pml": wl.n_pml, "order": wl.order, "nt": nt, "shots_per_gpu": S,
-                       "n_rec": wl.n_rec, "snapshots": f"checkpoint every {C} steps + segment replay",
+                       "n_rec": wl.n_rec, "snapshots": snapshot_desc(wl),
                        "l2": "inputs larger than L2 (one state buffer is "
                              f"{prob.p.n_shots * wl.ny * wl.nx * 12 / 1e6:.0f} MB)",
                        "parallelism": f"shots sharded, {world} rank(s)"},
             "value_fwd": round(value_fwd, 4),
             "value_interior": round(value * (wl.n_interior ** 2) / (wl.ny * wl.nx), 4),
             "hbm_frac_sweep": round(sweep_frac, 4),
-            "alg_bytes_per_cell": {"forward": round(b_fwd, 3), "replay": round(b_rep, 3),
-                                   "adjoint": round(b_adj, 3)},
-            "roofline": {"bound": "hbm", "kernel": "k_adjoint<2, kStoreF32, 1>",
+            "alg_bytes_per_cell": {k: round(v, 3) for k, v in passes.items()},
+            "roofline": {"bound": "hbm", "kernel": kernel_name,
                          "achieved": round(achieved, 1),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
-                         "traffic": traffic, "alg_bytes_per_launch": adj_bytes,
-                         "avg_launch_ms": round(adj_launch_ms, 4),
+                         "traffic": traffic, "alg_bytes_per_launch": top_bytes,
+                         "avg_launch_ms": round(top_launch_ms, 4),
                          "timing": "CUDA events around every launch, second pass of the same K steps"},
-            "kernel_ms": {"forward": round(fwd_launch_ms, 4), "forward_store": round(rep_launch_ms, 4),
-                          "adjoint": round(adj_launch_ms, 4), "launches": counts},
+            "kernel_ms": {**{k: round(v, 4) for k, v in launch_ms.items()},
+                          "launches": [int(c) for c in counts]},
             "gpu_launches": int(n_launch),
             "J": float(J.cpu()[0]),
             "clocks": clk,
