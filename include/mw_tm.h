@@ -18,9 +18,8 @@
  *  - Grid: ny rows (y = depth z) by nx columns (x), row-major; cell index
  *    j = y * nx + x.  Ey at (y, x), Hx at (y + 1/2, x), Hz at (y, x + 1/2).
  *    Every array cell of every field is updated; fields are zero outside the
- *    array.  nx must be a multiple of 4 (rows are read as float4; a multiple
- *    of 8 with bf16 snapshots) and n_pml at most 123 (a CPML band row is one
- *    TMA box of at most 256 floats).
+ *    array.  nx must be a multiple of 4 (rows are read as float4) and n_pml
+ *    at most 123 (a CPML band row is one TMA box of at most 256 floats).
  *  - Per-shot arrays are [S][ny][nx] float32, time series are time-major
  *    [nt][S][n] float32 (the page's source / receiver kernels).
  *  - Source / receiver positions are flat per-shot cell indices int64
@@ -31,7 +30,9 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Compute calls are asynchronous and stream-ordered; they
  *    return after enqueueing.  Errors found on the host return at once;
- *    device-side status (non-finite fields) is reported by mw_sync_status.
+ *    device-side status (an out-of-range index, a non-finite field with
+ *    check_finite, a stage wait that ran out) is recorded in the workspace
+ *    and reported by mw_sync_status.
  *  - Return codes: MW_OK (0) or a negative MW_ERR_*; mw_last_error() gives a
  *    thread-local message.  No entry point aborts the process.
  *
