@@ -85,6 +85,8 @@ def lib():
         L.orc_residual.restype = ctypes.c_double
         L.orc_num_threads.restype = ctypes.c_int
         _U8 = ctypes.POINTER(ctypes.c_uint8)
+        L.orc_born.argtypes = [ctypes.POINTER(_Sim), ctypes.c_int, _D, _D, _D, _D, _D, _D]
+        L.orc_born.restype = ctypes.c_int
         L.orc_quant_bf16.argtypes = [ctypes.c_int64, _D, _D]
         L.orc_fp8_encode.argtypes = [ctypes.c_int64, _D, _U8]
         L.orc_fp8_decode.argtypes = [ctypes.c_int64, _U8, _D]
@@ -295,6 +297,24 @@ class Sim:
         if rc != 0:
             raise RuntimeError(f"orc_adjoint failed: {rc}")
         return dict(gca=gca, gcb=gcb, grad_f=gf, adj=adj)
+
+    def born(self, snap_ey, snap_curl, dca, dcb, nt=None, state=None):
+        """Born (linearised) forward: records [nt, S, n_rec] of the derivative
+        of the forward's records in the direction (dCa, dCb), given the
+        background's snapshots (forward(..., snapshots=True)).  The
+        transpose of this map is the adjoint's (shot-summed) gradient."""
+        snap_ey, snap_curl = _f64(snap_ey), _f64(snap_curl)
+        nt = snap_ey.shape[0] if nt is None else nt
+        dca = _f64(np.broadcast_to(dca, self.ca.shape))
+        dcb = _f64(np.broadcast_to(dcb, self.ca.shape))
+        state = self.zero_state() if state is None else _f64(state).copy()
+        rec = np.zeros((nt, self.n_shots, self.n_rec))
+        st = self._struct()
+        rc = lib().orc_born(ctypes.byref(st), nt, _p(snap_ey), _p(snap_curl), _p(dca), _p(dcb),
+                            _p(state), _p(rec))
+        if rc != 0:
+            raise RuntimeError(f"orc_born failed: {rc}")
+        return rec
 
     def fwd_adj_ckpt(self, f, res, C, nt=None, state0=None, records=True, grad_f=True):
         """Checkpointed forward + replayed adjoint (memory O(nt/C state + C snapshots))."""

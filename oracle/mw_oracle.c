@@ -242,9 +242,15 @@ static inline double cq_at(const orc_sim *m, int s, int64_t j) {
 /* One forward time step t for all shots, in the page's order:
  * H update, E update (optionally saving Ey^t and curl^t), source injection,
  * receiver sampling.  `state` is [7][S][ny][nx]. */
+/* Born source of the linearised step (NULL for the plain forward): the
+ * perturbation dCa, dCb (model-shaped) and the background's E^t, curl^t. */
+typedef struct {
+  const double *dca, *dcb, *e0, *c0;
+} orc_born_src;
+
 static void forward_step(const orc_sim *m, int t, const double *f,
                          double *state, double *rec, double *snap_ey,
-                         double *snap_curl) {
+                         double *snap_curl, const orc_born_src *born) {
   const int ny = m->ny, nx = m->nx, S = m->n_shots;
   const int64_t N = (int64_t)ny * nx;
   double c[4];
@@ -292,6 +298,12 @@ static void forward_step(const orc_sim *m, int t, const double *f,
         if (snap_ey) snap_ey[((int64_t)t * S + s) * N + j] = ey[j];
         if (snap_curl) snap_curl[((int64_t)t * S + s) * N + j] = curl;
         ey[j] = ca[j] * ey[j] + cb[j] * curl;
+        if (born) {
+          /* linearised step: d(Ca E + Cb curl) = Ca dE + Cb dcurl + dCa E0 + dCb curl0 */
+          const int64_t k = ((int64_t)t * S + s) * N + j;
+          ey[j] += model_ptr(m, born->dca, s)[j] * born->e0[k] +
+                   model_ptr(m, born->dcb, s)[j] * born->c0[k];
+        }
       }
     }
   }
@@ -300,7 +312,7 @@ static void forward_step(const orc_sim *m, int t, const double *f,
     double *ey = state + (int64_t)s * N;
     for (int k = 0; k < m->n_src; ++k) {
       int64_t i = m->src_idx[(int64_t)s * m->n_src + k];
-      if (i >= 0) ey[i] += f[((int64_t)t * S + s) * m->n_src + k];
+      if (i >= 0 && f) ey[i] += f[((int64_t)t * S + s) * m->n_src + k];
     }
     for (int k = 0; k < m->n_rec; ++k) {
       int64_t i = m->rec_idx[(int64_t)s * m->n_rec + k];
@@ -317,7 +329,23 @@ int orc_forward(const orc_sim *m, int nt, const double *f, double *state,
   double c[4];
   if (!orc_coeffs(m->order, c)) return -1;
   for (int t = 0; t < nt; ++t)
-    forward_step(m, t, f, state, rec, snap_ey, snap_curl);
+    forward_step(m, t, f, state, rec, snap_ey, snap_curl, NULL);
+  return 0;
+}
+
+/* Born (linearised) forward: the derivative of the records with respect to
+ * (Ca, Cb) in the direction (dCa, dCb).  The perturbation state starts at
+ * zero and takes the forward step without sources, plus the term
+ * dCa E0^t + dCb curl0^t from the background's snapshots (the E^t and
+ * curl^t of the step, [nt][S][ny][nx]); records are sampled as in the
+ * forward.  Its transpose maps a record residual to the gradients
+ * sum_t E0^t lambda^{t+1}, sum_t curl0^t lambda^{t+1} of the adjoint. */
+int orc_born(const orc_sim *m, int nt, const double *snap_ey0, const double *snap_curl0,
+             const double *dca, const double *dcb, double *state, double *rec) {
+  double c[4];
+  if (!orc_coeffs(m->order, c)) return -1;
+  const orc_born_src b = {dca, dcb, snap_ey0, snap_curl0};
+  for (int t = 0; t < nt; ++t) forward_step(m, t, NULL, state, rec, NULL, NULL, &b);
   return 0;
 }
 
@@ -478,7 +506,7 @@ int orc_fwd_adj_ckpt(const orc_sim *m, int nt, int C, const double *f,
   if (state0) memcpy(st, state0, (size_t)SZ * sizeof(double));
   for (int t = 0; t < nt; ++t) {
     if (t % C == 0) memcpy(ck + (int64_t)(t / C) * SZ, st, (size_t)SZ * sizeof(double));
-    forward_step(m, t, f, st, rec, NULL, NULL);
+    forward_step(m, t, f, st, rec, NULL, NULL, NULL);
   }
   if (res_in) {
     for (int k = nseg - 1; k >= 0; --k) {
@@ -487,7 +515,7 @@ int orc_fwd_adj_ckpt(const orc_sim *m, int nt, int C, const double *f,
       /* replay: snapshots of step t go to slot t - t0 */
       for (int t = t0; t < t1; ++t)
         forward_step(m, t - t0, f + (int64_t)t0 * m->n_shots * m->n_src, st,
-                     NULL, sey, scu);
+                     NULL, sey, scu, NULL);
       for (int t = t1 - 1; t >= t0; --t)
         adjoint_step(m, t - t0, res_in + (int64_t)t0 * m->n_shots * m->n_rec,
                      sey, scu, adj, gca, gcb,

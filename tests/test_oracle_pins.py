@@ -642,3 +642,55 @@ def test_storage_formats_match_torch_casts():
     t = torch.tensor(x, dtype=torch.float32)
     assert np.array_equal(oracle.quant_fp8(x), t.to(torch.float8_e4m3fn).double().numpy())
     assert np.array_equal(oracle.quant_bf16(x), t.to(torch.bfloat16).double().numpy())
+
+
+# ----------------------------------------------------------------------------
+# Born (linearised) forward
+
+
+def _born_case(batched=False):
+    sim, dt, _ = small_sim(321, 24, 28, 2, 1, 5, 4, 4, batched=batched, round_f32=False,
+                           sigma_max=0.02)
+    nt = 40
+    g = synth.rng(3210)
+    f = g.normal(size=(nt, 2, 1))
+    dca = 0.01 * g.normal(size=sim.ca.shape)
+    dcb = 0.01 * float(np.mean(sim.cb)) * g.normal(size=sim.ca.shape)
+    return sim, f, dca, dcb, g
+
+
+def _with_model(sim, ca, cb):
+    return oracle.Sim(ny=sim.ny, nx=sim.nx, order=sim.order, dy=sim.dy, dx=sim.dx, ca=ca, cb=cb,
+                      cq=sim.cq if sim.cq_is_array else float(sim.cq[0]), prof_y=sim.prof_y,
+                      prof_x=sim.prof_x, src_idx=sim.src_idx, rec_idx=sim.rec_idx)
+
+
+def test_born_forward_is_the_derivative_of_the_records():
+    """Central difference of the forward's records along (dCa, dCb) against
+    the Born map (error O(h^2)), with the CPML band on."""
+    sim, f, dca, dcb, _ = _born_case()
+    fw = sim.forward(f, snapshots=True)
+    b = sim.born(fw["snap_ey"], fw["snap_curl"], dca, dcb)
+    h = 1e-4
+    rp = _with_model(sim, sim.ca + h * dca, sim.cb + h * dcb).forward(f)["rec"]
+    rm = _with_model(sim, sim.ca - h * dca, sim.cb - h * dcb).forward(f)["rec"]
+    fd = (rp - rm) / (2 * h)
+    assert np.abs(b).max() > 0
+    assert rel_l2(b, fd) <= 1e-6
+
+
+@pytest.mark.parametrize("batched", [False, True])
+def test_born_forward_is_the_transpose_of_the_gradient(batched):
+    """<B dm, r> = <dm, B^T r>, B^T r being the adjoint's gradient (summed
+    over shots for a shared model, per shot for a batched one)."""
+    sim, f, dca, dcb, g = _born_case(batched)
+    fw = sim.forward(f, snapshots=True)
+    res = g.normal(size=fw["rec"].shape)
+    b = sim.born(fw["snap_ey"], fw["snap_curl"], dca, dcb)
+    adj = sim.adjoint(res, fw["snap_ey"], fw["snap_curl"])
+    gca, gcb = adj["gca"], adj["gcb"]
+    if not batched:
+        gca, gcb = gca.sum(axis=0), gcb.sum(axis=0)
+    lhs = float(np.sum(b * res))
+    rhs = float(np.sum(dca * gca) + np.sum(dcb * gcb))
+    assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), abs(rhs))
