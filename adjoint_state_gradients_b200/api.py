@@ -117,6 +117,18 @@ class Problem:
                              self.src_idx, self.rec_idx, res, gca, gcb, gf, adj_state, self.workspace)
         return gca, gcb, gf
 
+    def born(self, dca, dcb, rec=None):
+        """Born (linearised) forward about the last forward's background:
+        records [nt, S, n_rec] of the perturbation (dca, dcb) of (Ca, Cb)."""
+        p = self.p
+        d = self.device
+        dca = _dev(dca, device=d).reshape(self.model_shape)
+        dcb = _dev(dcb, device=d).reshape(self.model_shape)
+        rec = torch.zeros((p.nt, self.S, max(p.n_rec, 1)), dtype=F32, device=d) if rec is None else rec
+        mwtm.tm_born(p, self.ca, self.cb, self.cq, self.cpml, dca, dcb, getattr(self, "_f", None),
+                     self.src_idx, self.rec_idx, rec, self.workspace)
+        return rec
+
     def combine(self, g_shot, out=None, accumulate=False):
         p = self.p
         out = torch.empty((p.ny, p.nx), dtype=F32, device=self.device) if out is None else out

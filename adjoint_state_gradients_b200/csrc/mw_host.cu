@@ -528,6 +528,30 @@ int fwd_maps(const mw_params *p, const Fields &in, const float *ca, const float 
   return MW_OK;
 }
 
+// Born forward: dCa / dCb (pair box when their distance allows) and the
+// background's snapshots (x, y, shot, step, field) as one box 144 wide.
+int born_maps(const mw_params *p, const float *dca, const float *dcb, const void *se,
+              const void *sc, int snap_elem, int snap_steps, int snap_pitch, FwdMaps *m) {
+  const uint64_t nx = p->nx, ny = p->ny, S = p->n_shots, Sm = p->model_batched ? p->n_shots : 1;
+  const MdPair bd = md_pairing(p, dca, dcb);
+  if (bd.pair) {
+    MW_TRY(encode_rows(&m->map[kMapBD], bd.swap ? dcb : dca, 4, 4, nx, ny, Sm, 2, 120, 2,
+                       bd.stride));
+  } else {
+    MW_TRY(encode_rows(&m->map[kMapBD], dca, 4, 3, nx, ny, Sm, 1, 120));
+    MW_TRY(encode_rows(&m->map[kMapBDB], dcb, 4, 3, nx, ny, Sm, 1, 120));
+  }
+  if ((const char *)sc <= (const char *)se)
+    return fail(MW_ERR_ARG, "internal: snapshot fields out of order");
+  const uint64_t e = (uint64_t)snap_elem, pitch = (uint64_t)snap_pitch;
+  const uint64_t dims[5] = {nx, ny, S, (uint64_t)snap_steps, 2};
+  const uint64_t strides[4] = {pitch * e, pitch * ny * e, pitch * ny * S * e,
+                               (uint64_t)((const char *)sc - (const char *)se)};
+  const uint32_t box[5] = {144, 1, 1, 1, 2};
+  MW_TRY(encode_map(&m->map[kMapBS], se, snap_elem, 5, dims, strides, box));
+  return MW_OK;
+}
+
 int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb,
              const float *cq, const float *gca, const float *gcb, const void *se, const void *sc,
              int snap_elem, int snap_steps, int snap_pitch, AdjMaps *m) {
@@ -598,7 +622,7 @@ void set_layout(StepArgs &a, const mw_params *p, bool adjoint) {
     a.gg_swap = gg.swap ? 1 : 0;
   } else {
     // forward: needs a.ca / a.cb (the Ca / Cb pair fetch)
-    forward_layout(p->order, bands(p).Wx, !p->cq_is_scalar, &a, &smem);
+    forward_layout(p->order, bands(p).Wx, !p->cq_is_scalar, false, &a, &smem);
     const MdPair md = md_pairing(p, a.ca, a.cb);
     a.md_pair = md.pair ? 1 : 0;
     a.md_swap = md.swap ? 1 : 0;
@@ -801,7 +825,7 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
     const FwdMaps &m = cur == bufA ? mA : mB;
     a.ctr_slot = t & 1;
     MW_CUDA(timed(store ? 1 : 0, st, [&] {
-      return launch_forward(m, a, p->order, store, p->model_batched != 0, !p->cq_is_scalar,
+      return launch_forward(m, a, p->order, store, kStoreNone, p->model_batched != 0, !p->cq_is_scalar,
                             lc.grid, st);
     }));
     if (host) {  // step t: ring slot -> host, on the copy stream
@@ -976,7 +1000,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
         const FwdMaps &fm = rc_ == rA ? fA : fB;
         fa.ctr_slot = (launch_idx++) & 1;
         MW_CUDA(timed(1, st, [&] {
-          return launch_forward(fm, fa, p->order, kStoreF32, p->model_batched != 0,
+          return launch_forward(fm, fa, p->order, kStoreF32, kStoreNone, p->model_batched != 0,
                                 !p->cq_is_scalar, lf.grid, st);
         }));
         MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
@@ -991,6 +1015,168 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   if (p->check_finite) {
     MW_CUDA(launch_check_finite(gca, SN, flags, st));
     MW_CUDA(launch_check_finite(gcb, SN, flags, st));
+  }
+  return MW_OK;
+}
+
+int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float *cq,
+               const float *cpml, const float *dca, const float *dcb, const float *f,
+               const int64_t *src_idx, const int64_t *rec_idx, float *rec, void *workspace,
+               size_t workspace_bytes, void *stream) {
+  g_err.clear();
+  int rc = check_params(p, true);
+  if (rc) return rc;
+  if ((rc = check_host_snap(p))) return rc;
+  if (p->snap_mode == MW_SNAP_NONE)
+    return fail(MW_ERR_ARG, "snap_mode NONE: the forward stored no background snapshots");
+  if ((rc = check_ptr(ca, "ca")) || (rc = check_ptr(cb, "cb")) || (rc = check_ptr(cpml, "cpml")) ||
+      (rc = check_ptr(dca, "dca")) || (rc = check_ptr(dcb, "dcb")))
+    return rc;
+  if (!cq) return fail(MW_ERR_ARG, "cq is NULL");
+  if (!p->cq_is_scalar && (rc = check_ptr(cq, "cq"))) return rc;
+  if (p->n_rec > 0 && (!rec || !rec_idx)) return fail(MW_ERR_ARG, "receivers need rec and rec_idx");
+  const bool ckpt = p->snap_mode == MW_SNAP_CKPT;
+  if (ckpt && p->n_src > 0 && (!f || !src_idx))
+    return fail(MW_ERR_ARG, "checkpoint replay needs f and src_idx");
+  if (!workspace) return fail(MW_ERR_WORKSPACE, "workspace is NULL");
+  const Layout L = layout(p);
+  if (workspace_bytes < L.total)
+    return fail(MW_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+  if (((uintptr_t)workspace) % 256 != 0) return fail(MW_ERR_WORKSPACE, "workspace not 256-aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  char *ws = (char *)workspace;
+  int *flags = (int *)(ws + L.flags);
+  const int64_t numel = (int64_t)p->ny * p->nx;
+  const Chains ch = chains_at(p, ws, L);
+  if (p->n_rec > 0)  // validates the receiver indices
+    MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
+                              flags, st));
+  if (ckpt && p->n_src > 0)
+    MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
+                              flags, st));
+  if (p->nt == 0) return MW_OK;
+
+  // the perturbation state lives in the adjoint's buffers, from zero
+  float *dA = (float *)(ws + L.adA), *dB = (float *)(ws + L.adB);
+  MW_CUDA(cudaMemsetAsync(dA, 0, L.state_bytes, st));
+  const Launch lc = plan(p, false);
+  StepArgs b{};
+  b.g = lc.g;
+  b.c = coef_of(p);
+  b.ca = ca;
+  b.cb = cb;
+  b.cq = cq;
+  b.flags = flags;
+  b.bt = (const float *)(ws + L.bandtab);
+  {
+    size_t smem;
+    forward_layout(p->order, bands(p).Wx, !p->cq_is_scalar, true, &b, &smem);
+    const MdPair md = md_pairing(p, ca, cb), bd = md_pairing(p, dca, dcb);
+    b.md_pair = md.pair ? 1 : 0;
+    b.md_swap = md.swap ? 1 : 0;
+    b.bd_pair = bd.pair ? 1 : 0;
+    b.bd_swap = bd.swap ? 1 : 0;
+  }
+  MW_TRY(stencil_prologue(p, cpml, ws, L, st));
+
+  // the background's snapshots: every step in the workspace, a 3-step ring
+  // fed from pinned host memory, or a replayed checkpoint segment (fp32)
+  const bool host = p->snap_host != 0;
+  const int kind = ckpt ? kStoreF32 : snap_store_kind(p->snap_mode);
+  const int elem = ckpt ? 4 : (int)snap_elem_bytes(p->snap_mode);
+  const int steps = ckpt ? p->ckpt_every : host ? kHostRing : p->nt;
+  const char *snap_e = ckpt ? ws + L.seg : ws + L.snap;
+  const char *snap_c = snap_e + (size_t)steps * L.snap_step_bytes;
+  FwdMaps mA, mB;
+  MW_TRY(fwd_maps(p, fields_at(p, dA), ca, cb, cq, &mA));
+  MW_TRY(fwd_maps(p, fields_at(p, dB), ca, cb, cq, &mB));
+  MW_TRY(born_maps(p, dca, dcb, snap_e, snap_c, elem, steps, L.snap_pitch, &mA));
+  MW_TRY(born_maps(p, dca, dcb, snap_e, snap_c, elem, steps, L.snap_pitch, &mB));
+
+  int launch_idx = 0;
+  float *cur = dA, *nxt = dB;
+  auto born_step = [&](int t, int slot) -> int {
+    b.in = fields_at(p, cur);
+    b.out = fields_at(p, nxt);
+    b.snap_t = slot;
+    b.ctr_slot = (launch_idx++) & 1;
+    const FwdMaps &m = cur == dA ? mA : mB;
+    MW_CUDA(launch_forward(m, b, p->order, kStoreNone, kind, p->model_batched != 0,
+                           !p->cq_is_scalar, lc.grid, st));
+    MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots, nullptr, nullptr, nullptr, nullptr, 0,
+                                 rec_idx, p->n_rec,
+                                 rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, st));
+    std::swap(cur, nxt);
+    return MW_OK;
+  };
+
+  if (host) {
+    HostCopies hc;
+    MW_TRY(hc.init());
+    MW_CUDA(cudaEventRecord(hc.start, st));
+    MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.start, 0));
+    const char *hbuf = (const char *)p->snap_host_ptr;
+    auto fetch = [&](int t) -> int {
+      const int slot = t % kHostRing;
+      if (t >= kHostRing) MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.freed[slot], 0));
+      const char *h = hbuf + 2 * (size_t)t * L.snap_step_bytes;
+      MW_CUDA(cudaMemcpyAsync((void *)(snap_e + (size_t)slot * L.snap_step_bytes), h,
+                              L.snap_step_bytes, cudaMemcpyHostToDevice, hc.cs));
+      MW_CUDA(cudaMemcpyAsync((void *)(snap_c + (size_t)slot * L.snap_step_bytes),
+                              h + L.snap_step_bytes, L.snap_step_bytes, cudaMemcpyHostToDevice,
+                              hc.cs));
+      MW_CUDA(cudaEventRecord(hc.filled[slot], hc.cs));
+      return MW_OK;
+    };
+    for (int t = 0; t < p->nt && t < kHostRing; ++t) MW_TRY(fetch(t));
+    for (int t = 0; t < p->nt; ++t) {
+      const int slot = t % kHostRing;
+      MW_CUDA(cudaStreamWaitEvent(st, hc.filled[slot], 0));
+      MW_TRY(born_step(t, slot));
+      MW_CUDA(cudaEventRecord(hc.freed[slot], st));
+      if (t + kHostRing < p->nt) MW_TRY(fetch(t + kHostRing));
+    }
+  } else if (!ckpt) {
+    for (int t = 0; t < p->nt; ++t) MW_TRY(born_step(t, t));
+  } else {
+    // replay each segment of the background from its checkpoint into the fp32
+    // segment buffer, then take the segment's linearised steps
+    const int C = p->ckpt_every;
+    StepArgs fa{};
+    fa.g = lc.g;
+    fa.c = b.c;
+    fa.ca = ca;
+    fa.cb = cb;
+    fa.cq = cq;
+    fa.flags = flags;
+    fa.bt = b.bt;
+    set_layout(fa, p, false);
+    fa.snap_pitch = p->nx;
+    float *rA = (float *)(ws + L.rpA), *rB = (float *)(ws + L.rpB);
+    FwdMaps fA, fB;
+    MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, cq, &fA));
+    MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, cq, &fB));
+    for (int k = 0; k < L.n_seg; ++k) {
+      const int t0 = k * C;
+      const int t1 = (t0 + C < p->nt) ? t0 + C : p->nt;
+      MW_CUDA(cudaMemcpyAsync(rA, ws + L.snap + (size_t)k * align256(L.state_bytes),
+                              L.state_bytes, cudaMemcpyDeviceToDevice, st));
+      float *rc_ = rA, *rn = rB;
+      for (int t = t0; t < t1; ++t) {
+        fa.in = fields_at(p, rc_);
+        fa.out = fields_at(p, rn);
+        fa.snap_e = (char *)snap_e + (size_t)(t - t0) * L.snap_step_bytes;
+        fa.snap_c = (char *)snap_c + (size_t)(t - t0) * L.snap_step_bytes;
+        fa.ctr_slot = (launch_idx++) & 1;
+        MW_CUDA(launch_forward(rc_ == rA ? fA : fB, fa, p->order, kStoreF32, kStoreNone,
+                               p->model_batched != 0, !p->cq_is_scalar, lc.grid, st));
+        MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
+                                     f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
+                                     ch.src_lead, ch.src_next, p->n_src, nullptr, 0, nullptr, st));
+        std::swap(rc_, rn);
+      }
+      for (int t = t0; t < t1; ++t) MW_TRY(born_step(t, t - t0));
+    }
   }
   return MW_OK;
 }
@@ -1205,7 +1391,7 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
       a.in = fields_at(p, cur);
       a.out = fields_at(p, nxt);
       a.ctr_slot = t & 1;
-      MW_CUDA(launch_forward(cur == bufA ? mA : mB, a, p->order, kStoreNone,
+      MW_CUDA(launch_forward(cur == bufA ? mA : mB, a, p->order, kStoreNone, kStoreNone,
                              p->model_batched != 0, !p->cq_is_scalar, lc.grid, st));
       MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots,
                                    f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,

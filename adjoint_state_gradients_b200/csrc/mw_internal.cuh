@@ -59,7 +59,7 @@ struct Fields {
 };
 
 // Forward stage slots placed by the host (float offsets within a stage).
-enum { kFoCqH = 0, kFoCqX, kFoMzh, kFoMze, kFoMxh, kFoMxe, kFoCount };
+enum { kFoCqH = 0, kFoCqX, kFoMzh, kFoMze, kFoMxh, kFoMxe, kFoBd, kFoBs, kFoCount };
 // Adjoint stage slots placed by the host.
 enum { kAoCqR = 0, kAoCqH, kAoMx, kAoMze, kAoMzh, kAoCount };
 
@@ -87,6 +87,7 @@ struct StepArgs {
   // forward only: optional stage slots (kFo*), Ca / Cb pair fetch and order
   int fo[kFoCount];
   int md_pair, md_swap;
+  int bd_pair, bd_swap;  // Born forward: dCa / dCb pair fetch and order
   // adjoint only: optional stage slots (kAo*), gCa / gCb pair fetch and order
   int ao[kAoCount];
   int gg_pair, gg_swap;
@@ -103,8 +104,12 @@ struct StepArgs {
 //   kMapCQ  Cq when it is an array: 128 wide from x0 - 4
 //   kMapMXH / kMapMXE  x-band memories, a whole band row (2*Wx)
 //   kMapMZH / kMapMZE  z-band memories, 120 wide from x0
+//   kMapBD / kMapBDB  Born forward: dCa and dCb (like kMapMD / kMapCB)
+//   kMapBS  Born forward: the background's E and curl snapshots of the step
+//           as one 5-D box, 144 wide from a 16-element boundary
 enum FwdMap {
-  kMapEH = 0, kMapHX, kMapMD, kMapCB, kMapCQ, kMapMXH, kMapMXE, kMapMZH, kMapMZE, kFwdMaps
+  kMapEH = 0, kMapHX, kMapMD, kMapCB, kMapCQ, kMapMXH, kMapMXE, kMapMZH, kMapMZE, kMapBD,
+  kMapBDB, kMapBS, kFwdMaps
 };
 struct FwdMaps {
   CUtensorMap map[kFwdMaps];
@@ -230,7 +235,9 @@ cudaError_t launch_dependent(void (*kern)(KArgs...), int grid, int block, size_t
 }
 
 // stencil launchers (mw_stencil.cu); return a cudaError_t
-cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int store,
+// born: kStoreNone, or the background snapshots' kind for the Born forward
+// (then store must be kStoreNone)
+cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int store, int born,
                            bool batched, bool cq_array, int grid, cudaStream_t st);
 // snap: the snapshot storage (kStoreF32, kStoreBF16 or kStoreFP8)
 cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int snap,
@@ -242,7 +249,7 @@ cudaError_t launch_snap_encode(int store, int64_t n, const float *x, void *out, 
 cudaError_t launch_wait_selftest(int *flags, cudaStream_t st);
 // forward / adjoint: the full stage layout (optional slots for a Cq array and
 // bands)
-void forward_layout(int order, int Wx, bool cq_array, StepArgs *a, size_t *smem_bytes);
+void forward_layout(int order, int Wx, bool cq_array, bool born, StepArgs *a, size_t *smem_bytes);
 void adjoint_layout(int order, int Wx, bool cq_array, bool bf16, StepArgs *a, size_t *smem_bytes);
 int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array);
 

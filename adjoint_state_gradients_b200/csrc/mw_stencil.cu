@@ -175,6 +175,7 @@ struct FwdWarp {
   uint32_t bars, stage0, hring;
   uint32_t stage_bytes;
   uint32_t ca_o, cb_o;  // byte offsets of the Ca / Cb rows in a stage
+  uint32_t dca_o, dcb_o;  // Born forward: byte offsets of the dCa / dCb rows
   int lane;
   Ring ring;
 };
@@ -183,7 +184,7 @@ struct FwdWarp {
 // rows are r (Ey, Hz; Cq), r - P (Hx; Cq, z-band memory of Hx) and
 // y = r - 2P + 1 (Ca, Cb; band memories of E); the x-band memory of Hz is
 // that of row r.  Rows outside the array read as zeros.
-template <int P, bool BAND>
+template <int P, bool BAND, int BORN>
 __device__ __forceinline__ void fwd_issue(const FwdMaps &m, const StepArgs &a, const Item &it,
                                           int i, uint32_t st, uint32_t bar, int cq_arr) {
   const int r = it.r0 + i;
@@ -201,9 +202,27 @@ __device__ __forceinline__ void fwd_issue(const FwdMaps &m, const StepArgs &a, c
     if (ze >= 0) bytes += 120 * 4;
     if (it.xb) bytes += (uint32_t)a.band_box_floats * 4 * (e_row ? 2 : 1);
   }
+  if constexpr (BORN != kStoreNone) {
+    constexpr uint32_t be = BORN == kStoreF32 ? 4 : BORN == kStoreBF16 ? 2 : 1;
+    if (e_row) bytes += 2 * 120 * 4 + 2 * 144 * be;
+  }
   expect_tx_s(bar, bytes);
   fence_proxy_async();
   tma4s(st + kF_EY * 4, &m.map[kMapEH], it.x0 - 8, r, it.s, 0, bar);
+  if constexpr (BORN != kStoreNone) {
+    if (e_row) {  // dCa, dCb and the background's E, curl of row y at this step
+      const int y = r - 2 * P + 1;
+      if (a.bd_pair) {
+        tma4s(st + a.fo[kFoBd] * 4, &m.map[kMapBD], it.x0, y, it.sm, 0, bar);
+      } else {
+        tma3s(st + a.fo[kFoBd] * 4, &m.map[kMapBD], it.x0, y, it.sm, bar);
+        tma3s(st + (a.fo[kFoBd] + 128) * 4, &m.map[kMapBDB], it.x0, y, it.sm, bar);
+      }
+      // a 16-element boundary, so that a byte-sized row stays TMA-aligned
+      const int xs = ((it.x0 - 4) >> 4) << 4;
+      tma5s(st + a.fo[kFoBs] * 4, &m.map[kMapBS], xs, y, it.s, a.snap_t, 0, bar);
+    }
+  }
   if (hx_in) tma3s(st + kF_HX * 4, &m.map[kMapHX], it.x0, r - P, it.s, bar);
   if (e_row) {
     if (a.md_pair) {
@@ -243,7 +262,7 @@ __device__ __noinline__ void give_up_s(int *flags, uint32_t bars, Ring ring, int
 // (owned rows); the row-range tests are warp-uniform, the per-lane ones only
 // predicate stores.  BAND adds the CPML recursions and the array-edge masks
 // that interior items do not need.
-template <int P, int STORE, int L, bool BAND>
+template <int P, int STORE, int L, bool BAND, int BORN>
 __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, const Item &it,
                                          FwdWarp &w, int cq_arr, float cqs) {
   constexpr int NQ = 2 * P;
@@ -271,7 +290,7 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
     Ring pr = w.ring;
     for (int j = 0; j < L && j < it.n_it; ++j) {
       if (lane == 0)
-        fwd_issue<P, BAND>(m, a, it, j, w.stage0 + pr.slot * w.stage_bytes, w.bars + 8 * pr.slot,
+        fwd_issue<P, BAND, BORN>(m, a, it, j, w.stage0 + pr.slot * w.stage_bytes, w.bars + 8 * pr.slot,
                            cq_arr);
       pr.next(NS);
     }
@@ -290,7 +309,7 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
       if (i < it.n_it) {
         if (i + L < it.n_it && lane == 0) {
           const int ps = w.ring.slot == 0 ? NS - 1 : w.ring.slot - 1;
-          fwd_issue<P, BAND>(m, a, it, i + L, w.stage0 + ps * w.stage_bytes, w.bars + 8 * ps,
+          fwd_issue<P, BAND, BORN>(m, a, it, i + L, w.stage0 + ps * w.stage_bytes, w.bars + 8 * ps,
                              cq_arr);
         }
         if (!mbar_wait_s(w.bars + 8 * w.ring.slot, w.ring.phase)) {
@@ -430,6 +449,17 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
             curl.v[q] = cx.v[q] - cz.v[q];
             en.v[q] = fmaf(ca4.v[q], e_old.v[q], cb4.v[q] * curl.v[q]);
           }
+          if constexpr (BORN != kStoreNone) {
+            // linearised step: + dCa E0 + dCb curl0 (the background's values)
+            constexpr uint32_t be = BORN == kStoreF32 ? 4 : BORN == kStoreBF16 ? 2 : 1;
+            const F4 dca4 = lds4s(st + w.dca_o + 16 * lane - 16);
+            const F4 dcb4 = lds4s(st + w.dcb_o + 16 * lane - 16);
+            const uint32_t sb = st + a.fo[kFoBs] * 4 + (((it.x0 - 4) & 15) + 4 * lane) * be;
+            const F4 e0 = snap_lds_s<BORN>(sb), c0 = snap_lds_s<BORN>(sb + 144 * be);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              en.v[q] += fmaf(dcb4.v[q], c0.v[q], dca4.v[q] * e0.v[q]);
+          }
           {
             const int off = ro - (2 * P - 1) * nx;
             if constexpr (STORE != kStoreNone) {
@@ -452,8 +482,9 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
   return true;
 }
 
-template <int P, int STORE, int L>
-__global__ void __launch_bounds__(128, P <= 3 ? 5 : 4) k_forward(const __grid_constant__ FwdMaps m,
+template <int P, int STORE, int L, int BORN>
+__global__ void __launch_bounds__(128, BORN != kStoreNone ? 3 : (P <= 3 ? 5 : 4))
+    k_forward(const __grid_constant__ FwdMaps m,
                                                  const StepArgs a, const int batched,
                                                  const int cq_arr) {
   constexpr int NS = L + 1;
@@ -472,6 +503,8 @@ __global__ void __launch_bounds__(128, P <= 3 ? 5 : 4) k_forward(const __grid_co
   // two boxes: Ca at kF_MD, Cb at kF_MD + 128 (every box starts 128-aligned)
   w.ca_o = (kF_MD + (a.md_pair && a.md_swap ? 120 : 0)) * 4;
   w.cb_o = (kF_MD + (a.md_pair ? (a.md_swap ? 0 : 120) : 128)) * 4;
+  w.dca_o = (a.fo[kFoBd] + (a.bd_pair && a.bd_swap ? 120 : 0)) * 4;
+  w.dcb_o = (a.fo[kFoBd] + (a.bd_pair ? (a.bd_swap ? 0 : 120) : 128)) * 4;
   w.ring = Ring{0, 0u};
   const Geom &g = a.g;
   const int n_items = g.S * g.n_strips * g.n_chunks;
@@ -498,8 +531,8 @@ __global__ void __launch_bounds__(128, P <= 3 ? 5 : 4) k_forward(const __grid_co
     if (item >= n_items) break;
     Item it;
     if (!make_item<P>(g, item, batched != 0, it)) continue;
-    const bool ok = it.edge ? fwd_walk<P, STORE, L, true>(m, a, it, w, cq_arr, cqs)
-                            : fwd_walk<P, STORE, L, false>(m, a, it, w, cq_arr, cqs);
+    const bool ok = it.edge ? fwd_walk<P, STORE, L, true, BORN>(m, a, it, w, cq_arr, cqs)
+                            : fwd_walk<P, STORE, L, false, BORN>(m, a, it, w, cq_arr, cqs);
     if (!ok) return;
   }
 }
@@ -879,7 +912,7 @@ constexpr int kAdjL = 1;  // adjoint lookahead
 // Forward stage: the fixed slots, then a Cq array's rows r and r - P, then
 // the z-band memory rows and the two x-band memory rows, each only if used.
 template <int P>
-void fwd_layout_t(int Wx, bool cq_arr, StepArgs *a, size_t *smem) {
+void fwd_layout_t(int Wx, bool cq_arr, bool born, StepArgs *a, size_t *smem) {
   const int bw = Wx > 0 ? ((2 * Wx + 31) / 32) * 32 : 0;
   int o = kF_FIXED;
   for (int k = 0; k < kFoCount; ++k) a->fo[k] = 0;
@@ -894,6 +927,11 @@ void fwd_layout_t(int Wx, bool cq_arr, StepArgs *a, size_t *smem) {
     a->fo[kFoMxh] = o + 256;
     a->fo[kFoMxe] = o + 256 + bw;
     o += 256 + 2 * bw;
+  }
+  if (born) {  // dCa / dCb (pair, or two 128-aligned boxes) and the snapshots
+    a->fo[kFoBd] = o;
+    a->fo[kFoBs] = o + 256;
+    o += 256 + 288;
   }
   int wf = (kFwdL + 1) * o + 2 * P * kFRing;
   wf = ((wf + 31) / 32) * 32;
@@ -942,7 +980,7 @@ void allow_big_smem(K kern, std::atomic<uint64_t> &done) {
     done.fetch_or(bit);
   }
 }
-template <int P, int STORE>
+template <int P, int STORE, int BORN = kStoreNone>
 std::atomic<uint64_t> &fwd_smem_flag() {
   static std::atomic<uint64_t> f{0};
   return f;
@@ -953,12 +991,12 @@ std::atomic<uint64_t> &adj_smem_flag() {
   return f;
 }
 
-template <int P, int STORE>
+template <int P, int STORE, int BORN = kStoreNone>
 cudaError_t fwd_t(const FwdMaps &m, const StepArgs &a, bool batched, bool cq_arr, int grid,
                   cudaStream_t st) {
   const size_t smem = (size_t)(32 + kWarpsPerCta * a.warp_floats) * sizeof(float) + 128;
-  allow_big_smem(k_forward<P, STORE, kFwdL>, fwd_smem_flag<P, STORE>());
-  const cudaError_t e = launch_dependent(k_forward<P, STORE, kFwdL>, grid, 128, smem, st, m, a,
+  allow_big_smem(k_forward<P, STORE, kFwdL, BORN>, fwd_smem_flag<P, STORE, BORN>());
+  const cudaError_t e = launch_dependent(k_forward<P, STORE, kFwdL, BORN>, grid, 128, smem, st, m, a,
                                          batched ? 1 : 0, cq_arr ? 1 : 0);
   if (e != cudaSuccess) return e;
   count_launches(1);
@@ -977,8 +1015,17 @@ cudaError_t adj_t(const AdjMaps &m, const StepArgs &a, bool batched, bool cq_arr
 }
 
 template <int P>
-cudaError_t fwd_store(const FwdMaps &m, const StepArgs &a, int store, bool batched, bool cq_arr,
-                      int grid, cudaStream_t st) {
+cudaError_t fwd_store(const FwdMaps &m, const StepArgs &a, int store, int born, bool batched,
+                      bool cq_arr, int grid, cudaStream_t st) {
+  if (born != kStoreNone) {
+    if (store != kStoreNone) return cudaErrorInvalidValue;
+    switch (born) {
+      case kStoreF32: return fwd_t<P, kStoreNone, kStoreF32>(m, a, batched, cq_arr, grid, st);
+      case kStoreBF16: return fwd_t<P, kStoreNone, kStoreBF16>(m, a, batched, cq_arr, grid, st);
+      case kStoreFP8: return fwd_t<P, kStoreNone, kStoreFP8>(m, a, batched, cq_arr, grid, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (store) {
     case kStoreNone: return fwd_t<P, kStoreNone>(m, a, batched, cq_arr, grid, st);
     case kStoreF32: return fwd_t<P, kStoreF32>(m, a, batched, cq_arr, grid, st);
@@ -1018,21 +1065,21 @@ int slots_t(bool adjoint, int Wx, bool cq_arr) {
                      adj_smem_flag<P, kStoreF32>()) *
            kAdjWarpsPerCta;
   }
-  fwd_layout_t<P>(Wx, cq_arr, &a, &smem);
-  return occupancy(k_forward<P, kStoreF32, kFwdL>, 32 * kWarpsPerCta, smem,
+  fwd_layout_t<P>(Wx, cq_arr, false, &a, &smem);
+  return occupancy(k_forward<P, kStoreF32, kFwdL, kStoreNone>, 32 * kWarpsPerCta, smem,
                    fwd_smem_flag<P, kStoreF32>()) *
          kWarpsPerCta;
 }
 
 }  // namespace
 
-cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int store, bool batched,
-                           bool cq_array, int grid, cudaStream_t st) {
+cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int store, int born,
+                           bool batched, bool cq_array, int grid, cudaStream_t st) {
   switch (order) {
-    case 2: return fwd_store<1>(m, a, store, batched, cq_array, grid, st);
-    case 4: return fwd_store<2>(m, a, store, batched, cq_array, grid, st);
-    case 6: return fwd_store<3>(m, a, store, batched, cq_array, grid, st);
-    case 8: return fwd_store<4>(m, a, store, batched, cq_array, grid, st);
+    case 2: return fwd_store<1>(m, a, store, born, batched, cq_array, grid, st);
+    case 4: return fwd_store<2>(m, a, store, born, batched, cq_array, grid, st);
+    case 6: return fwd_store<3>(m, a, store, born, batched, cq_array, grid, st);
+    case 8: return fwd_store<4>(m, a, store, born, batched, cq_array, grid, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -1067,12 +1114,12 @@ void adjoint_layout(int order, int Wx, bool cq_array, bool bf16, StepArgs *a, si
   }
 }
 
-void forward_layout(int order, int Wx, bool cq_array, StepArgs *a, size_t *smem) {
+void forward_layout(int order, int Wx, bool cq_array, bool born, StepArgs *a, size_t *smem) {
   switch (order) {
-    case 2: fwd_layout_t<1>(Wx, cq_array, a, smem); return;
-    case 4: fwd_layout_t<2>(Wx, cq_array, a, smem); return;
-    case 6: fwd_layout_t<3>(Wx, cq_array, a, smem); return;
-    default: fwd_layout_t<4>(Wx, cq_array, a, smem); return;
+    case 2: fwd_layout_t<1>(Wx, cq_array, born, a, smem); return;
+    case 4: fwd_layout_t<2>(Wx, cq_array, born, a, smem); return;
+    case 6: fwd_layout_t<3>(Wx, cq_array, born, a, smem); return;
+    default: fwd_layout_t<4>(Wx, cq_array, born, a, smem); return;
   }
 }
 

@@ -73,6 +73,7 @@ SIGNATURES = [
     ("mw_profile_read", ctypes.c_int, [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double),
                                        ctypes.c_int32]),
     ("mw_launch_count", ctypes.c_int64, []),
+    ("mw_tm_born", ctypes.c_int, [_P] + [ctypes.c_void_p] * 10 + [ctypes.c_size_t, ctypes.c_void_p]),
     ("mw_selftest_wait_timeout", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     ("mw_snapshot_encode", ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p,
                                           ctypes.c_void_p, ctypes.c_void_p]),
@@ -244,3 +245,12 @@ def snapshot_encode(snap_mode, x, out, stream=None):
 def selftest_wait_timeout(workspace, stream=None):
     """Run the bounded-wait self-test kernel on `workspace` (see mw_tm.h)."""
     return check(lib().mw_selftest_wait_timeout(ptr(workspace), stream_ptr(stream)))
+
+
+def tm_born(p, ca, cb, cq, cpml, dca, dcb, f, src_idx, rec_idx, rec, workspace, stream=None):
+    """Born (linearised) forward records of (dca, dcb) about the last forward's
+    background on this workspace (see mw_tm.h)."""
+    return check(lib().mw_tm_born(ctypes.byref(p), ptr(ca), ptr(cb), ptr(cq), ptr(cpml), ptr(dca),
+                                  ptr(dcb), ptr(f), ptr(src_idx), ptr(rec_idx), ptr(rec),
+                                  ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  stream_ptr(stream)))

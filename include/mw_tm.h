@@ -233,6 +233,25 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca_dev,
                        float *adj_state_dev, void *workspace_dev,
                        size_t workspace_bytes, void *stream);
 
+/* Born (linearised) forward: the derivative of the records with respect to
+ * (Ca, Cb) in the direction (dCa, dCb), the transpose of mw_tm_adjoint_grad's
+ * gradient map (LSRTM-style modelling / migration pairs; the PR page
+ * "DeepWave-KAUST/sweep #125", commits 1-2, describes such Born / adjoint
+ * pairs, checked by a dot test, for its acoustic and qP operators).  A perturbation state starts at zero and takes the
+ * forward step without sources, plus dCa E^t + dCb curl^t from the
+ * background's snapshots of that step; rec_dev [nt][S][n_rec] receives its
+ * records.  The background is the last mw_tm_forward on this workspace with
+ * the same p, ca, cb, cq, cpml: its stored snapshots (FP32, BF16 or FP8, on
+ * the device or in pinned host memory with snap_host, used exactly as
+ * stored) or, with MW_SNAP_CKPT, its checkpoints replayed segment by segment
+ * (which needs f and src_idx again).  dca_dev / dcb_dev are model-shaped
+ * float32.  The workspace's adjoint state buffers are overwritten; the
+ * snapshots and checkpoints are kept, so mw_tm_adjoint_grad may follow. */
+int mw_tm_born(const mw_params *p, const float *ca_dev, const float *cb_dev, const float *cq_dev,
+               const float *cpml_dev, const float *dca_dev, const float *dcb_dev,
+               const float *f_dev, const int64_t *src_idx_dev, const int64_t *rec_idx_dev,
+               float *rec_dev, void *workspace_dev, size_t workspace_bytes, void *stream);
+
 /* Shot reduction (the page's combine_grad, over every cell):
  * grad[j] (+)= sum_{s=0..S-1} grad_shot[s][j], shots summed in order in
  * float32.  accumulate = 0 overwrites, 1 adds. */
