@@ -1101,8 +1101,10 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
     b.snap_t = slot;
     b.ctr_slot = (launch_idx++) & 1;
     const FwdMaps &m = cur == dA ? mA : mB;
-    MW_CUDA(launch_forward(m, b, p->order, kStoreNone, kind, p->model_batched != 0,
-                           !p->cq_is_scalar, lc.grid, st));
+    MW_CUDA(timed(3, st, [&] {
+      return launch_forward(m, b, p->order, kStoreNone, kind, p->model_batched != 0,
+                            !p->cq_is_scalar, lc.grid, st);
+    }));
     MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots, nullptr, nullptr, nullptr, nullptr, 0,
                                  rec_idx, p->n_rec,
                                  rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, st));

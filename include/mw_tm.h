@@ -281,8 +281,8 @@ int mw_sync_status(void *workspace_dev, void *stream);
 /* Thread-local message of the last failing call ("" if none). */
 const char *mw_last_error(void);
 
-/* Per-kernel timing (CUDA events around each launch of the three stencil
- * kernels: 0 forward, 1 forward with snapshot store, 2 adjoint).  enable = 1
+/* Per-kernel timing (CUDA events around each launch of the stencil kernels:
+ * 0 forward, 1 forward with snapshot store, 2 adjoint, 3 Born forward).  enable = 1
  * clears and starts recording; mw_profile_read synchronizes the recorded
  * events and returns, per class, the launch count and total milliseconds. */
 int mw_profile_enable(int32_t enable);
