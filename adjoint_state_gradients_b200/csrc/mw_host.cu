@@ -629,6 +629,20 @@ void set_layout(StepArgs &a, const mw_params *p, bool adjoint) {
   }
 }
 
+// Step arguments shared by every stencil launch of a call.
+StepArgs step_args(const mw_params *p, const Launch &lc, const float *ca, const float *cb,
+                   const float *cq, int *flags, const char *ws, const Layout &L) {
+  StepArgs a{};
+  a.g = lc.g;
+  a.c = coef_of(p);
+  a.ca = ca;
+  a.cb = cb;
+  a.cq = cq;
+  a.flags = flags;
+  a.bt = (const float *)(ws + L.bandtab);
+  return a;
+}
+
 // ---- per-kernel event timing ------------------------------------------------
 struct Timer {
   std::mutex mu;
@@ -669,6 +683,98 @@ int check_ptr(const void *ptr, const char *name) {
   if (((uintptr_t)ptr) % 16 != 0) return fail(MW_ERR_ARG, "%s is not 16-byte aligned", name);
   return MW_OK;
 }
+
+// Checkpoint replay: re-runs the forward from checkpoint k over its segment
+// [k C, min((k + 1) C, nt)) and stores each step's E and curl (fp32) in the
+// segment buffer at slot t - k C.  Used by the adjoint (segments newest
+// first) and the Born forward (oldest first).
+struct Replay {
+  const mw_params *p = nullptr;
+  char *ws = nullptr;
+  Layout L{};
+  cudaStream_t st = nullptr;
+  const float *f = nullptr;
+  const int64_t *src_idx = nullptr;
+  Chains ch{};
+  Launch lf{};
+  StepArgs fa{};
+  FwdMaps fA, fB;
+  float *rA = nullptr, *rB = nullptr;
+
+  int init(const mw_params *p_, char *ws_, const Layout &L_, cudaStream_t st_, const float *ca,
+           const float *cb, const float *cq, int *flags, const float *f_,
+           const int64_t *src_idx_, const Chains &ch_) {
+    p = p_;
+    ws = ws_;
+    L = L_;
+    st = st_;
+    f = f_;
+    src_idx = src_idx_;
+    ch = ch_;
+    lf = plan(p, false);
+    fa = step_args(p, lf, ca, cb, cq, flags, ws, L);
+    set_layout(fa, p, false);
+    fa.snap_pitch = p->nx;  // the fp32 segment
+    rA = (float *)(ws + L.rpA);
+    rB = (float *)(ws + L.rpB);
+    MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, cq, &fA));
+    MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, cq, &fB));
+    return MW_OK;
+  }
+  // replay segment k; *t0 / *t1 receive its steps
+  int segment(int k, int *launch_idx, int *t0_out, int *t1_out) {
+    const int C = p->ckpt_every;
+    const int t0 = k * C;
+    const int t1 = (t0 + C < p->nt) ? t0 + C : p->nt;
+    const int64_t numel = (int64_t)p->ny * p->nx;
+    char *seg_e = ws + L.seg;
+    char *seg_c = seg_e + (size_t)C * L.snap_step_bytes;
+    MW_CUDA(cudaMemcpyAsync(rA, ws + L.snap + (size_t)k * align256(L.state_bytes),
+                            L.state_bytes, cudaMemcpyDeviceToDevice, st));
+    float *rc = rA, *rn = rB;
+    for (int t = t0; t < t1; ++t) {
+      fa.in = fields_at(p, rc);
+      fa.out = fields_at(p, rn);
+      fa.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
+      fa.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
+      fa.ctr_slot = ((*launch_idx)++) & 1;
+      const FwdMaps &fm = rc == rA ? fA : fB;
+      MW_CUDA(timed(1, st, [&] {
+        return launch_forward(fm, fa, p->order, kStoreF32, kStoreNone, p->model_batched != 0,
+                              !p->cq_is_scalar, lf.grid, st);
+      }));
+      MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
+                                   f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
+                                   ch.src_lead, ch.src_next, p->n_src, nullptr, 0, nullptr, st));
+      std::swap(rc, rn);
+    }
+    *t0_out = t0;
+    *t1_out = t1;
+    return MW_OK;
+  }
+};
+
+// Host -> device-ring copies of the pinned-host snapshot store: step t goes
+// to ring slot t % kHostRing, on the copy stream, after the slot's previous
+// reader (if any) has finished.
+struct HostFetch {
+  HostCopies *hc;
+  const char *hbuf;
+  const char *se, *sc;
+  size_t step_bytes;
+  int fetch(int t, bool slot_was_used) {
+    const int slot = t % kHostRing;
+    if (slot_was_used) MW_CUDA(cudaStreamWaitEvent(hc->cs, hc->freed[slot], 0));
+    const char *h = hbuf + 2 * (size_t)t * step_bytes;
+    MW_CUDA(cudaMemcpyAsync((void *)(se + (size_t)slot * step_bytes), h, step_bytes,
+                            cudaMemcpyHostToDevice, hc->cs));
+    MW_CUDA(cudaMemcpyAsync((void *)(sc + (size_t)slot * step_bytes), h + step_bytes, step_bytes,
+                            cudaMemcpyHostToDevice, hc->cs));
+    MW_CUDA(cudaEventRecord(hc->filled[slot], hc->cs));
+    return MW_OK;
+  }
+};
+
 
 }  // namespace
 }  // namespace mw
@@ -776,15 +882,8 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   if (!state) MW_CUDA(cudaMemsetAsync(bufA, 0, L.state_bytes, st));
   if (p->nt == 0) return MW_OK;
 
-  StepArgs a{};
   const Launch lc = plan(p, false);
-  a.g = lc.g;
-  a.c = coef_of(p);
-  a.ca = ca;
-  a.cb = cb;
-  a.cq = cq;
-  a.flags = flags;
-  a.bt = (const float *)(ws + L.bandtab);
+  StepArgs a = step_args(p, lc, ca, cb, cq, flags, ws, L);
   set_layout(a, p, false);
   a.snap_pitch = L.snap_pitch;
   MW_TRY(stencil_prologue(p, cpml, ws, L, st));
@@ -896,16 +995,9 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   if (p->nt == 0) return MW_OK;
 
   const Launch la = plan(p, true);
-  StepArgs a{};
-  a.g = la.g;
-  a.c = coef_of(p);
-  a.ca = ca;
-  a.cb = cb;
-  a.cq = cq;
+  StepArgs a = step_args(p, la, ca, cb, cq, flags, ws, L);
   a.gca = gca;
   a.gcb = gcb;
-  a.flags = flags;
-  a.bt = (const float *)(ws + L.bandtab);
   set_layout(a, p, true);
   MW_TRY(stencil_prologue(p, cpml, ws, L, st));
   int launch_idx = 0;  // alternates the work counter between stencil launches
@@ -950,64 +1042,24 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     MW_TRY(hc.init());
     MW_CUDA(cudaEventRecord(hc.start, st));
     MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.start, 0));
-    const char *hbuf = (const char *)p->snap_host_ptr;
-    auto fetch = [&](int t) -> int {
-      const int slot = t % kHostRing;
-      if (t + kHostRing <= p->nt - 1) MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.freed[slot], 0));
-      const char *h = hbuf + 2 * (size_t)t * L.snap_step_bytes;
-      MW_CUDA(cudaMemcpyAsync((void *)(snap_e + (size_t)slot * L.snap_step_bytes), h,
-                              L.snap_step_bytes, cudaMemcpyHostToDevice, hc.cs));
-      MW_CUDA(cudaMemcpyAsync((void *)(snap_c + (size_t)slot * L.snap_step_bytes),
-                              h + L.snap_step_bytes, L.snap_step_bytes, cudaMemcpyHostToDevice,
-                              hc.cs));
-      MW_CUDA(cudaEventRecord(hc.filled[slot], hc.cs));
-      return MW_OK;
-    };
-    for (int t = p->nt - 1; t >= 0 && t >= p->nt - kHostRing; --t) MW_TRY(fetch(t));
+    HostFetch hf{&hc, (const char *)p->snap_host_ptr, snap_e, snap_c, L.snap_step_bytes};
+    for (int t = p->nt - 1; t >= 0 && t >= p->nt - kHostRing; --t) MW_TRY(hf.fetch(t, false));
     for (int t = p->nt - 1; t >= 0; --t) {
       const int slot = t % kHostRing;
       MW_CUDA(cudaStreamWaitEvent(st, hc.filled[slot], 0));
       MW_TRY(adj_step(t, slot));
       MW_CUDA(cudaEventRecord(hc.freed[slot], st));
-      if (t - kHostRing >= 0) MW_TRY(fetch(t - kHostRing));
+      if (t - kHostRing >= 0) MW_TRY(hf.fetch(t - kHostRing, true));
     }
   } else if (!ckpt) {
     for (int t = p->nt - 1; t >= 0; --t) MW_TRY(adj_step(t, t));
   } else {
     // checkpoint mode: replay each segment from its checkpoint, newest first
-    const Launch lf = plan(p, false);
-    StepArgs fa = a;
-    fa.g = lf.g;
-    set_layout(fa, p, false);
-    fa.snap_pitch = p->nx;  // the fp32 segment
-    float *rA = (float *)(ws + L.rpA), *rB = (float *)(ws + L.rpB);
-    FwdMaps fA, fB;
-    MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, cq, &fA));
-    MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, cq, &fB));
-    char *seg_e = ws + L.seg;
-    char *seg_c = seg_e + (size_t)C * L.snap_step_bytes;
+    Replay rp;
+    MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, src_idx, ch));
     for (int k = L.n_seg - 1; k >= 0; --k) {
-      const int t0 = k * C;
-      const int t1 = (t0 + C < p->nt) ? t0 + C : p->nt;
-      MW_CUDA(cudaMemcpyAsync(rA, ws + L.snap + (size_t)k * align256(L.state_bytes),
-                              L.state_bytes, cudaMemcpyDeviceToDevice, st));
-      float *rc_ = rA, *rn = rB;
-      for (int t = t0; t < t1; ++t) {
-        fa.in = fields_at(p, rc_);
-        fa.out = fields_at(p, rn);
-        fa.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
-        fa.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
-        const FwdMaps &fm = rc_ == rA ? fA : fB;
-        fa.ctr_slot = (launch_idx++) & 1;
-        MW_CUDA(timed(1, st, [&] {
-          return launch_forward(fm, fa, p->order, kStoreF32, kStoreNone, p->model_batched != 0,
-                                !p->cq_is_scalar, lf.grid, st);
-        }));
-        MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
-                                     f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
-                                     ch.src_lead, ch.src_next, p->n_src, nullptr, 0, nullptr, st));
-        std::swap(rc_, rn);
-      }
+      int t0, t1;
+      MW_TRY(rp.segment(k, &launch_idx, &t0, &t1));
       for (int t = t1 - 1; t >= t0; --t) MW_TRY(adj_step(t, t - t0));
     }
   }
@@ -1060,14 +1112,7 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
   float *dA = (float *)(ws + L.adA), *dB = (float *)(ws + L.adB);
   MW_CUDA(cudaMemsetAsync(dA, 0, L.state_bytes, st));
   const Launch lc = plan(p, false);
-  StepArgs b{};
-  b.g = lc.g;
-  b.c = coef_of(p);
-  b.ca = ca;
-  b.cb = cb;
-  b.cq = cq;
-  b.flags = flags;
-  b.bt = (const float *)(ws + L.bandtab);
+  StepArgs b = step_args(p, lc, ca, cb, cq, flags, ws, L);
   {
     size_t smem;
     forward_layout(p->order, bands(p).Wx, !p->cq_is_scalar, true, &b, &smem);
@@ -1117,66 +1162,25 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
     MW_TRY(hc.init());
     MW_CUDA(cudaEventRecord(hc.start, st));
     MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.start, 0));
-    const char *hbuf = (const char *)p->snap_host_ptr;
-    auto fetch = [&](int t) -> int {
-      const int slot = t % kHostRing;
-      if (t >= kHostRing) MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.freed[slot], 0));
-      const char *h = hbuf + 2 * (size_t)t * L.snap_step_bytes;
-      MW_CUDA(cudaMemcpyAsync((void *)(snap_e + (size_t)slot * L.snap_step_bytes), h,
-                              L.snap_step_bytes, cudaMemcpyHostToDevice, hc.cs));
-      MW_CUDA(cudaMemcpyAsync((void *)(snap_c + (size_t)slot * L.snap_step_bytes),
-                              h + L.snap_step_bytes, L.snap_step_bytes, cudaMemcpyHostToDevice,
-                              hc.cs));
-      MW_CUDA(cudaEventRecord(hc.filled[slot], hc.cs));
-      return MW_OK;
-    };
-    for (int t = 0; t < p->nt && t < kHostRing; ++t) MW_TRY(fetch(t));
+    HostFetch hf{&hc, (const char *)p->snap_host_ptr, snap_e, snap_c, L.snap_step_bytes};
+    for (int t = 0; t < p->nt && t < kHostRing; ++t) MW_TRY(hf.fetch(t, false));
     for (int t = 0; t < p->nt; ++t) {
       const int slot = t % kHostRing;
       MW_CUDA(cudaStreamWaitEvent(st, hc.filled[slot], 0));
       MW_TRY(born_step(t, slot));
       MW_CUDA(cudaEventRecord(hc.freed[slot], st));
-      if (t + kHostRing < p->nt) MW_TRY(fetch(t + kHostRing));
+      if (t + kHostRing < p->nt) MW_TRY(hf.fetch(t + kHostRing, true));
     }
   } else if (!ckpt) {
     for (int t = 0; t < p->nt; ++t) MW_TRY(born_step(t, t));
   } else {
     // replay each segment of the background from its checkpoint into the fp32
     // segment buffer, then take the segment's linearised steps
-    const int C = p->ckpt_every;
-    StepArgs fa{};
-    fa.g = lc.g;
-    fa.c = b.c;
-    fa.ca = ca;
-    fa.cb = cb;
-    fa.cq = cq;
-    fa.flags = flags;
-    fa.bt = b.bt;
-    set_layout(fa, p, false);
-    fa.snap_pitch = p->nx;
-    float *rA = (float *)(ws + L.rpA), *rB = (float *)(ws + L.rpB);
-    FwdMaps fA, fB;
-    MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, cq, &fA));
-    MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, cq, &fB));
+    Replay rp;
+    MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, src_idx, ch));
     for (int k = 0; k < L.n_seg; ++k) {
-      const int t0 = k * C;
-      const int t1 = (t0 + C < p->nt) ? t0 + C : p->nt;
-      MW_CUDA(cudaMemcpyAsync(rA, ws + L.snap + (size_t)k * align256(L.state_bytes),
-                              L.state_bytes, cudaMemcpyDeviceToDevice, st));
-      float *rc_ = rA, *rn = rB;
-      for (int t = t0; t < t1; ++t) {
-        fa.in = fields_at(p, rc_);
-        fa.out = fields_at(p, rn);
-        fa.snap_e = (char *)snap_e + (size_t)(t - t0) * L.snap_step_bytes;
-        fa.snap_c = (char *)snap_c + (size_t)(t - t0) * L.snap_step_bytes;
-        fa.ctr_slot = (launch_idx++) & 1;
-        MW_CUDA(launch_forward(rc_ == rA ? fA : fB, fa, p->order, kStoreF32, kStoreNone,
-                               p->model_batched != 0, !p->cq_is_scalar, lc.grid, st));
-        MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
-                                     f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
-                                     ch.src_lead, ch.src_next, p->n_src, nullptr, 0, nullptr, st));
-        std::swap(rc_, rn);
-      }
+      int t0, t1;
+      MW_TRY(rp.segment(k, &launch_idx, &t0, &t1));
       for (int t = t0; t < t1; ++t) MW_TRY(born_step(t, t - t0));
     }
   }
@@ -1366,15 +1370,8 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
   float *bufA = state;
   float *bufB = (float *)(ws + off_state);
   if (p->nt > 0) {
-    StepArgs a{};
     const Launch lc = plan(p, false);
-    a.g = lc.g;
-    a.c = coef_of(p);
-    a.ca = ca;
-    a.cb = cb;
-    a.cq = cq;
-    a.flags = flags;
-    a.bt = (const float *)(ws + L.bandtab);
+    StepArgs a = step_args(p, lc, ca, cb, cq, flags, ws, L);
     set_layout(a, p, false);
     MW_TRY(stencil_prologue(p, cpml, ws, L, st));
     FwdMaps mA, mB;

@@ -503,8 +503,11 @@ __global__ void __launch_bounds__(128, BORN != kStoreNone ? 3 : (P <= 3 ? 5 : 4)
   // two boxes: Ca at kF_MD, Cb at kF_MD + 128 (every box starts 128-aligned)
   w.ca_o = (kF_MD + (a.md_pair && a.md_swap ? 120 : 0)) * 4;
   w.cb_o = (kF_MD + (a.md_pair ? (a.md_swap ? 0 : 120) : 128)) * 4;
-  w.dca_o = (a.fo[kFoBd] + (a.bd_pair && a.bd_swap ? 120 : 0)) * 4;
-  w.dcb_o = (a.fo[kFoBd] + (a.bd_pair ? (a.bd_swap ? 0 : 120) : 128)) * 4;
+  w.dca_o = w.dcb_o = 0;
+  if constexpr (BORN != kStoreNone) {
+    w.dca_o = (a.fo[kFoBd] + (a.bd_pair && a.bd_swap ? 120 : 0)) * 4;
+    w.dcb_o = (a.fo[kFoBd] + (a.bd_pair ? (a.bd_swap ? 0 : 120) : 128)) * 4;
+  }
   w.ring = Ring{0, 0u};
   const Geom &g = a.g;
   const int n_items = g.S * g.n_strips * g.n_chunks;
