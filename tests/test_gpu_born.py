@@ -77,3 +77,35 @@ def test_gpu_born_is_the_transpose_of_the_gpu_gradient(order):
     lhs = float(np.sum(born * r))
     rhs = float(np.sum(dca * gca.sum(0).cpu().numpy()) + np.sum(dcb * gcb.sum(0).cpu().numpy()))
     assert abs(lhs - rhs) <= 1e-5 * max(abs(lhs), abs(rhs))
+
+
+@pytest.mark.parametrize("mode", ["ckpt", "fp32", "fp8"])
+def test_workspace_reuse_adjoint_twice_and_born_around_it(mode):
+    """One forward, then adjoint, Born, adjoint, Born on the same workspace:
+    each repeated call returns bit-identical results (the checkpoint replays
+    and the Born state never disturb what a later call needs)."""
+    sim, dt, nt, f, dca, dcb, g = _case(4, False, 840)
+    prob = _problem(sim, nt, dt, mode)
+    run_forward(prob, f)
+    r = torch.as_tensor(f32(g.normal(size=(nt, 2, 6))), dtype=torch.float32).cuda()
+    dca_t = torch.as_tensor(dca, dtype=torch.float32)
+    dcb_t = torch.as_tensor(dcb, dtype=torch.float32)
+    g1 = [t.clone() for t in prob.adjoint(r)[:2]]
+    b1 = prob.born(dca_t, dcb_t).clone()
+    g2 = [t.clone() for t in prob.adjoint(r)[:2]]
+    b2 = prob.born(dca_t, dcb_t).clone()
+    torch.cuda.synchronize()
+    assert prob.status() == 0
+    assert torch.equal(g1[0], g2[0]) and torch.equal(g1[1], g2[1])
+    assert torch.equal(b1, b2)
+
+
+def test_born_with_no_steps_is_a_no_op():
+    sim, dt, _, f, dca, dcb, _ = _case(4, False, 850)
+    prob = problem_from_sim(sim, 0, dt, 6, snapshot="fp32")
+    rec = torch.full((1, 2, 6), 7.0, device="cuda")
+    prob.born(torch.as_tensor(dca, dtype=torch.float32), torch.as_tensor(dcb, dtype=torch.float32),
+              rec=rec)
+    torch.cuda.synchronize()
+    assert prob.status() == 0
+    assert float(rec.min()) == 7.0 and float(rec.max()) == 7.0
