@@ -1,0 +1,59 @@
+"""bench.py on the host: the algorithmic byte model per pass, the sample
+sizing of the oracle baseline, and the reference arm's JSON line (the fp64
+oracle timed on host cores), run as the driver runs it."""
+from __future__ import annotations
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from adjoint_state_gradients_b200 import synth  # noqa: E402
+
+
+def test_byte_model_of_the_headline_sweep():
+    wl = synth.WORKLOADS[4]
+    b = bench.alg_bytes(wl, wl.n_shots)
+    band = 16.0 * (2 * 40 / 2128 + 2 * 40 / 2128)
+    assert b["forward"] == pytest.approx(24 + 1 + band + 28 / 64)
+    assert b["replay"] == pytest.approx(24 + 1 + band + 8 + 28 / 64)
+    assert b["adjoint"] == pytest.approx(24 + 1 + band + 8 + 16)
+    assert sum(b.values()) == pytest.approx(111.49, abs=0.01)
+    assert bench.pass_classes(wl) == {"forward": 0, "replay": 1, "adjoint": 2}
+
+
+def test_byte_model_of_the_other_storage_modes():
+    w3, w5 = synth.WORKLOADS[3], synth.WORKLOADS[5]
+    b3, b5 = bench.alg_bytes(w3, w3.n_shots), bench.alg_bytes(w5, w5.n_shots)
+    assert b3["adjoint"] - b3["forward"] == pytest.approx(16.0)   # gradient read + write
+    assert set(b5) == {"forward"}
+    assert b5["forward"] > 24 + 8                                  # per-shot model: 8 B per cell
+    assert bench.pass_classes(w5) == {"forward": 0}
+
+
+def test_oracle_sample_is_bounded():
+    for n in range(1, 6):
+        wl = synth.WORKLOADS[n]
+        k = bench.sample_steps(wl, 1.2e9)
+        assert 16 <= k <= wl.nt
+        assert k * wl.ny * wl.nx <= max(1.2e9, 16 * wl.ny * wl.nx)
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "1", "--steps", "1", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["config"]["workload"] == synth.WORKLOADS[1].name
