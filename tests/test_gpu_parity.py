@@ -591,3 +591,29 @@ def test_host_side_argument_errors():
     with pytest.raises(mwtm.MWError) as e:
         mwtm.tm_forward(p, dummy, dummy, dummy, dummy, dummy, idx, idx, None, dummy, ws)
     assert e.value.code == mwtm.MW_ERR_WORKSPACE
+
+
+def test_no_sources_and_no_receivers():
+    """A problem with receivers but no sources (the field comes from a given
+    initial state), and one with sources but no receivers (the adjoint then
+    has no residual to inject, so its gradients vanish)."""
+    S, ny, nx, nt = 2, 44, 64, 40
+    sim0, dt, _ = small_sim(930, ny, nx, S, 0, 5, 4, 5, round_f32=True)
+    st0 = np.zeros((7, S, ny, nx))
+    st0[:3] = f32(synth.rng(931).normal(size=(3, S, ny, nx)))  # Ey, Hx, Hz; memories zero
+    fw = sim0.forward(np.zeros((nt, S, 0)), state=st0)
+    prob = problem_from_sim(sim0, nt, dt, 5)
+    state = prob.new_state()
+    SN = S * ny * nx
+    state[:3 * SN] = torch.as_tensor(st0[:3].reshape(-1), dtype=torch.float32)
+    rec = run_forward(prob, np.zeros((nt, S, 1)), state=state)
+    assert rel_l2(rec, fw["rec"]) <= REC_TOL
+    assert prob.status() == mwtm.MW_OK
+
+    sim1, dt1, _ = small_sim(932, ny, nx, S, 2, 0, 4, 5, round_f32=True)
+    f = f32(synth.rng(933).normal(size=(nt, S, 2)))
+    prob1 = problem_from_sim(sim1, nt, dt1, 5)
+    run_forward(prob1, f)
+    gca, gcb, gf = run_adjoint(prob1, np.zeros((nt, S, 1)))
+    assert np.all(gca == 0) and np.all(gcb == 0) and np.all(gf == 0)
+    assert prob1.status() == mwtm.MW_OK
