@@ -27,7 +27,9 @@ class Problem:
     """One 2-D TM setup: grid, stencil order, time step, shots, storage mode.
 
     src_idx [S, n_src] / rec_idx [S, n_rec] are flat cell indices y*nx + x
-    (-1 = inactive).  snapshot: "none" | "fp32" | "bf16" | "fp8" | "ckpt".
+    (-1 = inactive).  snapshot: "none" | "fp32" | "bf16" | "fp8" | "ckpt" |
+    "ckpt_ey" (checkpoints whose replay keeps E alone; the Cb gradient by
+    summation by parts).
     snapshot_host: keep the fp32 / bf16 / fp8 snapshots in page-locked host
     memory (staged through a 3-step device ring) instead of the workspace.
     """

@@ -52,7 +52,7 @@ __global__ void k_inject_sample(float *__restrict__ field, int64_t numel,
                                 const float *__restrict__ vals_t, const int64_t *__restrict__ idx_a,
                                 const int *__restrict__ lead, const int *__restrict__ next, int na,
                                 const int64_t *__restrict__ idx_b, int nb,
-                                float *__restrict__ out_t) {
+                                float *__restrict__ out_t, const SbpTerms sbp) {
   const int s = blockIdx.x;
   float *e = field + (int64_t)s * numel;
   // programmatic dependent launch (no-ops without the launch attribute):
@@ -62,6 +62,7 @@ __global__ void k_inject_sample(float *__restrict__ field, int64_t numel,
   if (vals_t != nullptr) {
     const int64_t base = (int64_t)s * na;
     for (int k = threadIdx.x; k < na; k += blockDim.x) {
+      if (sbp.acc_a != nullptr) sbp.acc_a[base + k] += vals_t[base + k] * sbp.pair_t[base + k];
       if (!lead[base + k]) continue;
       float v = vals_t[base + k];
       for (int j = next[base + k]; j >= 0; j = next[base + j]) v += vals_t[base + j];
@@ -71,9 +72,52 @@ __global__ void k_inject_sample(float *__restrict__ field, int64_t numel,
   __syncthreads();
   if (out_t != nullptr) {
     for (int k = threadIdx.x; k < nb; k += blockDim.x) {
-      const int64_t i = idx_b[(int64_t)s * nb + k];
-      out_t[(int64_t)s * nb + k] = (i >= 0 && i < numel) ? e[i] : 0.f;
+      const int64_t j = (int64_t)s * nb + k;
+      const int64_t i = idx_b[j];
+      const float v = (i >= 0 && i < numel) ? e[i] : 0.f;
+      out_t[j] = v;
+      if (sbp.acc_b != nullptr) sbp.acc_b[j] += sbp.w_t[j] * v;
     }
+  }
+}
+
+__global__ void k_sbp_init(float *__restrict__ P, const float *__restrict__ lam,
+                           const float *__restrict__ e, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    P[i] = lam[i] * e[i];
+}
+
+// One thread per shot, so that duplicate cells add in index order.
+__global__ void k_sbp_scatter(float *__restrict__ P, int64_t numel, int S,
+                              const int64_t *__restrict__ rec_idx,
+                              const float *__restrict__ acc_rec, int n_rec,
+                              const int64_t *__restrict__ src_idx,
+                              const float *__restrict__ acc_src, int n_src) {
+  const int s = blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= S) return;
+  float *p = P + (int64_t)s * numel;
+  for (int k = 0; k < n_rec; ++k) {
+    const int64_t i = rec_idx[(int64_t)s * n_rec + k];
+    if (i >= 0 && i < numel) p[i] += acc_rec[(int64_t)s * n_rec + k];
+  }
+  for (int k = 0; k < n_src; ++k) {
+    const int64_t i = src_idx[(int64_t)s * n_src + k];
+    if (i >= 0 && i < numel) p[i] -= acc_src[(int64_t)s * n_src + k];
+  }
+}
+
+__global__ void k_sbp_finish(const float *__restrict__ P, const float *__restrict__ cb,
+                             float *__restrict__ gcb, int S, int ny, int nx, int batched,
+                             int mask_pml) {
+  const int64_t numel = (int64_t)ny * nx, n = (int64_t)S * numel;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t s = i / numel, c = i - s * numel;
+    const int y = (int)(c / nx), x = (int)(c - (int64_t)y * nx);
+    if (mask_pml > 0 && (y < mask_pml || y >= ny - mask_pml || x < mask_pml || x >= nx - mask_pml))
+      continue;
+    gcb[i] += P[i] / cb[batched ? i : c];
   }
 }
 
@@ -236,12 +280,43 @@ cudaError_t launch_dup_chains(const int64_t *idx, int S, int n, int64_t numel, i
 
 cudaError_t launch_inject_sample(float *field, int64_t numel, int S, const float *vals_t,
                                  const int64_t *idx_a, const int *lead, const int *next, int na,
-                                 const int64_t *idx_b, int nb, float *out_t, cudaStream_t st) {
+                                 const int64_t *idx_b, int nb, float *out_t, cudaStream_t st,
+                                 const SbpTerms &sbp) {
   if ((na == 0 || vals_t == nullptr) && (nb == 0 || out_t == nullptr)) return cudaSuccess;
+  SbpTerms t = sbp;
+  if (na == 0 || vals_t == nullptr || t.pair_t == nullptr) t.acc_a = nullptr;
+  if (nb == 0 || out_t == nullptr || t.w_t == nullptr) t.acc_b = nullptr;
   const cudaError_t e = launch_dependent(k_inject_sample, S, 256, 0, st, field, numel,
                                          na > 0 ? vals_t : nullptr, idx_a, lead, next, na, idx_b,
-                                         nb, nb > 0 ? out_t : nullptr);
+                                         nb, nb > 0 ? out_t : nullptr, t);
   if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sbp_init(float *P, const float *lam, const float *e, int64_t n,
+                            cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  k_sbp_init<<<grid_for(n, 256), 256, 0, st>>>(P, lam, e, n);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sbp_scatter(float *P, int64_t numel, int S, const int64_t *rec_idx,
+                               const float *acc_rec, int n_rec, const int64_t *src_idx,
+                               const float *acc_src, int n_src, cudaStream_t st) {
+  if (S <= 0 || (n_rec == 0 && n_src == 0)) return cudaSuccess;
+  k_sbp_scatter<<<(S + 63) / 64, 64, 0, st>>>(P, numel, S, rec_idx, acc_rec, n_rec, src_idx,
+                                                acc_src, n_src);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sbp_finish(const float *P, const float *cb, float *gcb, int S, int ny, int nx,
+                              int batched, int mask_pml, cudaStream_t st) {
+  const int64_t n = (int64_t)S * ny * nx;
+  if (n <= 0) return cudaSuccess;
+  k_sbp_finish<<<grid_for(n, 256), 256, 0, st>>>(P, cb, gcb, S, ny, nx, batched, mask_pml);
   count_launches(1);
   return cudaGetLastError();
 }

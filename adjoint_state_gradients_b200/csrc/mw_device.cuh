@@ -59,7 +59,7 @@ __device__ __forceinline__ void fence_proxy_async() {
 // the largest finite value, no scaling: the maxwell.cu page's fp8 storage).
 template <int STORE>
 __device__ __forceinline__ void snap_store(void *base, int64_t elem, const F4 &v) {
-  if constexpr (STORE == kStoreF32) {
+  if constexpr (STORE == kStoreF32 || STORE == kStoreEy) {
     st4(reinterpret_cast<float *>(base) + elem, v);
   } else if constexpr (STORE == kStoreBF16) {
     __nv_bfloat162 lo = __floats2bfloat162_rn(v.v[0], v.v[1]);
@@ -150,10 +150,10 @@ __device__ __forceinline__ void tma5s(uint32_t dst, const CUtensorMap *map, int 
       : "memory");
 }
 // Staged snapshot float4 (4 cells) at byte address addr: float32, bf16 or
-// FP8 E4M3 (SNAP = kStoreF32 / kStoreBF16 / kStoreFP8).
+// FP8 E4M3 (SNAP = kStoreF32 or kStoreEy / kStoreBF16 / kStoreFP8).
 template <int SNAP>
 __device__ __forceinline__ F4 snap_lds_s(uint32_t addr) {
-  if constexpr (SNAP == kStoreF32) {
+  if constexpr (SNAP == kStoreF32 || SNAP == kStoreEy) {
     return lds4s(addr);
   } else if constexpr (SNAP == kStoreBF16) {
     uint32_t lo, hi;
@@ -191,7 +191,7 @@ __device__ __forceinline__ void sts4p(bool p, uint32_t addr, const F4 &v) {
 // Snapshot row store (4 cells) where p holds.
 template <int STORE>
 __device__ __forceinline__ void snap_store_p(bool p, void *base, int64_t elem, const F4 &v) {
-  if constexpr (STORE == kStoreF32) {
+  if constexpr (STORE == kStoreF32 || STORE == kStoreEy) {
     st4p(p, reinterpret_cast<float *>(base) + elem, v);
   } else if constexpr (STORE == kStoreBF16) {
     __nv_bfloat162 lo = __floats2bfloat162_rn(v.v[0], v.v[1]);

@@ -83,6 +83,12 @@ size_t state_floats(const mw_params *p) {
   return S * ny * nx * 3 + S * ny * 2 * b.Wx * 2 + S * 2 * b.Wz * nx * 2;
 }
 
+// checkpoint modes: segment replay (pair store), or the E snapshot alone with
+// the summation-by-parts Cb gradient
+bool is_ckpt(const mw_params *p) {
+  return p->snap_mode == MW_SNAP_CKPT || p->snap_mode == MW_SNAP_CKPT_EY;
+}
+
 int check_params(const mw_params *p, bool cfl) {
   if (!p) return fail(MW_ERR_ARG, "params is NULL");
   double c[4];
@@ -98,12 +104,12 @@ int check_params(const mw_params *p, bool cfl) {
   const Bands b = bands(p);
   if (2 * b.Wx > p->nx || 2 * b.Wz > p->ny)
     return fail(MW_ERR_ARG, "CPML band %d does not fit a %d x %d grid", p->n_pml, p->ny, p->nx);
-  if (p->snap_mode < MW_SNAP_NONE || p->snap_mode > MW_SNAP_FP8)
+  if (p->snap_mode < MW_SNAP_NONE || p->snap_mode > MW_SNAP_CKPT_EY)
     return fail(MW_ERR_ARG, "snap_mode = %d", p->snap_mode);
   if (p->snap_host && p->snap_mode != MW_SNAP_FP32 && p->snap_mode != MW_SNAP_BF16 &&
       p->snap_mode != MW_SNAP_FP8)
     return fail(MW_ERR_ARG, "snap_host needs snap_mode FP32, BF16 or FP8 (got %d)", p->snap_mode);
-  if (p->snap_mode == MW_SNAP_CKPT && p->ckpt_every < 1)
+  if (is_ckpt(p) && p->ckpt_every < 1)
     return fail(MW_ERR_ARG, "ckpt_every = %d", p->ckpt_every);
   if (2 * b.Wx > 256)
     return fail(MW_ERR_UNSUPPORTED, "n_pml = %d: a band row exceeds one TMA box (n_pml <= 123)",
@@ -168,7 +174,7 @@ Layout layout(const mw_params *p) {
     // ([2][kHostRing] step slots) that the host copies pass through
     const size_t steps = p->snap_host ? (size_t)kHostRing : (size_t)p->nt;
     off += align256(2 * steps * L.snap_step_bytes);
-  } else if (p->snap_mode == MW_SNAP_CKPT) {
+  } else if (is_ckpt(p)) {
     L.n_seg = p->nt > 0 ? (p->nt + p->ckpt_every - 1) / p->ckpt_every : 0;
     L.rpA = off; off += sb;
     L.rpB = off; off += sb;
@@ -177,6 +183,15 @@ Layout layout(const mw_params *p) {
     L.snap_step_bytes = SN * 4;
     L.seg = off;
     off += align256(2 * (size_t)p->ckpt_every * L.snap_step_bytes);
+  }
+  L.sbp = L.rcopy = L.acc = 0;
+  if (p->snap_mode == MW_SNAP_CKPT_EY) {
+    L.sbp = off; off += align256(SN * sizeof(float));
+    L.rcopy = off; off += align256((size_t)p->nt * p->n_shots * p->n_rec * sizeof(float));
+    // the receiver and source sums, then lambda_E sampled at the sources
+    // when the caller asks for no grad_f
+    L.acc = off;
+    off += align256((size_t)p->n_shots * (p->n_rec + 2 * (size_t)p->n_src) * sizeof(float));
   }
   L.total = off;
   return L;
@@ -554,7 +569,7 @@ int born_maps(const mw_params *p, const float *dca, const float *dcb, const void
 
 int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb,
              const float *cq, const float *gca, const float *gcb, const void *se, const void *sc,
-             int snap_elem, int snap_steps, int snap_pitch, AdjMaps *m) {
+             int snap_elem, int snap_steps, int snap_pitch, bool ey_only, AdjMaps *m) {
   memset(m, 0, sizeof *m);
   const Bands bd = bands(p);
   const uint64_t nx = p->nx, ny = p->ny, S = p->n_shots, Sm = p->model_batched ? p->n_shots : 1;
@@ -569,7 +584,15 @@ int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float 
     MW_TRY(encode_rows(&m->map[kAMapCB], cb, 4, 3, nx, ny, Sm, 1, 128));
   }
   MW_TRY(encode_rows(&m->map[kAMapHX], in.hx, 4, 3, nx, ny, S, 1, 112));
-  {
+  if (ey_only) {
+    // (x, y, shot, step): the E snapshots; and lambda_E of the input again
+    const uint64_t e = (uint64_t)snap_elem, pitch = (uint64_t)snap_pitch;
+    const uint64_t dims[4] = {nx, ny, S, (uint64_t)snap_steps};
+    const uint64_t strides[3] = {pitch * e, pitch * ny * e, pitch * ny * S * e};
+    const uint32_t box[4] = {112, 1, 1, 1};
+    MW_TRY(encode_map(&m->map[kAMapSS], se, snap_elem, 4, dims, strides, box));
+    MW_TRY(encode_rows(&m->map[kAMapLE], in.ey, 4, 3, nx, ny, S, 1, 112));
+  } else {
     // (x, y, shot, step, field): the curl snapshots follow the E snapshots
     const uint64_t e = (uint64_t)snap_elem;
     const uint64_t dims[5] = {nx, ny, S, (uint64_t)snap_steps, 2};
@@ -700,6 +723,8 @@ struct Replay {
   StepArgs fa{};
   FwdMaps fA, fB;
   float *rA = nullptr, *rB = nullptr;
+  int store = kStoreF32;  // the segment: E and curl, or E alone (kStoreEy)
+  float *last = nullptr;  // the state after the latest replayed segment
 
   int init(const mw_params *p_, char *ws_, const Layout &L_, cudaStream_t st_, const float *ca,
            const float *cb, const float *cq, int *flags, const float *f_,
@@ -740,7 +765,7 @@ struct Replay {
       fa.ctr_slot = ((*launch_idx)++) & 1;
       const FwdMaps &fm = rc == rA ? fA : fB;
       MW_CUDA(timed(1, st, [&] {
-        return launch_forward(fm, fa, p->order, kStoreF32, kStoreNone, p->model_batched != 0,
+        return launch_forward(fm, fa, p->order, store, kStoreNone, p->model_batched != 0,
                               !p->cq_is_scalar, lf.grid, st);
       }));
       MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
@@ -748,6 +773,7 @@ struct Replay {
                                    ch.src_lead, ch.src_next, p->n_src, nullptr, 0, nullptr, st));
       std::swap(rc, rn);
     }
+    last = rc;
     *t0_out = t0;
     *t1_out = t1;
     return MW_OK;
@@ -867,6 +893,10 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   if (!p->cq_is_scalar && (rc = check_ptr(cq, "cq"))) return rc;
   if (p->n_src > 0 && (!f || !src_idx)) return fail(MW_ERR_ARG, "sources need f and src_idx");
   if (p->n_rec > 0 && rec && !rec_idx) return fail(MW_ERR_ARG, "receivers need rec_idx");
+  // MW_SNAP_CKPT_EY keeps its own copy of the records for the adjoint
+  const bool ey_only = p->snap_mode == MW_SNAP_CKPT_EY;
+  if (ey_only && p->n_rec > 0 && !rec_idx)
+    return fail(MW_ERR_ARG, "snap_mode CKPT_EY: receivers need rec_idx");
   if (state && (rc = check_ptr(state, "state"))) return rc;
   if (!workspace) return fail(MW_ERR_WORKSPACE, "workspace is NULL");
   const Layout L = layout(p);
@@ -898,7 +928,8 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   if (p->n_src > 0)
     MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
                               flags, st));
-  if (p->n_rec > 0 && rec)  // chains unused here: this validates the receiver indices
+  float *rec_out = ey_only ? (float *)(ws + L.rcopy) : rec;
+  if (p->n_rec > 0 && rec_out)  // chains unused here: this validates the receiver indices
     MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
                               flags, st));
   const bool host = p->snap_host != 0;
@@ -910,7 +941,7 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   char *hbuf = (char *)p->snap_host_ptr;
   float *cur = bufA, *nxt = bufB;
   for (int t = 0; t < p->nt; ++t) {
-    if (p->snap_mode == MW_SNAP_CKPT && t % p->ckpt_every == 0) {
+    if (is_ckpt(p) && t % p->ckpt_every == 0) {
       char *ck = ws + L.snap + (size_t)(t / p->ckpt_every) * align256(L.state_bytes);
       MW_CUDA(cudaMemcpyAsync(ck, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
     }
@@ -939,9 +970,13 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
     MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots,
                                  f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
                                  ch.src_lead, ch.src_next, p->n_src, rec_idx, p->n_rec,
-                                 rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, st));
+                                 rec_out ? rec_out + (int64_t)t * p->n_shots * p->n_rec : nullptr,
+                                 st));
     std::swap(cur, nxt);
   }
+  if (ey_only && rec && p->n_rec > 0)
+    MW_CUDA(cudaMemcpyAsync(rec, rec_out, (size_t)p->nt * p->n_shots * p->n_rec * sizeof(float),
+                            cudaMemcpyDeviceToDevice, st));
   if (host)  // the call's stream completes only after every copy reached the host
     for (int k = 0; k < kHostRing && k < p->nt; ++k)
       MW_CUDA(cudaStreamWaitEvent(st, hc.freed[(p->nt - 1 - k) % kHostRing], 0));
@@ -968,7 +1003,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   if (!p->cq_is_scalar && (rc = check_ptr(cq, "cq"))) return rc;
   if (p->n_rec > 0 && (!res || !rec_idx)) return fail(MW_ERR_ARG, "receivers need res and rec_idx");
   if (p->n_src > 0 && grad_f && !src_idx) return fail(MW_ERR_ARG, "grad_f needs src_idx");
-  if (p->snap_mode == MW_SNAP_CKPT && p->n_src > 0 && (!f || !src_idx))
+  if (is_ckpt(p) && p->n_src > 0 && (!f || !src_idx))
     return fail(MW_ERR_ARG, "checkpoint replay needs f and src_idx");
   if (adj_state && (rc = check_ptr(adj_state, "adj_state"))) return rc;
   if (!workspace) return fail(MW_ERR_WORKSPACE, "workspace is NULL");
@@ -986,7 +1021,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   if (p->n_rec > 0)
     MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
                               flags, st));
-  if (p->n_src > 0 && p->snap_mode == MW_SNAP_CKPT)
+  if (p->n_src > 0 && is_ckpt(p))
     MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
                               flags, st));
   float *adA = adj_state ? adj_state : (float *)(ws + L.adA);
@@ -995,36 +1030,63 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   if (p->nt == 0) return MW_OK;
 
   const Launch la = plan(p, true);
+  // MW_SNAP_CKPT_EY: the Cb gradient accumulates E^t G^t into P (workspace)
+  // and the end-term sums beside it; grad_cb_shot receives P / Cb at the end
+  const bool ey_only = p->snap_mode == MW_SNAP_CKPT_EY;
+  float *sbp = ey_only ? (float *)(ws + L.sbp) : nullptr;
+  float *acc_rec = ey_only ? (float *)(ws + L.acc) : nullptr;
+  float *acc_src = ey_only ? acc_rec + (size_t)p->n_shots * p->n_rec : nullptr;
+  const float *rcopy = ey_only ? (const float *)(ws + L.rcopy) : nullptr;
+  if (ey_only) {
+    MW_CUDA(cudaMemsetAsync(sbp, 0, SN * sizeof(float), st));
+    if (p->n_rec + p->n_src > 0)
+      MW_CUDA(cudaMemsetAsync(acc_rec, 0,
+                              (size_t)p->n_shots * (p->n_rec + p->n_src) * sizeof(float), st));
+  }
   StepArgs a = step_args(p, la, ca, cb, cq, flags, ws, L);
   a.gca = gca;
-  a.gcb = gcb;
+  a.gcb = ey_only ? sbp : gcb;
   set_layout(a, p, true);
   MW_TRY(stencil_prologue(p, cpml, ws, L, st));
   int launch_idx = 0;  // alternates the work counter between stencil launches
 
   // snapshot source of the adjoint: the full store, or the replay segment
-  const bool ckpt = p->snap_mode == MW_SNAP_CKPT;
+  const bool ckpt = is_ckpt(p);
   // snapshots the adjoint reads: the full store, or the fp32 replay segment
-  const int snap = ckpt ? kStoreF32 : snap_store_kind(p->snap_mode);
+  // (E and curl, or E alone)
+  const int snap = ey_only ? kStoreEy : ckpt ? kStoreF32 : snap_store_kind(p->snap_mode);
   const int snap_elem = ckpt ? 4 : (int)snap_elem_bytes(p->snap_mode);
   const bool host = p->snap_host != 0;
   const int C = ckpt ? p->ckpt_every : host ? kHostRing : p->nt;
   const char *snap_e = ckpt ? ws + L.seg : ws + L.snap;
   const char *snap_c = snap_e + (size_t)C * L.snap_step_bytes;
   AdjMaps mA, mB;
-  MW_TRY(adj_maps(p, fields_at(p, adA), ca, cb, cq, gca, gcb, snap_e, snap_c, snap_elem, C, L.snap_pitch, &mA));
-  MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, cq, gca, gcb, snap_e, snap_c, snap_elem, C, L.snap_pitch, &mB));
+  MW_TRY(adj_maps(p, fields_at(p, adA), ca, cb, cq, gca, a.gcb, snap_e, snap_c, snap_elem, C,
+                  L.snap_pitch, ey_only, &mA));
+  MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, cq, gca, a.gcb, snap_e, snap_c, snap_elem, C,
+                  L.snap_pitch, ey_only, &mB));
 
   float *cur = adA, *nxt = adB;
+  // with the summation-by-parts Cb gradient the source term needs lambda_E at
+  // the sources every step, grad_f or not: sampled into the end of acc
+  float *gf_scratch = ey_only && !grad_f ? acc_src + (size_t)p->n_shots * p->n_src : nullptr;
   auto adj_step = [&](int t, int slot) -> int {
+    SbpTerms sb;
+    float *gf_t = grad_f ? grad_f + (int64_t)t * p->n_shots * p->n_src : gf_scratch;
+    if (ey_only) {
+      sb.pair_t = rcopy + (int64_t)t * p->n_shots * p->n_rec;
+      sb.acc_a = acc_rec;
+      sb.w_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
+      sb.acc_b = acc_src;
+    }
     MW_CUDA(launch_inject_sample(cur, numel, p->n_shots,
                                  res ? res + (int64_t)t * p->n_shots * p->n_rec : nullptr,
                                  rec_idx, ch.rec_lead, ch.rec_next, p->n_rec, src_idx, p->n_src,
-                                 grad_f ? grad_f + (int64_t)t * p->n_shots * p->n_src : nullptr,
-                                 st));
+                                 gf_t, st, sb));
     a.in = fields_at(p, cur);
     a.out = fields_at(p, nxt);
     a.snap_t = slot;
+    a.tzero = t == 0 ? 1 : 0;
     a.ctr_slot = (launch_idx++) & 1;
     const AdjMaps &m = cur == adA ? mA : mB;
     MW_CUDA(timed(2, st, [&] {
@@ -1057,13 +1119,24 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     // checkpoint mode: replay each segment from its checkpoint, newest first
     Replay rp;
     MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, src_idx, ch));
+    rp.store = ey_only ? kStoreEy : kStoreF32;
     for (int k = L.n_seg - 1; k >= 0; --k) {
       int t0, t1;
       MW_TRY(rp.segment(k, &launch_idx, &t0, &t1));
+      // a given adjoint start state meets the forward's final E: P starts
+      // at lambda~_E^{nt} E^{nt}
+      if (ey_only && adj_state && k == L.n_seg - 1)
+        MW_CUDA(launch_sbp_init(sbp, adA, rp.last, SN, st));
       for (int t = t1 - 1; t >= t0; --t) MW_TRY(adj_step(t, t - t0));
     }
   }
   if (cur != adA) MW_CUDA(cudaMemcpyAsync(adA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
+  if (ey_only) {
+    MW_CUDA(launch_sbp_scatter(sbp, numel, p->n_shots, rec_idx, acc_rec, res ? p->n_rec : 0,
+                               src_idx, acc_src, f ? p->n_src : 0, st));
+    MW_CUDA(launch_sbp_finish(sbp, cb, gcb, p->n_shots, p->ny, p->nx, p->model_batched,
+                              p->grad_mask_pml ? p->n_pml : 0, st));
+  }
   if (p->check_finite) {
     MW_CUDA(launch_check_finite(gca, SN, flags, st));
     MW_CUDA(launch_check_finite(gcb, SN, flags, st));
@@ -1087,7 +1160,7 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
   if (!cq) return fail(MW_ERR_ARG, "cq is NULL");
   if (!p->cq_is_scalar && (rc = check_ptr(cq, "cq"))) return rc;
   if (p->n_rec > 0 && (!rec || !rec_idx)) return fail(MW_ERR_ARG, "receivers need rec and rec_idx");
-  const bool ckpt = p->snap_mode == MW_SNAP_CKPT;
+  const bool ckpt = is_ckpt(p);
   if (ckpt && p->n_src > 0 && (!f || !src_idx))
     return fail(MW_ERR_ARG, "checkpoint replay needs f and src_idx");
   if (!workspace) return fail(MW_ERR_WORKSPACE, "workspace is NULL");

@@ -77,6 +77,7 @@ struct StepArgs {
   // snapshot tensor maps
   float *gca, *gcb;
   int snap_t;
+  int tzero;          // adjoint, kStoreEy: this launch is step t = 0
   int *flags;         // device status words (wait timeouts, work counters)
   int ctr_slot;       // work counter of this launch (flags[kCtrBase + ctr_slot])
   // CPML band coefficients (BandTab layout), float4-aligned, 1/k precomputed
@@ -128,9 +129,12 @@ struct FwdMaps {
 //   kAMapMX  the x-band memories at the H and E nodes (adjacent arrays) as
 //            one pair box of whole band rows
 //   kAMapMZE / kAMapMZH  z-band memories, 112 wide from x0
+//   kAMapLE  lambda_E of the input, 112 wide from x0 (kStoreEy: the gradients
+//            of a row are formed at its E update, 2P - 1 rows after its
+//            first fetch; kAMapSS is then the E snapshot alone, 4-D)
 enum AdjMap {
   kAMapEH = 0, kAMapMD, kAMapCB, kAMapHX, kAMapSS, kAMapGG, kAMapGB, kAMapCQ, kAMapMX,
-  kAMapMZE, kAMapMZH, kAdjMaps
+  kAMapMZE, kAMapMZH, kAMapLE, kAdjMaps
 };
 struct AdjMaps {
   CUtensorMap map[kAdjMaps];
@@ -187,6 +191,9 @@ struct Layout {
   size_t seg;         // checkpoint mode: fp32 segment snapshot buffer
   size_t chains;      // duplicate chains of the source / receiver indices
   size_t bandtab;     // CPML band coefficient table (BandTab)
+  // MW_SNAP_CKPT_EY: the Cb-gradient accumulator [S][ny][nx], the record copy
+  // [nt][S][n_rec] and the receiver / source end-term sums [S][n_rec + n_src]
+  size_t sbp, rcopy, acc;
   size_t total;
   size_t state_bytes;
   size_t snap_step_bytes;  // one step of one snapshot field ([S][ny][snap_pitch])
@@ -194,7 +201,9 @@ struct Layout {
   int n_seg;
 };
 
-enum StoreKind { kStoreNone = 0, kStoreF32 = 1, kStoreBF16 = 2, kStoreFP8 = 3 };
+// kStoreEy: the E snapshot alone, float32 (the summation-by-parts Cb
+// gradient needs no curl snapshot)
+enum StoreKind { kStoreNone = 0, kStoreF32 = 1, kStoreBF16 = 2, kStoreFP8 = 3, kStoreEy = 4 };
 
 // device status word indices in the flags area; kCtrBase, kCtrBase + 1: the
 // work-item counters that consecutive stencil launches alternate between
@@ -256,9 +265,32 @@ int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array);
 // small kernels (mw_aux.cu)
 cudaError_t launch_dup_chains(const int64_t *idx, int S, int n, int64_t numel, int *lead,
                               int *next, int *flags, cudaStream_t st);
+// End-term sums of the summation-by-parts Cb gradient, gathered by the
+// adjoint's injection launch of each step (all four null otherwise):
+// acc_a[s][k] += vals_t[s][k] * pair_t[s][k] (the residual times the
+// record it answers) and acc_b[s][k] += w_t[s][k] * out_t[s][k] (the source
+// wavelet times the sampled lambda_E).
+struct SbpTerms {
+  const float *pair_t = nullptr;
+  float *acc_a = nullptr;
+  const float *w_t = nullptr;
+  float *acc_b = nullptr;
+};
 cudaError_t launch_inject_sample(float *field, int64_t numel, int S, const float *vals_t,
                                  const int64_t *idx_a, const int *lead, const int *next, int na,
-                                 const int64_t *idx_b, int nb, float *out_t, cudaStream_t st);
+                                 const int64_t *idx_b, int nb, float *out_t, cudaStream_t st,
+                                 const SbpTerms &sbp = SbpTerms{});
+// summation-by-parts Cb gradient: P = lambda_E * E (the end term of a given
+// adjoint start state), the scatter of the end-term sums into P (sequential
+// per shot: duplicates add in index order), and grad_cb_shot += P / Cb at
+// the cells the gradient mask keeps
+cudaError_t launch_sbp_init(float *P, const float *lam, const float *e, int64_t n,
+                            cudaStream_t st);
+cudaError_t launch_sbp_scatter(float *P, int64_t numel, int S, const int64_t *rec_idx,
+                               const float *acc_rec, int n_rec, const int64_t *src_idx,
+                               const float *acc_src, int n_src, cudaStream_t st);
+cudaError_t launch_sbp_finish(const float *P, const float *cb, float *gcb, int S, int ny, int nx,
+                              int batched, int mask_pml, cudaStream_t st);
 cudaError_t launch_check_finite(const float *x, int64_t n, int *flags,
                                 cudaStream_t st);
 cudaError_t launch_model(int64_t n, const float *eps_r, const float *sigma,

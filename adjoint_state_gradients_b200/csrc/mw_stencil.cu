@@ -465,7 +465,7 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
             if constexpr (STORE != kStoreNone) {
               const int64_t so = ((int64_t)it.s * a.g.ny + (it.r0 + i - 2 * P + 1)) * a.snap_pitch + c;
               snap_store_p<STORE>(own, a.snap_e, so, e_old);
-              snap_store_p<STORE>(own, a.snap_c, so, curl);
+              if constexpr (STORE != kStoreEy) snap_store_p<STORE>(own, a.snap_c, so, curl);
             }
             st4p(own, ey_o + off, en);
           }
@@ -562,11 +562,17 @@ __device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, c
   const int r = it.r0 + i;
   const bool own_r = (unsigned)(i - (2 * P - 1)) < (unsigned)(it.yb - it.ya);
   const bool hx_in = i >= it.hx_lo && i <= it.hx_hi;
-  constexpr uint32_t snap_elem = SNAP == kStoreF32 ? 4 : SNAP == kStoreBF16 ? 2 : 1;
-  constexpr uint32_t snap_bytes = 2 * 112 * snap_elem;
+  constexpr bool EY = SNAP == kStoreEy;
+  constexpr uint32_t snap_elem = SNAP == kStoreF32 || EY ? 4 : SNAP == kStoreBF16 ? 2 : 1;
+  constexpr uint32_t snap_bytes = EY ? 2 * 112 * 4 : 2 * 112 * snap_elem;
+  // the gradient rows: this row's (snapshot pair), or with the E snapshot
+  // alone that of row r - 2P + 1, whose E update this iteration makes
+  // (lambda_E and the E snapshot)
+  const bool g_r = EY ? (unsigned)(i - (4 * P - 2)) < (unsigned)(it.yb - it.ya) : own_r;
+  const int rg = EY ? r - 2 * P + 1 : r;
   uint32_t bytes = 2 * 128 * 4 + 2 * 128 * 4;
   if (hx_in) bytes += 112 * 4;
-  if (own_r) bytes += snap_bytes + 2 * 112 * 4;
+  if (g_r) bytes += snap_bytes + 2 * 112 * 4;
   if (cq_arr) bytes += hx_in ? 2 * 128 * 4 : 128 * 4;
   int ze = -1, zh = -1;
   if constexpr (BAND) {
@@ -586,13 +592,18 @@ __device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, c
     tma3s(st + (kA_MD + 128) * 4, &m.map[kAMapCB], it.x0 - 8, r, it.sm, bar);
   }
   if (hx_in) tma3s(st + kA_HX * 4, &m.map[kAMapHX], it.x0, r - P, it.s, bar);
-  if (own_r) {
-    tma5s(st + kA_SS * 4, &m.map[kAMapSS], it.x0, r, it.s, a.snap_t, 0, bar);
-    if (a.gg_pair) {
-      tma4s(st + kA_GG * 4, &m.map[kAMapGG], it.x0, r, it.s, 0, bar);
+  if (g_r) {
+    if constexpr (EY) {
+      tma3s(st + kA_SS * 4, &m.map[kAMapLE], it.x0, rg, it.s, bar);
+      tma4s(st + (kA_SS + 128) * 4, &m.map[kAMapSS], it.x0, rg, it.s, a.snap_t, bar);
     } else {
-      tma3s(st + kA_GG * 4, &m.map[kAMapGG], it.x0, r, it.s, bar);
-      tma3s(st + (kA_GG + 128) * 4, &m.map[kAMapGB], it.x0, r, it.s, bar);
+      tma5s(st + kA_SS * 4, &m.map[kAMapSS], it.x0, rg, it.s, a.snap_t, 0, bar);
+    }
+    if (a.gg_pair) {
+      tma4s(st + kA_GG * 4, &m.map[kAMapGG], it.x0, rg, it.s, 0, bar);
+    } else {
+      tma3s(st + kA_GG * 4, &m.map[kAMapGG], it.x0, rg, it.s, bar);
+      tma3s(st + (kA_GG + 128) * 4, &m.map[kAMapGB], it.x0, rg, it.s, bar);
     }
   }
   if (cq_arr) {
@@ -721,7 +732,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
         }
         // ---- owned rows: gradients (lam = lambda_E^{t+1}) and px
         if (own_r) {
-          {  // every lane computes (in-bounds staged reads); owned lanes store
+          if constexpr (SNAP != kStoreEy) {  // every lane computes; owned lanes store
             const uint32_t sbase = st + kA_SS * 4;
             constexpr uint32_t selem = SNAP == kStoreF32 ? 4 : SNAP == kStoreBF16 ? 2 : 1;
             constexpr uint32_t sfield = 112 * selem, sstep = 4 * selem;
@@ -839,6 +850,28 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
             en.v[q] = cl[Q::at(u, NQ - 1)].v[q] - d_int<P>(wv, q, a.c.cx) - dz;
           }
           st4p(own, ey_o + (ro - (2 * P - 1) * nx), en);
+          if constexpr (SNAP == kStoreEy) {
+            // gradients of this row by summation by parts: gCa += E^t lam^{t+1};
+            // the Cb accumulator takes E^t times the E-update term
+            // G^t = lam~^t - Ca lam^{t+1} (at t = 0: E^0 times -Ca lam^1)
+            const int re = r - 2 * P + 1;
+            const F4 lv = lds4s(st + kA_SS * 4 + 16 * wo);
+            const F4 se = lds4s(st + (kA_SS + 128) * 4 + 16 * wo);
+            F4 gca = lds4s(st + w.gca_o + 16 * wo), gcb = lds4s(st + w.gcb_o + 16 * wo);
+            const bool rowmask =
+                !BAND || !a.g.grad_mask || (re >= a.g.n_pml && re < ny - a.g.n_pml);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (rowmask && colmask[q]) {
+                const float c = cl[Q::at(u, NQ - 1)].v[q];
+                gca.v[q] = fmaf(se.v[q], lv.v[q], gca.v[q]);
+                gcb.v[q] = fmaf(se.v[q], a.tzero ? -c : en.v[q] - c, gcb.v[q]);
+              }
+            }
+            const int go = ro - (2 * P - 1) * nx;
+            st4p(own, gca_o + go, gca);
+            st4p(own, gcb_o + go, gcb);
+          }
         }
         __syncwarp();
         w.ring.next(NS);
@@ -1034,6 +1067,7 @@ cudaError_t fwd_store(const FwdMaps &m, const StepArgs &a, int store, int born, 
     case kStoreF32: return fwd_t<P, kStoreF32>(m, a, batched, cq_arr, grid, st);
     case kStoreBF16: return fwd_t<P, kStoreBF16>(m, a, batched, cq_arr, grid, st);
     case kStoreFP8: return fwd_t<P, kStoreFP8>(m, a, batched, cq_arr, grid, st);
+    case kStoreEy: return fwd_t<P, kStoreEy>(m, a, batched, cq_arr, grid, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -1045,6 +1079,7 @@ cudaError_t adj_snap(const AdjMaps &m, const StepArgs &a, int snap, bool batched
     case kStoreF32: return adj_t<P, kStoreF32>(m, a, batched, cq_arr, grid, st);
     case kStoreBF16: return adj_t<P, kStoreBF16>(m, a, batched, cq_arr, grid, st);
     case kStoreFP8: return adj_t<P, kStoreFP8>(m, a, batched, cq_arr, grid, st);
+    case kStoreEy: return adj_t<P, kStoreEy>(m, a, batched, cq_arr, grid, st);
   }
   return cudaErrorInvalidValue;
 }

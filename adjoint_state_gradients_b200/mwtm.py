@@ -22,9 +22,9 @@ MW_ERR_NONFINITE = -5
 MW_ERR_TIMEOUT = -6
 MW_ERR_UNSUPPORTED = -7
 
-SNAP_NONE, SNAP_FP32, SNAP_BF16, SNAP_CKPT, SNAP_FP8 = 0, 1, 2, 3, 4
+SNAP_NONE, SNAP_FP32, SNAP_BF16, SNAP_CKPT, SNAP_FP8, SNAP_CKPT_EY = 0, 1, 2, 3, 4, 5
 SNAP_MODES = {"none": SNAP_NONE, "fp32": SNAP_FP32, "bf16": SNAP_BF16, "ckpt": SNAP_CKPT,
-              "fp8": SNAP_FP8}
+              "fp8": SNAP_FP8, "ckpt_ey": SNAP_CKPT_EY}
 
 
 class Params(ctypes.Structure):

@@ -23,7 +23,7 @@ def main():
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--shots", type=int, default=4)
     ap.add_argument("--nt", type=int, default=8)
-    ap.add_argument("--mode", default="fp32", choices=["fp32", "bf16", "ckpt", "none"])
+    ap.add_argument("--mode", default="fp32", choices=["fp32", "bf16", "fp8", "ckpt", "ckpt_ey", "none"])
     args = ap.parse_args()
     inp = synth.make_inputs(args.workload, n_shots=args.shots)
     wl = inp.wl

@@ -19,6 +19,7 @@ weak scaling) and all-reduce the gradients once per step over NCCL.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -57,6 +58,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--nt", type=int, default=None, help="override nt (profiling runs only)")
+    ap.add_argument("--snapshot", default=None, choices=["fp32", "bf16", "fp8", "ckpt", "ckpt_ey"],
+                    help="override the workload's snapshot storage")
     ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5],
                     help="workload to time (default: the 2048^2 order-4 checkpointed sweep)")
     return ap.parse_args()
@@ -73,18 +76,24 @@ def dist_env():
 # algorithmic bytes per cell-update (fixed before tuning)
 
 
+CKPT_MODES = ("ckpt", "ckpt_ey")
+
+
 def alg_bytes(wl, S):
     """Bytes per cell-update of each pass of the workload's sweep (fp32 fields):
     state read + write 24 B, Ca and Cb (shared by the shots unless the model is
     batched), the CPML band memories, snapshot write / read (8, 4 or 2 B), the
-    per-shot gradient read-modify-write 16 B, checkpoint copies 28 / C B."""
+    per-shot gradient read-modify-write 16 B, checkpoint copies 28 / C B.
+    With the E snapshot alone ("ckpt_ey") the replay writes and the adjoint
+    reads 4 B of snapshot instead of 8."""
     band = 16.0 * (2.0 * wl.n_pml / wl.nx + 2.0 * wl.n_pml / wl.ny)
     model = 8.0 if wl.batched else 8.0 / S
     base = 24.0 + model + band
-    if wl.snapshot == "ckpt":
+    if wl.snapshot in CKPT_MODES:
         C = wl.ckpt_every
-        return {"forward": base + 28.0 / C, "replay": base + 8.0 + 28.0 / C,
-                "adjoint": base + 8.0 + 16.0}
+        sb = 4.0 if wl.snapshot == "ckpt_ey" else 8.0
+        return {"forward": base + 28.0 / C, "replay": base + sb + 28.0 / C,
+                "adjoint": base + sb + 16.0}
     if wl.snapshot == "none":
         return {"forward": base}
     sb = {"fp32": 8.0, "bf16": 4.0, "fp8": 2.0}[wl.snapshot]
@@ -94,7 +103,7 @@ def alg_bytes(wl, S):
 # the library's per-launch timing classes: 0 forward, 1 forward with snapshot
 # store, 2 adjoint; which class each pass of a sweep uses
 def pass_classes(wl):
-    if wl.snapshot == "ckpt":
+    if wl.snapshot in CKPT_MODES:
         return {"forward": 0, "replay": 1, "adjoint": 2}
     if wl.snapshot == "none":
         return {"forward": 0}
@@ -169,13 +178,13 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-def traffic_record():
-    """DRAM bytes per adjoint launch from the committed ncu summary, if the
-    kernel source has not changed since it was taken."""
+def traffic_record(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
+    covers that kernel and its source has not changed since it was taken."""
     try:
         with open(os.path.join(PROFILES, "adjoint_traffic.json")) as fh:
             d = json.load(fh)
-        if d.get("stencil_sha") != stencil_sha():
+        if d.get("stencil_sha") != stencil_sha() or d.get("kernel") != kernel:
             return None
         return float(d["dram_bytes_per_launch_full"])
     except Exception:
@@ -205,7 +214,7 @@ def oracle_sample(number, nt_sample):
     f = inp.wavelet(dt, nt_sample)
     res = synth.rng(7).normal(size=(nt_sample, 1, wl.n_rec))
     t0 = time.perf_counter()
-    if wl.snapshot == "ckpt":
+    if wl.snapshot in CKPT_MODES:
         sim.fwd_adj_ckpt(f, res, wl.ckpt_every)
         what = f"checkpoint every {wl.ckpt_every}: forward + replay + adjoint"
     elif wl.snapshot == "none":
@@ -222,6 +231,9 @@ def oracle_sample(number, nt_sample):
 
 
 def snapshot_desc(wl):
+    if wl.snapshot == "ckpt_ey":
+        return (f"checkpoint every {wl.ckpt_every} steps + segment replay of E alone "
+                "(Cb gradient by summation by parts)")
     if wl.snapshot == "ckpt":
         return f"checkpoint every {wl.ckpt_every} steps + segment replay"
     if wl.snapshot == "none":
@@ -281,6 +293,8 @@ def main():
 
     number = args.workload
     wl = synth.WORKLOADS[number]
+    if args.snapshot:
+        wl = dataclasses.replace(wl, snapshot=args.snapshot)
     nt = args.nt or wl.nt
     S = wl.n_shots
     grad = wl.snapshot != "none"   # workload 5 times the forward alone
@@ -395,12 +409,13 @@ def main():
     top_launch_ms = launch_ms[top]
     top_bytes = passes[top] * wl.ny * wl.nx * S
     achieved = top_bytes / (top_launch_ms / 1e3) / 1e9
-    # the recorded ncu traffic is that of the 8-shot order-4 adjoint launch
-    traffic = traffic_record() if number == WORKLOAD else None
     kname = {("adjoint", "fp32"): "kStoreF32", ("adjoint", "ckpt"): "kStoreF32",
+             ("adjoint", "ckpt_ey"): "kStoreEy",
              ("adjoint", "bf16"): "kStoreBF16", ("adjoint", "fp8"): "kStoreFP8"}
     kernel_name = (f"k_adjoint<{wl.order // 2}, {kname[(top, wl.snapshot)]}, 1>" if grad
                    else f"k_forward<{wl.order // 2}, kStoreNone, 1>")
+    # the recorded ncu traffic is that of the 8-shot order-4 adjoint launch
+    traffic = traffic_record(kernel_name) if number == WORKLOAD else None
 
     # ---- end to end through the public API with host buffers
     e2e = None

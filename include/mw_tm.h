@@ -82,6 +82,13 @@ extern "C" {
                           saturating to +-448, no scaling), as the
                           maxwell.cu page's forward_kernel_e_with_storage_fp8
                           stores them                                        */
+#define MW_SNAP_CKPT_EY 5 /* checkpoints as MW_SNAP_CKPT, but the replayed
+                          segment keeps Ey^n alone and the adjoint forms the
+                          Cb gradient by summation by parts (below), which
+                          halves the segment's snapshot traffic; the forward
+                          keeps a copy of the records in the workspace (it
+                          then needs rec_idx when n_rec > 0), and Cb must be
+                          nonzero everywhere                                 */
 
 typedef struct mw_params {
   int32_t ny, nx;        /* array size incl. the CPML band                 */
@@ -224,6 +231,18 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca_dev,
  *   adj_state      in/out adjoint state, or NULL (start from zero)
  * In MW_SNAP_CKPT mode the forward is replayed segment by segment from the
  * checkpoints, which needs f and src_idx again. */
+/* MW_SNAP_CKPT_EY: with E^{t+1} = Ca E^t + Cb curl^t + s^t (s the source
+ * injection) and the adjoint's E update lam~^t = Ca lam^{t+1} + G^t
+ * (lam^{t+1} = lam~^{t+1} + the residual injected at step t), the sum
+ * Cb * grad_cb = sum_t curl^t lam^{t+1} * Cb regroups, exactly, into
+ *     sum_{t>=1} G^t E^t  -  Ca lam^1 E^0  +  lam~^{nt} E^{nt}
+ *   + sum_t res[t] rec[t]  (at the receiver cells)
+ *   - sum_t f[t] lam^{t+1} (at the source cells),
+ * which needs only E^t from the replay.  The kernel accumulates the first two
+ * terms row by row into a workspace array at each row's E update, the
+ * injection launches gather the last two, and the end of the call adds them
+ * and divides by Cb.  grad_ca_shot, grad_f and the adjoint state are
+ * bitwise those of MW_SNAP_CKPT; grad_cb_shot agrees to rounding. */
 int mw_tm_adjoint_grad(const mw_params *p, const float *ca_dev,
                        const float *cb_dev, const float *cq_dev,
                        const float *cpml_dev, const float *f_dev,

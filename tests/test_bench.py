@@ -3,6 +3,7 @@ sizing of the oracle baseline, and the reference arm's JSON line (the fp64
 oracle timed on host cores), run as the driver runs it."""
 from __future__ import annotations
 
+import dataclasses
 import json
 import os
 import subprocess
@@ -18,14 +19,22 @@ from adjoint_state_gradients_b200 import synth  # noqa: E402
 
 
 def test_byte_model_of_the_headline_sweep():
+    """Checkpoints every 64 steps with the E-alone segment: the replay writes
+    and the adjoint reads 4 B of snapshot per cell-update; with the pair
+    segment 8 B."""
     wl = synth.WORKLOADS[4]
+    assert wl.snapshot == "ckpt_ey"
     b = bench.alg_bytes(wl, wl.n_shots)
     band = 16.0 * (2 * 40 / 2128 + 2 * 40 / 2128)
     assert b["forward"] == pytest.approx(24 + 1 + band + 28 / 64)
-    assert b["replay"] == pytest.approx(24 + 1 + band + 8 + 28 / 64)
-    assert b["adjoint"] == pytest.approx(24 + 1 + band + 8 + 16)
-    assert sum(b.values()) == pytest.approx(111.49, abs=0.01)
+    assert b["replay"] == pytest.approx(24 + 1 + band + 4 + 28 / 64)
+    assert b["adjoint"] == pytest.approx(24 + 1 + band + 4 + 16)
+    assert sum(b.values()) == pytest.approx(103.49, abs=0.01)
     assert bench.pass_classes(wl) == {"forward": 0, "replay": 1, "adjoint": 2}
+    bp = bench.alg_bytes(dataclasses.replace(wl, snapshot="ckpt"), wl.n_shots)
+    assert bp["replay"] - b["replay"] == pytest.approx(4.0)
+    assert bp["adjoint"] - b["adjoint"] == pytest.approx(4.0)
+    assert sum(bp.values()) == pytest.approx(111.49, abs=0.01)
 
 
 def test_byte_model_of_the_other_storage_modes():

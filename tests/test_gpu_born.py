@@ -45,7 +45,7 @@ def _problem(sim, nt, dt, mode):
 
 @pytest.mark.parametrize("mode,order,batched", [
     ("fp32", 4, False), ("bf16", 4, False), ("fp8", 4, False), ("ckpt", 4, False),
-    ("fp32-host", 4, False), ("fp32", 8, True), ("ckpt", 8, False)])
+    ("fp32-host", 4, False), ("fp32", 8, True), ("ckpt", 8, False), ("ckpt_ey", 4, False)])
 def test_born_forward_matches_oracle(mode, order, batched):
     sim, dt, nt, f, dca, dcb, _ = _case(order, batched, 800 + order)
     fw = sim.forward(f, snapshots=True)

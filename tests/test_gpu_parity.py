@@ -293,15 +293,17 @@ def test_workload3_bf16_snapshots():
     assert e_ca <= 2e-2 and e_cb <= 2e-2
 
 
-def test_workload4_checkpoint_replay():
+@pytest.mark.parametrize("snapshot", ["ckpt", "ckpt_ey"])
+def test_workload4_checkpoint_replay(snapshot):
     """2128x2128 order 4, checkpoints every 64 steps: one shot, nt 200
-    (3 full segments + a partial one) against the oracle's own replay."""
+    (3 full segments + a partial one) against the oracle's own replay, with
+    the pair segment and with the E-alone segment."""
     nt = 200
     sim, inp, dt, f = workload_sim(4, n_shots=1, nt=nt)
     g = synth.rng(44)
     res = f32(g.normal(size=(nt, 1, inp.wl.n_rec)))
     ck = sim.fwd_adj_ckpt(f, res, 50)
-    prob = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot="ckpt", ckpt_every=64)
+    prob = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot=snapshot, ckpt_every=64)
     rec = run_forward(prob, f)
     assert rel_l2(rec, ck["rec"]) <= REC_TOL
     gca, gcb, gf = run_adjoint(prob, res)
@@ -334,15 +336,17 @@ def _subset_sim(inp, sel, dt, batched=False):
                       wl.f0, vmax=vmax, round_f32=True)
 
 
-def test_workload4_all_shots_sampled():
+@pytest.mark.parametrize("snapshot", ["ckpt", "ckpt_ey"])
+def test_workload4_all_shots_sampled(snapshot):
     """2128x2128 order 4, all 8 shots, checkpoints every 64 steps (the
-    benchmark's launch plan), nt 137 = two full segments + a partial one;
-    records and per-shot gradients of shots 0 and 7 against the oracle."""
+    benchmark's launch plan with "ckpt_ey"), nt 137 = two full segments + a
+    partial one; records and per-shot gradients of shots 0 and 7 against the
+    oracle."""
     nt, sel = 137, [0, 7]
     sim, inp, dt, f = workload_sim(4, n_shots=8, nt=nt)
     g = synth.rng(404)
     res = f32(g.normal(size=(nt, 8, inp.wl.n_rec)))
-    prob = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot="ckpt", ckpt_every=64)
+    prob = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot=snapshot, ckpt_every=64)
     rec = run_forward(prob, f)
     gca, gcb, gf = run_adjoint(prob, res)
     assert prob.status() == mwtm.MW_OK
