@@ -32,12 +32,14 @@ class Problem:
     summation by parts).
     snapshot_host: keep the fp32 / bf16 / fp8 snapshots in page-locked host
     memory (staged through a 3-step device ring) instead of the workspace.
+    ckpt_tail: checkpoint modes, the forward stores the snapshots of the last
+    ckpt_tail steps itself (HBM for replay work).
     """
 
     def __init__(self, ny, nx, order, dy, dx, dt, nt, n_pml, src_idx, rec_idx, *, vmax,
                  snapshot="fp32", ckpt_every=64, batched=False, cq_scalar=True,
                  grad_mask_pml=False, allow_unstable=False, check_finite=False, device="cuda",
-                 snapshot_host=False):
+                 snapshot_host=False, ckpt_tail=0):
         src_idx = np.asarray(src_idx, dtype=np.int64)
         rec_idx = np.asarray(rec_idx, dtype=np.int64)
         self.S = src_idx.shape[0]
@@ -47,7 +49,8 @@ class Problem:
             nt=nt, dt=dt, dy=dy, dx=dx, n_pml=n_pml, model_batched=int(batched),
             cq_is_scalar=int(cq_scalar), snap_mode=mwtm.SNAP_MODES[snapshot], ckpt_every=ckpt_every,
             grad_mask_pml=int(grad_mask_pml), vmax=vmax, allow_unstable=int(allow_unstable),
-            check_finite=int(check_finite), snap_host=int(bool(snapshot_host)))
+            check_finite=int(check_finite), snap_host=int(bool(snapshot_host)),
+            ckpt_tail=int(ckpt_tail))
         mwtm.check(mwtm.validate(self.p))
         self.host_snapshots = None
         if snapshot_host:

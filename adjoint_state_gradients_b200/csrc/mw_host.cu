@@ -111,6 +111,8 @@ int check_params(const mw_params *p, bool cfl) {
     return fail(MW_ERR_ARG, "snap_host needs snap_mode FP32, BF16 or FP8 (got %d)", p->snap_mode);
   if (is_ckpt(p) && p->ckpt_every < 1)
     return fail(MW_ERR_ARG, "ckpt_every = %d", p->ckpt_every);
+  if (p->ckpt_tail < 0 || (p->ckpt_tail > 0 && !is_ckpt(p)))
+    return fail(MW_ERR_ARG, "ckpt_tail = %d needs a checkpoint snap_mode", p->ckpt_tail);
   if (2 * b.Wx > 256)
     return fail(MW_ERR_UNSUPPORTED, "n_pml = %d: a band row exceeds one TMA box (n_pml <= 123)",
                 p->n_pml);
@@ -183,6 +185,15 @@ Layout layout(const mw_params *p) {
     L.snap_step_bytes = SN * 4;
     L.seg = off;
     off += align256(2 * (size_t)p->ckpt_every * L.snap_step_bytes);
+    // the tail the forward stores itself: [E slots][curl slots], or with E
+    // alone the E slots and one more for the final E (the adjoint's end term)
+    L.n_tail = p->ckpt_tail < p->nt ? p->ckpt_tail : p->nt;
+    L.tail = off;
+    if (L.n_tail > 0) {
+      const size_t slots = p->snap_mode == MW_SNAP_CKPT_EY ? (size_t)L.n_tail + 1
+                                                            : 2 * (size_t)L.n_tail;
+      off += align256(slots * L.snap_step_bytes);
+    }
   }
   L.sbp = L.rcopy = L.acc = 0;
   if (p->snap_mode == MW_SNAP_CKPT_EY) {
@@ -746,11 +757,11 @@ struct Replay {
     MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, cq, &fB));
     return MW_OK;
   }
-  // replay segment k; *t0 / *t1 receive its steps
-  int segment(int k, int *launch_idx, int *t0_out, int *t1_out) {
+  // replay segment k up to step t_end at most; *t0 / *t1 receive its steps
+  int segment(int k, int *launch_idx, int *t0_out, int *t1_out, int t_end) {
     const int C = p->ckpt_every;
     const int t0 = k * C;
-    const int t1 = (t0 + C < p->nt) ? t0 + C : p->nt;
+    const int t1 = (t0 + C < t_end) ? t0 + C : t_end;
     const int64_t numel = (int64_t)p->ny * p->nx;
     char *seg_e = ws + L.seg;
     char *seg_c = seg_e + (size_t)C * L.snap_step_bytes;
@@ -922,6 +933,11 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, cq, &mB));
 
   const int store = snap_store_kind(p->snap_mode);
+  // checkpoint modes: the last n_tail steps store their snapshots themselves
+  const int t_tail = p->nt - L.n_tail;
+  const int tail_store = ey_only ? kStoreEy : kStoreF32;
+  char *tail_e = ws + L.tail;
+  char *tail_c = tail_e + (size_t)L.n_tail * L.snap_step_bytes;
   const int64_t SN = (int64_t)p->n_shots * p->ny * p->nx;
   const int64_t numel = (int64_t)p->ny * p->nx;
   const Chains ch = chains_at(p, ws, L);
@@ -952,10 +968,16 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
     a.out = fields_at(p, nxt);
     a.snap_e = store ? snap_e + (size_t)slot * L.snap_step_bytes : nullptr;
     a.snap_c = store ? snap_c + (size_t)slot * L.snap_step_bytes : nullptr;
+    int kind = store;
+    if (t >= t_tail && L.n_tail > 0) {
+      kind = tail_store;
+      a.snap_e = tail_e + (size_t)(t - t_tail) * L.snap_step_bytes;
+      a.snap_c = tail_c + (size_t)(t - t_tail) * L.snap_step_bytes;
+    }
     const FwdMaps &m = cur == bufA ? mA : mB;
     a.ctr_slot = t & 1;
-    MW_CUDA(timed(store ? 1 : 0, st, [&] {
-      return launch_forward(m, a, p->order, store, kStoreNone, p->model_batched != 0, !p->cq_is_scalar,
+    MW_CUDA(timed(kind ? 1 : 0, st, [&] {
+      return launch_forward(m, a, p->order, kind, kStoreNone, p->model_batched != 0, !p->cq_is_scalar,
                             lc.grid, st);
     }));
     if (host) {  // step t: ring slot -> host, on the copy stream
@@ -981,6 +1003,9 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
     for (int k = 0; k < kHostRing && k < p->nt; ++k)
       MW_CUDA(cudaStreamWaitEvent(st, hc.freed[(p->nt - 1 - k) % kHostRing], 0));
   if (cur != bufA) MW_CUDA(cudaMemcpyAsync(bufA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
+  if (ey_only && L.n_tail > 0)  // the final E, for the adjoint's end term
+    MW_CUDA(cudaMemcpyAsync(tail_e + (size_t)L.n_tail * L.snap_step_bytes, bufA,
+                            SN * sizeof(float), cudaMemcpyDeviceToDevice, st));
   if (p->check_finite) MW_CUDA(launch_check_finite(bufA, 3 * SN, flags, st));
   return MW_OK;
 }
@@ -1065,6 +1090,16 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
                   L.snap_pitch, ey_only, &mA));
   MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, cq, gca, a.gcb, snap_e, snap_c, snap_elem, C,
                   L.snap_pitch, ey_only, &mB));
+  // checkpoint modes: the tail the forward stored, read in place
+  const int t_tail = ckpt ? p->nt - L.n_tail : p->nt;
+  AdjMaps tA, tB;
+  if (ckpt && L.n_tail > 0) {
+    const char *te = ws + L.tail, *tc = te + (size_t)L.n_tail * L.snap_step_bytes;
+    MW_TRY(adj_maps(p, fields_at(p, adA), ca, cb, cq, gca, a.gcb, te, tc, snap_elem, L.n_tail,
+                    L.snap_pitch, ey_only, &tA));
+    MW_TRY(adj_maps(p, fields_at(p, adB), ca, cb, cq, gca, a.gcb, te, tc, snap_elem, L.n_tail,
+                    L.snap_pitch, ey_only, &tB));
+  }
 
   float *cur = adA, *nxt = adB;
   // with the summation-by-parts Cb gradient the source term needs lambda_E at
@@ -1088,7 +1123,8 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     a.snap_t = slot;
     a.tzero = t == 0 ? 1 : 0;
     a.ctr_slot = (launch_idx++) & 1;
-    const AdjMaps &m = cur == adA ? mA : mB;
+    const bool in_tail = t >= t_tail;
+    const AdjMaps &m = cur == adA ? (in_tail ? tA : mA) : (in_tail ? tB : mB);
     MW_CUDA(timed(2, st, [&] {
       return launch_adjoint(m, a, p->order, snap, p->model_batched != 0, !p->cq_is_scalar,
                             la.grid, st);
@@ -1117,15 +1153,24 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     for (int t = p->nt - 1; t >= 0; --t) MW_TRY(adj_step(t, t));
   } else {
     // checkpoint mode: replay each segment from its checkpoint, newest first
+    // the tail first (no replay), then each earlier segment replayed from its
+    // checkpoint; a given adjoint start state meets the forward's final E:
+    // P starts at lambda~_E^{nt} E^{nt}
     Replay rp;
     MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, src_idx, ch));
     rp.store = ey_only ? kStoreEy : kStoreF32;
-    for (int k = L.n_seg - 1; k >= 0; --k) {
+    if (L.n_tail > 0) {
+      if (ey_only && adj_state)
+        MW_CUDA(launch_sbp_init(sbp, adA,
+                                (const float *)(ws + L.tail + (size_t)L.n_tail * L.snap_step_bytes),
+                                SN, st));
+      for (int t = p->nt - 1; t >= t_tail; --t) MW_TRY(adj_step(t, t - t_tail));
+    }
+    const int n_rep = (t_tail + p->ckpt_every - 1) / p->ckpt_every;
+    for (int k = n_rep - 1; k >= 0; --k) {
       int t0, t1;
-      MW_TRY(rp.segment(k, &launch_idx, &t0, &t1));
-      // a given adjoint start state meets the forward's final E: P starts
-      // at lambda~_E^{nt} E^{nt}
-      if (ey_only && adj_state && k == L.n_seg - 1)
+      MW_TRY(rp.segment(k, &launch_idx, &t0, &t1, t_tail));
+      if (ey_only && adj_state && L.n_tail == 0 && k == n_rep - 1)
         MW_CUDA(launch_sbp_init(sbp, adA, rp.last, SN, st));
       for (int t = t1 - 1; t >= t0; --t) MW_TRY(adj_step(t, t - t0));
     }
@@ -1253,7 +1298,7 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
     MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, src_idx, ch));
     for (int k = 0; k < L.n_seg; ++k) {
       int t0, t1;
-      MW_TRY(rp.segment(k, &launch_idx, &t0, &t1));
+      MW_TRY(rp.segment(k, &launch_idx, &t0, &t1, p->nt));
       for (int t = t0; t < t1; ++t) MW_TRY(born_step(t, t - t0));
     }
   }

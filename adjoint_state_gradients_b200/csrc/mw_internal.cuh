@@ -194,6 +194,9 @@ struct Layout {
   // MW_SNAP_CKPT_EY: the Cb-gradient accumulator [S][ny][nx], the record copy
   // [nt][S][n_rec] and the receiver / source end-term sums [S][n_rec + n_src]
   size_t sbp, rcopy, acc;
+  // checkpoint modes: snapshots of the last n_tail steps, stored by the forward
+  size_t tail;
+  int n_tail;
   size_t total;
   size_t state_bytes;
   size_t snap_step_bytes;  // one step of one snapshot field ([S][ny][snap_pitch])

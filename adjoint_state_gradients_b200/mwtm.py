@@ -36,7 +36,7 @@ class Params(ctypes.Structure):
                 ("ckpt_every", ctypes.c_int32), ("grad_mask_pml", ctypes.c_int32),
                 ("vmax", ctypes.c_double), ("allow_unstable", ctypes.c_int32),
                 ("check_finite", ctypes.c_int32), ("snap_host", ctypes.c_int32),
-                ("snap_host_ptr", ctypes.c_void_p)]
+                ("snap_host_ptr", ctypes.c_void_p), ("ckpt_tail", ctypes.c_int32)]
 
 
 class MWError(RuntimeError):

@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--nt", type=int, default=None, help="override nt (profiling runs only)")
     ap.add_argument("--snapshot", default=None, choices=["fp32", "bf16", "fp8", "ckpt", "ckpt_ey"],
                     help="override the workload's snapshot storage")
+    ap.add_argument("--ckpt-tail", type=int, default=None,
+                    help="override the workload's forward-stored tail (checkpoint modes)")
     ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5],
                     help="workload to time (default: the 2048^2 order-4 checkpointed sweep)")
     return ap.parse_args()
@@ -77,6 +79,19 @@ def dist_env():
 
 
 CKPT_MODES = ("ckpt", "ckpt_ey")
+
+
+def sweep_bytes_per_cell(wl, S, nt=None):
+    """Bytes per cell-update of the whole sweep: each pass weighted by the
+    share of the steps it runs (the replay skips the forward-stored tail,
+    whose forward steps write the snapshot instead)."""
+    b = alg_bytes(wl, S)
+    if wl.snapshot not in CKPT_MODES:
+        return sum(b.values())
+    nt = nt or wl.nt
+    tail = min(wl.ckpt_tail, nt) / nt
+    sb = 4.0 if wl.snapshot == "ckpt_ey" else 8.0
+    return b["forward"] + tail * sb + (1.0 - tail) * b["replay"] + b["adjoint"]
 
 
 def alg_bytes(wl, S):
@@ -232,8 +247,10 @@ def oracle_sample(number, nt_sample):
 
 def snapshot_desc(wl):
     if wl.snapshot == "ckpt_ey":
+        tail = (f"; the last {wl.ckpt_tail} steps' E kept from the forward (no replay)"
+                if wl.ckpt_tail else "")
         return (f"checkpoint every {wl.ckpt_every} steps + segment replay of E alone "
-                "(Cb gradient by summation by parts)")
+                f"(Cb gradient by summation by parts){tail}")
     if wl.snapshot == "ckpt":
         return f"checkpoint every {wl.ckpt_every} steps + segment replay"
     if wl.snapshot == "none":
@@ -295,6 +312,8 @@ def main():
     wl = synth.WORKLOADS[number]
     if args.snapshot:
         wl = dataclasses.replace(wl, snapshot=args.snapshot)
+    if args.ckpt_tail is not None:
+        wl = dataclasses.replace(wl, ckpt_tail=args.ckpt_tail)
     nt = args.nt or wl.nt
     S = wl.n_shots
     grad = wl.snapshot != "none"   # workload 5 times the forward alone
@@ -311,7 +330,8 @@ def main():
     C = wl.ckpt_every
 
     prob = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
-                       vmax=vmax, snapshot=wl.snapshot, ckpt_every=max(C, 1), batched=wl.batched)
+                       vmax=vmax, snapshot=wl.snapshot, ckpt_every=max(C, 1), batched=wl.batched,
+                       ckpt_tail=wl.ckpt_tail if wl.snapshot in CKPT_MODES else 0)
     f_host = inp.wavelet(dt, nt).astype(np.float32)
     eps_h = inp.eps_r.astype(np.float32)
     sig_h = inp.sigma.astype(np.float32)
@@ -402,7 +422,7 @@ def main():
     passes = alg_bytes(wl, S)
     classes = pass_classes(wl)
     peak, peak_kind = measured_peaks()
-    sweep_bytes = sum(passes.values()) * cells * args.steps
+    sweep_bytes = sweep_bytes_per_cell(wl, S, nt) * cells * args.steps
     sweep_frac = sweep_bytes / (total_ms / 1e3) / 1e9 / peak / world
     launch_ms = {k: ms[c] / max(counts[c], 1) for k, c in classes.items()}
     top = "adjoint" if grad else "forward"   # the dominant kernel
@@ -486,6 +506,7 @@ def main():
             "value_interior": round(value * (wl.n_interior ** 2) / (wl.ny * wl.nx), 4),
             "hbm_frac_sweep": round(sweep_frac, 4),
             "alg_bytes_per_cell": {k: round(v, 3) for k, v in passes.items()},
+            "sweep_bytes_per_cell": round(sweep_bytes_per_cell(wl, S, nt), 3),
             "roofline": {"bound": "hbm", "kernel": kernel_name,
                          "achieved": round(achieved, 1),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",

@@ -116,6 +116,13 @@ typedef struct mw_params {
                             own (the page's CPU snapshot storage with its
                             ring of device buffers and prefetch)           */
   void *snap_host_ptr;   /* page-locked host buffer for snap_host = 1        */
+  int32_t ckpt_tail;     /* checkpoint modes: the forward itself stores the
+                            snapshots of the last min(ckpt_tail, nt) steps (E
+                            and curl, or E alone for MW_SNAP_CKPT_EY) in the
+                            workspace, and the adjoint replays only the steps
+                            before them; it trades HBM for replay work (each
+                            tail step takes ny*nx*S*4 bytes per stored field).
+                            0: replay every step                            */
 } mw_params;
 
 /* Fill *p with defaults (zeros, cq_is_scalar = 1, snap_mode NONE). */

@@ -11,12 +11,13 @@ from adjoint_state_gradients_b200 import api, mwtm
 
 
 def problem_from_sim(sim, nt, dt, n_pml, snapshot="fp32", ckpt_every=64, grad_mask=False,
-                     check_finite=False, vmax=None):
+                     check_finite=False, vmax=None, ckpt_tail=0):
     kw = dict(vmax=vmax if vmax is not None else 1.0, allow_unstable=vmax is None)
     prob = api.Problem(sim.ny, sim.nx, sim.order, sim.dy, sim.dx, dt, nt, n_pml, sim.src_idx,
                        sim.rec_idx, snapshot=snapshot, ckpt_every=ckpt_every,
                        batched=bool(sim.model_batched), cq_scalar=not sim.cq_is_array,
-                       grad_mask_pml=grad_mask, check_finite=check_finite, **kw)
+                       grad_mask_pml=grad_mask, check_finite=check_finite,
+                       ckpt_tail=ckpt_tail, **kw)
     cpml = np.concatenate(list(sim.prof_y) + list(sim.prof_x))
     prob.set_coefficients(sim.ca, sim.cb, sim.cq, cpml)
     return prob

@@ -58,6 +58,26 @@ def test_host_only_entry_points():
     assert mwtm.workspace_bytes(p) == ws
 
 
+def test_checkpoint_modes_workspace_and_tail():
+    """The E-alone checkpoint mode adds its Cb accumulator, record copy and
+    end-term sums; a forward-stored tail adds its snapshot slots (pairs, or E
+    alone plus the final E); ckpt_tail needs a checkpoint mode."""
+    kw = dict(ny=84, nx=84, order=2, n_shots=2, n_src=1, n_rec=32, nt=300, dt=4.7e-11, dy=0.02,
+              dx=0.02, n_pml=10, vmax=1.5e8, ckpt_every=64)
+    step = 2 * 84 * 84 * 4
+    pair = mwtm.workspace_bytes(mwtm.make_params(snap_mode=mwtm.SNAP_CKPT, **kw))
+    ey = mwtm.workspace_bytes(mwtm.make_params(snap_mode=mwtm.SNAP_CKPT_EY, **kw))
+    assert ey >= pair + step + 300 * 2 * 32 * 4
+    for tail, slots_pair, slots_ey in ((10, 20, 11), (300, 600, 301), (1000, 600, 301)):
+        pt = mwtm.workspace_bytes(mwtm.make_params(snap_mode=mwtm.SNAP_CKPT, ckpt_tail=tail, **kw))
+        et = mwtm.workspace_bytes(mwtm.make_params(snap_mode=mwtm.SNAP_CKPT_EY, ckpt_tail=tail, **kw))
+        assert slots_pair * step <= pt - pair < slots_pair * step + 256
+        assert slots_ey * step <= et - ey < slots_ey * step + 256
+    for mode, tail in ((mwtm.SNAP_FP32, 5), (mwtm.SNAP_CKPT, -1)):
+        assert mwtm.validate(mwtm.make_params(snap_mode=mode, ckpt_tail=tail, **kw)) == mwtm.MW_ERR_ARG
+        assert "ckpt_tail" in mwtm.last_error()
+
+
 @pytest.mark.parametrize("order,s", [(2, 1.0), (4, 7 / 6), (6, 1.2416666666666667),
                                      (8, 1.2863095238095237)])
 def test_cfl_dt_matches_oracle(order, s):

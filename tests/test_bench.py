@@ -35,6 +35,12 @@ def test_byte_model_of_the_headline_sweep():
     assert bp["replay"] - b["replay"] == pytest.approx(4.0)
     assert bp["adjoint"] - b["adjoint"] == pytest.approx(4.0)
     assert sum(bp.values()) == pytest.approx(111.49, abs=0.01)
+    # the forward-stored tail: those steps write E (4 B) and skip the replay
+    assert wl.ckpt_tail == 640
+    want = b["forward"] + 0.16 * 4 + 0.84 * b["replay"] + b["adjoint"]
+    assert bench.sweep_bytes_per_cell(wl, wl.n_shots) == pytest.approx(want)
+    assert bench.sweep_bytes_per_cell(dataclasses.replace(wl, ckpt_tail=0), wl.n_shots) == \
+        pytest.approx(103.49, abs=0.01)
 
 
 def test_byte_model_of_the_other_storage_modes():

@@ -198,3 +198,53 @@ def test_ckpt_ey_no_sources_no_receivers():
     gca, gcb, _ = run_adjoint(prob, res)
     assert np.all(gca == 0) and np.all(gcb == 0)
     assert prob.status() == mwtm.MW_OK
+
+
+@pytest.mark.parametrize("mode", ["ckpt", "ckpt_ey"])
+def test_forward_stored_tail_is_bitwise_the_replay(mode):
+    """ckpt_tail: the forward stores the last steps' snapshots itself and the
+    adjoint replays only the steps before them.  The replay recomputes the
+    same values, so every output equals the tail-free run bit for bit, for
+    tails inside a segment, on a segment boundary, of the whole run and
+    longer than it; with a given adjoint start state (the final E then comes
+    from the tail store)."""
+    S, ny, nx, n_pml, nt, C = 2, 46, 72, 5, 40, 8
+    sim, dt, _ = small_sim(900, ny, nx, S, 2, 4, 4, n_pml, round_f32=True, sigma_max=0.02)
+    g = synth.rng(901)
+    f = torch.as_tensor(f32(g.normal(size=(nt, S, 2))), dtype=torch.float32).cuda()
+    res = torch.as_tensor(f32(g.normal(size=(nt, S, 4))), dtype=torch.float32).cuda()
+    ad0 = torch.as_tensor(f32(g.normal(size=(3 * S * ny * nx,))), dtype=torch.float32).cuda()
+    out = {}
+    for tail in (0, 3, 8, 21, 40, 100):
+        prob = problem_from_sim(sim, nt, dt, n_pml, snapshot=mode, ckpt_every=C, ckpt_tail=tail)
+        rec = prob.forward(f)
+        adj_state = prob.new_state()
+        adj_state[:ad0.numel()] = ad0
+        gca, gcb, gf = prob.adjoint(res, grad_f=True, adj_state=adj_state)
+        torch.cuda.synchronize()
+        assert prob.status() == mwtm.MW_OK
+        out[tail] = [t.cpu().numpy() for t in (rec, gca, gcb, gf, adj_state)]
+    for tail in (3, 8, 21, 40, 100):
+        for k, nm in enumerate(("rec", "gca", "gcb", "grad_f", "adj_state")):
+            assert np.array_equal(out[tail][k], out[0][k]), (tail, nm)
+
+
+def test_forward_stored_tail_matches_oracle_and_born():
+    S, ny, nx, n_pml, nt, C = 2, 46, 72, 5, 45, 16
+    sim, dt, _ = small_sim(902, ny, nx, S, 2, 4, 4, n_pml, round_f32=True, sigma_max=0.02)
+    g = synth.rng(903)
+    f = f32(g.normal(size=(nt, S, 2)))
+    res = f32(g.normal(size=(nt, S, 4)))
+    fw, ad = _oracle(sim, f, res)
+    dca = f32(1e-3 * g.normal(size=(ny, nx)))
+    dcb = f32(1e-3 * g.normal(size=(ny, nx)))
+    want_born = sim.born(fw["snap_ey"], fw["snap_curl"], dca, dcb)
+    prob = problem_from_sim(sim, nt, dt, n_pml, snapshot="ckpt_ey", ckpt_every=C, ckpt_tail=20)
+    rec = run_forward(prob, f)
+    assert rel_l2(rec, fw["rec"]) <= REC_TOL
+    born = prob.born(torch.as_tensor(dca, dtype=torch.float32),
+                     torch.as_tensor(dcb, dtype=torch.float32)).cpu().numpy().astype(np.float64)
+    assert rel_l2(born, want_born) <= REC_TOL
+    gca, gcb, gf = run_adjoint(prob, res)
+    _check_grads(gca, gcb, gf, ad)
+    assert prob.status() == mwtm.MW_OK
