@@ -315,6 +315,9 @@ def main():
     if args.ckpt_tail is not None:
         wl = dataclasses.replace(wl, ckpt_tail=args.ckpt_tail)
     nt = args.nt or wl.nt
+    if args.nt and args.ckpt_tail is None and wl.ckpt_tail:
+        # a shortened run keeps the tail's share of the steps
+        wl = dataclasses.replace(wl, ckpt_tail=wl.ckpt_tail * nt // wl.nt)
     S = wl.n_shots
     grad = wl.snapshot != "none"   # workload 5 times the forward alone
     # weak scaling: every rank simulates its own block of S shots of one
@@ -499,6 +502,8 @@ def main():
             "config": {"workload": wl.name, "grid": [wl.ny, wl.nx], "interior": wl.n_interior,
                        "n_pml": wl.n_pml, "order": wl.order, "nt": nt, "shots_per_gpu": S,
                        "n_rec": wl.n_rec, "snapshots": snapshot_desc(wl),
+                       "workspace_gb": round(prob.workspace.numel() * prob.workspace.element_size()
+                                             / 1e9, 1),
                        "l2": "inputs larger than L2 (one state buffer is "
                              f"{prob.p.n_shots * wl.ny * wl.nx * 12 / 1e6:.0f} MB)",
                        "parallelism": f"shots sharded, {world} rank(s)"},
