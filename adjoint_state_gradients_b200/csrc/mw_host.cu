@@ -224,6 +224,11 @@ Fields fields_at(const mw_params *p, float *base) {
   return f;
 }
 
+// checkpoint k of the checkpoint modes (a full state, 256-aligned)
+float *ckpt_slot(char *ws, const Layout &L, int k) {
+  return (float *)(ws + L.snap + (size_t)k * align256(L.state_bytes));
+}
+
 // Pinned-host snapshot store: the caller's page-locked buffer holds step t
 // as [E block][curl block] at 2 t step_bytes; a ring of kHostRing device
 // slots per field stages the copies, which run on a stream of their own and
@@ -718,10 +723,10 @@ int check_ptr(const void *ptr, const char *name) {
   return MW_OK;
 }
 
-// Checkpoint replay: re-runs the forward from checkpoint k over its segment
-// [k C, min((k + 1) C, nt)) and stores each step's E and curl (fp32) in the
-// segment buffer at slot t - k C.  Used by the adjoint (segments newest
-// first) and the Born forward (oldest first).
+// Checkpoint replay: re-runs the forward from checkpoint k (read in place)
+// over its segment [k C, min((k + 1) C, t_end)) and stores each step's E and
+// curl (fp32), or E alone, in the segment buffer at slot t - k C.  Used by
+// the adjoint (segments newest first) and the Born forward (oldest first).
 struct Replay {
   const mw_params *p = nullptr;
   char *ws = nullptr;
@@ -732,7 +737,8 @@ struct Replay {
   Chains ch{};
   Launch lf{};
   StepArgs fa{};
-  FwdMaps fA, fB;
+  FwdMaps fA, fB, fS;  // inputs rA, rB, the segment's checkpoint
+  const float *ca_ = nullptr, *cb_ = nullptr, *cq_ = nullptr;
   float *rA = nullptr, *rB = nullptr;
   int store = kStoreF32;  // the segment: E and curl, or E alone (kStoreEy)
   float *last = nullptr;  // the state after the latest replayed segment
@@ -753,6 +759,9 @@ struct Replay {
     fa.snap_pitch = p->nx;  // the fp32 segment
     rA = (float *)(ws + L.rpA);
     rB = (float *)(ws + L.rpB);
+    ca_ = ca;
+    cb_ = cb;
+    cq_ = cq;
     MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, cq, &fA));
     MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, cq, &fB));
     return MW_OK;
@@ -765,16 +774,17 @@ struct Replay {
     const int64_t numel = (int64_t)p->ny * p->nx;
     char *seg_e = ws + L.seg;
     char *seg_c = seg_e + (size_t)C * L.snap_step_bytes;
-    MW_CUDA(cudaMemcpyAsync(rA, ws + L.snap + (size_t)k * align256(L.state_bytes),
-                            L.state_bytes, cudaMemcpyDeviceToDevice, st));
-    float *rc = rA, *rn = rB;
+    // the first step reads the checkpoint in place
+    float *rc = ckpt_slot(ws, L, k), *rn = rA;
+    MW_TRY(fwd_maps(p, fields_at(p, rc), ca_, cb_, cq_, &fS));
     for (int t = t0; t < t1; ++t) {
+      rn = rc == rA ? rB : rA;
       fa.in = fields_at(p, rc);
       fa.out = fields_at(p, rn);
       fa.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
       fa.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
       fa.ctr_slot = ((*launch_idx)++) & 1;
-      const FwdMaps &fm = rc == rA ? fA : fB;
+      const FwdMaps &fm = rc == rA ? fA : rc == rB ? fB : fS;
       MW_CUDA(timed(1, st, [&] {
         return launch_forward(fm, fa, p->order, store, kStoreNone, p->model_batched != 0,
                               !p->cq_is_scalar, lf.grid, st);
@@ -782,7 +792,7 @@ struct Replay {
       MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
                                    f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
                                    ch.src_lead, ch.src_next, p->n_src, nullptr, 0, nullptr, st));
-      std::swap(rc, rn);
+      rc = rn;
     }
     last = rc;
     *t0_out = t0;
@@ -956,11 +966,16 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   if (host) MW_TRY(hc.init());
   char *hbuf = (char *)p->snap_host_ptr;
   float *cur = bufA, *nxt = bufB;
+  // checkpoint modes: checkpoint 0 is a copy of the initial state; the step
+  // that produces the state of checkpoint k >= 1 writes it into the slot
+  // directly and the next step reads it from there (no copies)
+  const bool ck = is_ckpt(p);
+  if (ck) MW_CUDA(cudaMemcpyAsync(ckpt_slot(ws, L, 0), bufA, L.state_bytes,
+                                  cudaMemcpyDeviceToDevice, st));
+  FwdMaps mS;  // input maps of a checkpoint slot
   for (int t = 0; t < p->nt; ++t) {
-    if (is_ckpt(p) && t % p->ckpt_every == 0) {
-      char *ck = ws + L.snap + (size_t)(t / p->ckpt_every) * align256(L.state_bytes);
-      MW_CUDA(cudaMemcpyAsync(ck, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
-    }
+    const int k_out = ck && (t + 1) % p->ckpt_every == 0 ? (t + 1) / p->ckpt_every : -1;
+    nxt = k_out > 0 && k_out < L.n_seg ? ckpt_slot(ws, L, k_out) : cur == bufA ? bufB : bufA;
     const int slot = host ? t % kHostRing : t;
     // the slot's previous step must have reached the host
     if (host && t >= kHostRing) MW_CUDA(cudaStreamWaitEvent(st, hc.freed[slot], 0));
@@ -974,7 +989,8 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
       a.snap_e = tail_e + (size_t)(t - t_tail) * L.snap_step_bytes;
       a.snap_c = tail_c + (size_t)(t - t_tail) * L.snap_step_bytes;
     }
-    const FwdMaps &m = cur == bufA ? mA : mB;
+    if (cur != bufA && cur != bufB) MW_TRY(fwd_maps(p, a.in, ca, cb, cq, &mS));
+    const FwdMaps &m = cur == bufA ? mA : cur == bufB ? mB : mS;
     a.ctr_slot = t & 1;
     MW_CUDA(timed(kind ? 1 : 0, st, [&] {
       return launch_forward(m, a, p->order, kind, kStoreNone, p->model_batched != 0, !p->cq_is_scalar,
@@ -994,7 +1010,7 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
                                  ch.src_lead, ch.src_next, p->n_src, rec_idx, p->n_rec,
                                  rec_out ? rec_out + (int64_t)t * p->n_shots * p->n_rec : nullptr,
                                  st));
-    std::swap(cur, nxt);
+    cur = nxt;
   }
   if (ey_only && rec && p->n_rec > 0)
     MW_CUDA(cudaMemcpyAsync(rec, rec_out, (size_t)p->nt * p->n_shots * p->n_rec * sizeof(float),

@@ -98,17 +98,17 @@ def alg_bytes(wl, S):
     """Bytes per cell-update of each pass of the workload's sweep (fp32 fields):
     state read + write 24 B, Ca and Cb (shared by the shots unless the model is
     batched), the CPML band memories, snapshot write / read (8, 4 or 2 B), the
-    per-shot gradient read-modify-write 16 B, checkpoint copies 28 / C B.
-    With the E snapshot alone ("ckpt_ey") the replay writes and the adjoint
-    reads 4 B of snapshot instead of 8."""
+    per-shot gradient read-modify-write 16 B.  Checkpoints cost nothing
+    beyond the state traffic: the step that produces one writes it into its
+    slot and the next step (and later the replay) reads it there.  With the E
+    snapshot alone ("ckpt_ey") the replay writes and the adjoint reads 4 B of
+    snapshot instead of 8."""
     band = 16.0 * (2.0 * wl.n_pml / wl.nx + 2.0 * wl.n_pml / wl.ny)
     model = 8.0 if wl.batched else 8.0 / S
     base = 24.0 + model + band
     if wl.snapshot in CKPT_MODES:
-        C = wl.ckpt_every
         sb = 4.0 if wl.snapshot == "ckpt_ey" else 8.0
-        return {"forward": base + 28.0 / C, "replay": base + sb + 28.0 / C,
-                "adjoint": base + sb + 16.0}
+        return {"forward": base, "replay": base + sb, "adjoint": base + sb + 16.0}
     if wl.snapshot == "none":
         return {"forward": base}
     sb = {"fp32": 8.0, "bf16": 4.0, "fp8": 2.0}[wl.snapshot]
