@@ -592,7 +592,10 @@ int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float 
   MW_TRY(encode_rows(&m->map[kAMapEH], in.ey, 4, 4, nx, ny, S, 2, 128, 2,
                      (uint64_t)(in.hz - in.ey) * sizeof(float)));
   const MdPair md = md_pairing(p, ca, cb);
-  if (md.pair) {
+  if (ey_only) {  // Cb of the row fetched, Ca of the row updated
+    MW_TRY(encode_rows(&m->map[kAMapCB], cb, 4, 3, nx, ny, Sm, 1, 128));
+    MW_TRY(encode_rows(&m->map[kAMapCA], ca, 4, 3, nx, ny, Sm, 1, 112));
+  } else if (md.pair) {
     MW_TRY(encode_rows(&m->map[kAMapMD], md.swap ? cb : ca, 4, 4, nx, ny, Sm, 2, 128, 2,
                        md.stride));
   } else {
@@ -601,13 +604,12 @@ int adj_maps(const mw_params *p, const Fields &in, const float *ca, const float 
   }
   MW_TRY(encode_rows(&m->map[kAMapHX], in.hx, 4, 3, nx, ny, S, 1, 112));
   if (ey_only) {
-    // (x, y, shot, step): the E snapshots; and lambda_E of the input again
+    // (x, y, shot, step): the E snapshots
     const uint64_t e = (uint64_t)snap_elem, pitch = (uint64_t)snap_pitch;
     const uint64_t dims[4] = {nx, ny, S, (uint64_t)snap_steps};
     const uint64_t strides[3] = {pitch * e, pitch * ny * e, pitch * ny * S * e};
     const uint32_t box[4] = {112, 1, 1, 1};
     MW_TRY(encode_map(&m->map[kAMapSS], se, snap_elem, 4, dims, strides, box));
-    MW_TRY(encode_rows(&m->map[kAMapLE], in.ey, 4, 3, nx, ny, S, 1, 112));
   } else {
     // (x, y, shot, step, field): the curl snapshots follow the E snapshots
     const uint64_t e = (uint64_t)snap_elem;

@@ -129,12 +129,13 @@ struct FwdMaps {
 //   kAMapMX  the x-band memories at the H and E nodes (adjacent arrays) as
 //            one pair box of whole band rows
 //   kAMapMZE / kAMapMZH  z-band memories, 112 wide from x0
-//   kAMapLE  lambda_E of the input, 112 wide from x0 (kStoreEy: the gradients
-//            of a row are formed at its E update, 2P - 1 rows after its
-//            first fetch; kAMapSS is then the E snapshot alone, 4-D)
+//   kAMapCA  Ca alone, 112 wide from x0 (kStoreEy: a row's E update and its
+//            gradients come 2P - 1 rows after its first fetch, which then
+//            needs Cb alone, kAMapCB; the walk carries lambda_E to the E
+//            update and kAMapSS is the E snapshot alone, 4-D)
 enum AdjMap {
   kAMapEH = 0, kAMapMD, kAMapCB, kAMapHX, kAMapSS, kAMapGG, kAMapGB, kAMapCQ, kAMapMX,
-  kAMapMZE, kAMapMZH, kAMapLE, kAdjMaps
+  kAMapMZE, kAMapMZH, kAMapCA, kAdjMaps
 };
 struct AdjMaps {
   CUtensorMap map[kAdjMaps];

@@ -554,8 +554,10 @@ struct AdjWarp {
 // Issue the loads of walk iteration i (lane 0 only): row r = r0 + i for
 // lambda_E / lambda_Hz, Ca / Cb, Cq, the snapshots, the gradients and the
 // band memories of the E nodes and (x band) H nodes; row r - P for
-// lambda_Hx, its Cq and its z-band memory.  Rows outside the array read as
-// zeros.
+// lambda_Hx, its Cq and its z-band memory.  With the E snapshot alone
+// (kStoreEy) row r brings Cb only, and Ca, the E snapshot and the gradients
+// come for row r - 2P + 1, whose E update this iteration makes.  Rows
+// outside the array read as zeros.
 template <int P, int SNAP, bool BAND>
 __device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, const Item &it,
                                           int i, uint32_t st, uint32_t bar, int cq_arr) {
@@ -570,7 +572,7 @@ __device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, c
   // (lambda_E and the E snapshot)
   const bool g_r = EY ? (unsigned)(i - (4 * P - 2)) < (unsigned)(it.yb - it.ya) : own_r;
   const int rg = EY ? r - 2 * P + 1 : r;
-  uint32_t bytes = 2 * 128 * 4 + 2 * 128 * 4;
+  uint32_t bytes = 2 * 128 * 4 + (EY ? 128 * 4 : 2 * 128 * 4);
   if (hx_in) bytes += 112 * 4;
   if (g_r) bytes += snap_bytes + 2 * 112 * 4;
   if (cq_arr) bytes += hx_in ? 2 * 128 * 4 : 128 * 4;
@@ -585,7 +587,9 @@ __device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, c
   expect_tx_s(bar, bytes);
   fence_proxy_async();
   tma4s(st + kA_EH * 4, &m.map[kAMapEH], it.x0 - 8, r, it.s, 0, bar);
-  if (a.md_pair) {
+  if constexpr (EY) {
+    tma3s(st + kA_MD * 4, &m.map[kAMapCB], it.x0 - 8, r, it.sm, bar);
+  } else if (a.md_pair) {
     tma4s(st + kA_MD * 4, &m.map[kAMapMD], it.x0 - 8, r, it.sm, 0, bar);
   } else {
     tma3s(st + kA_MD * 4, &m.map[kAMapMD], it.x0 - 8, r, it.sm, bar);
@@ -594,7 +598,7 @@ __device__ __forceinline__ void adj_issue(const AdjMaps &m, const StepArgs &a, c
   if (hx_in) tma3s(st + kA_HX * 4, &m.map[kAMapHX], it.x0, r - P, it.s, bar);
   if (g_r) {
     if constexpr (EY) {
-      tma3s(st + kA_SS * 4, &m.map[kAMapLE], it.x0, rg, it.s, bar);
+      tma3s(st + kA_SS * 4, &m.map[kAMapCA], it.x0, rg, it.sm, bar);
       tma4s(st + (kA_SS + 128) * 4, &m.map[kAMapSS], it.x0, rg, it.s, a.snap_t, bar);
     } else {
       tma5s(st + kA_SS * 4, &m.map[kAMapSS], it.x0, rg, it.s, a.snap_t, 0, bar);
@@ -701,12 +705,18 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
 
         const F4 lam = lds4s(st + kA_EH * 4 + 16 * lane);
         const F4 cbv = lds4s(st + w.cb_o + 16 * lane);
-        const F4 cav = lds4s(st + w.ca_o + 16 * lane);
         F4 gv;
+        if constexpr (SNAP == kStoreEy) {  // lambda_E itself goes to the E update
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          gv.v[q] = cbv.v[q] * lam.v[q];
-          cl[Q::at(u, 0)].v[q] = cav.v[q] * lam.v[q];
+          for (int q = 0; q < 4; ++q) gv.v[q] = cbv.v[q] * lam.v[q];
+          cl[Q::at(u, 0)] = lam;
+        } else {
+          const F4 cav = lds4s(st + w.ca_o + 16 * lane);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            gv.v[q] = cbv.v[q] * lam.v[q];
+            cl[Q::at(u, 0)].v[q] = cav.v[q] * lam.v[q];
+          }
         }
         // ---- pz at E nodes (every row; owned lanes matter)
         {
@@ -839,6 +849,14 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
         if (e_row) {
           float wv[12];
           win12s(w.qring + slot_r * kARing * 4 + 16 * wo, wv);
+          // Ca lam^{t+1} of this row: queued, or (kStoreEy) formed here from
+          // the queued lambda_E and the row's Ca
+          F4 cla = cl[Q::at(u, NQ - 1)];
+          if constexpr (SNAP == kStoreEy) {
+            const F4 ca_e = lds4s(st + kA_SS * 4 + 16 * wo);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cla.v[q] = ca_e.v[q] * cla.v[q];
+          }
           F4 en;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -847,7 +865,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
             for (int k = 1; k <= P; ++k)
               dz = fmaf(a.c.cy[k - 1], qq[Q::at(u, P - k)].v[q] - qq[Q::at(u, P - 1 + k)].v[q],
                         dz);
-            en.v[q] = cl[Q::at(u, NQ - 1)].v[q] - d_int<P>(wv, q, a.c.cx) - dz;
+            en.v[q] = cla.v[q] - d_int<P>(wv, q, a.c.cx) - dz;
           }
           st4p(own, ey_o + (ro - (2 * P - 1) * nx), en);
           if constexpr (SNAP == kStoreEy) {
@@ -855,7 +873,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
             // the Cb accumulator takes E^t times the E-update term
             // G^t = lam~^t - Ca lam^{t+1} (at t = 0: E^0 times -Ca lam^1)
             const int re = r - 2 * P + 1;
-            const F4 lv = lds4s(st + kA_SS * 4 + 16 * wo);
+            const F4 lv = cl[Q::at(u, NQ - 1)];
             const F4 se = lds4s(st + (kA_SS + 128) * 4 + 16 * wo);
             F4 gca = lds4s(st + w.gca_o + 16 * wo), gcb = lds4s(st + w.gcb_o + 16 * wo);
             const bool rowmask =
@@ -863,7 +881,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               if (rowmask && colmask[q]) {
-                const float c = cl[Q::at(u, NQ - 1)].v[q];
+                const float c = cla.v[q];
                 gca.v[q] = fmaf(se.v[q], lv.v[q], gca.v[q]);
                 gcb.v[q] = fmaf(se.v[q], a.tzero ? -c : en.v[q] - c, gcb.v[q]);
               }
@@ -908,6 +926,7 @@ __global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_c
   // array lies first; single boxes at 128-float slots
   w.ca_o = (kA_MD + (a.md_pair && a.md_swap ? 128 : 0)) * 4;
   w.cb_o = (kA_MD + (a.md_pair && a.md_swap ? 0 : 128)) * 4;
+  if constexpr (SNAP == kStoreEy) w.cb_o = kA_MD * 4;  // Cb alone
   w.gca_o = (kA_GG + (a.gg_pair && a.gg_swap ? 112 : 0)) * 4;
   w.gcb_o = (kA_GG + (a.gg_pair ? (a.gg_swap ? 0 : 112) : 128)) * 4;
   w.ring = Ring{0, 0u};
