@@ -18,7 +18,7 @@ import torch
 
 import oracle
 from adjoint_state_gradients_b200 import api, mwtm, synth
-from tests._cases import rel_l2, small_sim
+from tests._cases import rel_l2, small_sim, workload_sim
 from tests._gpu import f32, problem_from_sim, run_adjoint, run_forward
 
 pytestmark = pytest.mark.gpu
@@ -248,3 +248,32 @@ def test_forward_stored_tail_matches_oracle_and_born():
     gca, gcb, gf = run_adjoint(prob, res)
     _check_grads(gca, gcb, gf, ad)
     assert prob.status() == mwtm.MW_OK
+
+
+def test_full_length_sweep_matches_pair_checkpoints():
+    """The 2128^2 order-4 workload over its full 4000 steps (2 of its 8 shots):
+    the summation-by-parts dJ/dCb of the E-alone checkpoints, with and without
+    the forward-stored tail, against the direct sum of the pair checkpoints
+    (both fp32); dJ/dCa and dJ/df bitwise."""
+    nt = 4000
+    sim, inp, dt, f = workload_sim(4, n_shots=2, nt=nt)
+    g = synth.rng(4004)
+    res = torch.as_tensor(f32(g.normal(size=(nt, 2, inp.wl.n_rec))), dtype=torch.float32).cuda()
+    f_d = torch.as_tensor(np.asarray(f, dtype=np.float32)).cuda()
+    out = {}
+    for mode, tail in (("ckpt", 0), ("ckpt_ey", 0), ("ckpt_ey", 320)):
+        prob = problem_from_sim(sim, nt, dt, inp.wl.n_pml, snapshot=mode, ckpt_every=64,
+                                ckpt_tail=tail)
+        prob.forward(f_d)
+        gca, gcb, gf = prob.adjoint(res, grad_f=True)
+        torch.cuda.synchronize()
+        assert prob.status() == mwtm.MW_OK
+        out[(mode, tail)] = [t.cpu().numpy().astype(np.float64) for t in (gca, gcb, gf)]
+        del prob
+    ref = out[("ckpt", 0)]
+    for key in (("ckpt_ey", 0), ("ckpt_ey", 320)):
+        assert np.array_equal(out[key][0], ref[0]) and np.array_equal(out[key][2], ref[2])
+        err = rel_l2(out[key][1], ref[1])
+        print(f"{key}: rel-L2 of dJ/dCb against the direct sum {err:.2e}")
+        assert err <= GRAD_TOL
+    assert np.array_equal(out[("ckpt_ey", 0)][1], out[("ckpt_ey", 320)][1])
