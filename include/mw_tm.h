@@ -70,7 +70,7 @@ extern "C" {
 #define MW_ERR_NONFINITE (-5)   /* NaN / Inf found in a field (device flag) */
 #define MW_ERR_TIMEOUT (-6)     /* a kernel gave up waiting for its own copies
                                    (device flag; results of that call invalid) */
-#define MW_ERR_UNSUPPORTED (-7) /* valid request this build does not serve  */
+#define MW_ERR_UNSUPPORTED (-7) /* valid request the library does not serve */
 
 /* forward snapshot storage for the gradient */
 #define MW_SNAP_NONE 0 /* records only; mw_tm_adjoint_grad unavailable       */
