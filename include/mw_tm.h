@@ -238,8 +238,10 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca_dev,
  *   adj_state      in/out adjoint state, or NULL (start from zero)
  * In MW_SNAP_CKPT mode the forward is replayed segment by segment from the
  * checkpoints, which needs f and src_idx again. */
-/* MW_SNAP_CKPT_EY: with E^{t+1} = Ca E^t + Cb curl^t + s^t (s the source
- * injection) and the adjoint's E update lam~^t = Ca lam^{t+1} + G^t
+/* MW_SNAP_CKPT_EY: the same gradient (the maxwell.cu page's header comment:
+ * grad_cb = sum_t curl^t lambda_E^{t+1}), regrouped.  With
+ * E^{t+1} = Ca E^t + Cb curl^t + s^t (s the source injection; the page's
+ * forward equations) and the adjoint's E update lam~^t = Ca lam^{t+1} + G^t
  * (lam^{t+1} = lam~^{t+1} + the residual injected at step t), the sum
  * Cb * grad_cb = sum_t curl^t lam^{t+1} * Cb regroups, exactly, into
  *     sum_{t>=1} G^t E^t  -  Ca lam^1 E^0  +  lam~^{nt} E^{nt}
