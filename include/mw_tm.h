@@ -248,9 +248,11 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca_dev,
  *   + sum_t res[t] rec[t]  (at the receiver cells)
  *   - sum_t f[t] lam^{t+1} (at the source cells),
  * which needs only E^t from the replay.  The kernel accumulates the first two
- * terms row by row into a workspace array at each row's E update, the
- * injection launches gather the last two, and the end of the call adds them
- * and divides by Cb.  grad_ca_shot, grad_f and the adjoint state are
+ * terms row by row, at each row's E update, into a workspace array that
+ * starts at the third (zero unless adj_state is given; E^{nt} comes from the
+ * last replayed segment or the forward-stored tail), the injection launches
+ * gather the last two, and the end of the call adds them and divides by
+ * Cb.  grad_ca_shot, grad_f and the adjoint state are
  * bitwise those of MW_SNAP_CKPT; grad_cb_shot agrees to rounding. */
 int mw_tm_adjoint_grad(const mw_params *p, const float *ca_dev,
                        const float *cb_dev, const float *cq_dev,
