@@ -694,3 +694,60 @@ def test_born_forward_is_the_transpose_of_the_gradient(batched):
     lhs = float(np.sum(b * res))
     rhs = float(np.sum(dca * gca) + np.sum(dcb * gcb))
     assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), abs(rhs))
+
+
+@pytest.mark.parametrize("order,n_pml", [(2, 3), (4, 4), (8, 0)])
+def test_cb_gradient_regroups_by_summation_by_parts(order, n_pml):
+    """The identity the E-alone checkpoint mode evaluates, in fp64: with the
+    forward E^{t+1} = Ca E^t + Cb curl^t + s^t and the adjoint's E update
+    lam~^t = Ca lam^{t+1} + G^t (lam^{t+1} = lam~^{t+1} + the residual injected
+    at step t),
+        Cb sum_t curl^t lam^{t+1} = sum_{t>=1} G^t E^t - Ca lam^1 E^0
+            + lam~^{nt} E^{nt} + sum_t res[t] rec[t] (receiver cells)
+            - sum_t f[t] lam^{t+1} (source cells),
+    every end term live: given initial and adjoint states, duplicate and
+    inactive indices, a source on a receiver.  The left side is the oracle's
+    own gradient; the right side steps the oracle's adjoint one step at a time
+    to read lam~^t."""
+    S, ny, nx, nt = 2, 20, 24, 30
+    sim, dt, _ = small_sim(950 + order, ny, nx, S, 3, 4, order, n_pml, sigma_max=0.02)
+    sim.src_idx[0] = [50, 50, -1]
+    sim.rec_idx[0, :3] = [50, 77, 77]
+    sim.rec_idx[1, 1] = -1
+    g = synth.rng(951 + order)
+    st0 = np.zeros(sim.zero_state().shape)
+    st0[:3] = 0.1 * g.normal(size=st0[:3].shape)
+    ad0 = np.zeros_like(st0)
+    ad0[:3] = g.normal(size=ad0[:3].shape)
+    f = g.normal(size=(nt, S, 3))
+    res = g.normal(size=(nt, S, 4))
+    fw = sim.forward(f, state=st0, snapshots=True)
+    full = sim.adjoint(res, fw["snap_ey"], fw["snap_curl"], adj=ad0)
+    ca = np.broadcast_to(sim.ca, (S, ny, nx))
+    cb = np.broadcast_to(sim.cb, (S, ny, nx))
+
+    def scatter(idx, vals):  # per-entry values onto their cells; duplicates add
+        out = np.zeros((S, ny * nx))
+        for s in range(S):
+            for k, i in enumerate(idx[s]):
+                if i >= 0:
+                    out[s, i] += vals[s, k]
+        return out.reshape(S, ny, nx)
+
+    def gather(idx, field):
+        flat = field.reshape(S, -1)
+        return np.array([[flat[s, i] if i >= 0 else 0.0 for i in idx[s]] for s in range(S)])
+
+    rhs = ad0[0] * fw["state"][0]                      # lam~^{nt} E^{nt}
+    adj = ad0.copy()
+    for t in range(nt - 1, -1, -1):
+        lam = adj[0] + scatter(sim.rec_idx, res[t])   # lam^{t+1}
+        adj = sim.adjoint(res[t:t + 1], fw["snap_ey"][t:t + 1], fw["snap_curl"][t:t + 1],
+                          adj=adj, grad_f=False)["adj"]   # lam~^t
+        e_t = fw["snap_ey"][t]
+        rhs += (adj[0] - ca * lam) * e_t if t >= 1 else -ca * lam * e_t
+        rhs += scatter(sim.rec_idx, res[t] * fw["rec"][t])
+        rhs -= scatter(sim.src_idx, f[t] * gather(sim.src_idx, lam))
+    lhs = cb * full["gcb"]
+    assert np.abs(lhs).max() > 0
+    assert rel_l2(rhs, lhs) <= 1e-12
