@@ -315,6 +315,8 @@ def main():
     wl = synth.WORKLOADS[number]
     if args.snapshot:
         wl = dataclasses.replace(wl, snapshot=args.snapshot)
+        if wl.snapshot in CKPT_MODES and wl.ckpt_every < 1:  # a full-storage workload
+            wl = dataclasses.replace(wl, ckpt_every=64)
     if args.ckpt_tail is not None:
         wl = dataclasses.replace(wl, ckpt_tail=args.ckpt_tail)
     nt = args.nt or wl.nt
