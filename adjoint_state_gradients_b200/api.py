@@ -73,25 +73,36 @@ class Problem:
         p = self.p
         return (self.S, p.ny, p.nx) if p.model_batched else (p.ny, p.nx)
 
+    def _model_buffers(self):
+        """Ca, Cb, Cq buffers, allocated once: later model updates write into
+        them, so a captured SweepGraph sees the new model."""
+        d = self.device
+        cq_shape = (1,) if self.p.cq_is_scalar else self.model_shape
+        for name, shape in (("ca", self.model_shape), ("cb", self.model_shape), ("cq", cq_shape)):
+            t = getattr(self, name)
+            if t is None or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+                setattr(self, name, torch.empty(shape, dtype=F32, device=d))
+
     def set_model_eps_sigma(self, eps_r, sigma=None, mu_r=None, f0=0.0, R=1e-3):
-        """Ca, Cb, Cq from eps_r, sigma, mu_r (library kernel) and CPML profiles."""
+        """Ca, Cb, Cq from eps_r, sigma, mu_r (library kernel) and CPML profiles,
+        written into the problem's model buffers."""
         d = self.device
         eps_r = _dev(eps_r, device=d).reshape(self.model_shape)
         sigma = None if sigma is None else _dev(sigma, device=d).reshape(self.model_shape)
         mu_r = None if mu_r is None else _dev(mu_r, device=d).reshape(self.model_shape)
-        self.ca = torch.empty(self.model_shape, dtype=F32, device=d)
-        self.cb = torch.empty(self.model_shape, dtype=F32, device=d)
-        self.cq = torch.empty((1,) if self.p.cq_is_scalar else self.model_shape, dtype=F32, device=d)
+        self._model_buffers()
         mwtm.model_from_eps_sigma(self.p, eps_r, sigma, mu_r, self.ca, self.cb, self.cq)
         mwtm.cpml_profiles(self.p, f0, R, self.cpml)
         return self
 
     def set_coefficients(self, ca, cb, cq, cpml):
+        """Copy Ca, Cb, Cq and the 12 CPML profiles into the model buffers."""
         d = self.device
-        self.ca = _dev(ca, device=d).reshape(self.model_shape)
-        self.cb = _dev(cb, device=d).reshape(self.model_shape)
-        self.cq = _dev(cq, device=d).reshape(-1)
-        self.cpml = _dev(cpml, device=d).reshape(-1)
+        self._model_buffers()
+        self.ca.copy_(_dev(ca, device=d).reshape(self.model_shape))
+        self.cb.copy_(_dev(cb, device=d).reshape(self.model_shape))
+        self.cq.copy_(_dev(cq, device=d).reshape(self.cq.shape))
+        self.cpml.copy_(_dev(cpml, device=d).reshape(-1))
         return self
 
     # ---- sweeps ------------------------------------------------------------
@@ -206,6 +217,10 @@ class SweepGraph:
         else:
             self.gca = torch.zeros((p.ny, p.nx), dtype=F32, device=dev)
             self.gcb = torch.zeros((p.ny, p.nx), dtype=F32, device=dev)
+        # the buffers the capture bakes in (kept alive; replay() checks that
+        # the problem still uses them)
+        self._baked = (prob.ca, prob.cb, prob.cq, prob.cpml, prob.workspace, prob.src_idx,
+                       prob.rec_idx)
         # one eager sweep first: kernel attributes are set and the work
         # counters settle outside the capture
         self._body()
@@ -230,7 +245,13 @@ class SweepGraph:
 
     def replay(self):
         """Run the captured sweep on the current stream's device; returns
-        (J, rec, grad_Ca, grad_Cb) (the buffers above)."""
+        (J, rec, grad_Ca, grad_Cb) (the buffers above).  Model updates must go
+        through the problem's setters, which write in place."""
+        prob = self.prob
+        now = (prob.ca, prob.cb, prob.cq, prob.cpml, prob.workspace, prob.src_idx, prob.rec_idx)
+        if any(a is not b for a, b in zip(now, self._baked)):
+            raise RuntimeError("SweepGraph: a buffer of the problem was replaced after capture "
+                               "(update the model through set_model_eps_sigma / set_coefficients)")
         self.graph.replay()
         return self.J, self.rec, self.gca, self.gcb
 
