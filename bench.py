@@ -128,6 +128,20 @@ def pass_classes(wl):
     return {"forward": 1, "adjoint": 2}
 
 
+TAIL_RESERVE = 12e9  # device bytes left free beside the workspace
+
+
+def fit_tail(tail, base_bytes, step_bytes, free_bytes, C=64):
+    """The forward-stored tail that fits: at most `tail` steps, whole
+    C-step segments when cut, with the workspace (base_bytes without a tail,
+    step_bytes per tail step) at most free_bytes - TAIL_RESERVE."""
+    room = free_bytes - TAIL_RESERVE - base_bytes
+    if tail <= 0 or room <= 0:
+        return 0
+    k = int(room // step_bytes)
+    return tail if k >= tail else (k // C) * C
+
+
 def sample_steps(wl, target_cell_updates):
     """Steps of a one-shot oracle sample worth about target_cell_updates."""
     return int(max(16, min(wl.nt, target_cell_updates // (wl.ny * wl.nx))))
@@ -337,6 +351,19 @@ def main():
     dt = wl.cfl_fraction * mwtm.cfl_dt(wl.order, wl.h, wl.h, vmax)
     C = wl.ckpt_every
 
+    if wl.snapshot in CKPT_MODES and wl.ckpt_tail > 0:
+        # the tail trades spare HBM for replay work: shrink it to what is free
+        kw = dict(ny=wl.ny, nx=wl.nx, order=wl.order, n_shots=hi - lo if number == 4 else S,
+                  n_src=inp.src_idx.shape[1], n_rec=inp.rec_idx.shape[1], nt=nt, dt=dt, dy=wl.h,
+                  dx=wl.h, n_pml=wl.n_pml, snap_mode=mwtm.SNAP_MODES[wl.snapshot],
+                  ckpt_every=max(C, 1), vmax=vmax, model_batched=int(wl.batched))
+        # workspace = base + tail x step (the E-alone tail's extra final-E slot
+        # is in base)
+        w1 = mwtm.workspace_bytes(mwtm.make_params(ckpt_tail=1, **kw))
+        step_b = mwtm.workspace_bytes(mwtm.make_params(ckpt_tail=2, **kw)) - w1
+        free, _ = torch.cuda.mem_get_info(dev)
+        wl = dataclasses.replace(wl, ckpt_tail=fit_tail(wl.ckpt_tail, w1 - step_b, step_b, free,
+                                                        max(C, 1)))
     prob = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
                        vmax=vmax, snapshot=wl.snapshot, ckpt_every=max(C, 1), batched=wl.batched,
                        ckpt_tail=wl.ckpt_tail if wl.snapshot in CKPT_MODES else 0)

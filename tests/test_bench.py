@@ -72,3 +72,24 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["config"]["workload"] == synth.WORKLOADS[1].name
+
+
+def test_tail_fits_free_memory():
+    """The forward-stored tail shrinks, by whole segments, to what the free
+    device memory holds beside the reserve, and vanishes when nothing fits."""
+    from adjoint_state_gradients_b200 import mwtm
+    wl = synth.WORKLOADS[4]
+    kw = dict(ny=wl.ny, nx=wl.nx, order=4, n_shots=8, n_src=1, n_rec=512, nt=4000, dt=4.2e-11,
+              dy=0.02, dx=0.02, n_pml=40, snap_mode=mwtm.SNAP_CKPT_EY, ckpt_every=64, vmax=1.7e8)
+    w = {k: mwtm.workspace_bytes(mwtm.make_params(ckpt_tail=k, **kw)) for k in (1, 2, 640)}
+    step = w[2] - w[1]
+    base = w[1] - step
+    assert base + 640 * step == pytest.approx(w[640], abs=4096)
+    gb = 1e9
+    assert bench.fit_tail(640, base, step, 192 * gb) == 640            # a whole B200
+    k = bench.fit_tail(640, base, step, 120 * gb)                      # less free memory
+    assert k % 64 == 0 and 0 < k < 640
+    assert base + k * step <= 120 * gb - bench.TAIL_RESERVE
+    assert base + (k + 64) * step > 120 * gb - bench.TAIL_RESERVE
+    assert bench.fit_tail(640, base, step, 40 * gb) == 0                # not even the checkpoints
+    assert bench.fit_tail(0, base, step, 192 * gb) == 0
