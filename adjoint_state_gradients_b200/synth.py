@@ -76,10 +76,10 @@ WORKLOADS = {
     1: Workload("tm2d-84sq-o2-s1-nt300-fp32snap", 1, 64, 10, 2, 1, 300, 32, 0.02, 400e6, 0.5, "fp32"),
     2: Workload("tm2d-296sq-o4-s4-nt1000-fp32snap", 2, 256, 20, 4, 4, 1000, 128, 0.02, 400e6, 0.6, "fp32"),
     3: Workload("tm2d-1064sq-o8-s16-nt2000-bf16snap", 3, 1000, 32, 8, 16, 2000, 256, 0.01, 200e6, 0.6, "bf16"),
-    # the last 640 steps' E snapshots (92.9 GB) kept from the forward: about
-    # 143 GB of the 180 GB HBM in all
+    # the last 768 steps' E snapshots (111.3 GB) kept from the forward: about
+    # 162 GB of the 180 GB HBM in all
     4: Workload("tm2d-2128sq-o4-s8-nt4000-ckpt64", 4, 2048, 40, 4, 8, 4000, 512, 0.02, 200e6, 0.6,
-                "ckpt_ey", ckpt_every=64, ckpt_tail=640),
+                "ckpt_ey", ckpt_every=64, ckpt_tail=768),
     5: Workload("tm2d-552sq-o8-s256-nt2000-fwd", 5, 512, 20, 8, 256, 2000, 128, 0.02, 200e6, 0.6, "none",
                 batched=True),
 }

@@ -36,8 +36,8 @@ def test_byte_model_of_the_headline_sweep():
     assert bp["adjoint"] - b["adjoint"] == pytest.approx(4.0)
     assert sum(bp.values()) == pytest.approx(110.61, abs=0.01)
     # the forward-stored tail: those steps write E (4 B) and skip the replay
-    assert wl.ckpt_tail == 640
-    want = b["forward"] + 0.16 * 4 + 0.84 * b["replay"] + b["adjoint"]
+    assert wl.ckpt_tail == 768
+    want = b["forward"] + 0.192 * 4 + 0.808 * b["replay"] + b["adjoint"]
     assert bench.sweep_bytes_per_cell(wl, wl.n_shots) == pytest.approx(want)
     assert bench.sweep_bytes_per_cell(dataclasses.replace(wl, ckpt_tail=0), wl.n_shots) == \
         pytest.approx(102.61, abs=0.01)
@@ -87,6 +87,7 @@ def test_tail_fits_free_memory():
     assert base + 640 * step == pytest.approx(w[640], abs=4096)
     gb = 1e9
     assert bench.fit_tail(640, base, step, 192 * gb) == 640            # a whole B200
+    assert bench.fit_tail(768, base, step, 190 * gb) == 768
     k = bench.fit_tail(640, base, step, 120 * gb)                      # less free memory
     assert k % 64 == 0 and 0 < k < 640
     assert base + k * step <= 120 * gb - bench.TAIL_RESERVE
