@@ -34,6 +34,22 @@ def test_library_exports_every_declared_symbol():
     assert not missing, missing
 
 
+def test_binding_constants_match_the_header():
+    """Status codes and snapshot modes: the binding's values are the
+    header's, and every mode the header defines is reachable by name."""
+    text = open(HEADER).read()
+    defs = {k: int(v) for k, v in re.findall(r"#define\s+(MW_(?:ERR_[A-Z]+|OK|SNAP_[A-Z0-9_]+))\s+"
+                                              r"\(?(-?\d+)\)?", text)}
+    assert defs["MW_OK"] == mwtm.MW_OK
+    errs = {k: v for k, v in defs.items() if k.startswith("MW_ERR_")}
+    assert len(errs) >= 7
+    for k, v in errs.items():
+        assert getattr(mwtm, k) == v, k
+    modes = {k[len("MW_SNAP_"):].lower(): v for k, v in defs.items() if k.startswith("MW_SNAP_")}
+    assert modes == {"none": 0, "fp32": 1, "bf16": 2, "ckpt": 3, "fp8": 4, "ckpt_ey": 5}
+    assert mwtm.SNAP_MODES == modes
+
+
 def test_binding_covers_every_declared_symbol():
     bound = {name for name, _, _ in mwtm.SIGNATURES}
     missing = [n for n in declared_functions() if n not in bound]
