@@ -1433,30 +1433,23 @@ int mw_profile_read(int64_t *counts, double *total_ms, int32_t n_classes) {
 // The scratch of mw_tm_forward_noalloc: status words | duplicate chains | CPML
 // band table | the second state buffer of the ping-pong.  Host code must not
 // use the symbol itself (it is a host-side stand-in); it takes the device
-// address from cudaGetSymbolAddress, once per device.
+// address from cudaGetSymbolAddress with the calling device current.
 }  // extern "C"
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MW_NOALLOC_SCRATCH_BYTES];
 
 namespace mw {
 namespace {
-std::mutex g_noalloc_mu;
-void *g_noalloc_addr[64];
-
+// The array's device address in the current device's context, looked up on
+// every call: a cached address would dangle once the context is torn down
+// (cudaDeviceReset) and the module is loaded again at another address.
 int noalloc_scratch(char **out) {
-  int dev = 0;
-  MW_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return fail(MW_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void *ptr = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || !ptr)
-      return fail(MW_ERR_CUDA, "cudaGetSymbolAddress of the built-in scratch failed: %s",
-                  cudaGetErrorString(e));
-    g_noalloc_addr[dev] = ptr;
-  }
-  *out = (char *)g_noalloc_addr[dev];
+  void *ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess || !ptr)
+    return fail(MW_ERR_CUDA, "cudaGetSymbolAddress of the built-in scratch failed: %s",
+                cudaGetErrorString(e));
+  *out = (char *)ptr;
   return MW_OK;
 }
 }  // namespace

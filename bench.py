@@ -9,7 +9,11 @@ fused per-shot gradients, shot reduction of dJ/dCa and dJ/dCb.
 
 --workload picks another of the five workloads (default 4, the headline):
 1 and 2 store fp32 snapshots, 3 bf16 snapshots, 5 times the forward alone
-(records of 256 shots with per-shot models).
+(records of 256 shots with per-shot models).  The default one-GPU run also
+times, after the headline, the headline workload with every segment replayed
+from its checkpoint (no forward-stored tail; `value_strict` with E + curl
+segments, `value_strict_ey` with E alone) and short runs of the other four
+workloads (`other_configs`); --no-extras skips them.
 
 Prints one JSON line (rank 0).  --impl reference times the fp64 CPU oracle
 (the reference arm) on a bounded sample of the same workload.  Multi-GPU runs
@@ -67,6 +71,9 @@ def parse():
                     help="override the workload's forward-stored tail (checkpoint modes)")
     ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5],
                     help="workload to time (default: the 2048^2 order-4 checkpointed sweep)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default run only: skip the strict checkpoint configurations and the "
+                         "other four workloads")
     return ap.parse_args()
 
 
@@ -305,6 +312,274 @@ def run_reference(args):
 # ----------------------------------------------------------------------------
 
 
+class Sweep:
+    """One workload set up on this rank's GPU: the problem, its inputs, the
+    observed data, the gradient buffers and (unless --no-graph) the sweep
+    captured as one CUDA graph.  step() runs one whole sweep."""
+
+    def __init__(self, args, number, wl, nt, rank, world, dev, use_graph=True):
+        import torch
+
+        from adjoint_state_gradients_b200 import api, mwtm, shard, synth
+        self.torch, self.api, self.mwtm, self.shard = torch, api, mwtm, shard
+        self.number, self.nt, self.world, self.dev = number, nt, world, dev
+        S = wl.n_shots
+        self.grad = wl.snapshot != "none"   # workload 5 times the forward alone
+        # weak scaling: every rank simulates its own block of S shots of one
+        # survey of S * world shots (sources spread over the interior)
+        lo, hi = shard.shot_block(S * world, rank, world)
+        if number == 4:
+            inp = synth.make_inputs(number, n_shots=hi - lo, survey_shots=S * world, first_shot=lo)
+        else:  # the other workloads' shots are the same set on every rank
+            inp = synth.make_inputs(number)
+        c0 = 299792458.0
+        vmax = c0 / math.sqrt(inp.eps_min)
+        dt = wl.cfl_fraction * mwtm.cfl_dt(wl.order, wl.h, wl.h, vmax)
+        C = wl.ckpt_every
+        if wl.snapshot in CKPT_MODES and wl.ckpt_tail > 0:
+            # the tail trades spare HBM for replay work: shrink it to what is free
+            kw = dict(ny=wl.ny, nx=wl.nx, order=wl.order, n_shots=hi - lo if number == 4 else S,
+                      n_src=inp.src_idx.shape[1], n_rec=inp.rec_idx.shape[1], nt=nt, dt=dt,
+                      dy=wl.h, dx=wl.h, n_pml=wl.n_pml, snap_mode=mwtm.SNAP_MODES[wl.snapshot],
+                      ckpt_every=max(C, 1), vmax=vmax, model_batched=int(wl.batched))
+            # workspace = base + tail x step (the E-alone tail's extra final-E
+            # slot is in base)
+            w1 = mwtm.workspace_bytes(mwtm.make_params(ckpt_tail=1, **kw))
+            step_b = mwtm.workspace_bytes(mwtm.make_params(ckpt_tail=2, **kw)) - w1
+            free, _ = torch.cuda.mem_get_info(dev)
+            wl = dataclasses.replace(wl, ckpt_tail=fit_tail(wl.ckpt_tail, w1 - step_b, step_b,
+                                                            free, max(C, 1)))
+        self.wl = wl
+        self.prob = prob = api.Problem(
+            wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
+            vmax=vmax, snapshot=wl.snapshot, ckpt_every=max(C, 1), batched=wl.batched,
+            ckpt_tail=wl.ckpt_tail if wl.snapshot in CKPT_MODES else 0)
+        self.f_host = inp.wavelet(dt, nt).astype(np.float32)
+        self.eps_h = inp.eps_r.astype(np.float32)
+        self.sig_h = inp.sigma.astype(np.float32)
+        # observed data from the perturbed model (setup, outside the timed region)
+        obs = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx,
+                          inp.rec_idx, vmax=vmax, snapshot="none", batched=wl.batched)
+        obs.set_model_eps_sigma(inp.eps_r_true.astype(np.float32), self.sig_h, f0=wl.f0)
+        self.f_dev = torch.as_tensor(self.f_host, device=dev)
+        self.d_obs = obs.forward(self.f_dev).clone()
+        del obs
+        torch.cuda.synchronize()
+        prob.set_model_eps_sigma(self.eps_h, self.sig_h, f0=wl.f0)
+        self.gshape = (wl.ny, wl.nx) if self.grad else (1,)
+        self.gca = torch.empty(self.gshape, device=dev)
+        self.gcb = torch.empty(self.gshape, device=dev)
+        self.gca_s = torch.empty((S, wl.ny, wl.nx) if self.grad else (1,), device=dev)
+        self.gcb_s = torch.empty((S, wl.ny, wl.nx) if self.grad else (1,), device=dev)
+        self.rec = torch.empty((nt, S, wl.n_rec), device=dev)
+        self.res = torch.empty_like(self.rec)
+        self.J = torch.zeros(1, dtype=torch.float64, device=dev)
+        self.stream = torch.cuda.current_stream()
+        # the sweep captured once as a CUDA graph and replayed (the per-kernel
+        # event pass stays eager)
+        self.graph = api.SweepGraph(prob, self.f_dev, self.d_obs) if (
+            self.grad and use_graph) else None
+        self.cells = wl.ny * wl.nx * nt * S * world
+
+    def step(self, ev_fwd=None, eager=False):
+        prob, shard = self.prob, self.shard
+        if self.graph is not None and not eager:
+            self.graph.replay()
+            if ev_fwd is not None:  # no forward boundary inside a replay
+                ev_fwd.record(self.stream)
+            shard.sum_over_ranks_(self.graph.gca, self.graph.gcb)
+            return
+        prob.forward(self.f_dev, rec=self.rec)
+        if ev_fwd is not None:
+            ev_fwd.record(self.stream)
+        prob.residual(self.rec, self.d_obs, res=self.res, J=self.J)
+        if not self.grad:
+            return
+        self.gca_s.zero_()
+        self.gcb_s.zero_()
+        prob.adjoint(self.res, gca=self.gca_s, gcb=self.gcb_s)
+        prob.combine(self.gca_s, out=self.gca)
+        prob.combine(self.gcb_s, out=self.gcb)
+        shard.sum_over_ranks_(self.gca, self.gcb)
+
+    def measure(self, steps, warmup, clocks=None, flush_l2=False):
+        """Time `steps` sweeps after `warmup` untimed ones.  Returns the
+        numbers of the JSON line.  flush_l2: time each sweep alone with an
+        L2-sized write between sweeps (for workloads whose state fits in L2)."""
+        torch, mwtm, shard = self.torch, self.mwtm, self.shard
+        wl, world, dev, stream = self.wl, self.world, self.dev, self.stream
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        rc = self.prob.status()
+        if rc != mwtm.MW_OK:
+            raise RuntimeError(f"device status {rc}: {mwtm.last_error()}")
+        flush = torch.empty(64 << 20, dtype=torch.float32, device=dev) if flush_l2 else None
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        ev0, ev1 = ev(), ev()
+        evs = [(ev(), ev()) for _ in range(steps)]
+        evs_end = [ev() for _ in range(steps)]
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        # timed region: K steps, nothing recorded between the library's launches
+        mwtm.profile_enable(False)
+        n0 = mwtm.launch_count()
+        if clocks is not None:
+            clocks.start()
+        ev0.record(stream)
+        for k in range(steps):
+            if flush is not None:
+                flush.fill_(float(k))
+            evs[k][0].record(stream)
+            self.step(ev_fwd=evs[k][1])
+            evs_end[k].record(stream)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        n_launch = mwtm.launch_count() - n0
+        if self.graph is not None:  # replays count no host launches: the graph's own
+            n_launch = self.graph.launches * steps
+        clk = clocks.stop() if clocks is not None else None
+        if world > 1:
+            dist.barrier()
+        total_ms = (sum(a.elapsed_time(b) for (a, _), b in zip(evs, evs_end)) if flush is not None
+                    else ev0.elapsed_time(ev1))
+        # per-kernel durations for the roofline: the same K steps once more
+        # with CUDA events around every stencil launch on the launching stream
+        # (the events add a little time between kernels, so `value` comes from
+        # the pass above)
+        mwtm.profile_enable(True)
+        evs_e = [(ev(), ev()) for _ in range(steps)]
+        for k in range(steps):
+            evs_e[k][0].record(stream)
+            self.step(ev_fwd=evs_e[k][1], eager=True)
+        torch.cuda.synchronize()
+        counts, ms = mwtm.profile_read(3)
+        mwtm.profile_enable(False)
+        if world > 1:
+            dist.barrier()
+        # the forward alone: from the timed pass, or (graph replays have no
+        # forward boundary) from the eager pass with per-launch events
+        fwd_ms = sum(a.elapsed_time(b) for a, b in (evs if self.graph is None else evs_e))
+        total_ms = shard.max_over_ranks(total_ms, dev)
+        fwd_ms = shard.max_over_ranks(fwd_ms, dev)
+
+        S, nt = wl.n_shots, self.nt
+        value = self.cells * steps / (total_ms / 1e3) / 1e9
+        value_fwd = self.cells * steps / (fwd_ms / 1e3) / 1e9
+        passes = alg_bytes(wl, S)
+        classes = pass_classes(wl)
+        peak, peak_kind = measured_peaks()
+        sweep_bytes = sweep_bytes_per_cell(wl, S, nt) * self.cells * steps
+        sweep_frac = sweep_bytes / (total_ms / 1e3) / 1e9 / peak / world
+        launch_ms = {k: ms[c] / max(counts[c], 1) for k, c in classes.items()}
+        top = "adjoint" if self.grad else "forward"   # the dominant kernel
+        top_launch_ms = launch_ms[top]
+        top_bytes = passes[top] * wl.ny * wl.nx * S
+        achieved = top_bytes / (top_launch_ms / 1e3) / 1e9
+        kname = {("adjoint", "fp32"): "kStoreF32", ("adjoint", "ckpt"): "kStoreF32",
+                 ("adjoint", "ckpt_ey"): "kStoreEy",
+                 ("adjoint", "bf16"): "kStoreBF16", ("adjoint", "fp8"): "kStoreFP8"}
+        kernel_name = (f"k_adjoint<{wl.order // 2}, {kname[(top, wl.snapshot)]}, 1>" if self.grad
+                       else f"k_forward<{wl.order // 2}, kStoreNone, 1>")
+        return dict(value=value, value_fwd=value_fwd, total_ms=total_ms, steps=steps,
+                    passes=passes, sweep_frac=sweep_frac, launch_ms=launch_ms, counts=counts,
+                    top=top, top_bytes=top_bytes, top_launch_ms=top_launch_ms, achieved=achieved,
+                    peak=peak, peak_kind=peak_kind, kernel_name=kernel_name, n_launch=n_launch,
+                    clocks=clk)
+
+    def e2e(self, steps):
+        """The same metric end to end through the public API with host
+        buffers: model, wavelet and observed data copied in, J and the
+        gradients (records for the records-only workload) copied out."""
+        torch, shard = self.torch, self.shard
+        prob, dev, wl, grad = self.prob, self.dev, self.wl, self.grad
+        pin = lambda a: torch.as_tensor(a).pin_memory()
+        f_p, eps_p, sig_p = pin(self.f_host), pin(self.eps_h), pin(self.sig_h)
+        dobs_p = self.d_obs.cpu().pin_memory()
+        outs = [torch.empty(1, dtype=torch.float64).pin_memory(),
+                torch.empty(self.gshape).pin_memory(), torch.empty(self.gshape).pin_memory()]
+        if not grad:  # records-only workload: the result is the records
+            outs = [torch.empty(1, dtype=torch.float64).pin_memory(),
+                    torch.empty(self.rec.shape).pin_memory()]
+
+        def e2e_step():
+            prob.set_model_eps_sigma(eps_p.to(dev, non_blocking=True),
+                                     sig_p.to(dev, non_blocking=True), f0=wl.f0)
+            fd = f_p.to(dev, non_blocking=True)
+            do = dobs_p.to(dev, non_blocking=True)
+            prob.forward(fd, rec=self.rec)
+            prob.residual(self.rec, do, res=self.res, J=self.J)
+            if grad:
+                self.gca_s.zero_()
+                self.gcb_s.zero_()
+                prob.adjoint(self.res, gca=self.gca_s, gcb=self.gcb_s)
+                prob.combine(self.gca_s, out=self.gca)
+                prob.combine(self.gcb_s, out=self.gcb)
+                shard.sum_over_ranks_(self.gca, self.gcb)
+            for o, src in zip(outs, (self.J, self.gca, self.gcb) if grad else (self.J, self.rec)):
+                o.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(self.stream)
+        for _ in range(steps):
+            e2e_step()
+        b.record(self.stream)
+        torch.cuda.synchronize()
+        e_ms = shard.max_over_ranks(a.elapsed_time(b), dev)
+        h2d = sum(x.numel() * x.element_size() for x in (f_p, eps_p, sig_p, dobs_p))
+        d2h = sum(x.numel() * x.element_size() for x in outs)
+        return {"value": round(self.cells * steps / (e_ms / 1e3) / 1e9, 4), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    def workspace_gb(self):
+        w = self.prob.workspace
+        return round(w.numel() * w.element_size() / 1e9, 1)
+
+    def close(self):
+        self.graph = None
+        self.prob = None
+        import gc
+        gc.collect()
+        self.torch.cuda.synchronize()
+        self.torch.cuda.empty_cache()
+
+
+def summary(m, wl, nt, ws_gb=None):
+    """Short record of one extra measurement (the default run's other
+    configurations)."""
+    d = {"workload": wl.name, "snapshots": snapshot_desc(wl), "nt": nt,
+         "value": round(m["value"], 4), "ms_per_step": round(m["total_ms"] / m["steps"], 3),
+         "steps": m["steps"], "hbm_frac_sweep": round(m["sweep_frac"], 4),
+         "sweep_bytes_per_cell": round(sweep_bytes_per_cell(wl, wl.n_shots, nt), 3),
+         "kernel": m["kernel_name"], "kernel_frac": round(m["achieved"] / m["peak"], 4),
+         "kernel_ms": {k: round(v, 4) for k, v in m["launch_ms"].items()}}
+    if ws_gb is not None:
+        d["workspace_gb"] = ws_gb
+    return d
+
+
+# The default run's extra measurements: (key, workload, overrides, steps,
+# warm-up, flush L2 between sweeps).  The strict reading of the headline
+# workload replays every segment from its checkpoint (no forward-stored tail),
+# with the E + curl pair and with E alone; workloads 1 and 2 fit in L2, so
+# their sweeps are timed one at a time with an L2 flush between them.
+EXTRAS = (
+    ("strict_pair", 4, dict(snapshot="ckpt", ckpt_tail=0), 2, 3, False),
+    ("strict_ey", 4, dict(snapshot="ckpt_ey", ckpt_tail=0), 2, 3, False),
+    ("workload1", 1, {}, 20, 5, True),
+    ("workload2", 2, {}, 10, 3, True),
+    ("workload3", 3, {}, 2, 3, False),
+    ("workload5", 5, {}, 2, 3, False),
+)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -313,7 +588,7 @@ def main():
     import torch
     import torch.distributed as dist
 
-    from adjoint_state_gradients_b200 import api, mwtm, shard, synth
+    from adjoint_state_gradients_b200 import synth
 
     rank, world, local = dist_env()
     if world != args.gpus:
@@ -337,203 +612,38 @@ def main():
     if args.nt and args.ckpt_tail is None and wl.ckpt_tail:
         # a shortened run keeps the tail's share of the steps
         wl = dataclasses.replace(wl, ckpt_tail=wl.ckpt_tail * nt // wl.nt)
+
+    sw = Sweep(args, number, wl, nt, rank, world, dev, use_graph=not args.no_graph)
+    wl = sw.wl
     S = wl.n_shots
-    grad = wl.snapshot != "none"   # workload 5 times the forward alone
-    # weak scaling: every rank simulates its own block of S shots of one
-    # survey of S * world shots (sources spread over the interior)
-    lo, hi = shard.shot_block(S * world, rank, world)
-    if number == 4:
-        inp = synth.make_inputs(number, n_shots=hi - lo, survey_shots=S * world, first_shot=lo)
-    else:  # the other workloads' shots are the same set on every rank
-        inp = synth.make_inputs(number)
-    c0 = 299792458.0
-    vmax = c0 / math.sqrt(inp.eps_min)
-    dt = wl.cfl_fraction * mwtm.cfl_dt(wl.order, wl.h, wl.h, vmax)
-    C = wl.ckpt_every
-
-    if wl.snapshot in CKPT_MODES and wl.ckpt_tail > 0:
-        # the tail trades spare HBM for replay work: shrink it to what is free
-        kw = dict(ny=wl.ny, nx=wl.nx, order=wl.order, n_shots=hi - lo if number == 4 else S,
-                  n_src=inp.src_idx.shape[1], n_rec=inp.rec_idx.shape[1], nt=nt, dt=dt, dy=wl.h,
-                  dx=wl.h, n_pml=wl.n_pml, snap_mode=mwtm.SNAP_MODES[wl.snapshot],
-                  ckpt_every=max(C, 1), vmax=vmax, model_batched=int(wl.batched))
-        # workspace = base + tail x step (the E-alone tail's extra final-E slot
-        # is in base)
-        w1 = mwtm.workspace_bytes(mwtm.make_params(ckpt_tail=1, **kw))
-        step_b = mwtm.workspace_bytes(mwtm.make_params(ckpt_tail=2, **kw)) - w1
-        free, _ = torch.cuda.mem_get_info(dev)
-        wl = dataclasses.replace(wl, ckpt_tail=fit_tail(wl.ckpt_tail, w1 - step_b, step_b, free,
-                                                        max(C, 1)))
-    prob = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
-                       vmax=vmax, snapshot=wl.snapshot, ckpt_every=max(C, 1), batched=wl.batched,
-                       ckpt_tail=wl.ckpt_tail if wl.snapshot in CKPT_MODES else 0)
-    f_host = inp.wavelet(dt, nt).astype(np.float32)
-    eps_h = inp.eps_r.astype(np.float32)
-    sig_h = inp.sigma.astype(np.float32)
-    # observed data from the perturbed model (setup, outside the timed region)
-    obs = api.Problem(wl.ny, wl.nx, wl.order, wl.h, wl.h, dt, nt, wl.n_pml, inp.src_idx, inp.rec_idx,
-                      vmax=vmax, snapshot="none", batched=wl.batched)
-    obs.set_model_eps_sigma(inp.eps_r_true.astype(np.float32), sig_h, f0=wl.f0)
-    f_dev = torch.as_tensor(f_host, device=dev)
-    d_obs = obs.forward(f_dev).clone()
-    del obs
-    torch.cuda.synchronize()
-    prob.set_model_eps_sigma(eps_h, sig_h, f0=wl.f0)
-    gshape = (wl.ny, wl.nx) if grad else (1,)
-    gca = torch.empty(gshape, device=dev)
-    gcb = torch.empty(gshape, device=dev)
-    gca_s = torch.empty((S, wl.ny, wl.nx) if grad else (1,), device=dev)
-    gcb_s = torch.empty((S, wl.ny, wl.nx) if grad else (1,), device=dev)
-    rec = torch.empty((nt, S, wl.n_rec), device=dev)
-    res = torch.empty_like(rec)
-    J = torch.zeros(1, dtype=torch.float64, device=dev)
-    stream = torch.cuda.current_stream()
-
-    # --graph: the sweep captured once as a CUDA graph and replayed (the
-    # per-kernel event pass below stays eager)
-    graph = api.SweepGraph(prob, f_dev, d_obs) if grad and not args.no_graph else None
-
-    def step(ev_fwd=None, eager=False):
-        if graph is not None and not eager:
-            graph.replay()
-            if ev_fwd is not None:  # no forward boundary inside a replay
-                ev_fwd.record(stream)
-            shard.sum_over_ranks_(graph.gca, graph.gcb)
-            return
-        prob.forward(f_dev, rec=rec)
-        if ev_fwd is not None:
-            ev_fwd.record(stream)
-        prob.residual(rec, d_obs, res=res, J=J)
-        if not grad:
-            return
-        gca_s.zero_()
-        gcb_s.zero_()
-        prob.adjoint(res, gca=gca_s, gcb=gcb_s)
-        prob.combine(gca_s, out=gca)
-        prob.combine(gcb_s, out=gcb)
-        shard.sum_over_ranks_(gca, gcb)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    rc = prob.status()
-    if rc != mwtm.MW_OK:
-        raise RuntimeError(f"device status {rc}: {mwtm.last_error()}")
-
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     if not uuid.startswith("GPU-"):
         uuid = "GPU-" + uuid
-    clocks = Clocks(uuid)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    # timed region: K steps, nothing recorded between the library's launches
-    mwtm.profile_enable(False)
-    n0 = mwtm.launch_count()
-    clocks.start()
-    ev0.record(stream)
-    for k in range(args.steps):
-        evs[k][0].record(stream)
-        step(ev_fwd=evs[k][1])
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    n_launch = mwtm.launch_count() - n0
-    if graph is not None:  # replays count no host launches: the graph's own
-        n_launch = graph.launches * args.steps
-    clk = clocks.stop()
-    if world > 1:
-        dist.barrier()
-    total_ms = ev0.elapsed_time(ev1)
-    # per-kernel durations for the roofline: the same K steps once more with
-    # CUDA events around every stencil launch on the launching stream (the
-    # events add a little time between kernels, so `value` comes from the pass
-    # above)
-    mwtm.profile_enable(True)
-    evs_e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
-    for k in range(args.steps):
-        evs_e[k][0].record(stream)
-        step(ev_fwd=evs_e[k][1], eager=True)
-    torch.cuda.synchronize()
-    counts, ms = mwtm.profile_read(3)
-    mwtm.profile_enable(False)
-    if world > 1:
-        dist.barrier()
-    # the forward alone: from the timed pass, or (graph replays have no
-    # forward boundary) from the eager pass with per-launch events
-    fwd_ms = sum(a.elapsed_time(b) for a, b in (evs if graph is None else evs_e))
-    total_ms = shard.max_over_ranks(total_ms, dev)
-    fwd_ms = shard.max_over_ranks(fwd_ms, dev)
-
-    cells = wl.ny * wl.nx * nt * S * world
-    state_mb = prob.p.n_shots * wl.ny * wl.nx * 12 / 1e6
-    value = cells * args.steps / (total_ms / 1e3) / 1e9
-    value_fwd = cells * args.steps / (fwd_ms / 1e3) / 1e9
-    passes = alg_bytes(wl, S)
-    classes = pass_classes(wl)
-    peak, peak_kind = measured_peaks()
-    sweep_bytes = sweep_bytes_per_cell(wl, S, nt) * cells * args.steps
-    sweep_frac = sweep_bytes / (total_ms / 1e3) / 1e9 / peak / world
-    launch_ms = {k: ms[c] / max(counts[c], 1) for k, c in classes.items()}
-    top = "adjoint" if grad else "forward"   # the dominant kernel
-    top_launch_ms = launch_ms[top]
-    top_bytes = passes[top] * wl.ny * wl.nx * S
-    achieved = top_bytes / (top_launch_ms / 1e3) / 1e9
-    kname = {("adjoint", "fp32"): "kStoreF32", ("adjoint", "ckpt"): "kStoreF32",
-             ("adjoint", "ckpt_ey"): "kStoreEy",
-             ("adjoint", "bf16"): "kStoreBF16", ("adjoint", "fp8"): "kStoreFP8"}
-    kernel_name = (f"k_adjoint<{wl.order // 2}, {kname[(top, wl.snapshot)]}, 1>" if grad
-                   else f"k_forward<{wl.order // 2}, kStoreNone, 1>")
+    m = sw.measure(args.steps, args.warmup, clocks=Clocks(uuid))
     # the recorded ncu traffic is that of the 8-shot order-4 adjoint launch
-    traffic = traffic_record(kernel_name) if number == WORKLOAD else None
+    traffic = traffic_record(m["kernel_name"]) if number == WORKLOAD else None
+    e2e = None if args.no_e2e else sw.e2e(args.steps)
+    ws_gb = sw.workspace_gb()
+    J = float(sw.J.cpu()[0])
+    graph_used = sw.graph is not None
+    state_mb = sw.prob.p.n_shots * wl.ny * wl.nx * 12 / 1e6
+    sw.close()
+    del sw
 
-    # ---- end to end through the public API with host buffers
-    e2e = None
-    if not args.no_e2e:
-        pin = lambda a: torch.as_tensor(a).pin_memory()
-        f_p, eps_p, sig_p = pin(f_host), pin(eps_h), pin(sig_h)
-        dobs_p = d_obs.cpu().pin_memory()
-        outs = [torch.empty(1, dtype=torch.float64).pin_memory(),
-                torch.empty(gshape).pin_memory(), torch.empty(gshape).pin_memory()]
-        if not grad:  # records-only workload: the result is the records
-            outs = [torch.empty(1, dtype=torch.float64).pin_memory(),
-                    torch.empty(rec.shape).pin_memory()]
-
-        def e2e_step():
-            prob.set_model_eps_sigma(eps_p.to(dev, non_blocking=True), sig_p.to(dev, non_blocking=True),
-                                     f0=wl.f0)
-            fd = f_p.to(dev, non_blocking=True)
-            do = dobs_p.to(dev, non_blocking=True)
-            prob.forward(fd, rec=rec)
-            prob.residual(rec, do, res=res, J=J)
-            if grad:
-                gca_s.zero_()
-                gcb_s.zero_()
-                prob.adjoint(res, gca=gca_s, gcb=gcb_s)
-                prob.combine(gca_s, out=gca)
-                prob.combine(gcb_s, out=gcb)
-                shard.sum_over_ranks_(gca, gcb)
-            for o, src in zip(outs, (J, gca, gcb) if grad else (J, rec)):
-                o.copy_(src, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e_ms = shard.max_over_ranks(a.elapsed_time(b), dev)
-        h2d = sum(x.numel() * x.element_size() for x in (f_p, eps_p, sig_p, dobs_p))
-        d2h = sum(x.numel() * x.element_size() for x in outs)
-        e2e = {"value": round(cells * args.steps / (e_ms / 1e3) / 1e9, 4), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    # the default run also times the other configurations (one GPU only)
+    extras = None
+    if world == 1 and number == WORKLOAD and not args.nt and not args.snapshot \
+            and args.ckpt_tail is None and not args.no_extras:
+        extras = {}
+        for key, num, over, k_steps, k_warm, flush in EXTRAS:
+            wk = dataclasses.replace(synth.WORKLOADS[num], **over)
+            if wk.snapshot in CKPT_MODES and wk.ckpt_every < 1:
+                wk = dataclasses.replace(wk, ckpt_every=64)
+            x = Sweep(args, num, wk, wk.nt, rank, world, dev, use_graph=not args.no_graph)
+            mx = x.measure(k_steps, k_warm, flush_l2=flush)
+            extras[key] = summary(mx, x.wl, wk.nt, x.workspace_gb())
+            x.close()
+            del x
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -545,42 +655,46 @@ def main():
         dist.barrier()
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3),
+            "metric": METRIC, "value": round(m["value"], 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(m["total_ms"] / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": {"workload": wl.name, "grid": [wl.ny, wl.nx], "interior": wl.n_interior,
                        "n_pml": wl.n_pml, "order": wl.order, "nt": nt, "shots_per_gpu": S,
                        "n_rec": wl.n_rec, "snapshots": snapshot_desc(wl),
-                       "workspace_gb": round(prob.workspace.numel() * prob.workspace.element_size()
-                                             / 1e9, 1),
+                       "workspace_gb": ws_gb,
                        "l2": ("inputs larger than L2 (one state buffer is "
                               f"{state_mb:.0f} MB)" if state_mb > 126 else
                               f"one state buffer ({state_mb:.1f} MB) fits in L2: no flush "
                               "(a small workload; the 126 MB rule holds for the headline)"),
-                       "execution": "one CUDA graph per sweep" if graph is not None
+                       "execution": "one CUDA graph per sweep" if graph_used
                                     else "stream launches",
                        "parallelism": f"shots sharded, {world} rank(s)"},
-            "value_fwd": round(value_fwd, 4),
-            "value_interior": round(value * (wl.n_interior ** 2) / (wl.ny * wl.nx), 4),
-            "hbm_frac_sweep": round(sweep_frac, 4),
-            "alg_bytes_per_cell": {k: round(v, 3) for k, v in passes.items()},
+            "value_fwd": round(m["value_fwd"], 4),
+            "value_interior": round(m["value"] * (wl.n_interior ** 2) / (wl.ny * wl.nx), 4),
+            "hbm_frac_sweep": round(m["sweep_frac"], 4),
+            "alg_bytes_per_cell": {k: round(v, 3) for k, v in m["passes"].items()},
             "sweep_bytes_per_cell": round(sweep_bytes_per_cell(wl, S, nt), 3),
-            "roofline": {"bound": "hbm", "kernel": kernel_name,
-                         "achieved": round(achieved, 1),
-                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4),
-                         "traffic": traffic, "alg_bytes_per_launch": top_bytes,
-                         "avg_launch_ms": round(top_launch_ms, 4),
+            "roofline": {"bound": "hbm", "kernel": m["kernel_name"],
+                         "achieved": round(m["achieved"], 1),
+                         "peak": m["peak"], "peak_kind": m["peak_kind"], "unit": "GB/s",
+                         "frac": round(m["achieved"] / m["peak"], 4),
+                         "traffic": traffic, "alg_bytes_per_launch": m["top_bytes"],
+                         "avg_launch_ms": round(m["top_launch_ms"], 4),
                          "timing": "CUDA events around every launch, second pass of the same K steps"},
-            "kernel_ms": {**{k: round(v, 4) for k, v in launch_ms.items()},
-                          "launches": [int(c) for c in counts]},
-            "gpu_launches": int(n_launch),
-            "J": float(J.cpu()[0]),
-            "clocks": clk,
+            "kernel_ms": {**{k: round(v, 4) for k, v in m["launch_ms"].items()},
+                          "launches": [int(c) for c in m["counts"]]},
+            "gpu_launches": int(m["n_launch"]),
+            "J": J,
+            "clocks": m["clocks"],
             "cpu_baseline": cpu,
             "e2e": e2e,
         }
+        if extras is not None:
+            line["value_strict"] = extras["strict_pair"]["value"]
+            line["value_strict_ey"] = extras["strict_ey"]["value"]
+            line["other_configs"] = extras
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

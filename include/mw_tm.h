@@ -210,13 +210,15 @@ int mw_tm_forward(const mw_params *p, const float *ca_dev, const float *cb_dev,
  *     memory; every GPU that loads the library holds that array until the
  *     process exits.  A problem needing more than that is rejected with
  *     MW_ERR_WORKSPACE before any work is queued;
- *   - the call waits for its work on `stream` to finish and returns the
- *     device status of this call (MW_ERR_ARG for an out-of-range index,
- *     MW_ERR_TIMEOUT, MW_ERR_NONFINITE with check_finite), so no
- *     mw_sync_status call is needed;
- *   - the first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before any
- *     stream capture;
+ *   - the call is synchronous: it waits for its work on `stream` to finish
+ *     (cudaStreamSynchronize) and reads back the device status of this call
+ *     (MW_ERR_ARG for an out-of-range index, MW_ERR_TIMEOUT,
+ *     MW_ERR_NONFINITE with check_finite), so no mw_sync_status call is
+ *     needed; the status words are cleared at the start of every call, so a
+ *     failed call leaves nothing behind for the next one;
+ *   - every call looks up the array's device address (cudaGetSymbolAddress)
+ *     with the calling thread's current device, so the address stays valid
+ *     after a context teardown such as cudaDeviceReset;
  *   - every call shares the one array: calls that overlap on the GPU (other
  *     threads, other streams) race and corrupt each other's results. */
 #define MW_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)

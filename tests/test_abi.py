@@ -50,6 +50,15 @@ def test_binding_constants_match_the_header():
     assert mwtm.SNAP_MODES == modes
 
 
+def test_binding_scratch_size_matches_the_header():
+    """The scratch-free forward's built-in scratch size: the binding's copy
+    is the header's MW_NOALLOC_SCRATCH_BYTES."""
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+MW_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", text)
+    assert m, "MW_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert mwtm.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
 def test_binding_covers_every_declared_symbol():
     bound = {name for name, _, _ in mwtm.SIGNATURES}
     missing = [n for n in declared_functions() if n not in bound]

@@ -338,14 +338,19 @@ def test_dot_product_state_map(order):
 
 
 def _misfit(sim, f, d_obs):
-    r = sim.forward(f)["rec"]
-    return 0.5 * float(np.sum((r - d_obs) ** 2))
+    """J = 1/2 ||d - d_obs||^2 as the oracle's residual routine returns it."""
+    return oracle.residual(sim.forward(f)["rec"], d_obs)[1]
 
 
 @pytest.mark.parametrize("order,n_pml", [(2, 3), (4, 3), (4, 0)])
 def test_model_gradient_matches_central_differences_16x16(order, n_pml):
     """dJ/dCa and dJ/dCb on every cell of a 16x16 grid (10x10 interior + 3-cell
-    CPML, and a no-PML variant), J = 1/2 ||d - d_obs||^2, two shots summed."""
+    CPML, and a no-PML variant), J = 1/2 ||d - d_obs||^2, two shots summed.
+
+    Both the misfit J the differences are taken of and the residual the
+    adjoint is driven by come from the oracle's residual routine, so a wrong
+    factor or sign in it (J without the 1/2, res = d_obs - d) breaks the
+    agreement."""
     n = 16
     sim, dt, (eps, sig, _) = small_sim(31 + order, n, n, 2, 1, 4, order, n_pml, sigma_max=0.02)
     nt = 80
@@ -353,7 +358,7 @@ def test_model_gradient_matches_central_differences_16x16(order, n_pml):
     g = synth.rng(5)
     d_obs = sim.forward(f)["rec"] * (1 + 0.1 * g.normal(size=(nt, 2, sim.n_rec)))
     fw = sim.forward(f, snapshots=True)
-    res = fw["rec"] - d_obs
+    res, _ = oracle.residual(fw["rec"], d_obs)
     adj = sim.adjoint(res, fw["snap_ey"], fw["snap_curl"])
     gca = oracle.combine(adj["gca"])
     gcb = oracle.combine(adj["gcb"])
@@ -565,6 +570,13 @@ def test_combine_is_fixed_order_shot_sum():
     out = oracle.combine(gs)
     ref = gs[0] + gs[1] + gs[2] + gs[3] + gs[4]
     assert np.array_equal(out, ref)
+
+
+def test_residual_worked_example():
+    """d = (3, 1, -2), d_obs = (1, 2, -2): residual (2, -1, 0), J = (4 + 1) / 2."""
+    res, J = oracle.residual(np.array([3.0, 1.0, -2.0]), np.array([1.0, 2.0, -2.0]))
+    assert list(res) == [2.0, -1.0, 0.0]
+    assert J == 2.5
 
 
 def test_residual_and_misfit():

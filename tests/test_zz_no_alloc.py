@@ -3,7 +3,10 @@ allocate device memory: it keeps its scratch in an array the library defines
 in device memory instead of a caller-provided workspace.  Called through the
 C ABI twice in a row, it must reproduce the workspace forward (mw_tm_forward)
 within the records tolerance, and a problem too large for its scratch must be
-refused before any work runs.  Collected last on purpose; runs alone too.
+refused before any work runs.  It reports the device status of its own call:
+an out-of-range receiver index (which the kernels flag and skip, never
+access) gives MW_ERR_ARG, and the next valid call starts from clean status
+words and returns MW_OK.  Collected last on purpose; runs alone too.
 """
 from __future__ import annotations
 
@@ -54,3 +57,27 @@ def test_noalloc_forward_refuses_a_problem_larger_than_its_scratch():
     rc = mwtm.tm_forward_noalloc(p, dummy, dummy, dummy, dummy, None, idx, idx, dummy, None)
     assert rc == mwtm.MW_ERR_WORKSPACE
     assert "built-in scratch" in mwtm.last_error()
+
+
+def test_noalloc_forward_reports_its_own_status_and_clears_it():
+    n_pml, nt = 8, 40
+    sim, dt, _ = small_sim(919, 64, 96, 1, 1, 4, 4, n_pml, round_f32=True)
+    g = synth.rng(19)
+    f = f32(g.normal(size=(nt, 1, 1)))
+    prob = problem_from_sim(sim, nt, dt, n_pml, snapshot="none")
+    rec_ref = run_forward(prob, f)
+    f_dev = torch.as_tensor(np.asarray(f, dtype=np.float32)).cuda()
+    bad_idx = prob.rec_idx.clone()
+    bad_idx[0, 2] = sim.ny * sim.nx + 5  # one receiver past the last cell
+    state = prob.new_state()
+    rec = torch.zeros((nt, 1, 4), device="cuda")
+    rc = mwtm.tm_forward_noalloc(prob.p, prob.ca, prob.cb, prob.cq, prob.cpml, f_dev,
+                                 prob.src_idx, bad_idx, state, rec)
+    assert rc == mwtm.MW_ERR_ARG
+    assert "out of range" in mwtm.last_error()
+    state = prob.new_state()
+    rec = torch.zeros((nt, 1, 4), device="cuda")
+    rc = mwtm.tm_forward_noalloc(prob.p, prob.ca, prob.cb, prob.cq, prob.cpml, f_dev,
+                                 prob.src_idx, prob.rec_idx, state, rec)
+    assert rc == mwtm.MW_OK, mwtm.last_error()
+    assert rel_l2(rec.cpu().numpy().astype(np.float64), rec_ref) <= REC_TOL
