@@ -1,6 +1,7 @@
-// Small kernels of the mw_tm library: source injection / receiver sampling
-// and their transposes, model coefficients, CPML profiles, shot reduction,
-// epsilon / sigma chain rule, residual and misfit, non-finite scan.
+// Small kernels of the mw_tm library: the sorted source / receiver tables the
+// stencil kernels inject and sample from, model coefficients, CPML profiles,
+// shot reduction, epsilon / sigma chain rule, residual and misfit, non-finite
+// scan, the summation-by-parts end terms.
 //
 // Method: page "tide-GPR 0.0.9 ... tide/csrc/maxwell.cu" -- add_sources_ey,
 // record_receivers_ey, add_adjoint_sources_ey, record_adjoint_at_sources,
@@ -16,68 +17,123 @@ namespace {
 constexpr double kEps0 = 8.8541878128e-12;  // F/m (the page's EP0)
 constexpr double kMu0 = 1.25663706212e-6;   // H/m (CODATA 2018)
 
-// Duplicate chains of a per-shot index list idx [S][n] (one block per shot):
-// lead[k] = 1 when k is the first entry with its cell, next[k] = the next
-// entry with the same cell (-1 at the end of the chain).  Inactive (-1)
-// entries are never leaders; out-of-range entries set a status flag.
-__global__ void k_dup_chains(const int64_t *__restrict__ idx, int n, int64_t numel,
-                             int *__restrict__ lead, int *__restrict__ next,
-                             int *__restrict__ flags) {
+// Entry table of one shot's index list v[0..n) (one block per shot; the
+// EntrySet layout).  Pass 1 ranks every valid entry by (cell, k) and places
+// it; pass 2 marks the runs of equal cells and the distinct rows.  Invalid
+// entries (-1, or out of range, which also sets the bad-index flag) get no
+// place; with `out` their outputs out[t][s][k] are zeroed for every step.
+// O(n^2 / blockDim) per shot, once per call.
+__global__ void k_entry_table(const int64_t *__restrict__ idx, int n, int nx, int64_t numel,
+                              int4 *__restrict__ ent_all, int *__restrict__ arow_all,
+                              int *__restrict__ abeg_all, int *__restrict__ flags,
+                              float *__restrict__ out, int nt, int S) {
   const int s = blockIdx.x;
   const int64_t *v = idx + (int64_t)s * n;
+  int4 *ent = ent_all + (int64_t)s * n;
+  int *arow = arow_all + (int64_t)s * (n + 1);
+  int *abeg = abeg_all + (int64_t)s * (n + 1);
+  __shared__ int s_nv, s_nact;
+  if (threadIdx.x == 0) s_nv = 0;
+  __syncthreads();
   for (int k = threadIdx.x; k < n; k += blockDim.x) {
     const int64_t c = v[k];
     const bool ok = c >= 0 && c < numel;
-    if (!ok && c != -1 && flags) atomicOr(flags + kFlagBadIndex, 1);
-    int first = ok ? 1 : 0, nx = -1;
-    for (int j = 0; j < n && ok; ++j) {
-      if (v[j] != c) continue;
-      if (j < k) first = 0;
-      if (j > k) {
-        nx = j;
-        break;
-      }
+    if (!ok) {
+      if (c != -1 && flags) atomicOr(flags + kFlagBadIndex, 1);
+      if (out)
+        for (int t = 0; t < nt; ++t) out[((int64_t)t * S + s) * n + k] = 0.f;
+      continue;
     }
-    lead[(int64_t)s * n + k] = first;
-    next[(int64_t)s * n + k] = nx;
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const int64_t cj = v[j];
+      if (cj >= 0 && cj < numel && (cj < c || (cj == c && j < k))) ++rank;
+    }
+    ent[rank] = make_int4((int)(c / nx), (int)(c % nx), k, 0);
+    atomicAdd(&s_nv, 1);
+  }
+  __syncthreads();
+  const int nv = s_nv;
+  // runs of equal cells and the distinct rows; only the (row, column) half of
+  // an entry is read here, only its run half is written
+  const int2 *rc = reinterpret_cast<const int2 *>(ent);
+  for (int j = threadIdx.x; j < nv; j += blockDim.x) {
+    const int2 e = rc[2 * j];
+    int len = 0;
+    if (j == 0 || rc[2 * (j - 1)].x != e.x || rc[2 * (j - 1)].y != e.y) {
+      len = 1;
+      while (j + len < nv && rc[2 * (j + len)].x == e.x && rc[2 * (j + len)].y == e.y) ++len;
+    }
+    ent[j].w = len;
+    if (j > 0 && rc[2 * (j - 1)].x == e.x) continue;
+    int a = 0;  // the a-th row start: the number of row starts before j
+    for (int i = 1; i <= j; ++i) a += rc[2 * i].x != rc[2 * (i - 1)].x;
+    arow[a] = e.x;
+    abeg[a] = j;
+  }
+  if (threadIdx.x == 0) {
+    int na = 0;
+    for (int j = 0; j < nv; ++j) na += (j == 0 || rc[2 * j].x != rc[2 * (j - 1)].x);
+    s_nact = na;
+  }
+  __syncthreads();
+  for (int a = s_nact + threadIdx.x; a <= n; a += blockDim.x) {
+    arow[a] = 0x7fffffff;
+    abeg[a] = nv;
   }
 }
 
-// One block per shot: add vals_t[s][k] into field cells idx_a[s][k] -- each
-// chain leader sums its duplicates in index order, so the result does not
-// depend on scheduling -- then sample the field at idx_b into out_t
-// (inactive or out-of-range entries give 0).  Forward: sources then
-// receivers; adjoint: receiver residuals then the source gradient.
-__global__ void k_inject_sample(float *__restrict__ field, int64_t numel,
-                                const float *__restrict__ vals_t, const int64_t *__restrict__ idx_a,
-                                const int *__restrict__ lead, const int *__restrict__ next, int na,
-                                const int64_t *__restrict__ idx_b, int nb,
-                                float *__restrict__ out_t, const SbpTerms sbp) {
+// Fix-ups of a whole E field [S][ny][nx] (one block per shot): add vals[s][k]
+// at the entries of set `ea` (one thread per cell, duplicates added up in
+// index order first), then read the field at the entries of set `eb` into
+// out[s][k].  The stencil kernels make the same fix-ups row by row.
+__global__ void k_fix_field(float *__restrict__ field, int64_t numel, int nx, EntrySet ea,
+                            const float *__restrict__ vals, EntrySet eb, float *__restrict__ out) {
   const int s = blockIdx.x;
   float *e = field + (int64_t)s * numel;
   // programmatic dependent launch (no-ops without the launch attribute):
   // let the next stencil launch begin, then wait for the previous one
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (vals_t != nullptr) {
-    const int64_t base = (int64_t)s * na;
-    for (int k = threadIdx.x; k < na; k += blockDim.x) {
-      if (sbp.acc_a != nullptr) sbp.acc_a[base + k] += vals_t[base + k] * sbp.pair_t[base + k];
-      if (!lead[base + k]) continue;
-      float v = vals_t[base + k];
-      for (int j = next[base + k]; j >= 0; j = next[base + j]) v += vals_t[base + j];
-      e[idx_a[base + k]] += v;
+  if (vals != nullptr && ea.n > 0) {
+    const int nv = ea.abeg[(int64_t)s * (ea.n + 1) + ea.n];
+    const int4 *en = ea.ent + (int64_t)s * ea.n;
+    const float *vs = vals + (int64_t)s * ea.n;
+    for (int j = threadIdx.x; j < nv; j += blockDim.x) {
+      const int4 q = en[j];
+      if (q.w == 0) continue;
+      float v = vs[q.z];
+      for (int u = 1; u < q.w; ++u) v += vs[en[j + u].z];
+      e[(int64_t)q.x * nx + q.y] += v;
     }
   }
   __syncthreads();
-  if (out_t != nullptr) {
-    for (int k = threadIdx.x; k < nb; k += blockDim.x) {
-      const int64_t j = (int64_t)s * nb + k;
-      const int64_t i = idx_b[j];
-      const float v = (i >= 0 && i < numel) ? e[i] : 0.f;
-      out_t[j] = v;
-      if (sbp.acc_b != nullptr) sbp.acc_b[j] += sbp.w_t[j] * v;
+  if (out != nullptr && eb.n > 0) {
+    const int nv = eb.abeg[(int64_t)s * (eb.n + 1) + eb.n];
+    const int4 *en = eb.ent + (int64_t)s * eb.n;
+    for (int j = threadIdx.x; j < nv; j += blockDim.x) {
+      const int4 q = en[j];
+      out[(int64_t)s * eb.n + q.z] = e[(int64_t)q.x * nx + q.y];
     }
+  }
+}
+
+// One thread per (shot, entry): the end-term sums in the adjoint's order.
+__global__ void k_sbp_sums(int nt, int S, const float *__restrict__ res,
+                           const float *__restrict__ rec, int n_rec, float *__restrict__ acc_rec,
+                           const float *__restrict__ f, const float *__restrict__ lam, int n_src,
+                           float *__restrict__ acc_src) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nr = res ? S * n_rec : 0, ns = f ? S * n_src : 0;
+  if (i < nr) {
+    float acc = 0.f;
+    for (int t = nt - 1; t >= 0; --t) acc += res[(int64_t)t * nr + i] * rec[(int64_t)t * nr + i];
+    acc_rec[i] = acc;
+  } else if (i < nr + ns) {
+    const int j = i - nr;
+    float acc = 0.f;
+    for (int t = nt - 1; t >= 0; --t) acc += f[(int64_t)t * ns + j] * lam[(int64_t)t * ns + j];
+    acc_src[j] = acc;
   }
 }
 
@@ -270,26 +326,54 @@ int grid_for(int64_t n, int block) {
 
 }  // namespace
 
-cudaError_t launch_dup_chains(const int64_t *idx, int S, int n, int64_t numel, int *lead,
-                              int *next, int *flags, cudaStream_t st) {
+size_t entry_table_bytes(int S, int n) {
+  if (n <= 0) return 0;
+  const size_t e = (size_t)S * n * sizeof(int4);
+  const size_t r = (size_t)S * (n + 1) * sizeof(int);
+  return ((e + 255) & ~(size_t)255) + 2 * ((r + 255) & ~(size_t)255);
+}
+
+EntrySet entry_set_at(void *base, int S, int n) {
+  EntrySet es{nullptr, nullptr, nullptr, 0};
+  if (n <= 0 || base == nullptr) return es;
+  char *b = (char *)base;
+  const size_t e = (((size_t)S * n * sizeof(int4)) + 255) & ~(size_t)255;
+  const size_t r = (((size_t)S * (n + 1) * sizeof(int)) + 255) & ~(size_t)255;
+  es.ent = (const int4 *)b;
+  es.arow = (const int *)(b + e);
+  es.abeg = (const int *)(b + e + r);
+  es.n = n;
+  return es;
+}
+
+cudaError_t launch_entry_table(const int64_t *idx, int S, int n, int ny, int nx, void *base,
+                               int *flags, float *out, int nt, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  k_dup_chains<<<S, 256, 0, st>>>(idx, n, numel, lead, next, flags);
+  const EntrySet es = entry_set_at(base, S, n);
+  k_entry_table<<<S, 256, 0, st>>>(idx, n, nx, (int64_t)ny * nx, const_cast<int4 *>(es.ent),
+                                   const_cast<int *>(es.arow), const_cast<int *>(es.abeg), flags,
+                                   out, nt, S);
   count_launches(1);
   return cudaGetLastError();
 }
 
-cudaError_t launch_inject_sample(float *field, int64_t numel, int S, const float *vals_t,
-                                 const int64_t *idx_a, const int *lead, const int *next, int na,
-                                 const int64_t *idx_b, int nb, float *out_t, cudaStream_t st,
-                                 const SbpTerms &sbp) {
-  if ((na == 0 || vals_t == nullptr) && (nb == 0 || out_t == nullptr)) return cudaSuccess;
-  SbpTerms t = sbp;
-  if (na == 0 || vals_t == nullptr || t.pair_t == nullptr) t.acc_a = nullptr;
-  if (nb == 0 || out_t == nullptr || t.w_t == nullptr) t.acc_b = nullptr;
-  const cudaError_t e = launch_dependent(k_inject_sample, S, 256, 0, st, field, numel,
-                                         na > 0 ? vals_t : nullptr, idx_a, lead, next, na, idx_b,
-                                         nb, nb > 0 ? out_t : nullptr, t);
+cudaError_t launch_fix_field(float *field, int S, int ny, int nx, const EntrySet &ea,
+                             const float *vals, const EntrySet &eb, float *out, cudaStream_t st) {
+  if ((vals == nullptr || ea.n == 0) && (out == nullptr || eb.n == 0)) return cudaSuccess;
+  const cudaError_t e = launch_dependent(k_fix_field, S, 128, 0, st, field, (int64_t)ny * nx, nx,
+                                         ea, vals, eb, out);
   if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sbp_sums(int nt, int S, const float *res, const float *rec, int n_rec,
+                            float *acc_rec, const float *f, const float *lam, int n_src,
+                            float *acc_src, cudaStream_t st) {
+  const int n = (res ? S * n_rec : 0) + (f ? S * n_src : 0);
+  if (n <= 0) return cudaSuccess;
+  k_sbp_sums<<<(n + 127) / 128, 128, 0, st>>>(nt, S, res, rec, n_rec, acc_rec, f, lam, n_src,
+                                              acc_src);
   count_launches(1);
   return cudaGetLastError();
 }

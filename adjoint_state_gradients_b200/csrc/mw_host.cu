@@ -148,8 +148,8 @@ Layout layout(const mw_params *p) {
   const size_t sb = align256(L.state_bytes);
   size_t off = 0;
   L.flags = off; off += 256;
-  L.chains = off;
-  off += align256(2 * sizeof(int) * (size_t)p->n_shots * (p->n_src + p->n_rec));
+  L.tab_src = off; off += entry_table_bytes(p->n_shots, p->n_src);
+  L.tab_rec = off; off += entry_table_bytes(p->n_shots, p->n_rec);
   L.bandtab = off;
   {
     const Bands b = bands(p);
@@ -195,14 +195,17 @@ Layout layout(const mw_params *p) {
       off += align256(slots * L.snap_step_bytes);
     }
   }
-  L.sbp = L.rcopy = L.acc = 0;
+  L.sbp = L.rcopy = L.acc = L.gfbuf = 0;
   if (p->snap_mode == MW_SNAP_CKPT_EY) {
     L.sbp = off; off += align256(SN * sizeof(float));
     L.rcopy = off; off += align256((size_t)p->nt * p->n_shots * p->n_rec * sizeof(float));
-    // the receiver and source sums, then lambda_E sampled at the sources
-    // when the caller asks for no grad_f
+    // the receiver and source sums
     L.acc = off;
-    off += align256((size_t)p->n_shots * (p->n_rec + 2 * (size_t)p->n_src) * sizeof(float));
+    off += align256((size_t)p->n_shots * (p->n_rec + (size_t)p->n_src) * sizeof(float));
+    // lambda_E sampled at the sources every step, when the caller asks for
+    // no grad_f (the source end term needs it)
+    L.gfbuf = off;
+    off += align256((size_t)p->nt * p->n_shots * p->n_src * sizeof(float));
   }
   L.total = off;
   return L;
@@ -268,14 +271,21 @@ struct HostCopies {
   }
 };
 
-// Duplicate-chain arrays (lead, next) of the sources and receivers.
-struct Chains {
-  int *src_lead, *src_next, *rec_lead, *rec_next;
+// Entry tables of the sources and the receivers (built per call).
+struct Tables {
+  EntrySet src, rec;
 };
-Chains chains_at(const mw_params *p, char *ws, const Layout &L) {
-  int *c = (int *)(ws + L.chains);
-  const size_t ns = (size_t)p->n_shots * p->n_src, nr = (size_t)p->n_shots * p->n_rec;
-  return Chains{c, c + ns, c + 2 * ns, c + 2 * ns + nr};
+Tables tables_at(const mw_params *p, char *ws, const Layout &L) {
+  return Tables{entry_set_at(ws + L.tab_src, p->n_shots, p->n_src),
+                entry_set_at(ws + L.tab_rec, p->n_shots, p->n_rec)};
+}
+// Build the table of one index set (n > 0); `out` [nt][S][n] gets zeros at
+// the invalid entries.
+int build_table(const mw_params *p, const int64_t *idx, int n, char *ws, size_t off, int *flags,
+                float *out, cudaStream_t st) {
+  if (n <= 0) return MW_OK;
+  MW_CUDA(launch_entry_table(idx, p->n_shots, n, p->ny, p->nx, ws + off, flags, out, p->nt, st));
+  return MW_OK;
 }
 
 // ---- launch geometry ------------------------------------------------------
@@ -735,8 +745,7 @@ struct Replay {
   Layout L{};
   cudaStream_t st = nullptr;
   const float *f = nullptr;
-  const int64_t *src_idx = nullptr;
-  Chains ch{};
+  EntrySet src{};
   Launch lf{};
   StepArgs fa{};
   FwdMaps fA, fB, fS;  // inputs rA, rB, the segment's checkpoint
@@ -747,17 +756,17 @@ struct Replay {
 
   int init(const mw_params *p_, char *ws_, const Layout &L_, cudaStream_t st_, const float *ca,
            const float *cb, const float *cq, int *flags, const float *f_,
-           const int64_t *src_idx_, const Chains &ch_) {
+           const EntrySet &src_) {
     p = p_;
     ws = ws_;
     L = L_;
     st = st_;
     f = f_;
-    src_idx = src_idx_;
-    ch = ch_;
+    src = src_;
     lf = plan(p, false);
     fa = step_args(p, lf, ca, cb, cq, flags, ws, L);
     set_layout(fa, p, false);
+    fa.ea = src;  // sources injected, nothing recorded
     fa.snap_pitch = p->nx;  // the fp32 segment
     rA = (float *)(ws + L.rpA);
     rB = (float *)(ws + L.rpB);
@@ -773,7 +782,6 @@ struct Replay {
     const int C = p->ckpt_every;
     const int t0 = k * C;
     const int t1 = (t0 + C < t_end) ? t0 + C : t_end;
-    const int64_t numel = (int64_t)p->ny * p->nx;
     char *seg_e = ws + L.seg;
     char *seg_c = seg_e + (size_t)C * L.snap_step_bytes;
     // the first step reads the checkpoint in place
@@ -786,14 +794,12 @@ struct Replay {
       fa.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
       fa.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
       fa.ctr_slot = ((*launch_idx)++) & 1;
+      fa.vals_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
       const FwdMaps &fm = rc == rA ? fA : rc == rB ? fB : fS;
       MW_CUDA(timed(1, st, [&] {
         return launch_forward(fm, fa, p->order, store, kStoreNone, p->model_batched != 0,
                               !p->cq_is_scalar, lf.grid, st);
       }));
-      MW_CUDA(launch_inject_sample(rn, numel, p->n_shots,
-                                   f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
-                                   ch.src_lead, ch.src_next, p->n_src, nullptr, 0, nullptr, st));
       rc = rn;
     }
     last = rc;
@@ -951,15 +957,12 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   char *tail_e = ws + L.tail;
   char *tail_c = tail_e + (size_t)L.n_tail * L.snap_step_bytes;
   const int64_t SN = (int64_t)p->n_shots * p->ny * p->nx;
-  const int64_t numel = (int64_t)p->ny * p->nx;
-  const Chains ch = chains_at(p, ws, L);
-  if (p->n_src > 0)
-    MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
-                              flags, st));
+  const Tables tb = tables_at(p, ws, L);
   float *rec_out = ey_only ? (float *)(ws + L.rcopy) : rec;
-  if (p->n_rec > 0 && rec_out)  // chains unused here: this validates the receiver indices
-    MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
-                              flags, st));
+  MW_TRY(build_table(p, src_idx, p->n_src, ws, L.tab_src, flags, nullptr, st));
+  if (rec_out) MW_TRY(build_table(p, rec_idx, p->n_rec, ws, L.tab_rec, flags, rec_out, st));
+  a.ea = tb.src;
+  if (rec_out) a.eb = tb.rec;
   const bool host = p->snap_host != 0;
   const size_t ring_steps = host ? (size_t)kHostRing : (size_t)p->nt;
   char *snap_e = ws + L.snap;
@@ -994,6 +997,8 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
     if (cur != bufA && cur != bufB) MW_TRY(fwd_maps(p, a.in, ca, cb, cq, &mS));
     const FwdMaps &m = cur == bufA ? mA : cur == bufB ? mB : mS;
     a.ctr_slot = t & 1;
+    a.vals_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
+    a.out_t = rec_out ? rec_out + (int64_t)t * p->n_shots * p->n_rec : nullptr;
     MW_CUDA(timed(kind ? 1 : 0, st, [&] {
       return launch_forward(m, a, p->order, kind, kStoreNone, p->model_batched != 0, !p->cq_is_scalar,
                             lc.grid, st);
@@ -1007,11 +1012,6 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
                               cudaMemcpyDeviceToHost, hc.cs));
       MW_CUDA(cudaEventRecord(hc.freed[slot], hc.cs));
     }
-    MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots,
-                                 f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
-                                 ch.src_lead, ch.src_next, p->n_src, rec_idx, p->n_rec,
-                                 rec_out ? rec_out + (int64_t)t * p->n_shots * p->n_rec : nullptr,
-                                 st));
     cur = nxt;
   }
   if (ey_only && rec && p->n_rec > 0)
@@ -1060,13 +1060,15 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   const int64_t numel = (int64_t)p->ny * p->nx;
   const int64_t SN = p->n_shots * numel;
 
-  const Chains ch = chains_at(p, ws, L);
-  if (p->n_rec > 0)
-    MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
-                              flags, st));
-  if (p->n_src > 0 && is_ckpt(p))
-    MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
-                              flags, st));
+  // MW_SNAP_CKPT_EY: lambda_E at the sources of every step (the source end
+  // term), in grad_f or in the workspace
+  const bool ey_only = p->snap_mode == MW_SNAP_CKPT_EY;
+  float *gf_all = grad_f ? grad_f : ey_only ? (float *)(ws + L.gfbuf) : nullptr;
+  const Tables tb = tables_at(p, ws, L);
+  MW_TRY(build_table(p, rec_idx, p->n_rec, ws, L.tab_rec, flags, nullptr, st));
+  // the sources: sampled (grad_f, the end term) and injected by the replay
+  if (src_idx && (gf_all || is_ckpt(p)))
+    MW_TRY(build_table(p, src_idx, p->n_src, ws, L.tab_src, flags, gf_all, st));
   float *adA = adj_state ? adj_state : (float *)(ws + L.adA);
   float *adB = (float *)(ws + L.adB);
   if (!adj_state) MW_CUDA(cudaMemsetAsync(adA, 0, L.state_bytes, st));
@@ -1075,17 +1077,11 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   const Launch la = plan(p, true);
   // MW_SNAP_CKPT_EY: the Cb gradient accumulates E^t G^t into P (workspace)
   // and the end-term sums beside it; grad_cb_shot receives P / Cb at the end
-  const bool ey_only = p->snap_mode == MW_SNAP_CKPT_EY;
   float *sbp = ey_only ? (float *)(ws + L.sbp) : nullptr;
   float *acc_rec = ey_only ? (float *)(ws + L.acc) : nullptr;
   float *acc_src = ey_only ? acc_rec + (size_t)p->n_shots * p->n_rec : nullptr;
   const float *rcopy = ey_only ? (const float *)(ws + L.rcopy) : nullptr;
-  if (ey_only) {
-    MW_CUDA(cudaMemsetAsync(sbp, 0, SN * sizeof(float), st));
-    if (p->n_rec + p->n_src > 0)
-      MW_CUDA(cudaMemsetAsync(acc_rec, 0,
-                              (size_t)p->n_shots * (p->n_rec + p->n_src) * sizeof(float), st));
-  }
+  if (ey_only) MW_CUDA(cudaMemsetAsync(sbp, 0, SN * sizeof(float), st));
   StepArgs a = step_args(p, la, ca, cb, cq, flags, ws, L);
   a.gca = gca;
   a.gcb = ey_only ? sbp : gcb;
@@ -1120,22 +1116,19 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   }
 
   float *cur = adA, *nxt = adB;
-  // with the summation-by-parts Cb gradient the source term needs lambda_E at
-  // the sources every step, grad_f or not: sampled into the end of acc
-  float *gf_scratch = ey_only && !grad_f ? acc_src + (size_t)p->n_shots * p->n_src : nullptr;
+  a.ea = tb.rec;  // residuals injected
+  if (gf_all && src_idx) a.eb = tb.src;  // lambda_E sampled at the sources
+  const bool sample_src = gf_all && src_idx;
   auto adj_step = [&](int t, int slot) -> int {
-    SbpTerms sb;
-    float *gf_t = grad_f ? grad_f + (int64_t)t * p->n_shots * p->n_src : gf_scratch;
-    if (ey_only) {
-      sb.pair_t = rcopy + (int64_t)t * p->n_shots * p->n_rec;
-      sb.acc_a = acc_rec;
-      sb.w_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
-      sb.acc_b = acc_src;
-    }
-    MW_CUDA(launch_inject_sample(cur, numel, p->n_shots,
-                                 res ? res + (int64_t)t * p->n_shots * p->n_rec : nullptr,
-                                 rec_idx, ch.rec_lead, ch.rec_next, p->n_rec, src_idx, p->n_src,
-                                 gf_t, st, sb));
+    // step t's residuals and source gradient: the step t + 1 launch applies
+    // them to its output (the first step applies its own to the start state)
+    if (t == p->nt - 1)
+      MW_CUDA(launch_fix_field(cur, p->n_shots, p->ny, p->nx, tb.rec,
+                               res ? res + (int64_t)t * p->n_shots * p->n_rec : nullptr, tb.src,
+                               sample_src ? gf_all + (int64_t)t * p->n_shots * p->n_src : nullptr,
+                               st));
+    a.vals_t = res && t > 0 ? res + (int64_t)(t - 1) * p->n_shots * p->n_rec : nullptr;
+    a.out_t = sample_src && t > 0 ? gf_all + (int64_t)(t - 1) * p->n_shots * p->n_src : nullptr;
     a.in = fields_at(p, cur);
     a.out = fields_at(p, nxt);
     a.snap_t = slot;
@@ -1175,7 +1168,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     // checkpoint; a given adjoint start state meets the forward's final E:
     // P starts at lambda~_E^{nt} E^{nt}
     Replay rp;
-    MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, src_idx, ch));
+    MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, tb.src));
     rp.store = ey_only ? kStoreEy : kStoreF32;
     if (L.n_tail > 0) {
       if (ey_only && adj_state)
@@ -1195,8 +1188,10 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   }
   if (cur != adA) MW_CUDA(cudaMemcpyAsync(adA, cur, L.state_bytes, cudaMemcpyDeviceToDevice, st));
   if (ey_only) {
+    MW_CUDA(launch_sbp_sums(p->nt, p->n_shots, res, rcopy, p->n_rec, acc_rec,
+                            src_idx ? f : nullptr, gf_all, p->n_src, acc_src, st));
     MW_CUDA(launch_sbp_scatter(sbp, numel, p->n_shots, rec_idx, acc_rec, res ? p->n_rec : 0,
-                               src_idx, acc_src, f ? p->n_src : 0, st));
+                               src_idx, acc_src, f && src_idx ? p->n_src : 0, st));
     MW_CUDA(launch_sbp_finish(sbp, cb, gcb, p->n_shots, p->ny, p->nx, p->model_batched,
                               p->grad_mask_pml ? p->n_pml : 0, st));
   }
@@ -1234,14 +1229,9 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
   cudaStream_t st = (cudaStream_t)stream;
   char *ws = (char *)workspace;
   int *flags = (int *)(ws + L.flags);
-  const int64_t numel = (int64_t)p->ny * p->nx;
-  const Chains ch = chains_at(p, ws, L);
-  if (p->n_rec > 0)  // validates the receiver indices
-    MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
-                              flags, st));
-  if (ckpt && p->n_src > 0)
-    MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
-                              flags, st));
+  const Tables tb = tables_at(p, ws, L);
+  MW_TRY(build_table(p, rec_idx, p->n_rec, ws, L.tab_rec, flags, rec, st));
+  if (ckpt) MW_TRY(build_table(p, src_idx, p->n_src, ws, L.tab_src, flags, nullptr, st));
   if (p->nt == 0) return MW_OK;
 
   // the perturbation state lives in the adjoint's buffers, from zero
@@ -1258,6 +1248,7 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
     b.bd_pair = bd.pair ? 1 : 0;
     b.bd_swap = bd.swap ? 1 : 0;
   }
+  b.eb = tb.rec;  // the perturbation's records; no sources
   MW_TRY(stencil_prologue(p, cpml, ws, L, st));
 
   // the background's snapshots: every step in the workspace, a 3-step ring
@@ -1281,14 +1272,12 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
     b.out = fields_at(p, nxt);
     b.snap_t = slot;
     b.ctr_slot = (launch_idx++) & 1;
+    b.out_t = rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr;
     const FwdMaps &m = cur == dA ? mA : mB;
     MW_CUDA(timed(3, st, [&] {
       return launch_forward(m, b, p->order, kStoreNone, kind, p->model_batched != 0,
                             !p->cq_is_scalar, lc.grid, st);
     }));
-    MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots, nullptr, nullptr, nullptr, nullptr, 0,
-                                 rec_idx, p->n_rec,
-                                 rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, st));
     std::swap(cur, nxt);
     return MW_OK;
   };
@@ -1313,7 +1302,7 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
     // replay each segment of the background from its checkpoint into the fp32
     // segment buffer, then take the segment's linearised steps
     Replay rp;
-    MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, src_idx, ch));
+    MW_TRY(rp.init(p, ws, L, st, ca, cb, cq, flags, f, tb.src));
     for (int k = 0; k < L.n_seg; ++k) {
       int t0, t1;
       MW_TRY(rp.segment(k, &launch_idx, &t0, &t1, p->nt));
@@ -1430,8 +1419,8 @@ int mw_profile_read(int64_t *counts, double *total_ms, int32_t n_classes) {
 }
 
 // ---- forward without allocations -------------------------------------------
-// The scratch of mw_tm_forward_noalloc: status words | duplicate chains | CPML
-// band table | the second state buffer of the ping-pong.  Host code must not
+// The scratch of mw_tm_forward_noalloc: status words | source and receiver
+// tables | CPML band table | the second state buffer of the ping-pong.  Host code must not
 // use the symbol itself (it is a host-side stand-in); it takes the device
 // address from cudaGetSymbolAddress with the calling device current.
 }  // extern "C"
@@ -1477,8 +1466,9 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
   const Bands bd = bands(p);
   Layout L{};
   L.flags = 0;
-  L.chains = 256;
-  L.bandtab = L.chains + align256(2 * sizeof(int) * (size_t)p->n_shots * (p->n_src + p->n_rec));
+  L.tab_src = 256;
+  L.tab_rec = L.tab_src + entry_table_bytes(p->n_shots, p->n_src);
+  L.bandtab = L.tab_rec + entry_table_bytes(p->n_shots, p->n_rec);
   L.state_bytes = state_floats(p) * sizeof(float);
   const size_t off_state =
       L.bandtab + align256(sizeof(float) * (size_t)BandTab{bd.Wx, bd.Wz}.floats() + 16);
@@ -1493,7 +1483,8 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
   cudaStream_t st = (cudaStream_t)stream;
   int *flags = (int *)(ws + L.flags);
   // the array keeps the previous call's contents: clear the status words
-  // (the band table, chains and state buffer are fully rewritten below)
+  // (the band table, source / receiver tables and state buffer are fully
+  // rewritten below)
   MW_CUDA(cudaMemsetAsync(ws, 0, 256, st));
 
   float *bufA = state;
@@ -1507,24 +1498,20 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
     MW_TRY(fwd_maps(p, fields_at(p, bufA), ca, cb, cq, &mA));
     MW_TRY(fwd_maps(p, fields_at(p, bufB), ca, cb, cq, &mB));
     const int64_t numel = (int64_t)p->ny * p->nx;
-    const Chains ch = chains_at(p, ws, L);
-    if (p->n_src > 0)
-      MW_CUDA(launch_dup_chains(src_idx, p->n_shots, p->n_src, numel, ch.src_lead, ch.src_next,
-                                flags, st));
-    if (p->n_rec > 0 && rec)
-      MW_CUDA(launch_dup_chains(rec_idx, p->n_shots, p->n_rec, numel, ch.rec_lead, ch.rec_next,
-                                flags, st));
+    const Tables tb = tables_at(p, ws, L);
+    MW_TRY(build_table(p, src_idx, p->n_src, ws, L.tab_src, flags, nullptr, st));
+    if (rec) MW_TRY(build_table(p, rec_idx, p->n_rec, ws, L.tab_rec, flags, rec, st));
+    a.ea = tb.src;
+    if (rec) a.eb = tb.rec;
     float *cur = bufA, *nxt = bufB;
     for (int t = 0; t < p->nt; ++t) {
       a.in = fields_at(p, cur);
       a.out = fields_at(p, nxt);
       a.ctr_slot = t & 1;
+      a.vals_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
+      a.out_t = rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr;
       MW_CUDA(launch_forward(cur == bufA ? mA : mB, a, p->order, kStoreNone, kStoreNone,
                              p->model_batched != 0, !p->cq_is_scalar, lc.grid, st));
-      MW_CUDA(launch_inject_sample(nxt, numel, p->n_shots,
-                                   f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr, src_idx,
-                                   ch.src_lead, ch.src_next, p->n_src, rec_idx, p->n_rec,
-                                   rec ? rec + (int64_t)t * p->n_shots * p->n_rec : nullptr, st));
       std::swap(cur, nxt);
     }
     if (cur != bufA)

@@ -58,6 +58,23 @@ struct Fields {
   float *mze_node;  // z-band memory at the E nodes
 };
 
+// Sorted source or receiver entries of one index set idx [S][n] (built once
+// per call by launch_entry_table), so that the stencil kernels inject and
+// sample them in the rows they compute:
+//   ent  [S][n]    the valid entries of each shot sorted by (cell, k):
+//                  {row, column, k, run}; run = the number of consecutive
+//                  entries with this cell when this is the first of them,
+//                  else 0 (duplicates add up in index order)
+//   arow [S][n+1]  the distinct rows holding entries, ascending, then INT_MAX
+//   abeg [S][n+1]  the first sorted position of each of those rows, then the
+//                  number of valid entries
+// An empty set has n == 0 and null pointers.
+struct EntrySet {
+  const int4 *ent;
+  const int *arow, *abeg;
+  int n;
+};
+
 // Forward stage slots placed by the host (float offsets within a stage).
 enum { kFoCqH = 0, kFoCqX, kFoMzh, kFoMze, kFoMxh, kFoMxe, kFoBd, kFoBs, kFoCount };
 // Adjoint stage slots placed by the host.
@@ -92,6 +109,14 @@ struct StepArgs {
   // adjoint only: optional stage slots (kAo*), gCa / gCb pair fetch and order
   int ao[kAoCount];
   int gg_pair, gg_swap;
+  // sources / receivers of this step: set `ea` is injected (forward: the
+  // sources, vals_t = f[t]; adjoint: the receivers, vals_t = res[t]), set
+  // `eb` is sampled after the injection (forward: the receivers, out_t =
+  // rec[t]; adjoint: the sources, out_t = grad_f[t]); vals_t / out_t are
+  // [S][n] slices, null when there is nothing to inject / record
+  EntrySet ea, eb;
+  const float *vals_t;
+  float *out_t;
 };
 
 // TMA tensor maps of one forward launch (the input buffer set and model).
@@ -190,11 +215,13 @@ struct Layout {
   size_t rpA, rpB;    // replay ping-pong state buffers (checkpoint mode)
   size_t snap;        // snapshots / checkpoints
   size_t seg;         // checkpoint mode: fp32 segment snapshot buffer
-  size_t chains;      // duplicate chains of the source / receiver indices
+  size_t tab_src, tab_rec;  // entry tables of the sources and of the receivers
   size_t bandtab;     // CPML band coefficient table (BandTab)
   // MW_SNAP_CKPT_EY: the Cb-gradient accumulator [S][ny][nx], the record copy
-  // [nt][S][n_rec] and the receiver / source end-term sums [S][n_rec + n_src]
-  size_t sbp, rcopy, acc;
+  // [nt][S][n_rec], the receiver / source end-term sums [S][n_rec + n_src] and
+  // lambda_E sampled at the sources [nt][S][n_src] (when the caller asks for
+  // no grad_f)
+  size_t sbp, rcopy, acc, gfbuf;
   // checkpoint modes: snapshots of the last n_tail steps, stored by the forward
   size_t tail;
   int n_tail;
@@ -267,23 +294,30 @@ void adjoint_layout(int order, int Wx, bool cq_array, bool bf16, StepArgs *a, si
 int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array);
 
 // small kernels (mw_aux.cu)
-cudaError_t launch_dup_chains(const int64_t *idx, int S, int n, int64_t numel, int *lead,
-                              int *next, int *flags, cudaStream_t st);
-// End-term sums of the summation-by-parts Cb gradient, gathered by the
-// adjoint's injection launch of each step (all four null otherwise):
-// acc_a[s][k] += vals_t[s][k] * pair_t[s][k] (the residual times the
-// record it answers) and acc_b[s][k] += w_t[s][k] * out_t[s][k] (the source
-// wavelet times the sampled lambda_E).
-struct SbpTerms {
-  const float *pair_t = nullptr;
-  float *acc_a = nullptr;
-  const float *w_t = nullptr;
-  float *acc_b = nullptr;
-};
-cudaError_t launch_inject_sample(float *field, int64_t numel, int S, const float *vals_t,
-                                 const int64_t *idx_a, const int *lead, const int *next, int na,
-                                 const int64_t *idx_b, int nb, float *out_t, cudaStream_t st,
-                                 const SbpTerms &sbp = SbpTerms{});
+// Bytes of the entry table of an index set [S][n] (EntrySet layout).
+size_t entry_table_bytes(int S, int n);
+// The EntrySet of an index set whose table starts at `base`.
+EntrySet entry_set_at(void *base, int S, int n);
+// Build the entry table of idx [S][n] (cells y * nx + x, -1 inactive) into
+// the table at `base`; out-of-range entries set the bad-index flag.  Entries
+// that are not valid record nothing: with `out` ([nt][S][n]) their outputs
+// are zeroed for every step.
+cudaError_t launch_entry_table(const int64_t *idx, int S, int n, int ny, int nx, void *base,
+                               int *flags, float *out, int nt, cudaStream_t st);
+// Add vals [S][ea.n] at the cells of set `ea` of the E field [S][ny][nx]
+// (duplicates added up in index order first), then read the field at the
+// cells of set `eb` into out [S][eb.n]; either part is skipped when its
+// pointer is null.
+cudaError_t launch_fix_field(float *field, int S, int ny, int nx, const EntrySet &ea,
+                             const float *vals, const EntrySet &eb, float *out, cudaStream_t st);
+// End-term sums of the summation-by-parts Cb gradient, in the adjoint's
+// order t = nt - 1 .. 0: acc_rec[s][k] = sum_t res[t][s][k] rec[t][s][k] (the
+// residual times the record it answers) and acc_src[s][k] = sum_t
+// f[t][s][k] lam[t][s][k] (the source wavelet times lambda_E sampled at the
+// source).  A null pair skips that sum.
+cudaError_t launch_sbp_sums(int nt, int S, const float *res, const float *rec, int n_rec,
+                            float *acc_rec, const float *f, const float *lam, int n_src,
+                            float *acc_src, cudaStream_t st);
 // summation-by-parts Cb gradient: P = lambda_E * E (the end term of a given
 // adjoint start state), the scatter of the end-term sums into P (sequential
 // per shot: duplicates add in index order), and grad_cb_shot += P / Cb at

@@ -142,6 +142,77 @@ __host__ __device__ constexpr int walk_group() {
   return ADJ && P <= 2 ? 2 * P : 2;
 }
 
+// ---- sources and receivers in the rows a walk computes -------------------
+// A walk meets the rows of an EntrySet in ascending order: `Cursor` is the
+// next active row at or after the walk's position (INT_MAX when none).
+struct Cursor {
+  int a, row;
+};
+__device__ __forceinline__ Cursor cursor_at(const EntrySet &e, int s, int y0) {
+  if (e.n == 0) return Cursor{0, 0x7fffffff};
+  const int *ar = e.arow + (int64_t)s * (e.n + 1);
+  int lo = 0, hi = e.n;  // ar[e.n] is INT_MAX
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(ar + mid) < y0) lo = mid + 1;
+    else hi = mid;
+  }
+  return Cursor{lo, __ldg(ar + lo)};
+}
+__device__ __forceinline__ void cursor_next(const EntrySet &e, int s, Cursor &c) {
+  ++c.a;
+  c.row = __ldg(e.arow + (int64_t)s * (e.n + 1) + c.a);
+}
+
+// Fix-ups of one E row that the warp has just stored (row base `row`, the
+// warp's stores made visible by __syncwarp): add vals_t[s][k] into the cells
+// of the entries of active row c.a whose column lies in [lo, hi) -- the
+// entries of one cell add up first, in index order, then join the field,
+// like a serial loop over the duplicates -- or read those cells into
+// out_t[s][k].  One lane per entry; every cell is owned by exactly one warp.
+__device__ __forceinline__ void fix_inject(const EntrySet &e, int s, const Cursor &c,
+                                           const float *vals_t, int lo, int hi, float *row,
+                                           int lane) {
+  const int *ab = e.abeg + (int64_t)s * (e.n + 1);
+  const int j0 = __ldg(ab + c.a), j1 = __ldg(ab + c.a + 1);
+  const int4 *en = e.ent + (int64_t)s * e.n;
+  const float *vs = vals_t + (int64_t)s * e.n;
+  for (int j = j0 + lane; j < j1; j += 32) {
+    const int4 q = __ldg(en + j);
+    if (q.w > 0 && q.y >= lo && q.y < hi) {
+      float v = __ldg(vs + q.z);
+      for (int u = 1; u < q.w; ++u) v += __ldg(vs + __ldg(en + j + u).z);
+      row[q.y] += v;
+    }
+  }
+}
+__device__ __forceinline__ void fix_sample(const EntrySet &e, int s, const Cursor &c, float *out_t,
+                                           int lo, int hi, const float *row, int lane) {
+  const int *ab = e.abeg + (int64_t)s * (e.n + 1);
+  const int j0 = __ldg(ab + c.a), j1 = __ldg(ab + c.a + 1);
+  const int4 *en = e.ent + (int64_t)s * e.n;
+  for (int j = j0 + lane; j < j1; j += 32) {
+    const int4 q = __ldg(en + j);
+    if (q.y >= lo && q.y < hi) out_t[(int64_t)s * e.n + q.z] = row[q.y];
+  }
+}
+// Both fix-ups of output row y (sources first, then receivers), when y is
+// the next active row of either set; advances the cursors.
+__device__ __forceinline__ void fix_row(const StepArgs &a, int s, int y, int lo, int hi,
+                                        float *row, int lane, Cursor &ca, Cursor &cb) {
+  if (y != ca.row && y != cb.row) return;
+  __syncwarp();
+  if (y == ca.row) {
+    if (a.vals_t) fix_inject(a.ea, s, ca, a.vals_t, lo, hi, row, lane);
+    cursor_next(a.ea, s, ca);
+    __syncwarp();
+  }
+  if (y == cb.row) {
+    if (a.out_t) fix_sample(a.eb, s, cb, a.out_t, lo, hi, row, lane);
+    cursor_next(a.eb, s, cb);
+  }
+}
+
 // Strip / chunk of one work item.
 struct Item {
   int s, sm, x0, ya, yb, r0, n_it;
@@ -295,6 +366,8 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
       pr.next(NS);
     }
   }
+  // sources injected into and receivers sampled from the E rows [ya, yb)
+  Cursor cur_a = cursor_at(a.ea, it.s, it.ya), cur_b = cursor_at(a.eb, it.s, it.ya);
   constexpr int M = walk_group<P, false>();
   using Q = Queue<NQ, M>;
   F4 eq[Q::kSize], hq[Q::kSize];
@@ -468,6 +541,10 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
               if constexpr (STORE != kStoreEy) snap_store_p<STORE>(own, a.snap_c, so, curl);
             }
             st4p(own, ey_o + off, en);
+            // this step's sources, then its receivers, in the owned cells
+            const int y = it.r0 + i - 2 * P + 1;
+            fix_row(a, it.s, y, it.x0, min(it.x0 + a.g.strip_cols, nx),
+                    a.out.ey + (int64_t)it.s * a.g.numel + (int64_t)y * nx, lane, cur_a, cur_b);
           }
         }
         __syncwarp();
@@ -671,6 +748,9 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
       pr.next(NS);
     }
   }
+  // the next step's residuals injected into the lambda_E rows this walk
+  // writes, then lambda_E sampled at the sources there
+  Cursor cur_a = cursor_at(a.ea, it.s, it.ya), cur_b = cursor_at(a.eb, it.s, it.ya);
   constexpr int M = walk_group<P, true>();
   using Q = Queue<NQ, M>;
   F4 pq[Q::kSize], qq[Q::kSize], cl[Q::kSize];
@@ -868,6 +948,11 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
             en.v[q] = cla.v[q] - d_int<P>(wv, q, a.c.cx) - dz;
           }
           st4p(own, ey_o + (ro - (2 * P - 1) * nx), en);
+          {  // the next step's residuals, then its source gradient (owned cells)
+            const int y = r - 2 * P + 1;
+            fix_row(a, it.s, y, it.x0, min(it.x0 + a.g.strip_cols, nx),
+                    a.out.ey + (int64_t)it.s * a.g.numel + (int64_t)y * nx, lane, cur_a, cur_b);
+          }
           if constexpr (SNAP == kStoreEy) {
             // gradients of this row by summation by parts: gCa += E^t lam^{t+1};
             // the Cb accumulator takes E^t times the E-update term
