@@ -23,10 +23,10 @@ constexpr double kMu0 = 1.25663706212e-6;   // H/m (CODATA 2018)
 // entries (-1, or out of range, which also sets the bad-index flag) get no
 // place; with `out` their outputs out[t][s][k] are zeroed for every step.
 // O(n^2 / blockDim) per shot, once per call.
-__global__ void k_entry_table(const int64_t *__restrict__ idx, int n, int nx, int64_t numel,
-                              int4 *__restrict__ ent_all, int *__restrict__ arow_all,
-                              int *__restrict__ abeg_all, int *__restrict__ flags,
-                              float *__restrict__ out, int nt, int S) {
+__global__ void k_entry_table(const int64_t *__restrict__ idx, int n, int ny, int nx,
+                              int64_t numel, int4 *__restrict__ ent_all, int *__restrict__ arow_all,
+                              int *__restrict__ abeg_all, int2 *__restrict__ rcur_all,
+                              int *__restrict__ flags, float *__restrict__ out, int nt, int S) {
   const int s = blockIdx.x;
   const int64_t *v = idx + (int64_t)s * n;
   int4 *ent = ent_all + (int64_t)s * n;
@@ -80,6 +80,18 @@ __global__ void k_entry_table(const int64_t *__restrict__ idx, int n, int nx, in
   for (int a = s_nact + threadIdx.x; a <= n; a += blockDim.x) {
     arow[a] = 0x7fffffff;
     abeg[a] = nv;
+  }
+  __syncthreads();
+  // per row: the first active row at or after it (binary search over arow)
+  int2 *rcur = rcur_all + (int64_t)s * (ny + 1);
+  for (int y = threadIdx.x; y <= ny; y += blockDim.x) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (arow[mid] < y) lo = mid + 1;
+      else hi = mid;
+    }
+    rcur[y] = make_int2(lo, arow[lo]);
   }
 }
 
@@ -326,22 +338,24 @@ int grid_for(int64_t n, int block) {
 
 }  // namespace
 
-size_t entry_table_bytes(int S, int n) {
+size_t entry_table_bytes(int S, int n, int ny) {
   if (n <= 0) return 0;
-  const size_t e = (size_t)S * n * sizeof(int4);
-  const size_t r = (size_t)S * (n + 1) * sizeof(int);
-  return ((e + 255) & ~(size_t)255) + 2 * ((r + 255) & ~(size_t)255);
+  auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return a256((size_t)S * n * sizeof(int4)) + 2 * a256((size_t)S * (n + 1) * sizeof(int)) +
+         a256((size_t)S * (ny + 1) * sizeof(int2));
 }
 
-EntrySet entry_set_at(void *base, int S, int n) {
-  EntrySet es{nullptr, nullptr, nullptr, 0};
+EntrySet entry_set_at(void *base, int S, int n, int ny) {
+  EntrySet es{nullptr, nullptr, nullptr, nullptr, 0, ny};
   if (n <= 0 || base == nullptr) return es;
+  auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
   char *b = (char *)base;
-  const size_t e = (((size_t)S * n * sizeof(int4)) + 255) & ~(size_t)255;
-  const size_t r = (((size_t)S * (n + 1) * sizeof(int)) + 255) & ~(size_t)255;
+  const size_t e = a256((size_t)S * n * sizeof(int4));
+  const size_t r = a256((size_t)S * (n + 1) * sizeof(int));
   es.ent = (const int4 *)b;
   es.arow = (const int *)(b + e);
   es.abeg = (const int *)(b + e + r);
+  es.rcur = (const int2 *)(b + e + 2 * r);
   es.n = n;
   return es;
 }
@@ -349,10 +363,10 @@ EntrySet entry_set_at(void *base, int S, int n) {
 cudaError_t launch_entry_table(const int64_t *idx, int S, int n, int ny, int nx, void *base,
                                int *flags, float *out, int nt, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  const EntrySet es = entry_set_at(base, S, n);
-  k_entry_table<<<S, 256, 0, st>>>(idx, n, nx, (int64_t)ny * nx, const_cast<int4 *>(es.ent),
-                                   const_cast<int *>(es.arow), const_cast<int *>(es.abeg), flags,
-                                   out, nt, S);
+  const EntrySet es = entry_set_at(base, S, n, ny);
+  k_entry_table<<<S, 256, 0, st>>>(idx, n, ny, nx, (int64_t)ny * nx, const_cast<int4 *>(es.ent),
+                                   const_cast<int *>(es.arow), const_cast<int *>(es.abeg),
+                                   const_cast<int2 *>(es.rcur), flags, out, nt, S);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -148,8 +148,8 @@ Layout layout(const mw_params *p) {
   const size_t sb = align256(L.state_bytes);
   size_t off = 0;
   L.flags = off; off += 256;
-  L.tab_src = off; off += entry_table_bytes(p->n_shots, p->n_src);
-  L.tab_rec = off; off += entry_table_bytes(p->n_shots, p->n_rec);
+  L.tab_src = off; off += entry_table_bytes(p->n_shots, p->n_src, p->ny);
+  L.tab_rec = off; off += entry_table_bytes(p->n_shots, p->n_rec, p->ny);
   L.bandtab = off;
   {
     const Bands b = bands(p);
@@ -276,8 +276,8 @@ struct Tables {
   EntrySet src, rec;
 };
 Tables tables_at(const mw_params *p, char *ws, const Layout &L) {
-  return Tables{entry_set_at(ws + L.tab_src, p->n_shots, p->n_src),
-                entry_set_at(ws + L.tab_rec, p->n_shots, p->n_rec)};
+  return Tables{entry_set_at(ws + L.tab_src, p->n_shots, p->n_src, p->ny),
+                entry_set_at(ws + L.tab_rec, p->n_shots, p->n_rec, p->ny)};
 }
 // Build the table of one index set (n > 0); `out` [nt][S][n] gets zeros at
 // the invalid entries.
@@ -1467,8 +1467,8 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
   Layout L{};
   L.flags = 0;
   L.tab_src = 256;
-  L.tab_rec = L.tab_src + entry_table_bytes(p->n_shots, p->n_src);
-  L.bandtab = L.tab_rec + entry_table_bytes(p->n_shots, p->n_rec);
+  L.tab_rec = L.tab_src + entry_table_bytes(p->n_shots, p->n_src, p->ny);
+  L.bandtab = L.tab_rec + entry_table_bytes(p->n_shots, p->n_rec, p->ny);
   L.state_bytes = state_floats(p) * sizeof(float);
   const size_t off_state =
       L.bandtab + align256(sizeof(float) * (size_t)BandTab{bd.Wx, bd.Wz}.floats() + 16);

@@ -68,11 +68,14 @@ struct Fields {
 //   arow [S][n+1]  the distinct rows holding entries, ascending, then INT_MAX
 //   abeg [S][n+1]  the first sorted position of each of those rows, then the
 //                  number of valid entries
+//   rcur [S][ny+1] for each row y: {a, arow[a]} with a the first active row
+//                  at or after y (where a walk starting at row y begins)
 // An empty set has n == 0 and null pointers.
 struct EntrySet {
   const int4 *ent;
   const int *arow, *abeg;
-  int n;
+  const int2 *rcur;
+  int n, ny;
 };
 
 // Forward stage slots placed by the host (float offsets within a stage).
@@ -294,10 +297,10 @@ void adjoint_layout(int order, int Wx, bool cq_array, bool bf16, StepArgs *a, si
 int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array);
 
 // small kernels (mw_aux.cu)
-// Bytes of the entry table of an index set [S][n] (EntrySet layout).
-size_t entry_table_bytes(int S, int n);
+// Bytes of the entry table of an index set [S][n] on ny rows (EntrySet layout).
+size_t entry_table_bytes(int S, int n, int ny);
 // The EntrySet of an index set whose table starts at `base`.
-EntrySet entry_set_at(void *base, int S, int n);
+EntrySet entry_set_at(void *base, int S, int n, int ny);
 // Build the entry table of idx [S][n] (cells y * nx + x, -1 inactive) into
 // the table at `base`; out-of-range entries set the bad-index flag.  Entries
 // that are not valid record nothing: with `out` ([nt][S][n]) their outputs

@@ -150,14 +150,9 @@ struct Cursor {
 };
 __device__ __forceinline__ Cursor cursor_at(const EntrySet &e, int s, int y0) {
   if (e.n == 0) return Cursor{0, 0x7fffffff};
-  const int *ar = e.arow + (int64_t)s * (e.n + 1);
-  int lo = 0, hi = e.n;  // ar[e.n] is INT_MAX
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(ar + mid) < y0) lo = mid + 1;
-    else hi = mid;
-  }
-  return Cursor{lo, __ldg(ar + lo)};
+  const int y = y0 < 0 ? 0 : y0 > e.ny ? e.ny : y0;
+  const int2 c = __ldg(e.rcur + (int64_t)s * (e.ny + 1) + y);
+  return Cursor{c.x, c.y};
 }
 __device__ __forceinline__ void cursor_next(const EntrySet &e, int s, Cursor &c) {
   ++c.a;
@@ -196,20 +191,26 @@ __device__ __forceinline__ void fix_sample(const EntrySet &e, int s, const Curso
     if (q.y >= lo && q.y < hi) out_t[(int64_t)s * e.n + q.z] = row[q.y];
   }
 }
-// Both fix-ups of output row y (sources first, then receivers), when y is
-// the next active row of either set; advances the cursors.
-__device__ __forceinline__ void fix_row(const StepArgs &a, int s, int y, int lo, int hi,
-                                        float *row, int lane, Cursor &ca, Cursor &cb) {
-  if (y != ca.row && y != cb.row) return;
-  __syncwarp();
-  if (y == ca.row) {
-    if (a.vals_t) fix_inject(a.ea, s, ca, a.vals_t, lo, hi, row, lane);
-    cursor_next(a.ea, s, ca);
+// The fix-ups of the E rows [ya, yb) of one item once its walk has stored
+// them all (sources first, then receivers, row by row), in the columns
+// [lo, hi) the item owns.  Outside the walk loop, so the walk's code is
+// untouched by them.
+__device__ __forceinline__ void fix_item(const StepArgs &a, int s, int ya, int yb, int lo, int hi,
+                                         float *field, int nx, int lane) {
+  Cursor ca = cursor_at(a.ea, s, ya), cb = cursor_at(a.eb, s, ya);
+  while (ca.row < yb || cb.row < yb) {
+    const int y = ca.row < cb.row ? ca.row : cb.row;
+    float *row = field + (int64_t)y * nx;
     __syncwarp();
-  }
-  if (y == cb.row) {
-    if (a.out_t) fix_sample(a.eb, s, cb, a.out_t, lo, hi, row, lane);
-    cursor_next(a.eb, s, cb);
+    if (y == ca.row) {
+      if (a.vals_t) fix_inject(a.ea, s, ca, a.vals_t, lo, hi, row, lane);
+      cursor_next(a.ea, s, ca);
+      __syncwarp();
+    }
+    if (y == cb.row) {
+      if (a.out_t) fix_sample(a.eb, s, cb, a.out_t, lo, hi, row, lane);
+      cursor_next(a.eb, s, cb);
+    }
   }
 }
 
@@ -366,8 +367,6 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
       pr.next(NS);
     }
   }
-  // sources injected into and receivers sampled from the E rows [ya, yb)
-  Cursor cur_a = cursor_at(a.ea, it.s, it.ya), cur_b = cursor_at(a.eb, it.s, it.ya);
   constexpr int M = walk_group<P, false>();
   using Q = Queue<NQ, M>;
   F4 eq[Q::kSize], hq[Q::kSize];
@@ -541,10 +540,6 @@ __device__ __forceinline__ bool fwd_walk(const FwdMaps &m, const StepArgs &a, co
               if constexpr (STORE != kStoreEy) snap_store_p<STORE>(own, a.snap_c, so, curl);
             }
             st4p(own, ey_o + off, en);
-            // this step's sources, then its receivers, in the owned cells
-            const int y = it.r0 + i - 2 * P + 1;
-            fix_row(a, it.s, y, it.x0, min(it.x0 + a.g.strip_cols, nx),
-                    a.out.ey + (int64_t)it.s * a.g.numel + (int64_t)y * nx, lane, cur_a, cur_b);
           }
         }
         __syncwarp();
@@ -614,6 +609,9 @@ __global__ void __launch_bounds__(128, BORN != kStoreNone ? 3 : (P <= 3 ? 5 : 4)
     const bool ok = it.edge ? fwd_walk<P, STORE, L, true, BORN>(m, a, it, w, cq_arr, cqs)
                             : fwd_walk<P, STORE, L, false, BORN>(m, a, it, w, cq_arr, cqs);
     if (!ok) return;
+    // this step's sources, then its receivers, in the item's cells
+    fix_item(a, it.s, it.ya, it.yb, it.x0, min(it.x0 + g.strip_cols, g.nx),
+             a.out.ey + (int64_t)it.s * g.numel, g.nx, lane);
   }
 }
 
@@ -748,9 +746,6 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
       pr.next(NS);
     }
   }
-  // the next step's residuals injected into the lambda_E rows this walk
-  // writes, then lambda_E sampled at the sources there
-  Cursor cur_a = cursor_at(a.ea, it.s, it.ya), cur_b = cursor_at(a.eb, it.s, it.ya);
   constexpr int M = walk_group<P, true>();
   using Q = Queue<NQ, M>;
   F4 pq[Q::kSize], qq[Q::kSize], cl[Q::kSize];
@@ -948,11 +943,6 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
             en.v[q] = cla.v[q] - d_int<P>(wv, q, a.c.cx) - dz;
           }
           st4p(own, ey_o + (ro - (2 * P - 1) * nx), en);
-          {  // the next step's residuals, then its source gradient (owned cells)
-            const int y = r - 2 * P + 1;
-            fix_row(a, it.s, y, it.x0, min(it.x0 + a.g.strip_cols, nx),
-                    a.out.ey + (int64_t)it.s * a.g.numel + (int64_t)y * nx, lane, cur_a, cur_b);
-          }
           if constexpr (SNAP == kStoreEy) {
             // gradients of this row by summation by parts: gCa += E^t lam^{t+1};
             // the Cb accumulator takes E^t times the E-update term
@@ -1041,6 +1031,9 @@ __global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_c
     const bool ok = it.edge ? adj_walk<P, SNAP, L, true>(m, a, it, w, cq_arr, cqs)
                             : adj_walk<P, SNAP, L, false>(m, a, it, w, cq_arr, cqs);
     if (!ok) return;
+    // the next step's residuals, then its source gradient, in the item's cells
+    fix_item(a, it.s, it.ya, it.yb, it.x0, min(it.x0 + g.strip_cols, g.nx),
+             a.out.ey + (int64_t)it.s * g.numel, g.nx, lane);
   }
 }
 
