@@ -309,18 +309,20 @@ struct Launch {
 };
 
 // Interior rectangle of the item grid (the same edge rule as the kernels'
-// make_item): strip x0 with its 8-column halo clear of the x bands and the
-// array's sides; chunk [ya, yb) whose walk rows ya - 2P + 1 .. yb + 2P - 2
-// stay clear of the z bands.  Checked to give a bijection of the items.
-void interior_rect(Geom &g, int P) {
+// make_item / make_item2): strip x0 with an xh-column margin clear of the x
+// bands and the array's sides; chunk [ya, yb) whose walk rows ya - zw ..
+// yb + zw - 1 stay clear of the z bands (one-step kernels: xh = 8, zw =
+// 2P - 1; two-step forward: xh = halo + 4, zw = 4P - 2).  Checked to give a
+// bijection of the items.
+void interior_rect(Geom &g, int xh, int zw) {
   auto strip_edge = [&](int k) {
     const int x0 = k * g.strip_cols;
-    return x0 - 8 < g.Wx || x0 + g.strip_cols + 8 > g.nx - g.Wx;
+    return x0 - xh < g.Wx || x0 + g.strip_cols + xh > g.nx - g.Wx;
   };
   auto chunk_edge = [&](int k) {
     int ya, yb;
     chunk_rows(g, k, &ya, &yb);
-    return g.Wz > 0 && (ya - (2 * P - 1) < g.Wz || yb + 2 * P - 1 > g.ny - g.Wz);
+    return g.Wz > 0 && (ya - zw < g.Wz || yb + zw > g.ny - g.Wz);
   };
   int a = 0, b = g.n_strips;
   while (a < b && strip_edge(a)) ++a;
@@ -356,7 +358,9 @@ void interior_rect(Geom &g, int P) {
 
 // Choose the row-chunk height so that the warps' work items fill whole waves
 // of resident warps: cost ~ waves x (rows per item + warm-up rows).
-Launch plan(const mw_params *p, bool adjoint) {
+enum PlanKind { kPlanFwd = 0, kPlanAdj = 1, kPlanFwd2 = 2 };
+Launch plan(const mw_params *p, int kind) {
+  const bool adjoint = kind == kPlanAdj, two = kind == kPlanFwd2;
   Launch Lc{};
   Geom &g = Lc.g;
   const Bands b = bands(p);
@@ -368,10 +372,11 @@ Launch plan(const mw_params *p, bool adjoint) {
   g.n_pml = p->n_pml;
   g.grad_mask = p->grad_mask_pml ? 1 : 0;
   g.numel = (int64_t)p->ny * p->nx;
-  g.strip_cols = adjoint ? kAdjStripCols : kFwdStripCols;
-  g.n_strips = (p->nx + g.strip_cols - 1) / g.strip_cols;
   const int P = p->order / 2;
-  const int warps_sm = stencil_slots_per_sm(p->order, adjoint, b.Wx, !p->cq_is_scalar);
+  g.strip_cols = adjoint ? kAdjStripCols : two ? fwd2_width(P) : kFwdStripCols;
+  g.n_strips = (p->nx + g.strip_cols - 1) / g.strip_cols;
+  const int warps_sm = two ? forward2_slots_per_sm(p->order, b.Wx)
+                           : stencil_slots_per_sm(p->order, adjoint, b.Wx, !p->cq_is_scalar);
   const int64_t slots = (int64_t)sm_count() * warps_sm;
   const int64_t cols_items = (int64_t)g.S * g.n_strips;
   // Items are claimed dynamically by resident warps.  Each item walks its
@@ -380,7 +385,7 @@ Launch plan(const mw_params *p, bool adjoint) {
   // long chunks of H1 rows first and short chunks of H2 rows after them, the
   // last long items must also end in time:
   //   cost = max(W / slots + (H2 + w), W_long / slots + (H1 + w)).
-  const int w = 4 * P - 2;
+  const int w = two ? 8 * P - 4 : 4 * P - 2;
   const double cols = (double)cols_items, sl = (double)slots;
   int best_h1 = p->ny, best_h2 = p->ny, best_n1 = 1;
   double best_cost = 1e300;
@@ -422,7 +427,8 @@ Launch plan(const mw_params *p, bool adjoint) {
     g.n_chunks = rest > 0 ? best_n1 + (rest + best_h2 - 1) / best_h2 : (p->ny + best_h1 - 1) / best_h1;
     if (rest <= 0) g.n_big = g.n_chunks;
   }
-  interior_rect(g, P);
+  if (two) interior_rect(g, fwd2_halo(P) + 4, 4 * P - 2);
+  else interior_rect(g, 8, 2 * P - 1);
   const int64_t items = cols_items * g.n_chunks;
   const int wpc = adjoint ? kAdjWarpsPerCta : kWarpsPerCta;
   int64_t grid = (items + wpc - 1) / wpc;
@@ -569,6 +575,32 @@ int fwd_maps(const mw_params *p, const Fields &in, const float *ca, const float 
   return MW_OK;
 }
 
+// Two-step forward: every box 128 wide (the walk's columns), Ca / Cb a pair
+// box when their distance allows.
+int fwd2_maps(const mw_params *p, const Fields &in, const float *ca, const float *cb,
+              Fwd2Maps *m) {
+  memset(m, 0, sizeof *m);
+  const Bands bd = bands(p);
+  const uint64_t nx = p->nx, ny = p->ny, S = p->n_shots, Sm = p->model_batched ? p->n_shots : 1;
+  MW_TRY(encode_rows(&m->map[kM2E], in.ey, 4, 3, nx, ny, S, 1, 128));
+  MW_TRY(encode_rows(&m->map[kM2HZ], in.hz, 4, 3, nx, ny, S, 1, 128));
+  MW_TRY(encode_rows(&m->map[kM2HX], in.hx, 4, 3, nx, ny, S, 1, 128));
+  const MdPair md = md_pairing(p, ca, cb);
+  if (md.pair) {
+    MW_TRY(encode_rows(&m->map[kM2MD], md.swap ? cb : ca, 4, 4, nx, ny, Sm, 2, 128, 2, md.stride));
+  } else {
+    MW_TRY(encode_rows(&m->map[kM2MD], ca, 4, 3, nx, ny, Sm, 1, 128));
+    MW_TRY(encode_rows(&m->map[kM2CB], cb, 4, 3, nx, ny, Sm, 1, 128));
+  }
+  if (bd.Wx > 0) {
+    MW_TRY(encode_rows(&m->map[kM2MXH], in.mxh_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
+    MW_TRY(encode_rows(&m->map[kM2MXE], in.mxe_node, 4, 3, 2 * bd.Wx, ny, S, 1, 2 * bd.Wx));
+    MW_TRY(encode_rows(&m->map[kM2MZH], in.mzh_node, 4, 3, nx, 2 * bd.Wz, S, 1, 128));
+    MW_TRY(encode_rows(&m->map[kM2MZE], in.mze_node, 4, 3, nx, 2 * bd.Wz, S, 1, 128));
+  }
+  return MW_OK;
+}
+
 // Born forward: dCa / dCb (pair box when their distance allows) and the
 // background's snapshots (x, y, shot, step, field) as one box 144 wide.
 int born_maps(const mw_params *p, const float *dca, const float *dcb, const void *se,
@@ -680,6 +712,32 @@ void set_layout(StepArgs &a, const mw_params *p, bool adjoint) {
   }
 }
 
+// Two-step forward launches of a call: their plan, arguments (the one-step
+// forward's, re-laid-out) and the maps of each input buffer they read.  Used
+// only where the two-step kernel applies (orders 2-6, scalar Cq); otherwise
+// `on` is false and every step runs the one-step kernel.
+struct Pairs {
+  bool on = false;
+  Launch lc{};
+  StepArgs a{};
+  int init(const mw_params *p, const StepArgs &one) {
+    on = forward2_supported(p->order) && p->cq_is_scalar && !pairs_disabled();
+    if (!on) return MW_OK;
+    lc = plan(p, kPlanFwd2);
+    a = one;
+    a.g = lc.g;
+    size_t smem;
+    forward2_layout(p->order, bands(p).Wx, &a, &smem);
+    return MW_OK;
+  }
+  // MW_NO_TWO_STEP=1 in the environment runs every step with the one-step
+  // kernel (for comparisons)
+  static bool pairs_disabled() {
+    const char *e = getenv("MW_NO_TWO_STEP");
+    return e && e[0] == '1';
+  }
+};
+
 // Step arguments shared by every stencil launch of a call.
 StepArgs step_args(const mw_params *p, const Launch &lc, const float *ca, const float *cb,
                    const float *cq, int *flags, const char *ws, const Layout &L) {
@@ -749,6 +807,8 @@ struct Replay {
   Launch lf{};
   StepArgs fa{};
   FwdMaps fA, fB, fS;  // inputs rA, rB, the segment's checkpoint
+  Pairs pr;            // two steps per launch within a segment
+  Fwd2Maps f2A, f2B, f2S;
   const float *ca_ = nullptr, *cb_ = nullptr, *cq_ = nullptr;
   float *rA = nullptr, *rB = nullptr;
   int store = kStoreF32;  // the segment: E and curl, or E alone (kStoreEy)
@@ -763,7 +823,7 @@ struct Replay {
     st = st_;
     f = f_;
     src = src_;
-    lf = plan(p, false);
+    lf = plan(p, kPlanFwd);
     fa = step_args(p, lf, ca, cb, cq, flags, ws, L);
     set_layout(fa, p, false);
     fa.ea = src;  // sources injected, nothing recorded
@@ -775,6 +835,11 @@ struct Replay {
     cq_ = cq;
     MW_TRY(fwd_maps(p, fields_at(p, rA), ca, cb, cq, &fA));
     MW_TRY(fwd_maps(p, fields_at(p, rB), ca, cb, cq, &fB));
+    MW_TRY(pr.init(p, fa));
+    if (pr.on) {
+      MW_TRY(fwd2_maps(p, fields_at(p, rA), ca, cb, &f2A));
+      MW_TRY(fwd2_maps(p, fields_at(p, rB), ca, cb, &f2B));
+    }
     return MW_OK;
   }
   // replay segment k up to step t_end at most; *t0 / *t1 receive its steps
@@ -787,19 +852,41 @@ struct Replay {
     // the first step reads the checkpoint in place
     float *rc = ckpt_slot(ws, L, k), *rn = rA;
     MW_TRY(fwd_maps(p, fields_at(p, rc), ca_, cb_, cq_, &fS));
-    for (int t = t0; t < t1; ++t) {
+    if (pr.on) MW_TRY(fwd2_maps(p, fields_at(p, rc), ca_, cb_, &f2S));
+    for (int t = t0; t < t1;) {
+      const bool pair = pr.on && t + 1 < t1;
       rn = rc == rA ? rB : rA;
-      fa.in = fields_at(p, rc);
-      fa.out = fields_at(p, rn);
-      fa.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
-      fa.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
-      fa.ctr_slot = ((*launch_idx)++) & 1;
-      fa.vals_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
-      const FwdMaps &fm = rc == rA ? fA : rc == rB ? fB : fS;
-      MW_CUDA(timed(1, st, [&] {
-        return launch_forward(fm, fa, p->order, store, kStoreNone, p->model_batched != 0,
-                              !p->cq_is_scalar, lf.grid, st);
-      }));
+      const float *f_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
+      if (pair) {
+        StepArgs &b = pr.a;
+        b.in = fields_at(p, rc);
+        b.out = fields_at(p, rn);
+        b.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
+        b.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
+        b.snap_e2 = seg_e + (size_t)(t + 1 - t0) * L.snap_step_bytes;
+        b.snap_c2 = seg_c + (size_t)(t + 1 - t0) * L.snap_step_bytes;
+        b.vals_t = f_t;
+        b.vals_t2 = f ? f_t + (int64_t)p->n_shots * p->n_src : nullptr;
+        b.ctr_slot = ((*launch_idx)++) & 1;
+        const Fwd2Maps &fm = rc == rA ? f2A : rc == rB ? f2B : f2S;
+        MW_CUDA(timed(5, st, [&] {
+          return launch_forward2(fm, b, p->order, store, p->model_batched != 0, pr.lc.grid, st);
+        }));
+        t += 2;
+      } else {
+        fa.in = fields_at(p, rc);
+        fa.out = fields_at(p, rn);
+        fa.snap_e = seg_e + (size_t)(t - t0) * L.snap_step_bytes;
+        fa.snap_c = seg_c + (size_t)(t - t0) * L.snap_step_bytes;
+        fa.ctr_slot = ((*launch_idx)++) & 1;
+        fa.vals_t = f_t;
+        const FwdMaps &fm = rc == rA ? fA : rc == rB ? fB : fS;
+        MW_CUDA(timed(1, st, [&] {
+          return launch_forward(fm, fa, p->order, store, kStoreNone, p->model_batched != 0,
+                                !p->cq_is_scalar, lf.grid, st);
+        }));
+        t += 1;
+      }
       rc = rn;
     }
     last = rc;
@@ -941,7 +1028,7 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   if (!state) MW_CUDA(cudaMemsetAsync(bufA, 0, L.state_bytes, st));
   if (p->nt == 0) return MW_OK;
 
-  const Launch lc = plan(p, false);
+  const Launch lc = plan(p, kPlanFwd);
   StepArgs a = step_args(p, lc, ca, cb, cq, flags, ws, L);
   set_layout(a, p, false);
   a.snap_pitch = L.snap_pitch;
@@ -977,42 +1064,83 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   const bool ck = is_ckpt(p);
   if (ck) MW_CUDA(cudaMemcpyAsync(ckpt_slot(ws, L, 0), bufA, L.state_bytes,
                                   cudaMemcpyDeviceToDevice, st));
+  // the snapshot destination and store kind of step t
+  auto snap_of = [&](int t, void **e, void **c) -> int {
+    const int slot = host ? t % kHostRing : t;
+    if (t >= t_tail && L.n_tail > 0) {
+      *e = tail_e + (size_t)(t - t_tail) * L.snap_step_bytes;
+      *c = tail_c + (size_t)(t - t_tail) * L.snap_step_bytes;
+      return tail_store;
+    }
+    *e = store ? snap_e + (size_t)slot * L.snap_step_bytes : nullptr;
+    *c = store ? snap_c + (size_t)slot * L.snap_step_bytes : nullptr;
+    return store;
+  };
+  // two steps per launch where the state between them is not needed (no
+  // checkpoint after the first) and both store alike; not with the host
+  // snapshot ring, which copies every step out on its own
+  Pairs pr;
+  MW_TRY(pr.init(p, a));
+  Fwd2Maps m2A, m2B, m2S;
+  if (pr.on && !host) {
+    MW_TRY(fwd2_maps(p, fields_at(p, bufA), ca, cb, &m2A));
+    MW_TRY(fwd2_maps(p, fields_at(p, bufB), ca, cb, &m2B));
+  }
   FwdMaps mS;  // input maps of a checkpoint slot
-  for (int t = 0; t < p->nt; ++t) {
-    const int k_out = ck && (t + 1) % p->ckpt_every == 0 ? (t + 1) / p->ckpt_every : -1;
+  int launch_idx = 0;
+  const int C = ck ? p->ckpt_every : 0;
+  for (int t = 0; t < p->nt;) {
+    const bool pair = pr.on && !host && t + 1 < p->nt && !(ck && (t + 1) % C == 0) &&
+                      (L.n_tail == 0 || (t >= t_tail) == (t + 1 >= t_tail));
+    const int tn = pair ? t + 2 : t + 1;  // steps done after this launch
+    const int k_out = ck && tn % C == 0 ? tn / C : -1;
     nxt = k_out > 0 && k_out < L.n_seg ? ckpt_slot(ws, L, k_out) : cur == bufA ? bufB : bufA;
     const int slot = host ? t % kHostRing : t;
     // the slot's previous step must have reached the host
     if (host && t >= kHostRing) MW_CUDA(cudaStreamWaitEvent(st, hc.freed[slot], 0));
-    a.in = fields_at(p, cur);
-    a.out = fields_at(p, nxt);
-    a.snap_e = store ? snap_e + (size_t)slot * L.snap_step_bytes : nullptr;
-    a.snap_c = store ? snap_c + (size_t)slot * L.snap_step_bytes : nullptr;
-    int kind = store;
-    if (t >= t_tail && L.n_tail > 0) {
-      kind = tail_store;
-      a.snap_e = tail_e + (size_t)(t - t_tail) * L.snap_step_bytes;
-      a.snap_c = tail_c + (size_t)(t - t_tail) * L.snap_step_bytes;
-    }
-    if (cur != bufA && cur != bufB) MW_TRY(fwd_maps(p, a.in, ca, cb, cq, &mS));
-    const FwdMaps &m = cur == bufA ? mA : cur == bufB ? mB : mS;
-    a.ctr_slot = t & 1;
-    a.vals_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
-    a.out_t = rec_out ? rec_out + (int64_t)t * p->n_shots * p->n_rec : nullptr;
-    MW_CUDA(timed(kind ? 1 : 0, st, [&] {
-      return launch_forward(m, a, p->order, kind, kStoreNone, p->model_batched != 0, !p->cq_is_scalar,
-                            lc.grid, st);
-    }));
-    if (host) {  // step t: ring slot -> host, on the copy stream
-      MW_CUDA(cudaEventRecord(hc.filled[slot], st));
-      MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.filled[slot], 0));
-      char *h = hbuf + 2 * (size_t)t * L.snap_step_bytes;
-      MW_CUDA(cudaMemcpyAsync(h, a.snap_e, L.snap_step_bytes, cudaMemcpyDeviceToHost, hc.cs));
-      MW_CUDA(cudaMemcpyAsync(h + L.snap_step_bytes, a.snap_c, L.snap_step_bytes,
-                              cudaMemcpyDeviceToHost, hc.cs));
-      MW_CUDA(cudaEventRecord(hc.freed[slot], hc.cs));
+    const float *f_t = f ? f + (int64_t)t * p->n_shots * p->n_src : nullptr;
+    float *rec_t = rec_out ? rec_out + (int64_t)t * p->n_shots * p->n_rec : nullptr;
+    if (pair) {
+      StepArgs &b = pr.a;
+      b.in = fields_at(p, cur);
+      b.out = fields_at(p, nxt);
+      const int kind = snap_of(t, &b.snap_e, &b.snap_c);
+      snap_of(t + 1, &b.snap_e2, &b.snap_c2);
+      b.vals_t = f_t;
+      b.vals_t2 = f ? f_t + (int64_t)p->n_shots * p->n_src : nullptr;
+      b.out_t = rec_t;
+      b.out_t2 = rec_out ? rec_t + (int64_t)p->n_shots * p->n_rec : nullptr;
+      b.ctr_slot = (launch_idx++) & 1;
+      if (cur != bufA && cur != bufB) MW_TRY(fwd2_maps(p, b.in, ca, cb, &m2S));
+      const Fwd2Maps &m2 = cur == bufA ? m2A : cur == bufB ? m2B : m2S;
+      MW_CUDA(timed(kind ? 5 : 4, st, [&] {
+        return launch_forward2(m2, b, p->order, kind, p->model_batched != 0, pr.lc.grid, st);
+      }));
+    } else {
+      a.in = fields_at(p, cur);
+      a.out = fields_at(p, nxt);
+      const int kind = snap_of(t, &a.snap_e, &a.snap_c);
+      if (cur != bufA && cur != bufB) MW_TRY(fwd_maps(p, a.in, ca, cb, cq, &mS));
+      const FwdMaps &m = cur == bufA ? mA : cur == bufB ? mB : mS;
+      a.ctr_slot = (launch_idx++) & 1;
+      a.vals_t = f_t;
+      a.out_t = rec_t;
+      MW_CUDA(timed(kind ? 1 : 0, st, [&] {
+        return launch_forward(m, a, p->order, kind, kStoreNone, p->model_batched != 0,
+                              !p->cq_is_scalar, lc.grid, st);
+      }));
+      if (host) {  // step t: ring slot -> host, on the copy stream
+        MW_CUDA(cudaEventRecord(hc.filled[slot], st));
+        MW_CUDA(cudaStreamWaitEvent(hc.cs, hc.filled[slot], 0));
+        char *h = hbuf + 2 * (size_t)t * L.snap_step_bytes;
+        MW_CUDA(cudaMemcpyAsync(h, a.snap_e, L.snap_step_bytes, cudaMemcpyDeviceToHost, hc.cs));
+        MW_CUDA(cudaMemcpyAsync(h + L.snap_step_bytes, a.snap_c, L.snap_step_bytes,
+                                cudaMemcpyDeviceToHost, hc.cs));
+        MW_CUDA(cudaEventRecord(hc.freed[slot], hc.cs));
+      }
     }
     cur = nxt;
+    t = tn;
   }
   if (ey_only && rec && p->n_rec > 0)
     MW_CUDA(cudaMemcpyAsync(rec, rec_out, (size_t)p->nt * p->n_shots * p->n_rec * sizeof(float),
@@ -1074,7 +1202,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   if (!adj_state) MW_CUDA(cudaMemsetAsync(adA, 0, L.state_bytes, st));
   if (p->nt == 0) return MW_OK;
 
-  const Launch la = plan(p, true);
+  const Launch la = plan(p, kPlanAdj);
   // MW_SNAP_CKPT_EY: the Cb gradient accumulates E^t G^t into P (workspace)
   // and the end-term sums beside it; grad_cb_shot receives P / Cb at the end
   float *sbp = ey_only ? (float *)(ws + L.sbp) : nullptr;
@@ -1237,7 +1365,7 @@ int mw_tm_born(const mw_params *p, const float *ca, const float *cb, const float
   // the perturbation state lives in the adjoint's buffers, from zero
   float *dA = (float *)(ws + L.adA), *dB = (float *)(ws + L.adB);
   MW_CUDA(cudaMemsetAsync(dA, 0, L.state_bytes, st));
-  const Launch lc = plan(p, false);
+  const Launch lc = plan(p, kPlanFwd);
   StepArgs b = step_args(p, lc, ca, cb, cq, flags, ws, L);
   {
     size_t smem;
@@ -1490,7 +1618,7 @@ int mw_tm_forward_noalloc(const mw_params *p, const float *ca, const float *cb, 
   float *bufA = state;
   float *bufB = (float *)(ws + off_state);
   if (p->nt > 0) {
-    const Launch lc = plan(p, false);
+    const Launch lc = plan(p, kPlanFwd);
     StepArgs a = step_args(p, lc, ca, cb, cq, flags, ws, L);
     set_layout(a, p, false);
     MW_TRY(stencil_prologue(p, cpml, ws, L, st));

@@ -105,6 +105,7 @@ struct StepArgs {
   // shared-memory layout of one warp (floats): stage size, warp area, band
   // row width (the x-band memory TMA box, 2*Wx)
   int stage_floats, warp_floats, band_box_floats;
+  int band_ring;  // two-step forward: floats per band row of the x-band carry rings
   // forward only: optional stage slots (kFo*), Ca / Cb pair fetch and order
   int fo[kFoCount];
   int md_pair, md_swap;
@@ -120,6 +121,12 @@ struct StepArgs {
   EntrySet ea, eb;
   const float *vals_t;
   float *out_t;
+  // two-step forward launches (k_forward2): the second step's snapshots,
+  // source values and records (the first step's are snap_e / snap_c,
+  // vals_t, out_t)
+  void *snap_e2, *snap_c2;
+  const float *vals_t2;
+  float *out_t2;
 };
 
 // TMA tensor maps of one forward launch (the input buffer set and model).
@@ -168,6 +175,22 @@ enum AdjMap {
 struct AdjMaps {
   CUtensorMap map[kAdjMaps];
 };
+
+// TMA tensor maps of one two-step forward launch (k_forward2).  Boxes are one
+// row high and 128 wide from the walk's first column x0 - H (H the x halo):
+//   kM2E, kM2HZ, kM2HX  Ey (row r), Hz (row r - 2P + 1), Hx (row r - P)
+//   kM2MD / kM2CB  Ca and Cb as one pair box when md_pair, else two boxes
+//   kM2MXH / kM2MXE  x-band memories, a whole band row (2*Wx)
+//   kM2MZH / kM2MZE  z-band memories
+enum Fwd2Map { kM2E = 0, kM2HZ, kM2HX, kM2MD, kM2CB, kM2MXH, kM2MXE, kM2MZH, kM2MZE, kFwd2Maps };
+struct Fwd2Maps {
+  CUtensorMap map[kFwd2Maps];
+};
+// Two-step forward: columns of x halo on each side of the owned strip, and
+// the owned strip width (the walk covers 128 columns).  The halo holds the
+// 4P - 2 columns two steps consume, rounded up to whole float4s.
+__host__ __device__ constexpr int fwd2_halo(int P) { return P <= 2 ? 8 : P == 3 ? 12 : 16; }
+__host__ __device__ constexpr int fwd2_width(int P) { return 128 - 2 * fwd2_halo(P); }
 
 // Rows [ya, yb) of row chunk k.
 __host__ __device__ inline void chunk_rows(const Geom &g, int k, int *ya, int *yb) {
@@ -277,6 +300,13 @@ cudaError_t launch_dependent(void (*kern)(KArgs...), int grid, int block, size_t
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// two-step forward (steps t and t + 1 in one launch): scalar Cq, orders 2-6,
+// no Born term; store as in launch_forward (both steps' snapshots)
+cudaError_t launch_forward2(const Fwd2Maps &m, const StepArgs &a, int order, int store,
+                            bool batched, int grid, cudaStream_t st);
+void forward2_layout(int order, int Wx, StepArgs *a, size_t *smem_bytes);
+int forward2_slots_per_sm(int order, int Wx);
+bool forward2_supported(int order);
 // stencil launchers (mw_stencil.cu); return a cudaError_t
 // born: kStoreNone, or the background snapshots' kind for the Born forward
 // (then store must be kStoreNone)

@@ -196,19 +196,20 @@ __device__ __forceinline__ void fix_sample(const EntrySet &e, int s, const Curso
 // [lo, hi) the item owns.  Outside the walk loop, so the walk's code is
 // untouched by them.
 __device__ __forceinline__ void fix_item(const StepArgs &a, int s, int ya, int yb, int lo, int hi,
-                                         float *field, int nx, int lane) {
+                                         float *field, int nx, int lane, const float *vals_t,
+                                         float *out_t) {
   Cursor ca = cursor_at(a.ea, s, ya), cb = cursor_at(a.eb, s, ya);
   while (ca.row < yb || cb.row < yb) {
     const int y = ca.row < cb.row ? ca.row : cb.row;
     float *row = field + (int64_t)y * nx;
     __syncwarp();
     if (y == ca.row) {
-      if (a.vals_t) fix_inject(a.ea, s, ca, a.vals_t, lo, hi, row, lane);
+      if (vals_t) fix_inject(a.ea, s, ca, vals_t, lo, hi, row, lane);
       cursor_next(a.ea, s, ca);
       __syncwarp();
     }
     if (y == cb.row) {
-      if (a.out_t) fix_sample(a.eb, s, cb, a.out_t, lo, hi, row, lane);
+      if (out_t) fix_sample(a.eb, s, cb, out_t, lo, hi, row, lane);
       cursor_next(a.eb, s, cb);
     }
   }
@@ -611,7 +612,7 @@ __global__ void __launch_bounds__(128, BORN != kStoreNone ? 3 : (P <= 3 ? 5 : 4)
     if (!ok) return;
     // this step's sources, then its receivers, in the item's cells
     fix_item(a, it.s, it.ya, it.yb, it.x0, min(it.x0 + g.strip_cols, g.nx),
-             a.out.ey + (int64_t)it.s * g.numel, g.nx, lane);
+             a.out.ey + (int64_t)it.s * g.numel, g.nx, lane, a.vals_t, a.out_t);
   }
 }
 
@@ -1033,7 +1034,522 @@ __global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_c
     if (!ok) return;
     // the next step's residuals, then its source gradient, in the item's cells
     fix_item(a, it.s, it.ya, it.yb, it.x0, min(it.x0 + g.strip_cols, g.nx),
-             a.out.ey + (int64_t)it.s * g.numel, g.nx, lane);
+             a.out.ey + (int64_t)it.s * g.numel, g.nx, lane, a.vals_t, a.out_t);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// two-step forward (temporal blocking): steps t and t + 1 in one walk, so the
+// state is read and written once per two steps.
+//
+// Iteration i of an item's walk (row r = r0 + i) stages row r of Ey (step-t
+// input), row y1 = r - 2P + 1 of Hz, row h1 = r - P of Hx and the Ca / Cb rows
+// of the two E updates, and computes
+//   step t:      Hx1(h1), then Hz1(y1) and E1(y1)
+//   step t + 1:  Hx2(y1 - P), then Hz2(y2) and E2(y2), y2 = y1 - 2P + 1.
+// Lane l holds the float4 at column xb + 4l, xb = x0 - H; every x window comes
+// from the neighbouring lanes (shuffles), so each level loses a few columns
+// at the warp's edges and the halo H covers the 4P - 2 columns that two
+// steps consume on each side.  Register queues of 2P rows hold Ey, Hx1, E1,
+// Hx2 (the z-stencils) and Hz1 (Hz2 starts from it 2P - 1 rows later); band
+// items carry the step-t CPML memories to step t + 1 in per-warp shared
+// rings.  Every update is that of k_forward, operation for operation, so the
+// two steps give the bits two k_forward launches give.
+
+// stage slots (floats): Ey row r, Hz row y1, Hx row h1, Ca / Cb rows y1 and
+// y2 (pairs of 128); the band slots follow at host-given offsets
+constexpr int kF2_E = 0, kF2_HZ = 128, kF2_HX = 256, kF2_MD1 = 384, kF2_MD2 = 640,
+              kF2_FIXED = 896;
+
+// x window w[0..12) of columns c - 4 .. c + 8 (c this lane's first column)
+// from lanes l - 1, l, l + 1; only the entries [LO, HI] the stencil reads.
+template <int LO, int HI>
+__device__ __forceinline__ void win_lanes(const F4 &v, float w[12]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    w[4 + j] = v.v[j];
+    w[j] = j >= LO ? __shfl_up_sync(kFull, v.v[j], 1) : 0.f;
+    w[8 + j] = 8 + j <= HI ? __shfl_down_sync(kFull, v.v[j], 1) : 0.f;
+  }
+}
+
+// Sources of active row c.a added into the float4 v of every lane whose
+// columns [xb + 4l, xb + 4l + 4) hold one (entries of one cell added up first,
+// in index order).  A serial loop: source rows hold few entries.
+__device__ __forceinline__ void inject_lanes(const EntrySet &e, int s, const Cursor &c,
+                                             const float *vals_t, int xb, int lane, F4 &v) {
+  const int *ab = e.abeg + (int64_t)s * (e.n + 1);
+  const int j0 = __ldg(ab + c.a), j1 = __ldg(ab + c.a + 1);
+  const int4 *en = e.ent + (int64_t)s * e.n;
+  const float *vs = vals_t + (int64_t)s * e.n;
+  for (int j = j0; j < j1; ++j) {
+    const int4 q = __ldg(en + j);
+    const int d = q.y - xb;
+    if (q.w == 0 || d < 0 || d >= 128) continue;
+    float val = __ldg(vs + q.z);
+    for (int u = 1; u < q.w; ++u) val += __ldg(vs + __ldg(en + j + u).z);
+    if (lane == (d >> 2)) {
+      const int k = d & 3;
+      if (k == 0) v.v[0] += val;
+      else if (k == 1) v.v[1] += val;
+      else if (k == 2) v.v[2] += val;
+      else v.v[3] += val;
+    }
+  }
+}
+// Receivers of active row c.a in the columns [lo, hi): the warp's row v goes
+// to the shared row `buf` (xb at offset 0), then one lane per entry reads it.
+__device__ __forceinline__ void sample_lanes(const EntrySet &e, int s, const Cursor &c,
+                                             float *out_t, int xb, int lo, int hi, uint32_t buf,
+                                             int lane, const F4 &v) {
+  sts4s(buf + 16 * lane, v);
+  __syncwarp();
+  const int *ab = e.abeg + (int64_t)s * (e.n + 1);
+  const int j0 = __ldg(ab + c.a), j1 = __ldg(ab + c.a + 1);
+  const int4 *en = e.ent + (int64_t)s * e.n;
+  for (int j = j0 + lane; j < j1; j += 32) {
+    const int4 q = __ldg(en + j);
+    if (q.y >= lo && q.y < hi) {
+      float x;
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x) : "r"(buf + 4u * (uint32_t)(q.y - xb)) : "memory");
+      out_t[(int64_t)s * e.n + q.z] = x;
+    }
+  }
+  __syncwarp();
+}
+
+template <int P>
+__device__ __forceinline__ bool make_item2(const Geom &g, int item, bool batched, Item &it) {
+  constexpr int H = fwd2_halo(P), W = fwd2_width(P);
+  int strip, chunk;
+  item_coords(g, item, &it.s, &strip, &chunk);
+  it.sm = batched ? it.s : 0;
+  it.x0 = strip * W;
+  chunk_rows(g, chunk, &it.ya, &it.yb);
+  it.r0 = it.ya - (4 * P - 2);
+  it.n_it = (it.yb - it.ya) + 8 * P - 4;
+  const bool near_x = it.x0 - H - 4 < g.Wx || it.x0 + W + H + 4 > g.nx - g.Wx;
+  it.xb = g.Wx > 0 && near_x;
+  it.edge = near_x || (g.Wz > 0 && (it.r0 < g.Wz || it.r0 + it.n_it > g.ny - g.Wz));
+  it.hx_lo = it.hx_hi = 0;
+  return it.ya < it.yb;
+}
+
+struct Fwd2Warp {
+  uint32_t bars, stage0, carry;
+  uint32_t stage_bytes;
+  uint32_t ca_o, cb_o;  // byte offsets of Ca / Cb within a stage's Ca / Cb slot
+  int lane;
+  Ring ring;
+};
+
+template <int P, bool BAND>
+__device__ __forceinline__ void md2_issue(const Fwd2Maps &m, const StepArgs &a, const Item &it,
+                                          int x, int y, uint32_t dst, uint32_t bar) {
+  if (a.md_pair) {
+    tma4s(dst, &m.map[kM2MD], x, y, it.sm, 0, bar);
+  } else {
+    tma3s(dst, &m.map[kM2MD], x, y, it.sm, bar);
+    tma3s(dst + 128 * 4, &m.map[kM2CB], x, y, it.sm, bar);
+  }
+}
+
+// Loads of iteration i (lane 0): Ey row r; Hx row h1 (from iteration 2P - 1);
+// Hz row y1 and Ca / Cb row y1 (from 4P - 2, rows inside the array); Ca / Cb
+// row y2 (from 8P - 4); band items add the memories the step-t updates read
+// (z band: Hx nodes row h1, E nodes row y1; x band: rows y1).
+template <int P, bool BAND>
+__device__ __forceinline__ void fwd2_issue(const Fwd2Maps &m, const StepArgs &a, const Item &it,
+                                           int i, uint32_t st, uint32_t bar) {
+  constexpr int H = fwd2_halo(P);
+  const int xb = it.x0 - H, ny = a.g.ny;
+  const int r = it.r0 + i, y1 = r - 2 * P + 1, y2 = y1 - 2 * P + 1, h1 = r - P;
+  const bool hx1 = i >= 2 * P - 1 && h1 >= 0 && h1 < ny;
+  const bool e1 = i >= 4 * P - 2 && y1 >= 0 && y1 < ny;
+  const bool e2 = i >= 8 * P - 4;
+  uint32_t bytes = 128 * 4;
+  if (hx1) bytes += 128 * 4;
+  if (e1) bytes += 3 * 128 * 4;
+  if (e2) bytes += 2 * 128 * 4;
+  int zh = -1, ze = -1;
+  if constexpr (BAND) {
+    if (hx1) zh = zband_row(h1, ny, a.g.Wz);
+    if (e1) ze = zband_row(y1, ny, a.g.Wz);
+    if (zh >= 0) bytes += 128 * 4;
+    if (ze >= 0) bytes += 128 * 4;
+    if (it.xb && e1) bytes += 2 * (uint32_t)a.band_box_floats * 4;
+  }
+  expect_tx_s(bar, bytes);
+  fence_proxy_async();
+  tma3s(st + kF2_E * 4, &m.map[kM2E], xb, r, it.s, bar);
+  if (hx1) tma3s(st + kF2_HX * 4, &m.map[kM2HX], xb, h1, it.s, bar);
+  if (e1) {
+    tma3s(st + kF2_HZ * 4, &m.map[kM2HZ], xb, y1, it.s, bar);
+    md2_issue<P, BAND>(m, a, it, xb, y1, st + kF2_MD1 * 4, bar);
+  }
+  if (e2) md2_issue<P, BAND>(m, a, it, xb, y2, st + kF2_MD2 * 4, bar);
+  if constexpr (BAND) {
+    if (zh >= 0) tma3s(st + a.fo[kFoMzh] * 4, &m.map[kM2MZH], xb, zh, it.s, bar);
+    if (ze >= 0) tma3s(st + a.fo[kFoMze] * 4, &m.map[kM2MZE], xb, ze, it.s, bar);
+    if (it.xb && e1) {
+      tma3s(st + a.fo[kFoMxh] * 4, &m.map[kM2MXH], 0, y1, it.s, bar);
+      tma3s(st + a.fo[kFoMxe] * 4, &m.map[kM2MXE], 0, y1, it.s, bar);
+    }
+  }
+}
+
+template <int P, int STORE, bool BAND>
+__device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, const Item &it,
+                                          Fwd2Warp &w, float cqs) {
+  constexpr int NQ = 2 * P;
+  constexpr int NS = 2;
+  constexpr int H = fwd2_halo(P), W = fwd2_width(P);
+  constexpr int M = NQ;  // ring-indexed queues: no moves
+  using Q = Queue<NQ, M>;
+  const int lane = w.lane;
+  const int nx = a.g.nx, ny = a.g.ny;
+  const int xb = it.x0 - H;
+  const int c = xb + 4 * lane;
+  const bool c_ok = !BAND || (c >= 0 && c < nx);
+  const bool own = lane >= H / 4 && lane < H / 4 + W / 4 && c_ok;
+  const int64_t pb = (int64_t)it.s * a.g.numel + c;
+  float *const hz_o = a.out.hz + pb;
+  float *const hx_o = a.out.hx + pb;
+  float *const ey_o = a.out.ey + pb;
+  const BandTab T{a.g.Wx, a.g.Wz};
+  const int bcol = BAND ? xband_col(c, nx, a.g.Wx) : -1;
+  const int64_t xbw = BAND ? (int64_t)it.s * ny * 2 * a.g.Wx + bcol : 0;
+  const int64_t zbw = BAND ? (int64_t)it.s * 2 * a.g.Wz * nx + c : 0;
+  // carry rings: x band at the H and E nodes (NQ band rows each), z band at
+  // the H and E nodes (NQ rows of 32 float4 each)
+  const uint32_t rxh = w.carry, rxe = rxh + NQ * a.band_ring * 4;
+  const uint32_t rzh = rxe + NQ * a.band_ring * 4, rze = rzh + NQ * 128 * 4;
+  // step-t sources into every E1 row computed, receivers of the owned rows
+  Cursor c1a = cursor_at(a.ea, it.s, it.ya - 2 * P + 1), c1b = cursor_at(a.eb, it.s, it.ya);
+
+  if (lane == 0) fwd2_issue<P, BAND>(m, a, it, 0, w.stage0 + w.ring.slot * w.stage_bytes,
+                                     w.bars + 8 * w.ring.slot);
+  F4 eq[NQ], hq[NQ], e1q[NQ], h2q[NQ], z1q[NQ];
+#pragma unroll
+  for (int k = 0; k < NQ; ++k) eq[k] = hq[k] = e1q[k] = h2q[k] = z1q[k] = zero4();
+
+  for (int i0 = 0; i0 < it.n_it; i0 += M) {
+#pragma unroll
+    for (int u = 0; u < M; ++u) {
+      const int i = i0 + u;
+      if (i < it.n_it) {
+        if (i + 1 < it.n_it && lane == 0) {
+          const int ps = w.ring.slot ^ 1;
+          fwd2_issue<P, BAND>(m, a, it, i + 1, w.stage0 + ps * w.stage_bytes, w.bars + 8 * ps);
+        }
+        if (!mbar_wait_s(w.bars + 8 * w.ring.slot, w.ring.phase)) {
+          give_up_s<1>(a.flags, w.bars, w.ring, i, it.n_it, lane);
+          return false;
+        }
+        const uint32_t st = w.stage0 + w.ring.slot * w.stage_bytes;
+        const int r = it.r0 + i, y1 = r - 2 * P + 1, y2 = y1 - 2 * P + 1;
+        const int h1 = r - P, h2 = y1 - P;
+        const bool hx1 = i >= 2 * P - 1 && h1 >= 0 && h1 < ny;
+        const bool e1 = i >= 4 * P - 2 && y1 >= 0 && y1 < ny;
+        const bool e1_own = y1 >= it.ya && y1 < it.yb;
+        const bool hx2 = i >= 6 * P - 3 && h2 >= 0 && h2 < ny;
+        const bool hx2_own = h2 >= it.ya && h2 < it.yb;
+        const bool e2 = i >= 8 * P - 4;
+
+        eq[Q::at(u, 0)] = lds4s(st + kF2_E * 4 + 16 * lane);
+
+        // ---- step t: Hx1, row h1 (z-stencil of the Ey queue)
+        {
+          const F4 hx_old = lds4s(st + kF2_HX * 4 + 16 * lane);
+          F4 d;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float s = 0.f;
+#pragma unroll
+            for (int k = 1; k <= P; ++k)
+              s = fmaf(a.c.cy[k - 1], eq[Q::at(u, P - k)].v[q] - eq[Q::at(u, P + k - 1)].v[q], s);
+            d.v[q] = s;
+          }
+          if constexpr (BAND) {
+            const int zr = hx1 ? zband_row(h1, ny, a.g.Wz) : -1;
+            if (zr >= 0) {
+              F4 mz = lds4s(st + a.fo[kFoMzh] * 4 + 16 * lane);
+              const float ayh = __ldg(a.bt + T.z(3) + zr), byh = __ldg(a.bt + T.z(4) + zr);
+              const float rkyh = __ldg(a.bt + T.z(5) + zr);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mz.v[q] = fmaf(byh, mz.v[q], ayh * d.v[q]);
+                d.v[q] = fmaf(d.v[q], rkyh, mz.v[q]);
+              }
+              sts4s(rzh + Q::at(u, 0) * 512 + 16 * lane, mz);
+            }
+          }
+          F4 hn;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) hn.v[q] = fmaf(-cqs, d.v[q], hx_old.v[q]);
+          hq[Q::at(u, 0)] = hx1 ? hn : zero4();
+        }
+
+        // ---- step t: Hz1 and E1, row y1
+        F4 hz1 = zero4(), e1v = zero4();
+        if (e1) {
+          const F4 &e0 = eq[Q::at(u, NQ - 1)];
+          {
+            float wv[12];
+            win_lanes<5 - P, 7 + P>(e0, wv);
+            const F4 hz_old = lds4s(st + kF2_HZ * 4 + 16 * lane);
+            if (!BAND || bcol < 0) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                hz1.v[q] = fmaf(cqs, d_half<P>(wv, q, a.c.cx), hz_old.v[q]);
+            } else {
+              F4 mn = lds4s(st + (a.fo[kFoMxh] + bcol) * 4);
+              const F4 ah = ld4(a.bt + T.x(3) + bcol), bh = ld4(a.bt + T.x(4) + bcol);
+              const F4 rk = ld4(a.bt + T.x(5) + bcol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float d = d_half<P>(wv, q, a.c.cx);
+                mn.v[q] = fmaf(bh.v[q], mn.v[q], ah.v[q] * d);
+                hz1.v[q] = fmaf(cqs, fmaf(d, rk.v[q], mn.v[q]), hz_old.v[q]);
+              }
+              sts4s(rxh + (Q::at(u, 0) * a.band_ring + bcol) * 4, mn);
+            }
+            if (!c_ok) hz1 = zero4();
+          }
+          float wh[12];
+          win_lanes<4 - P, 6 + P>(hz1, wh);
+          const F4 ca4 = lds4s(st + kF2_MD1 * 4 + w.ca_o + 16 * lane);
+          const F4 cb4 = lds4s(st + kF2_MD1 * 4 + w.cb_o + 16 * lane);
+          F4 cx, cz;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            cx.v[q] = d_int<P>(wh, q, a.c.cx);
+            float s = 0.f;
+#pragma unroll
+            for (int k = 1; k <= P; ++k)
+              s = fmaf(a.c.cy[k - 1], hq[Q::at(u, P - k)].v[q] - hq[Q::at(u, P - 1 + k)].v[q], s);
+            cz.v[q] = s;
+          }
+          if constexpr (BAND) {
+            if (bcol >= 0) {
+              F4 mx = lds4s(st + (a.fo[kFoMxe] + bcol) * 4);
+              const F4 ax = ld4(a.bt + T.x(0) + bcol), bx = ld4(a.bt + T.x(1) + bcol);
+              const F4 rk = ld4(a.bt + T.x(2) + bcol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mx.v[q] = fmaf(bx.v[q], mx.v[q], ax.v[q] * cx.v[q]);
+                cx.v[q] = fmaf(cx.v[q], rk.v[q], mx.v[q]);
+              }
+              sts4s(rxe + (Q::at(u, 0) * a.band_ring + bcol) * 4, mx);
+            }
+            const int zr = zband_row(y1, ny, a.g.Wz);
+            if (zr >= 0) {
+              F4 mz = lds4s(st + a.fo[kFoMze] * 4 + 16 * lane);
+              const float ay = __ldg(a.bt + T.z(0) + zr), by = __ldg(a.bt + T.z(1) + zr);
+              const float rky = __ldg(a.bt + T.z(2) + zr);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mz.v[q] = fmaf(by, mz.v[q], ay * cz.v[q]);
+                cz.v[q] = fmaf(cz.v[q], rky, mz.v[q]);
+              }
+              sts4s(rze + Q::at(u, 0) * 512 + 16 * lane, mz);
+            }
+          }
+          F4 curl, en;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            curl.v[q] = cx.v[q] - cz.v[q];
+            en.v[q] = fmaf(ca4.v[q], e0.v[q], cb4.v[q] * curl.v[q]);
+          }
+          if constexpr (STORE != kStoreNone) {  // step t's snapshots
+            const int64_t so = ((int64_t)it.s * ny + y1) * a.snap_pitch + c;
+            snap_store_p<STORE>(own && e1_own, a.snap_e, so, e0);
+            if constexpr (STORE != kStoreEy) snap_store_p<STORE>(own && e1_own, a.snap_c, so, curl);
+          }
+          // step t's sources (every lane holding the cell), then its receivers
+          if (y1 == c1a.row) {
+            if (a.vals_t) inject_lanes(a.ea, it.s, c1a, a.vals_t, xb, lane, en);
+            cursor_next(a.ea, it.s, c1a);
+          }
+          if (y1 == c1b.row) {
+            if (a.out_t && y1 < it.yb)
+              sample_lanes(a.eb, it.s, c1b, a.out_t, xb, it.x0, min(it.x0 + W, nx),
+                           st + kF2_E * 4, lane, en);
+            cursor_next(a.eb, it.s, c1b);
+          }
+          e1v = c_ok ? en : zero4();
+        }
+        z1q[Q::at(u, 0)] = hz1;
+        e1q[Q::at(u, 0)] = e1v;
+
+        // ---- step t + 1: Hx2, row h2 (z-stencil of the E1 queue)
+        {
+          const F4 &hx_old = hq[Q::at(u, NQ - 1)];
+          F4 d;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float s = 0.f;
+#pragma unroll
+            for (int k = 1; k <= P; ++k)
+              s = fmaf(a.c.cy[k - 1], e1q[Q::at(u, P - k)].v[q] - e1q[Q::at(u, P + k - 1)].v[q],
+                       s);
+            d.v[q] = s;
+          }
+          if constexpr (BAND) {
+            const int zr = hx2 ? zband_row(h2, ny, a.g.Wz) : -1;
+            if (zr >= 0) {
+              F4 mz = lds4s(rzh + Q::at(u, NQ - 1) * 512 + 16 * lane);
+              const float ayh = __ldg(a.bt + T.z(3) + zr), byh = __ldg(a.bt + T.z(4) + zr);
+              const float rkyh = __ldg(a.bt + T.z(5) + zr);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mz.v[q] = fmaf(byh, mz.v[q], ayh * d.v[q]);
+                d.v[q] = fmaf(d.v[q], rkyh, mz.v[q]);
+              }
+              st4p(own && hx2_own, a.out.mzh_node + zbw + (int64_t)zr * nx, mz);
+            }
+          }
+          F4 hn;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) hn.v[q] = fmaf(-cqs, d.v[q], hx_old.v[q]);
+          h2q[Q::at(u, 0)] = hx2 ? hn : zero4();
+          st4p(own && hx2_own, hx_o + (int64_t)h2 * nx, hn);
+        }
+
+        // ---- step t + 1: Hz2 and E2, row y2
+        if (e2) {
+          const F4 &e1o = e1q[Q::at(u, NQ - 1)];
+          const F4 &hz1o = z1q[Q::at(u, NQ - 1)];
+          F4 hz2;
+          {
+            float wv[12];
+            win_lanes<5 - P, 7 + P>(e1o, wv);
+            if (!BAND || bcol < 0) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) hz2.v[q] = fmaf(cqs, d_half<P>(wv, q, a.c.cx), hz1o.v[q]);
+            } else {
+              F4 mn = lds4s(rxh + (Q::at(u, NQ - 1) * a.band_ring + bcol) * 4);
+              const F4 ah = ld4(a.bt + T.x(3) + bcol), bh = ld4(a.bt + T.x(4) + bcol);
+              const F4 rk = ld4(a.bt + T.x(5) + bcol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float d = d_half<P>(wv, q, a.c.cx);
+                mn.v[q] = fmaf(bh.v[q], mn.v[q], ah.v[q] * d);
+                hz2.v[q] = fmaf(cqs, fmaf(d, rk.v[q], mn.v[q]), hz1o.v[q]);
+              }
+              st4p(own, a.out.mxh_node + xbw + (int64_t)y2 * 2 * a.g.Wx, mn);
+            }
+            st4p(own, hz_o + (int64_t)y2 * nx, hz2);
+            if (!c_ok) hz2 = zero4();
+          }
+          float wh[12];
+          win_lanes<4 - P, 6 + P>(hz2, wh);
+          const F4 ca4 = lds4s(st + kF2_MD2 * 4 + w.ca_o + 16 * lane);
+          const F4 cb4 = lds4s(st + kF2_MD2 * 4 + w.cb_o + 16 * lane);
+          F4 cx, cz;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            cx.v[q] = d_int<P>(wh, q, a.c.cx);
+            float s = 0.f;
+#pragma unroll
+            for (int k = 1; k <= P; ++k)
+              s = fmaf(a.c.cy[k - 1], h2q[Q::at(u, P - k)].v[q] - h2q[Q::at(u, P - 1 + k)].v[q], s);
+            cz.v[q] = s;
+          }
+          if constexpr (BAND) {
+            if (bcol >= 0) {
+              F4 mx = lds4s(rxe + (Q::at(u, NQ - 1) * a.band_ring + bcol) * 4);
+              const F4 ax = ld4(a.bt + T.x(0) + bcol), bx = ld4(a.bt + T.x(1) + bcol);
+              const F4 rk = ld4(a.bt + T.x(2) + bcol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mx.v[q] = fmaf(bx.v[q], mx.v[q], ax.v[q] * cx.v[q]);
+                cx.v[q] = fmaf(cx.v[q], rk.v[q], mx.v[q]);
+              }
+              st4p(own, a.out.mxe_node + xbw + (int64_t)y2 * 2 * a.g.Wx, mx);
+            }
+            const int zr = zband_row(y2, ny, a.g.Wz);
+            if (zr >= 0) {
+              F4 mz = lds4s(rze + Q::at(u, NQ - 1) * 512 + 16 * lane);
+              const float ay = __ldg(a.bt + T.z(0) + zr), by = __ldg(a.bt + T.z(1) + zr);
+              const float rky = __ldg(a.bt + T.z(2) + zr);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                mz.v[q] = fmaf(by, mz.v[q], ay * cz.v[q]);
+                cz.v[q] = fmaf(cz.v[q], rky, mz.v[q]);
+              }
+              st4p(own, a.out.mze_node + zbw + (int64_t)zr * nx, mz);
+            }
+          }
+          F4 curl, en;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            curl.v[q] = cx.v[q] - cz.v[q];
+            en.v[q] = fmaf(ca4.v[q], e1o.v[q], cb4.v[q] * curl.v[q]);
+          }
+          if constexpr (STORE != kStoreNone) {  // step t + 1's snapshots
+            const int64_t so = ((int64_t)it.s * ny + y2) * a.snap_pitch + c;
+            snap_store_p<STORE>(own, a.snap_e2, so, e1o);
+            if constexpr (STORE != kStoreEy) snap_store_p<STORE>(own, a.snap_c2, so, curl);
+          }
+          st4p(own, ey_o + (int64_t)y2 * nx, en);
+        }
+        __syncwarp();
+        w.ring.next(NS);
+      }
+    }
+  }
+  return true;
+}
+
+template <int P, int STORE>
+__global__ void __launch_bounds__(128, 3)
+    k_forward2(const __grid_constant__ Fwd2Maps m, const StepArgs a, const int batched) {
+  constexpr int NS = 2;
+  extern __shared__ __align__(128) float smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 127u) & ~127u;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  Fwd2Warp w;
+  w.lane = lane;
+  w.bars = base + warp * NS * 8;
+  w.stage_bytes = (uint32_t)a.stage_floats * 4;
+  w.stage0 = base + 128 + warp * a.warp_floats * 4;
+  w.carry = w.stage0 + NS * w.stage_bytes;
+  // a pair box is [Ca][Cb] (or [Cb][Ca] when Cb lies first); two boxes put
+  // Ca first, each 128 wide
+  w.ca_o = a.md_pair && a.md_swap ? 512 : 0;
+  w.cb_o = a.md_pair && a.md_swap ? 0 : 512;
+  w.ring = Ring{0, 0u};
+  const Geom &g = a.g;
+  const int n_items = g.S * g.n_strips * g.n_chunks;
+  grid_dep_launch();
+  if (lane == 0) {
+    for (int k = 0; k < NS; ++k)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(w.bars + 8 * k), "r"(1)
+                   : "memory");
+    fence_mbar_init();
+  }
+  __syncwarp();
+  grid_dep_wait();  // everything below reads what earlier kernels wrote
+  if (__any_sync(kFull, *reinterpret_cast<volatile int *>(a.flags + kFlagTimeout) != 0)) return;
+  const float cqs = __ldg(a.cq);
+  int *ctr = a.flags + kCtrBase + a.ctr_slot;
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.flags[kCtrBase + (a.ctr_slot ^ 1)] = 0;
+
+  for (;;) {
+    int item = 0;
+    if (lane == 0) item = atomicAdd(ctr, 1);
+    item = __shfl_sync(kFull, item, 0);
+    if (item >= n_items) break;
+    Item it;
+    if (!make_item2<P>(g, item, batched != 0, it)) continue;
+    const bool ok = it.edge ? fwd2_walk<P, STORE, true>(m, a, it, w, cqs)
+                            : fwd2_walk<P, STORE, false>(m, a, it, w, cqs);
+    if (!ok) return;
+    // step t + 1's sources, then its receivers, in the item's cells
+    fix_item(a, it.s, it.ya, it.yb, it.x0, min(it.x0 + fwd2_width(P), g.nx),
+             a.out.ey + (int64_t)it.s * g.numel, g.nx, lane, a.vals_t2, a.out_t2);
   }
 }
 
@@ -1147,6 +1663,62 @@ cudaError_t adj_t(const AdjMaps &m, const StepArgs &a, bool batched, bool cq_arr
   return cudaGetLastError();
 }
 
+// Two-step forward stage: the fixed slots, then (with a band) the z-band
+// memory rows of the H and E nodes and the two x-band memory rows.  The warp
+// area adds the band items' carry rings: NQ x-band rows at each node, NQ
+// rows of 128 floats at each z-band node.
+template <int P>
+void fwd2_layout_t(int Wx, StepArgs *a, size_t *smem) {
+  const int bw = Wx > 0 ? ((2 * Wx + 31) / 32) * 32 : 0;
+  int o = kF2_FIXED;
+  for (int k = 0; k < kFoCount; ++k) a->fo[k] = 0;
+  if (Wx > 0) {
+    a->fo[kFoMzh] = o;
+    a->fo[kFoMze] = o + 128;
+    a->fo[kFoMxh] = o + 256;
+    a->fo[kFoMxe] = o + 256 + bw;
+    o += 256 + 2 * bw;
+  }
+  const int carry = Wx > 0 ? 2 * (2 * P) * bw + 2 * (2 * P) * 128 : 0;
+  int wf = 2 * o + carry;
+  wf = ((wf + 31) / 32) * 32;
+  a->stage_floats = o;
+  a->warp_floats = wf;
+  a->band_box_floats = 2 * Wx;
+  a->band_ring = bw;
+  *smem = (size_t)(32 + kWarpsPerCta * wf) * sizeof(float) + 128;
+}
+
+template <int P, int STORE>
+std::atomic<uint64_t> &fwd2_smem_flag() {
+  static std::atomic<uint64_t> f{0};
+  return f;
+}
+
+template <int P, int STORE>
+cudaError_t fwd2_t(const Fwd2Maps &m, const StepArgs &a, bool batched, int grid, cudaStream_t st) {
+  const size_t smem = (size_t)(32 + kWarpsPerCta * a.warp_floats) * sizeof(float) + 128;
+  allow_big_smem(k_forward2<P, STORE>, fwd2_smem_flag<P, STORE>());
+  const cudaError_t e = launch_dependent(k_forward2<P, STORE>, grid, 128, smem, st, m, a,
+                                         batched ? 1 : 0);
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <int P>
+cudaError_t fwd2_store(const Fwd2Maps &m, const StepArgs &a, int store, bool batched, int grid,
+                       cudaStream_t st) {
+  switch (store) {
+    case kStoreNone: return fwd2_t<P, kStoreNone>(m, a, batched, grid, st);
+    case kStoreF32: return fwd2_t<P, kStoreF32>(m, a, batched, grid, st);
+    case kStoreBF16: return fwd2_t<P, kStoreBF16>(m, a, batched, grid, st);
+    case kStoreFP8: return fwd2_t<P, kStoreFP8>(m, a, batched, grid, st);
+    case kStoreEy: return fwd2_t<P, kStoreEy>(m, a, batched, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int P>
 cudaError_t fwd_store(const FwdMaps &m, const StepArgs &a, int store, int born, bool batched,
                       bool cq_arr, int grid, cudaStream_t st) {
@@ -1206,6 +1778,15 @@ int slots_t(bool adjoint, int Wx, bool cq_arr) {
          kWarpsPerCta;
 }
 
+template <int P>
+int fwd2_slots_t(int Wx) {
+  size_t smem;
+  StepArgs a{};
+  fwd2_layout_t<P>(Wx, &a, &smem);
+  return occupancy(k_forward2<P, kStoreF32>, 128, smem, fwd2_smem_flag<P, kStoreF32>()) *
+         kWarpsPerCta;
+}
+
 }  // namespace
 
 cudaError_t launch_forward(const FwdMaps &m, const StepArgs &a, int order, int store, int born,
@@ -1228,6 +1809,34 @@ cudaError_t launch_adjoint(const AdjMaps &m, const StepArgs &a, int order, int s
     case 8: return adj_snap<4>(m, a, snap, batched, cq_array, grid, st);
   }
   return cudaErrorInvalidValue;
+}
+
+bool forward2_supported(int order) { return order >= 2 && order <= 6; }
+
+cudaError_t launch_forward2(const Fwd2Maps &m, const StepArgs &a, int order, int store,
+                            bool batched, int grid, cudaStream_t st) {
+  switch (order) {
+    case 2: return fwd2_store<1>(m, a, store, batched, grid, st);
+    case 4: return fwd2_store<2>(m, a, store, batched, grid, st);
+    case 6: return fwd2_store<3>(m, a, store, batched, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+void forward2_layout(int order, int Wx, StepArgs *a, size_t *smem) {
+  switch (order) {
+    case 2: fwd2_layout_t<1>(Wx, a, smem); return;
+    case 4: fwd2_layout_t<2>(Wx, a, smem); return;
+    default: fwd2_layout_t<3>(Wx, a, smem); return;
+  }
+}
+
+int forward2_slots_per_sm(int order, int Wx) {
+  switch (order) {
+    case 2: return fwd2_slots_t<1>(Wx);
+    case 4: return fwd2_slots_t<2>(Wx);
+    default: return fwd2_slots_t<3>(Wx);
+  }
 }
 
 int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array) {

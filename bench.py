@@ -91,11 +91,11 @@ def dist_env():
 CKPT_MODES = ("ckpt", "ckpt_ey")
 
 
-def sweep_bytes_per_cell(wl, S, nt=None):
+def sweep_bytes_per_cell(wl, S, nt=None, one_pass=False):
     """Bytes per cell-update of the whole sweep: each pass weighted by the
     share of the steps it runs (the replay skips the forward-stored tail,
     whose forward steps write the snapshot instead)."""
-    b = alg_bytes(wl, S)
+    b = alg_bytes(wl, S, one_pass)
     if wl.snapshot not in CKPT_MODES:
         return sum(b.values())
     nt = nt or wl.nt
@@ -104,7 +104,13 @@ def sweep_bytes_per_cell(wl, S, nt=None):
     return b["forward"] + tail * sb + (1.0 - tail) * b["replay"] + b["adjoint"]
 
 
-def alg_bytes(wl, S):
+def two_step(wl):
+    """Whether the library runs the workload's forward passes two steps per
+    launch (orders 2-6 with a scalar Cq, unless MW_NO_TWO_STEP=1)."""
+    return wl.order <= 6 and os.environ.get("MW_NO_TWO_STEP") != "1"
+
+
+def alg_bytes(wl, S, one_pass=False):
     """Bytes per cell-update of each pass of the workload's sweep (fp32 fields):
     state read + write 24 B, Ca and Cb (shared by the shots unless the model is
     batched), the CPML band memories, snapshot write / read (8, 4 or 2 B), the
@@ -112,27 +118,45 @@ def alg_bytes(wl, S):
     beyond the state traffic: the step that produces one writes it into its
     slot and the next step (and later the replay) reads it there.  With the E
     snapshot alone ("ckpt_ey") the replay writes and the adjoint reads 4 B of
-    snapshot instead of 8."""
+    snapshot instead of 8.  Forward passes that take two steps per launch read
+    and write the state and the band memories once per two steps (12 B of
+    state per cell-update) and still read Ca, Cb for each step; one_pass gives
+    the one-step-per-pass figures."""
     band = 16.0 * (2.0 * wl.n_pml / wl.nx + 2.0 * wl.n_pml / wl.ny)
     model = 8.0 if wl.batched else 8.0 / S
     base = 24.0 + model + band
+    fwd = 12.0 + model + band / 2.0 if (two_step(wl) and not one_pass) else base
     if wl.snapshot in CKPT_MODES:
         sb = 4.0 if wl.snapshot == "ckpt_ey" else 8.0
-        return {"forward": base, "replay": base + sb, "adjoint": base + sb + 16.0}
+        return {"forward": fwd, "replay": fwd + sb, "adjoint": base + sb + 16.0}
     if wl.snapshot == "none":
-        return {"forward": base}
+        return {"forward": fwd}
     sb = {"fp32": 8.0, "bf16": 4.0, "fp8": 2.0}[wl.snapshot]
-    return {"forward": base + sb, "adjoint": base + sb + 16.0}
+    return {"forward": fwd + sb, "adjoint": base + sb + 16.0}
 
 
 # the library's per-launch timing classes: 0 forward, 1 forward with snapshot
-# store, 2 adjoint; which class each pass of a sweep uses
+# store, 2 adjoint, 3 Born, 4 / 5 two-step forward launches without / with
+# snapshot store (two steps per launch); which classes each pass of a sweep
+# uses, as (one-step class, two-step class or None)
+N_CLASSES = 6
+
+
 def pass_classes(wl):
     if wl.snapshot in CKPT_MODES:
-        return {"forward": 0, "replay": 1, "adjoint": 2}
+        return {"forward": (0, 4), "replay": (1, 5), "adjoint": (2, None)}
     if wl.snapshot == "none":
-        return {"forward": 0}
-    return {"forward": 1, "adjoint": 2}
+        return {"forward": (0, 4)}
+    return {"forward": (1, 5), "adjoint": (2, None)}
+
+
+def per_step_ms(counts, ms, classes):
+    """Mean device time per step of one pass (a two-step launch counts as two
+    steps)."""
+    a, b = classes
+    n = counts[a] + (2 * counts[b] if b is not None else 0)
+    t = ms[a] + (ms[b] if b is not None else 0.0)
+    return t / max(n, 1)
 
 
 TAIL_RESERVE = 12e9  # device bytes left free beside the workspace
@@ -455,7 +479,7 @@ class Sweep:
             evs_e[k][0].record(stream)
             self.step(ev_fwd=evs_e[k][1], eager=True)
         torch.cuda.synchronize()
-        counts, ms = mwtm.profile_read(3)
+        counts, ms = mwtm.profile_read(N_CLASSES)
         mwtm.profile_enable(False)
         if world > 1:
             dist.barrier()
@@ -473,7 +497,7 @@ class Sweep:
         peak, peak_kind = measured_peaks()
         sweep_bytes = sweep_bytes_per_cell(wl, S, nt) * self.cells * steps
         sweep_frac = sweep_bytes / (total_ms / 1e3) / 1e9 / peak / world
-        launch_ms = {k: ms[c] / max(counts[c], 1) for k, c in classes.items()}
+        launch_ms = {k: per_step_ms(counts, ms, c) for k, c in classes.items()}
         top = "adjoint" if self.grad else "forward"   # the dominant kernel
         top_launch_ms = launch_ms[top]
         top_bytes = passes[top] * wl.ny * wl.nx * S
@@ -676,6 +700,9 @@ def main():
             "hbm_frac_sweep": round(m["sweep_frac"], 4),
             "alg_bytes_per_cell": {k: round(v, 3) for k, v in m["passes"].items()},
             "sweep_bytes_per_cell": round(sweep_bytes_per_cell(wl, S, nt), 3),
+            "sweep_bytes_per_cell_one_step_per_pass": round(
+                sweep_bytes_per_cell(wl, S, nt, one_pass=True), 3),
+            "forward_steps_per_launch": 2 if two_step(wl) else 1,
             "roofline": {"bound": "hbm", "kernel": m["kernel_name"],
                          "achieved": round(m["achieved"], 1),
                          "peak": m["peak"], "peak_kind": m["peak_kind"], "unit": "GB/s",

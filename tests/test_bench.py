@@ -21,26 +21,42 @@ from adjoint_state_gradients_b200 import synth  # noqa: E402
 def test_byte_model_of_the_headline_sweep():
     """Checkpoints every 64 steps with the E-alone segment: the replay writes
     and the adjoint reads 4 B of snapshot per cell-update; with the pair
-    segment 8 B.  Checkpoints add no bytes (written and read in place)."""
+    segment 8 B.  Checkpoints add no bytes (written and read in place).  One
+    step per forward launch (MW_NO_TWO_STEP=1 / one_pass)."""
     wl = synth.WORKLOADS[4]
     assert wl.snapshot == "ckpt_ey"
-    b = bench.alg_bytes(wl, wl.n_shots)
+    b = bench.alg_bytes(wl, wl.n_shots, one_pass=True)
     band = 16.0 * (2 * 40 / 2128 + 2 * 40 / 2128)
     assert b["forward"] == pytest.approx(24 + 1 + band)
     assert b["replay"] == pytest.approx(24 + 1 + band + 4)
     assert b["adjoint"] == pytest.approx(24 + 1 + band + 4 + 16)
     assert sum(b.values()) == pytest.approx(102.61, abs=0.01)
-    assert bench.pass_classes(wl) == {"forward": 0, "replay": 1, "adjoint": 2}
-    bp = bench.alg_bytes(dataclasses.replace(wl, snapshot="ckpt"), wl.n_shots)
+    assert bench.pass_classes(wl) == {"forward": (0, 4), "replay": (1, 5), "adjoint": (2, None)}
+    bp = bench.alg_bytes(dataclasses.replace(wl, snapshot="ckpt"), wl.n_shots, one_pass=True)
     assert bp["replay"] - b["replay"] == pytest.approx(4.0)
     assert bp["adjoint"] - b["adjoint"] == pytest.approx(4.0)
     assert sum(bp.values()) == pytest.approx(110.61, abs=0.01)
     # the forward-stored tail: those steps write E (4 B) and skip the replay
     assert wl.ckpt_tail == 768
     want = b["forward"] + 0.192 * 4 + 0.808 * b["replay"] + b["adjoint"]
-    assert bench.sweep_bytes_per_cell(wl, wl.n_shots) == pytest.approx(want)
-    assert bench.sweep_bytes_per_cell(dataclasses.replace(wl, ckpt_tail=0), wl.n_shots) == \
-        pytest.approx(102.61, abs=0.01)
+    assert bench.sweep_bytes_per_cell(wl, wl.n_shots, one_pass=True) == pytest.approx(want)
+    assert bench.sweep_bytes_per_cell(dataclasses.replace(wl, ckpt_tail=0), wl.n_shots,
+                                      one_pass=True) == pytest.approx(102.61, abs=0.01)
+
+
+def test_byte_model_of_two_step_forward_passes():
+    """Two steps per forward launch: the state (24 B) and the band memories
+    move once per two steps, Ca / Cb and the snapshots once per step; the
+    adjoint is unchanged."""
+    wl = synth.WORKLOADS[4]
+    one, two = bench.alg_bytes(wl, 8, one_pass=True), bench.alg_bytes(wl, 8)
+    band = 16.0 * (2 * 40 / 2128 + 2 * 40 / 2128)
+    assert bench.two_step(wl) and not bench.two_step(synth.WORKLOADS[5])
+    assert two["forward"] == pytest.approx(12 + 1 + band / 2)
+    assert two["replay"] == pytest.approx(12 + 1 + band / 2 + 4)
+    assert two["adjoint"] == one["adjoint"]
+    assert bench.alg_bytes(synth.WORKLOADS[5], 256) == bench.alg_bytes(synth.WORKLOADS[5], 256,
+                                                                       one_pass=True)
 
 
 def test_byte_model_of_the_other_storage_modes():
@@ -49,7 +65,7 @@ def test_byte_model_of_the_other_storage_modes():
     assert b3["adjoint"] - b3["forward"] == pytest.approx(16.0)   # gradient read + write
     assert set(b5) == {"forward"}
     assert b5["forward"] > 24 + 8                                  # per-shot model: 8 B per cell
-    assert bench.pass_classes(w5) == {"forward": 0}
+    assert bench.pass_classes(w5) == {"forward": (0, 4)}
 
 
 def test_oracle_sample_is_bounded():
