@@ -1204,7 +1204,10 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
   constexpr int NQ = 2 * P;
   constexpr int NS = 2;
   constexpr int H = fwd2_halo(P), W = fwd2_width(P);
-  constexpr int M = NQ;  // ring-indexed queues: no moves
+  // one iteration per loop trip (a longer unrolled body overflows the
+  // instruction cache): the register queues shift once per iteration and the
+  // carry rings rotate by a running slot
+  constexpr int M = 1;
   using Q = Queue<NQ, M>;
   const int lane = w.lane;
   const int nx = a.g.nx, ny = a.g.ny;
@@ -1229,9 +1232,11 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
 
   if (lane == 0) fwd2_issue<P, BAND>(m, a, it, 0, w.stage0 + w.ring.slot * w.stage_bytes,
                                      w.bars + 8 * w.ring.slot);
-  F4 eq[NQ], hq[NQ], e1q[NQ], h2q[NQ], z1q[NQ];
+  F4 eq[Q::kSize], hq[Q::kSize], e1q[Q::kSize], h2q[Q::kSize], z1q[Q::kSize];
 #pragma unroll
-  for (int k = 0; k < NQ; ++k) eq[k] = hq[k] = e1q[k] = h2q[k] = z1q[k] = zero4();
+  for (int k = 0; k < Q::kSize; ++k) eq[k] = hq[k] = e1q[k] = h2q[k] = z1q[k] = zero4();
+  // carry ring slots: written this iteration, written 2P - 1 iterations ago
+  int cw = 0, cr = 1;
 
   for (int i0 = 0; i0 < it.n_it; i0 += M) {
 #pragma unroll
@@ -1281,7 +1286,7 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
                 mz.v[q] = fmaf(byh, mz.v[q], ayh * d.v[q]);
                 d.v[q] = fmaf(d.v[q], rkyh, mz.v[q]);
               }
-              sts4s(rzh + Q::at(u, 0) * 512 + 16 * lane, mz);
+              sts4s(rzh + cw * 512 + 16 * lane, mz);
             }
           }
           F4 hn;
@@ -1312,7 +1317,7 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
                 mn.v[q] = fmaf(bh.v[q], mn.v[q], ah.v[q] * d);
                 hz1.v[q] = fmaf(cqs, fmaf(d, rk.v[q], mn.v[q]), hz_old.v[q]);
               }
-              sts4s(rxh + (Q::at(u, 0) * a.band_ring + bcol) * 4, mn);
+              sts4s(rxh + (cw * a.band_ring + bcol) * 4, mn);
             }
             if (!c_ok) hz1 = zero4();
           }
@@ -1340,7 +1345,7 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
                 mx.v[q] = fmaf(bx.v[q], mx.v[q], ax.v[q] * cx.v[q]);
                 cx.v[q] = fmaf(cx.v[q], rk.v[q], mx.v[q]);
               }
-              sts4s(rxe + (Q::at(u, 0) * a.band_ring + bcol) * 4, mx);
+              sts4s(rxe + (cw * a.band_ring + bcol) * 4, mx);
             }
             const int zr = zband_row(y1, ny, a.g.Wz);
             if (zr >= 0) {
@@ -1352,7 +1357,7 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
                 mz.v[q] = fmaf(by, mz.v[q], ay * cz.v[q]);
                 cz.v[q] = fmaf(cz.v[q], rky, mz.v[q]);
               }
-              sts4s(rze + Q::at(u, 0) * 512 + 16 * lane, mz);
+              sts4s(rze + cw * 512 + 16 * lane, mz);
             }
           }
           F4 curl, en;
@@ -1398,7 +1403,7 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
           if constexpr (BAND) {
             const int zr = hx2 ? zband_row(h2, ny, a.g.Wz) : -1;
             if (zr >= 0) {
-              F4 mz = lds4s(rzh + Q::at(u, NQ - 1) * 512 + 16 * lane);
+              F4 mz = lds4s(rzh + cr * 512 + 16 * lane);
               const float ayh = __ldg(a.bt + T.z(3) + zr), byh = __ldg(a.bt + T.z(4) + zr);
               const float rkyh = __ldg(a.bt + T.z(5) + zr);
 #pragma unroll
@@ -1428,7 +1433,7 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
 #pragma unroll
               for (int q = 0; q < 4; ++q) hz2.v[q] = fmaf(cqs, d_half<P>(wv, q, a.c.cx), hz1o.v[q]);
             } else {
-              F4 mn = lds4s(rxh + (Q::at(u, NQ - 1) * a.band_ring + bcol) * 4);
+              F4 mn = lds4s(rxh + (cr * a.band_ring + bcol) * 4);
               const F4 ah = ld4(a.bt + T.x(3) + bcol), bh = ld4(a.bt + T.x(4) + bcol);
               const F4 rk = ld4(a.bt + T.x(5) + bcol);
 #pragma unroll
@@ -1458,7 +1463,7 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
           }
           if constexpr (BAND) {
             if (bcol >= 0) {
-              F4 mx = lds4s(rxe + (Q::at(u, NQ - 1) * a.band_ring + bcol) * 4);
+              F4 mx = lds4s(rxe + (cr * a.band_ring + bcol) * 4);
               const F4 ax = ld4(a.bt + T.x(0) + bcol), bx = ld4(a.bt + T.x(1) + bcol);
               const F4 rk = ld4(a.bt + T.x(2) + bcol);
 #pragma unroll
@@ -1470,7 +1475,7 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
             }
             const int zr = zband_row(y2, ny, a.g.Wz);
             if (zr >= 0) {
-              F4 mz = lds4s(rze + Q::at(u, NQ - 1) * 512 + 16 * lane);
+              F4 mz = lds4s(rze + cr * 512 + 16 * lane);
               const float ay = __ldg(a.bt + T.z(0) + zr), by = __ldg(a.bt + T.z(1) + zr);
               const float rky = __ldg(a.bt + T.z(2) + zr);
 #pragma unroll
@@ -1496,8 +1501,17 @@ __device__ __forceinline__ bool fwd2_walk(const Fwd2Maps &m, const StepArgs &a, 
         }
         __syncwarp();
         w.ring.next(NS);
+        if constexpr (BAND) {
+          cw = cw + 1 == NQ ? 0 : cw + 1;
+          cr = cr + 1 == NQ ? 0 : cr + 1;
+        }
       }
     }
+    shift_queue<NQ, M>(eq);
+    shift_queue<NQ, M>(hq);
+    shift_queue<NQ, M>(e1q);
+    shift_queue<NQ, M>(h2q);
+    shift_queue<NQ, M>(z1q);
   }
   return true;
 }
