@@ -1,6 +1,6 @@
 """One forward + adjoint sweep of a reduced 2128^2 order-4 case, for profilers.
 
-    python -m adjoint_state_gradients_b200.profile_case [--shots 4] [--nt 8] [--mode fp32]
+    python -m adjoint_state_gradients_b200.profile_case [--shots 4] [--nt 8] [--mode fp32] [--born]
 
 Same grid, stencil, CPML band and launch configuration as the benchmark
 workload, with fewer shots and steps so that an ncu capture of a single
@@ -24,6 +24,8 @@ def main():
     ap.add_argument("--shots", type=int, default=4)
     ap.add_argument("--nt", type=int, default=8)
     ap.add_argument("--mode", default="fp32", choices=["fp32", "bf16", "fp8", "ckpt", "ckpt_ey", "none"])
+    ap.add_argument("--born", action="store_true",
+                    help="after the forward, the Born forward about it (instead of the adjoint)")
     args = ap.parse_args()
     inp = synth.make_inputs(args.workload, n_shots=args.shots)
     wl = inp.wl
@@ -34,7 +36,12 @@ def main():
     prob.set_model_eps_sigma(inp.eps_r.astype(np.float32), inp.sigma.astype(np.float32), f0=wl.f0)
     f = torch.as_tensor(inp.wavelet(dt, args.nt).astype(np.float32)).cuda()
     rec = prob.forward(f)
-    if args.mode != "none":
+    if args.born and args.mode != "none":
+        g = torch.Generator(device="cuda").manual_seed(1)
+        shape = prob.model_shape
+        prob.born(1e-3 * torch.randn(shape, device="cuda", generator=g) * prob.ca,
+                  1e-3 * torch.randn(shape, device="cuda", generator=g) * prob.cb)
+    elif args.mode != "none":
         prob.adjoint(rec.contiguous())
     torch.cuda.synchronize()
     rc = prob.status()
