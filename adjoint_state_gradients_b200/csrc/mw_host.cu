@@ -787,6 +787,54 @@ cudaError_t timed(int cls, cudaStream_t st, F &&launch) {
   return e;
 }
 
+// Small grids (at most kSmallCells cells over all shots) with every snapshot
+// on the device, or none, run each sweep as one cooperative launch
+// (mw_small.cu); MW_NO_SMALL=1 in the environment keeps the step-by-step
+// launches (for comparisons).
+constexpr int64_t kSmallCells = (int64_t)1 << 20;
+bool small_path(const mw_params *p) {
+  const char *e = getenv("MW_NO_SMALL");
+  if (e && e[0] == '1') return false;
+  if (p->snap_host || is_ckpt(p)) return false;
+  return (int64_t)p->n_shots * p->ny * p->nx <= kSmallCells;
+}
+SmallArgs small_args(const mw_params *p, const float *ca, const float *cb, const float *cq,
+                     char *ws, const Layout &L, int *flags) {
+  SmallArgs s{};
+  const Bands b = bands(p);
+  s.S = p->n_shots;
+  s.ny = p->ny;
+  s.nx = p->nx;
+  s.Wx = b.Wx;
+  s.Wz = b.Wz;
+  s.n_pml = p->n_pml;
+  s.grad_mask = p->grad_mask_pml ? 1 : 0;
+  s.batched = p->model_batched ? 1 : 0;
+  s.cq_arr = p->cq_is_scalar ? 0 : 1;
+  s.nt = p->nt;
+  s.numel = (int64_t)p->ny * p->nx;
+  s.c = coef_of(p);
+  s.ca = ca;
+  s.cb = cb;
+  s.cq = cq;
+  s.bt = (const float *)(ws + L.bandtab);
+  s.snap_pitch = L.snap_pitch;
+  s.flags = flags;
+  if (p->snap_mode != MW_SNAP_NONE) {
+    s.snap_e = ws + L.snap;
+    s.snap_c = ws + L.snap + (size_t)p->nt * L.snap_step_bytes;
+    s.step_elems = (int64_t)(L.snap_step_bytes / snap_elem_bytes(p->snap_mode));
+  }
+  return s;
+}
+int run_small(const mw_params *p, SmallArgs &s, bool adjoint, int store, cudaStream_t st) {
+  int block = 256, cluster = 16;
+  small_config(p->order, (int64_t)p->ny * (p->nx / 4), &block, &cluster);
+  MW_CUDA(timed(adjoint ? 2 : (store ? 1 : 0), st,
+                [&] { return launch_small(s, adjoint, p->order, store, cluster, block, st); }));
+  return MW_OK;
+}
+
 int check_ptr(const void *ptr, const char *name) {
   if (!ptr) return fail(MW_ERR_ARG, "%s is NULL", name);
   if (((uintptr_t)ptr) % 16 != 0) return fail(MW_ERR_ARG, "%s is not 16-byte aligned", name);
@@ -1050,6 +1098,19 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   if (rec_out) MW_TRY(build_table(p, rec_idx, p->n_rec, ws, L.tab_rec, flags, rec_out, st));
   a.ea = tb.src;
   if (rec_out) a.eb = tb.rec;
+  if (small_path(p)) {  // every step in one launch, the state in place
+    SmallArgs sa = small_args(p, ca, cb, cq, ws, L, flags);
+    sa.st = fields_at(p, bufA);
+    sa.src = tb.src;
+    sa.f = f;
+    if (rec_out) {
+      sa.rec = tb.rec;
+      sa.rec_out = rec_out;
+    }
+    MW_TRY(run_small(p, sa, false, store, st));
+    if (p->check_finite) MW_CUDA(launch_check_finite(bufA, 3 * SN, flags, st));
+    return MW_OK;
+  }
   const bool host = p->snap_host != 0;
   const size_t ring_steps = host ? (size_t)kHostRing : (size_t)p->nt;
   char *snap_e = ws + L.snap;
@@ -1201,6 +1262,31 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   float *adB = (float *)(ws + L.adB);
   if (!adj_state) MW_CUDA(cudaMemsetAsync(adA, 0, L.state_bytes, st));
   if (p->nt == 0) return MW_OK;
+  if (small_path(p)) {  // every step in one launch, the adjoint state in place
+    MW_TRY(stencil_prologue(p, cpml, ws, L, st));
+    SmallArgs sa = small_args(p, ca, cb, cq, ws, L, flags);
+    sa.st = fields_at(p, adA);
+    sa.rec = tb.rec;
+    sa.res = res;
+    if (gf_all && src_idx) {
+      sa.src = tb.src;
+      sa.grad_f = gf_all;
+    }
+    sa.gca = gca;
+    sa.gcb = gcb;
+    // scratch: the second adjoint buffer's fields and the forward's spare one
+    const Fields s1 = fields_at(p, adB), s2 = fields_at(p, (float *)(ws + L.stB));
+    sa.px = s1.ey;
+    sa.pz = s1.hx;
+    sa.qx = s1.hz;
+    sa.qz = s2.ey;
+    MW_TRY(run_small(p, sa, true, snap_store_kind(p->snap_mode), st));
+    if (p->check_finite) {
+      MW_CUDA(launch_check_finite(gca, SN, flags, st));
+      MW_CUDA(launch_check_finite(gcb, SN, flags, st));
+    }
+    return MW_OK;
+  }
 
   const Launch la = plan(p, kPlanAdj);
   // MW_SNAP_CKPT_EY: the Cb gradient accumulates E^t G^t into P (workspace)

@@ -326,6 +326,34 @@ void forward_layout(int order, int Wx, bool cq_array, bool born, StepArgs *a, si
 void adjoint_layout(int order, int Wx, bool cq_array, bool bf16, StepArgs *a, size_t *smem_bytes);
 int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array);
 
+// Whole-sweep launches for small grids (mw_small.cu): one cooperative launch
+// runs every step of the forward or the adjoint, the state updated in place.
+struct SmallArgs {
+  int S, ny, nx, Wx, Wz, n_pml, grad_mask, batched, cq_arr, nt;
+  int64_t numel;
+  Coef c;
+  Fields st;                 // the state, updated in place
+  const float *ca, *cb, *cq;
+  const float *bt;           // CPML band table (BandTab)
+  void *snap_e, *snap_c;     // snapshots [nt][S][ny][pitch]: step t at t * step_elems
+  int64_t step_elems;
+  int snap_pitch;
+  EntrySet src, rec;
+  const float *f;            // forward: [nt][S][n_src] or null
+  float *rec_out;            // forward: [nt][S][n_rec] or null
+  const float *res;          // adjoint: [nt][S][n_rec] or null
+  float *grad_f;             // adjoint: [nt][S][n_src] or null
+  float *gca, *gcb;          // adjoint: per-shot gradients (+=)
+  float *px, *pz, *qx, *qz;  // adjoint: scratch [S][ny][nx] each
+  int *flags;                // status words
+};
+// threads per block and blocks per shot's cluster of the launches
+void small_config(int order, int64_t groups_per_shot, int *block, int *cluster);
+// store: the forward's snapshot kind (kStoreNone / F32 / BF16 / FP8), or the
+// adjoint's (kStoreF32 / BF16 / FP8); one cluster per shot
+cudaError_t launch_small(const SmallArgs &a, bool adjoint, int order, int store, int cluster,
+                         int block, cudaStream_t st);
+
 // small kernels (mw_aux.cu)
 // Bytes of the entry table of an index set [S][n] on ny rows (EntrySet layout).
 size_t entry_table_bytes(int S, int n, int ny);

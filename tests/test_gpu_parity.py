@@ -41,7 +41,15 @@ def _oracle_pair(sim, f, res, snapshots=True):
     (8, 33, 40, 1, 0, False, False),
     (4, 150, 20, 2, 3, True, True),
 ])
-def test_small_forward_adjoint_parity(order, ny, nx, S, n_pml, batched, cq_array):
+@pytest.mark.parametrize("path", ["whole_sweep", "step_by_step"])
+def test_small_forward_adjoint_parity(order, ny, nx, S, n_pml, batched, cq_array, path,
+                                      monkeypatch):
+    """Both the whole-sweep launch small grids take and the step-by-step
+    launches (MW_NO_SMALL=1) against the oracle."""
+    if path == "step_by_step":
+        monkeypatch.setenv("MW_NO_SMALL", "1")
+    else:
+        monkeypatch.delenv("MW_NO_SMALL", raising=False)
     sim, dt, _ = small_sim(100 + order + ny, ny, nx, S, 2, 5, order, n_pml, batched=batched,
                            cq_array=cq_array, round_f32=True, sigma_max=0.02)
     nt = 57

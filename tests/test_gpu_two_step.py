@@ -44,6 +44,7 @@ def _indices(seed, ny, nx, S, n_pml, n):
 
 
 def _run(prob, f, res, one_step, monkeypatch):
+    monkeypatch.setenv("MW_NO_SMALL", "1")  # the step-by-step launches on every grid
     if one_step:
         monkeypatch.setenv("MW_NO_TWO_STEP", "1")
     else:
