@@ -792,11 +792,13 @@ cudaError_t timed(int cls, cudaStream_t st, F &&launch) {
 // (mw_small.cu); MW_NO_SMALL=1 in the environment keeps the step-by-step
 // launches (for comparisons).
 constexpr int64_t kSmallCells = (int64_t)1 << 20;
-bool small_path(const mw_params *p) {
+bool small_path(const mw_params *p, bool adjoint, int store, SmallPlan *pl) {
   const char *e = getenv("MW_NO_SMALL");
   if (e && e[0] == '1') return false;
   if (p->snap_host || is_ckpt(p)) return false;
-  return (int64_t)p->n_shots * p->ny * p->nx <= kSmallCells;
+  if ((int64_t)p->n_shots * p->ny * p->nx > kSmallCells) return false;
+  const Bands b = bands(p);
+  return small_plan(p->order, adjoint, store, p->ny, p->nx, b.Wx, b.Wz, p->n_src, p->n_rec, pl);
 }
 SmallArgs small_args(const mw_params *p, const float *ca, const float *cb, const float *cq,
                      char *ws, const Layout &L, int *flags) {
@@ -827,11 +829,12 @@ SmallArgs small_args(const mw_params *p, const float *ca, const float *cb, const
   }
   return s;
 }
-int run_small(const mw_params *p, SmallArgs &s, bool adjoint, int store, cudaStream_t st) {
-  int block = 256, cluster = 16;
-  small_config(p->order, (int64_t)p->ny * (p->nx / 4), &block, &cluster);
-  MW_CUDA(timed(adjoint ? 2 : (store ? 1 : 0), st,
-                [&] { return launch_small(s, adjoint, p->order, store, cluster, block, st); }));
+int run_small(const mw_params *p, SmallArgs &s, bool adjoint, int store, const SmallPlan &pl,
+              cudaStream_t st) {
+  // profile classes of whole-sweep launches: 6 / 7 / 8 resident, 9 / 10 / 11
+  // state in global memory (forward, forward with snapshots, adjoint)
+  const int cls = (pl.resident ? 6 : 9) + (adjoint ? 2 : (store ? 1 : 0));
+  MW_CUDA(timed(cls, st, [&] { return launch_small(s, adjoint, p->order, store, pl, st); }));
   return MW_OK;
 }
 
@@ -1098,7 +1101,8 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
   if (rec_out) MW_TRY(build_table(p, rec_idx, p->n_rec, ws, L.tab_rec, flags, rec_out, st));
   a.ea = tb.src;
   if (rec_out) a.eb = tb.rec;
-  if (small_path(p)) {  // every step in one launch, the state in place
+  SmallPlan spl{};
+  if (small_path(p, false, store, &spl)) {  // every step in one launch, the state in place
     SmallArgs sa = small_args(p, ca, cb, cq, ws, L, flags);
     sa.st = fields_at(p, bufA);
     sa.src = tb.src;
@@ -1107,7 +1111,7 @@ int mw_tm_forward(const mw_params *p, const float *ca, const float *cb, const fl
       sa.rec = tb.rec;
       sa.rec_out = rec_out;
     }
-    MW_TRY(run_small(p, sa, false, store, st));
+    MW_TRY(run_small(p, sa, false, store, spl, st));
     if (p->check_finite) MW_CUDA(launch_check_finite(bufA, 3 * SN, flags, st));
     return MW_OK;
   }
@@ -1262,7 +1266,9 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
   float *adB = (float *)(ws + L.adB);
   if (!adj_state) MW_CUDA(cudaMemsetAsync(adA, 0, L.state_bytes, st));
   if (p->nt == 0) return MW_OK;
-  if (small_path(p)) {  // every step in one launch, the adjoint state in place
+  SmallPlan spl{};
+  if (small_path(p, true, snap_store_kind(p->snap_mode), &spl)) {
+    // every step in one launch, the adjoint state in place
     MW_TRY(stencil_prologue(p, cpml, ws, L, st));
     SmallArgs sa = small_args(p, ca, cb, cq, ws, L, flags);
     sa.st = fields_at(p, adA);
@@ -1280,7 +1286,7 @@ int mw_tm_adjoint_grad(const mw_params *p, const float *ca, const float *cb, con
     sa.pz = s1.hx;
     sa.qx = s1.hz;
     sa.qz = s2.ey;
-    MW_TRY(run_small(p, sa, true, snap_store_kind(p->snap_mode), st));
+    MW_TRY(run_small(p, sa, true, snap_store_kind(p->snap_mode), spl, st));
     if (p->check_finite) {
       MW_CUDA(launch_check_finite(gca, SN, flags, st));
       MW_CUDA(launch_check_finite(gcb, SN, flags, st));

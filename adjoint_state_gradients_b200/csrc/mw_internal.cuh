@@ -330,6 +330,9 @@ int stencil_slots_per_sm(int order, bool adjoint, int Wx, bool cq_array);
 // runs every step of the forward or the adjoint, the state updated in place.
 struct SmallArgs {
   int S, ny, nx, Wx, Wz, n_pml, grad_mask, batched, cq_arr, nt;
+  // resident variant (set by launch_small): rows a block; steps a chunk of
+  // the global traffic; ring entries a step for sources and receivers
+  int rows, kchunk, csrc, crec;
   int64_t numel;
   Coef c;
   Fields st;                 // the state, updated in place
@@ -347,12 +350,22 @@ struct SmallArgs {
   float *px, *pz, *qx, *qz;  // adjoint: scratch [S][ny][nx] each
   int *flags;                // status words
 };
-// threads per block and blocks per shot's cluster of the launches
-void small_config(int order, int64_t groups_per_shot, int *block, int *cluster);
+// Shape of a whole-sweep launch: the resident variant (each block's rows in
+// shared memory, `rows` rows a block) or the L2 variant (the state in global
+// memory); `cluster` blocks per shot, `block` threads a block.
+struct SmallPlan {
+  bool resident;
+  int block, cluster, rows, kchunk, csrc, crec;
+  size_t smem;
+};
+// The shape for one direction (store: the forward's snapshot kind, or the
+// adjoint's) of a shot of ny x nx cells; false when no cluster fits.
+bool small_plan(int order, bool adjoint, int store, int ny, int nx, int Wx, int Wz, int n_src,
+                int n_rec, SmallPlan *pl);
 // store: the forward's snapshot kind (kStoreNone / F32 / BF16 / FP8), or the
 // adjoint's (kStoreF32 / BF16 / FP8); one cluster per shot
-cudaError_t launch_small(const SmallArgs &a, bool adjoint, int order, int store, int cluster,
-                         int block, cudaStream_t st);
+cudaError_t launch_small(const SmallArgs &a, bool adjoint, int order, int store,
+                         const SmallPlan &pl, cudaStream_t st);
 
 // small kernels (mw_aux.cu)
 // Bytes of the entry table of an index set [S][n] on ny rows (EntrySet layout).

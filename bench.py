@@ -137,25 +137,28 @@ def alg_bytes(wl, S, one_pass=False):
 
 # the library's per-launch timing classes: 0 forward, 1 forward with snapshot
 # store, 2 adjoint, 3 Born, 4 / 5 two-step forward launches without / with
-# snapshot store (two steps per launch); which classes each pass of a sweep
-# uses, as (one-step class, two-step class or None)
-N_CLASSES = 6
+# snapshot store (two steps per launch), and the whole-sweep launches of small
+# grids (all nt steps in one launch): 6 / 7 / 8 state in shared memory, 9 /
+# 10 / 11 state in global memory (forward, forward with store, adjoint);
+# which classes each pass of a sweep uses, as (one-step class, two-step class
+# or None, whole-sweep classes)
+N_CLASSES = 12
 
 
 def pass_classes(wl):
     if wl.snapshot in CKPT_MODES:
-        return {"forward": (0, 4), "replay": (1, 5), "adjoint": (2, None)}
+        return {"forward": (0, 4, ()), "replay": (1, 5, ()), "adjoint": (2, None, ())}
     if wl.snapshot == "none":
-        return {"forward": (0, 4)}
-    return {"forward": (1, 5), "adjoint": (2, None)}
+        return {"forward": (0, 4, (6, 9))}
+    return {"forward": (1, 5, (7, 10)), "adjoint": (2, None, (8, 11))}
 
 
-def per_step_ms(counts, ms, classes):
+def per_step_ms(counts, ms, classes, nt):
     """Mean device time per step of one pass (a two-step launch counts as two
-    steps)."""
-    a, b = classes
-    n = counts[a] + (2 * counts[b] if b is not None else 0)
-    t = ms[a] + (ms[b] if b is not None else 0.0)
+    steps, a whole-sweep launch as nt)."""
+    a, b, w = classes
+    n = counts[a] + (2 * counts[b] if b is not None else 0) + nt * sum(counts[c] for c in w)
+    t = ms[a] + (ms[b] if b is not None else 0.0) + sum(ms[c] for c in w)
     return t / max(n, 1)
 
 
@@ -497,9 +500,16 @@ class Sweep:
         peak, peak_kind = measured_peaks()
         sweep_bytes = sweep_bytes_per_cell(wl, S, nt) * self.cells * steps
         sweep_frac = sweep_bytes / (total_ms / 1e3) / 1e9 / peak / world
-        launch_ms = {k: per_step_ms(counts, ms, c) for k, c in classes.items()}
+        launch_ms = {k: per_step_ms(counts, ms, c, nt) for k, c in classes.items()}
         top = "adjoint" if self.grad else "forward"   # the dominant kernel
         top_launch_ms = launch_ms[top]
+
+        def steps_per_launch(c):
+            a, b, w = c
+            n = counts[a] + (counts[b] if b is not None else 0) + sum(counts[k] for k in w)
+            st = counts[a] + (2 * counts[b] if b is not None else 0) + nt * sum(counts[k] for k in w)
+            return st / n if n else 1.0
+        spl = {k: steps_per_launch(c) for k, c in classes.items()}
         top_bytes = passes[top] * wl.ny * wl.nx * S
         achieved = top_bytes / (top_launch_ms / 1e3) / 1e9
         kname = {("adjoint", "fp32"): "kStoreF32", ("adjoint", "ckpt"): "kStoreF32",
@@ -507,10 +517,18 @@ class Sweep:
                  ("adjoint", "bf16"): "kStoreBF16", ("adjoint", "fp8"): "kStoreFP8"}
         kernel_name = (f"k_adjoint<{wl.order // 2}, {kname[(top, wl.snapshot)]}, 1>" if self.grad
                        else f"k_forward<{wl.order // 2}, kStoreNone, 1>")
+        whole = classes[top][2]  # whole-sweep launches of a small grid
+        if whole and counts[whole[0]] > 0:
+            kernel_name = (f"k_res_adj<{wl.order // 2}, {kname[(top, wl.snapshot)]}>" if self.grad
+                           else f"k_res_fwd<{wl.order // 2}, kStoreNone>")
+        elif whole and counts[whole[1]] > 0:
+            kernel_name = (f"k_small_adj<{wl.order // 2}, {kname[(top, wl.snapshot)]}>" if self.grad
+                           else f"k_small_fwd<{wl.order // 2}, kStoreNone>")
         return dict(value=value, value_fwd=value_fwd, total_ms=total_ms, steps=steps,
                     passes=passes, sweep_frac=sweep_frac, launch_ms=launch_ms, counts=counts,
                     top=top, top_bytes=top_bytes, top_launch_ms=top_launch_ms, achieved=achieved,
                     peak=peak, peak_kind=peak_kind, kernel_name=kernel_name, n_launch=n_launch,
+                    steps_per_launch=spl,
                     clocks=clk)
 
     def e2e(self, steps):
@@ -702,13 +720,15 @@ def main():
             "sweep_bytes_per_cell": round(sweep_bytes_per_cell(wl, S, nt), 3),
             "sweep_bytes_per_cell_one_step_per_pass": round(
                 sweep_bytes_per_cell(wl, S, nt, one_pass=True), 3),
-            "forward_steps_per_launch": 2 if two_step(wl) else 1,
+            "forward_steps_per_launch": round(m["steps_per_launch"]["forward"], 3),
             "roofline": {"bound": "hbm", "kernel": m["kernel_name"],
                          "achieved": round(m["achieved"], 1),
                          "peak": m["peak"], "peak_kind": m["peak_kind"], "unit": "GB/s",
                          "frac": round(m["achieved"] / m["peak"], 4),
-                         "traffic": traffic, "alg_bytes_per_launch": m["top_bytes"],
-                         "avg_launch_ms": round(m["top_launch_ms"], 4),
+                         "traffic": traffic,
+                         "alg_bytes_per_launch": round(m["top_bytes"] * m["steps_per_launch"][m["top"]]),
+                         "avg_launch_ms": round(m["top_launch_ms"] * m["steps_per_launch"][m["top"]], 4),
+                         "steps_per_launch": round(m["steps_per_launch"][m["top"]], 3),
                          "timing": "CUDA events around every launch, second pass of the same K steps"},
             "kernel_ms": {**{k: round(v, 4) for k, v in m["launch_ms"].items()},
                           "launches": [int(c) for c in m["counts"]]},

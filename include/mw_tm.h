@@ -313,10 +313,14 @@ int mw_sync_status(void *workspace_dev, void *stream);
 /* Thread-local message of the last failing call ("" if none). */
 const char *mw_last_error(void);
 
-/* Per-kernel timing (CUDA events around each launch of the stencil kernels:
- * 0 forward, 1 forward with snapshot store, 2 adjoint, 3 Born forward).  enable = 1
- * clears and starts recording; mw_profile_read synchronizes the recorded
- * events and returns, per class, the launch count and total milliseconds. */
+/* Per-kernel timing (CUDA events around each launch of the stencil kernels,
+ * by class: 0 forward, 1 forward with snapshot store, 2 adjoint, 3 Born
+ * forward, 4 / 5 two-step forward without / with snapshot store; whole-sweep
+ * launches of small grids, each covering all nt steps: 6 / 7 / 8 with the
+ * state in shared memory, 9 / 10 / 11 with the state in global memory
+ * (forward, forward with snapshot store, adjoint)).  enable = 1 clears and
+ * starts recording; mw_profile_read synchronizes the recorded events and
+ * returns, per class, the launch count and total milliseconds. */
 int mw_profile_enable(int32_t enable);
 int mw_profile_read(int64_t *counts, double *total_ms, int32_t n_classes);
 

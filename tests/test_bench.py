@@ -31,7 +31,8 @@ def test_byte_model_of_the_headline_sweep():
     assert b["replay"] == pytest.approx(24 + 1 + band + 4)
     assert b["adjoint"] == pytest.approx(24 + 1 + band + 4 + 16)
     assert sum(b.values()) == pytest.approx(102.61, abs=0.01)
-    assert bench.pass_classes(wl) == {"forward": (0, 4), "replay": (1, 5), "adjoint": (2, None)}
+    assert bench.pass_classes(wl) == {"forward": (0, 4, ()), "replay": (1, 5, ()),
+                                      "adjoint": (2, None, ())}
     bp = bench.alg_bytes(dataclasses.replace(wl, snapshot="ckpt"), wl.n_shots, one_pass=True)
     assert bp["replay"] - b["replay"] == pytest.approx(4.0)
     assert bp["adjoint"] - b["adjoint"] == pytest.approx(4.0)
@@ -65,7 +66,18 @@ def test_byte_model_of_the_other_storage_modes():
     assert b3["adjoint"] - b3["forward"] == pytest.approx(16.0)   # gradient read + write
     assert set(b5) == {"forward"}
     assert b5["forward"] > 24 + 8                                  # per-shot model: 8 B per cell
-    assert bench.pass_classes(w5) == {"forward": (0, 4)}
+    assert bench.pass_classes(w5) == {"forward": (0, 4, (6, 9))}
+
+
+def test_per_step_time_of_each_launch_kind():
+    """One-step launches count one step, two-step launches two, whole-sweep
+    launches nt."""
+    counts = [10, 0, 0, 0, 5, 0, 0, 0, 0, 0, 0, 0]
+    ms = [1.0, 0, 0, 0, 2.0, 0, 0, 0, 0, 0, 0, 0]
+    assert bench.per_step_ms(counts, ms, (0, 4, (6, 9)), 300) == pytest.approx(3.0 / 20)
+    counts[8], ms[8] = 2, 6.0
+    assert bench.per_step_ms(counts, ms, (2, None, (8, 11)), 300) == pytest.approx(6.0 / 600)
+    assert bench.N_CLASSES == 12
 
 
 def test_oracle_sample_is_bounded():

@@ -1,6 +1,10 @@
 """The whole-sweep launch of small grids (every step of the forward, or of
 the adjoint, in one cooperative launch) against the step-by-step launches,
-bit for bit.
+bit for bit, in both variants: the resident one (each block's rows in shared
+memory, halo rows read from the neighbouring blocks), with the library's
+cluster and chunks of global traffic, with at most 4 blocks a shot, and with
+chunks of 2 steps, and the one whose state stays in global memory
+(MW_SMALL_L2=1).
 
 Both paths make the same floating-point operations in the same order for
 every update, source sum, receiver sample and gradient term, so records,
@@ -24,9 +28,17 @@ from tests._gpu import f32, problem_from_sim
 pytestmark = pytest.mark.gpu
 
 
-def _run(prob, f, res, state0, adj0, small, monkeypatch):
+VARIANTS = {"resident": {}, "resident-4": {"MW_SMALL_CLUSTER": "4"},
+            "resident-chunk2": {"MW_SMALL_CHUNK": "2"}, "l2": {"MW_SMALL_L2": "1"}}
+
+
+def _run(prob, f, res, state0, adj0, small, monkeypatch, variant="resident"):
+    for k in ("MW_SMALL_CLUSTER", "MW_SMALL_CHUNK", "MW_SMALL_L2"):
+        monkeypatch.delenv(k, raising=False)
     if small:
         monkeypatch.delenv("MW_NO_SMALL", raising=False)
+        for k, v in VARIANTS[variant].items():
+            monkeypatch.setenv(k, v)
     else:
         monkeypatch.setenv("MW_NO_SMALL", "1")
     state = state0.clone()
@@ -50,9 +62,13 @@ def _run(prob, f, res, state0, adj0, small, monkeypatch):
     (4, 150, 20, 2, 3, True, True, "fp32", True),
     (4, 33, 40, 1, 0, False, False, "none", False),
     (4, 84, 84, 1, 10, False, False, "fp32", True),
+    (8, 64, 96, 2, 5, False, False, "fp32", False),    # 4 rows a block: the halo is a whole block
+    (8, 61, 40, 1, 3, False, False, "bf16", False),    # a last block of one row
+    (4, 200, 264, 2, 8, False, False, "fp32", False),  # up to 2 groups a thread
 ])
+@pytest.mark.parametrize("variant", list(VARIANTS))
 def test_whole_sweep_is_bitwise_step_by_step(order, ny, nx, S, n_pml, batched, cq_array,
-                                             snapshot, mask, monkeypatch):
+                                             snapshot, mask, variant, monkeypatch):
     sim, dt, _ = small_sim(900 + order + ny, ny, nx, S, 3, 7, order, n_pml, batched=batched,
                            cq_array=cq_array, round_f32=True, sigma_max=0.02)
     src, rec = sim.src_idx.copy(), sim.rec_idx.copy()
@@ -69,7 +85,7 @@ def test_whole_sweep_is_bitwise_step_by_step(order, ny, nx, S, n_pml, batched, c
     state0 = torch.as_tensor(f32(1e-3 * g.normal(size=n)), dtype=torch.float32).cuda()
     adj0 = torch.as_tensor(f32(1e-3 * g.normal(size=n)), dtype=torch.float32).cuda()
     step = _run(prob, f, res, state0, adj0, False, monkeypatch)
-    whole = _run(prob, f, res, state0, adj0, True, monkeypatch)
+    whole = _run(prob, f, res, state0, adj0, True, monkeypatch, variant)
     names = ["records", "state", "dJ/dCa", "dJ/dCb", "dJ/df", "adjoint state"]
     for nm, x, y in zip(names, step, whole):
         assert np.array_equal(x, y), nm
