@@ -355,7 +355,7 @@ struct SmallArgs {
 // memory); `cluster` blocks per shot, `block` threads a block.
 struct SmallPlan {
   bool resident;
-  int block, cluster, rows, kchunk, csrc, crec;
+  int block, cluster, rows, kchunk, csrc, crec, width;  // width: cells a thread's group
   size_t smem;
 };
 // The shape for one direction (store: the forward's snapshot kind, or the

@@ -562,6 +562,13 @@ __device__ __forceinline__ int opaque(int x) {
   asm volatile("" : "+r"(x));
   return x;
 }
+// a group coordinate for the phase: opaque with several groups a thread
+// (registers are scarce), else as is (its addresses are kept across steps)
+template <int G>
+__device__ __forceinline__ int gco(int x) {
+  if constexpr (G > 1) return opaque(x);
+  else return x;
+}
 
 // ---------------------------------------------------------------------------
 // Resident variants: every block keeps its rows of the state -- and, in the
@@ -634,46 +641,110 @@ __device__ __forceinline__ F4 lds4(const float *p) {
   const float4 t = *reinterpret_cast<const float4 *>(p);
   return F4{{t.x, t.y, t.z, t.w}};
 }
+// W consecutive cells (a group of 4, or of 2 on small blocks, where twice
+// the threads each take half a float4's work)
+template <int W>
+struct VW {
+  float v[W];
+};
+template <int W>
+__device__ __forceinline__ VW<W> ldv(const float *p) {
+  VW<W> r;
+  if constexpr (W == 4) {
+    const float4 t = *reinterpret_cast<const float4 *>(p);
+    r.v[0] = t.x, r.v[1] = t.y, r.v[2] = t.z, r.v[3] = t.w;
+  } else {
+    const float2 t = *reinterpret_cast<const float2 *>(p);
+    r.v[0] = t.x, r.v[1] = t.y;
+  }
+  return r;
+}
+template <int W>
+__device__ __forceinline__ VW<W> ldgv(const float *p) {  // read-only global data
+  VW<W> r;
+  if constexpr (W == 4) {
+    const float4 t = __ldg(reinterpret_cast<const float4 *>(p));
+    r.v[0] = t.x, r.v[1] = t.y, r.v[2] = t.z, r.v[3] = t.w;
+  } else {
+    const float2 t = __ldg(reinterpret_cast<const float2 *>(p));
+    r.v[0] = t.x, r.v[1] = t.y;
+  }
+  return r;
+}
+template <int W>
+__device__ __forceinline__ void stv(float *p, const VW<W> &a) {
+  if constexpr (W == 4)
+    *reinterpret_cast<float4 *>(p) = make_float4(a.v[0], a.v[1], a.v[2], a.v[3]);
+  else
+    *reinterpret_cast<float2 *>(p) = make_float2(a.v[0], a.v[1]);
+}
+template <int W>
+__device__ __forceinline__ VW<W> zerov() {
+  VW<W> r;
+#pragma unroll
+  for (int q = 0; q < W; ++q) r.v[q] = 0.f;
+  return r;
+}
+template <int W>
+__device__ __forceinline__ VW<W> splatv(float x) {
+  VW<W> r;
+#pragma unroll
+  for (int q = 0; q < W; ++q) r.v[q] = x;
+  return r;
+}
 
 // The rows [r0, r1) of one block (R rows per block; block b - 1 holds
 // [r0 - R, r0), block b + 1 starts at r1) of a shot with ny rows; rows of
 // `np` floats, cells from offset 4.
 struct RBlk {
   int r0, r1, R, ny, np;
-  // float4 at (y, c) of a cluster field, zero outside the array (column c
-  // is a group's own column; |y - row| <= P <= R)
-  __device__ __forceinline__ F4 zrow(const CRows &f, int y, int c) const {
+  // the W cells at (y, c) of a cluster field, zero outside the array
+  // (column c is a group's own column; |y - row| <= P <= R)
+  template <int W>
+  __device__ __forceinline__ VW<W> zrow(const CRows &f, int y, int c) const {
     const bool in = y >= 0 && y < ny;
     const float *p = f.loc + 4 + c;
     if (in)
       p = (y < r0 ? f.up + (y - r0 + R) * np : y < r1 ? f.loc + (y - r0) * np : f.dn + (y - r1) * np) +
           4 + c;
-    const F4 v = lds4(p);
-    return in ? v : zero4();
+    const VW<W> v = ldv<W>(p);
+    return in ? v : zerov<W>();
   }
   // out[j] = field at row y + D0 - j, j < N, of the group at (y, c): from
   // this block's rows at constant offsets when all of them are here
-  template <int N, int D0>
-  __device__ __forceinline__ void zwin(const CRows &f, int y, int c, F4 out[N]) const {
+  template <int W, int N, int D0>
+  __device__ __forceinline__ void zwin(const CRows &f, int y, int c, VW<W> out[N]) const {
     if (y - r0 + D0 - (N - 1) >= 0 && y - r0 + D0 < r1 - r0) {
       const float *p = f.loc + (y - r0 + D0) * np + 4 + c;
 #pragma unroll
-      for (int j = 0; j < N; ++j) out[j] = lds4(p - j * np);
+      for (int j = 0; j < N; ++j) out[j] = ldv<W>(p - j * np);
     } else {
 #pragma unroll
-      for (int j = 0; j < N; ++j) out[j] = zrow(f, y + D0 - j, c);
+      for (int j = 0; j < N; ++j) out[j] = zrow<W>(f, y + D0 - j, c);
     }
   }
 };
 // x window w[0..12) = columns c - 4 .. c + 8 of a padded row (cells from
-// offset 4; the zero columns stand for the cells outside the array)
+// offset 4; the zero columns stand for the cells outside the array); with
+// W = 2 only w[0..10) (columns c - 4 .. c + 6) is read
+template <int W>
 __device__ __forceinline__ void xwin(const float *row, int c, float w[12]) {
-  const F4 A = lds4(row + c), B = lds4(row + c + 4), D = lds4(row + c + 8);
+  if constexpr (W == 4) {
+    const VW<4> A = ldv<4>(row + c), B = ldv<4>(row + c + 4), D = ldv<4>(row + c + 8);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    w[q] = A.v[q];
-    w[q + 4] = B.v[q];
-    w[q + 8] = D.v[q];
+    for (int q = 0; q < 4; ++q) {
+      w[q] = A.v[q];
+      w[q + 4] = B.v[q];
+      w[q + 8] = D.v[q];
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 5; ++j) {
+      const VW<2> t = ldv<2>(row + c + 2 * j);
+      w[2 * j] = t.v[0];
+      w[2 * j + 1] = t.v[1];
+    }
+    w[10] = w[11] = 0.f;
   }
 }
 
@@ -827,33 +898,53 @@ __device__ __forceinline__ bool res_start(const cg::cluster_group &cl, const int
   return stop;
 }
 
-// Copy one group's staged snapshot words (4 cells of the store type) from
-// shared memory to the snapshot array.
-template <int STORE>
-__device__ __forceinline__ void stage_out(const void *stage, int64_t li, void *dst, int64_t so) {
-  if constexpr (STORE == kStoreF32) {
-    *(reinterpret_cast<uint4 *>(dst) + so / 4) = *(reinterpret_cast<const uint4 *>(stage) + li / 4);
+// Snapshot store of W cells at element `elem` (the 4-cell form is
+// snap_store; 2 cells: the same conversions on one pair).
+template <int STORE, int W>
+__device__ __forceinline__ void snap_store_w(void *base, int64_t elem, const VW<W> &v) {
+  if constexpr (W == 4) {
+    snap_store<STORE>(base, elem, F4{{v.v[0], v.v[1], v.v[2], v.v[3]}});
+  } else if constexpr (STORE == kStoreF32) {
+    *reinterpret_cast<float2 *>(reinterpret_cast<float *>(base) + elem) = make_float2(v.v[0], v.v[1]);
   } else if constexpr (STORE == kStoreBF16) {
-    *(reinterpret_cast<uint2 *>(dst) + so / 4) = *(reinterpret_cast<const uint2 *>(stage) + li / 4);
+    __nv_bfloat162 pr = __floats2bfloat162_rn(v.v[0], v.v[1]);
+    *reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(base) + elem) =
+        *reinterpret_cast<uint32_t *>(&pr);
   } else if constexpr (STORE == kStoreFP8) {
-    *(reinterpret_cast<uint32_t *>(dst) + so / 4) =
-        *(reinterpret_cast<const uint32_t *>(stage) + li / 4);
+    const uint32_t pr =
+        __nv_cvt_float2_to_fp8x2(make_float2(v.v[0], v.v[1]), __NV_SATFINITE, __NV_E4M3);
+    *reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(base) + elem) = (uint16_t)pr;
   }
+}
+// Copy one group's staged snapshot words (W cells of the store type) from
+// shared memory to the snapshot array.
+template <typename T>
+__device__ __forceinline__ void copy_words(const void *src, int64_t i, void *dst, int64_t j) {
+  *(reinterpret_cast<T *>(dst) + j) = *(reinterpret_cast<const T *>(src) + i);
+}
+template <int STORE, int W>
+__device__ __forceinline__ void stage_out(const void *stage, int64_t li, void *dst, int64_t so) {
+  constexpr int bytes = W * (STORE == kStoreF32 ? 4 : STORE == kStoreBF16 ? 2 : 1);
+  if constexpr (bytes == 16) copy_words<uint4>(stage, li / W, dst, so / W);
+  else if constexpr (bytes == 8) copy_words<uint2>(stage, li / W, dst, so / W);
+  else if constexpr (bytes == 4) copy_words<uint32_t>(stage, li / W, dst, so / W);
+  else if constexpr (bytes == 2) copy_words<uint16_t>(stage, li / W, dst, so / W);
 }
 __host__ __device__ constexpr int stage_bytes(int store) {
   return store == kStoreF32 ? 4 : store == kStoreBF16 ? 2 : store == kStoreFP8 ? 1 : 0;
 }
 
-template <int P, int STORE, int NT, int G>
+template <int P, int STORE, int NT, int G, int W>
 __global__ void __launch_bounds__(NT, 1) k_res_fwd(const SmallArgs a) {
   constexpr int KM = res_kmax(G);
+  using V = VW<W>;
   __shared__ int s_stop;
   const cg::cluster_group cl = cg::this_cluster();
   if (res_start(cl, a.flags, &s_stop)) return;
   const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
   const int s = (int)(blockIdx.x / cs);
-  const int ny = a.ny, nx = a.nx, nx4 = nx >> 2, R = a.rows, K = a.kchunk, km = K - 1;
-  const int r0 = rank * R, r1 = min(ny, r0 + R), Rb = r1 - r0, ng = Rb * nx4;
+  const int ny = a.ny, nx = a.nx, nxw = nx / W, R = a.rows, K = a.kchunk, km = K - 1;
+  const int r0 = rank * R, r1 = min(ny, r0 + R), Rb = r1 - r0, ng = Rb * nxw;
   const ResLayout Ly{R, nx, a.Wx, a.Wz, kResFieldsFwd, K, a.csrc, a.crec, stage_bytes(STORE),
                      STORE != kStoreNone ? K : 0};
   const int np = Ly.pitch();
@@ -873,20 +964,20 @@ __global__ void __launch_bounds__(NT, 1) k_res_fwd(const SmallArgs a) {
   const int64_t sb = (int64_t)s * a.numel;
   // the thread's groups: row and column, and their Ca, Cb
   int gy[G], gc[G];
-  F4 ca[G], cb[G];
+  V ca[G], cb[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const int k = (int)threadIdx.x + g * NT;
     gy[g] = -1;
     gc[g] = 0;
-    ca[g] = cb[g] = zero4();
+    ca[g] = cb[g] = zerov<W>();
     if (k < ng) {
-      const int ly = k / nx4;
+      const int ly = k / nxw;
       gy[g] = r0 + ly;
-      gc[g] = (k - ly * nx4) * 4;
+      gc[g] = (k - ly * nxw) * W;
       const int64_t mb = (a.batched ? sb : 0) + (int64_t)gy[g] * nx + gc[g];
-      ca[g] = ld4(a.ca + mb);
-      cb[g] = ld4(a.cb + mb);
+      ca[g] = ldgv<W>(a.ca + mb);
+      cb[g] = ldgv<W>(a.cb + mb);
     }
   }
   res_state<true>(a.st, sm, Ly, a.bt, s, r0, Rb, ny, a.numel);
@@ -896,18 +987,20 @@ __global__ void __launch_bounds__(NT, 1) k_res_fwd(const SmallArgs a) {
   const int64_t fstep = (int64_t)a.S * a.src.n, rstep = (int64_t)a.S * a.rec.n;
   // steps [t0, t0 + cnt) of the rings to the snapshot arrays and the records
   auto flush = [&](int t0, int cnt) {
-    for (int i = 0; i < cnt; ++i) {
+#pragma unroll
+    for (int i = 0; i < KM; ++i) {
+      if (i >= cnt) break;
       const int t = t0 + i, k = t & km;
       if constexpr (STORE != kStoreNone) {
         const char *se = slots + k * slot_b, *sc = se + slot_b / 2;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           if (gy[g] < 0) continue;
-          const int y = opaque(gy[g]), c = gc[g];
+          const int y = gco<G>(gy[g]), c = gc[g];
           const int64_t li = (int64_t)(y - r0) * nx + c;
           const int64_t so = (int64_t)t * a.step_elems + ((int64_t)s * ny + y) * a.snap_pitch + c;
-          stage_out<STORE>(se, li, a.snap_e, so);
-          stage_out<STORE>(sc, li, a.snap_c, so);
+          stage_out<STORE, W>(se, li, a.snap_e, so);
+          stage_out<STORE, W>(sc, li, a.snap_c, so);
         }
       }
       if (a.rec_out && rec.mine())
@@ -931,44 +1024,47 @@ __global__ void __launch_bounds__(NT, 1) k_res_fwd(const SmallArgs a) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (gy[g] < 0) continue;
-      const int y = opaque(gy[g]), c = opaque(gc[g]), ly = y - r0;
+      const int y = gco<G>(gy[g]), c = gco<G>(gc[g]), ly = y - r0;
       const int64_t mb = (a.batched ? sb : 0) + (int64_t)y * nx + c;
-      const F4 cq = a.cq_arr ? ld4(a.cq + mb) : splat4(cqs);
+      const V cq = a.cq_arr ? ldgv<W>(a.cq + mb) : splatv<W>(cqs);
+      // the z window of E rows y - P + 1 .. y + P first: rows of the
+      // neighbouring blocks take longest, and the stores below would keep
+      // the compiler from hoisting their loads
+      V e[2 * P];
+      B.zwin<W, 2 * P, P>(fE, y, c, e);  // e[j] = E(y + P - j)
       // Hz(y, c..c+3) at the half nodes
       {
         float w[12];
-        xwin(sE + ly * np, c, w);
+        xwin<W>(sE + ly * np, c, w);
         float *hp = sHz + ly * np + 4 + c;
-        const F4 hz_old = lds4(hp);
-        F4 hn;
+        const V hz_old = ldv<W>(hp);
+        V hn;
         const int bc = xband(c, nx, a.Wx);
         if (bc < 0) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) hn.v[q] = fmaf(cq.v[q], dh<P>(w, q, a.c.cx), hz_old.v[q]);
+          for (int q = 0; q < W; ++q) hn.v[q] = fmaf(cq.v[q], dh<P>(w, q, a.c.cx), hz_old.v[q]);
         } else {
           float *mp = sMxh + ly * 2 * a.Wx + bc;
-          F4 mn = lds4(mp);
-          const F4 ah = lds4(bt + T.x(3) + bc), bh = lds4(bt + T.x(4) + bc);
-          const F4 rk = lds4(bt + T.x(5) + bc);
+          V mn = ldv<W>(mp);
+          const V ah = ldv<W>(bt + T.x(3) + bc), bh = ldv<W>(bt + T.x(4) + bc);
+          const V rk = ldv<W>(bt + T.x(5) + bc);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < W; ++q) {
             const float d = dh<P>(w, q, a.c.cx);
             mn.v[q] = fmaf(bh.v[q], mn.v[q], ah.v[q] * d);
             hn.v[q] = fmaf(cq.v[q], fmaf(d, rk.v[q], mn.v[q]), hz_old.v[q]);
           }
-          st4(mp, mn);
+          stv<W>(mp, mn);
         }
-        st4(hp, hn);
+        stv<W>(hp, hn);
       }
-      // Hx(y + 1/2, c..c+3): z window of E rows y - P + 1 .. y + P
+      // Hx(y + 1/2, c..c+3) from the z window of E
       {
-        F4 e[2 * P];
-        B.zwin<2 * P, P>(fE, y, c, e);  // e[j] = E(y + P - j)
         float *hp = sHx + ly * np + 4 + c;
-        const F4 hx_old = lds4(hp);
-        F4 d;
+        const V hx_old = ldv<W>(hp);
+        V d;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < W; ++q) {
           float sacc = 0.f;
 #pragma unroll
           for (int k = 1; k <= P; ++k)  // E(y + k) - E(y - k + 1)
@@ -978,20 +1074,20 @@ __global__ void __launch_bounds__(NT, 1) k_res_fwd(const SmallArgs a) {
         const int zr = zband(y, ny, a.Wz);
         if (zr >= 0) {
           float *mp = sMzh + ly * nx + c;
-          F4 mz = lds4(mp);
+          V mz = ldv<W>(mp);
           const float ayh = bt[T.z(3) + zr], byh = bt[T.z(4) + zr];
           const float rkyh = bt[T.z(5) + zr];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < W; ++q) {
             mz.v[q] = fmaf(byh, mz.v[q], ayh * d.v[q]);
             d.v[q] = fmaf(d.v[q], rkyh, mz.v[q]);
           }
-          st4(mp, mz);
+          stv<W>(mp, mz);
         }
-        F4 hn;
+        V hn;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) hn.v[q] = fmaf(-cq.v[q], d.v[q], hx_old.v[q]);
-        st4(hp, hn);
+        for (int q = 0; q < W; ++q) hn.v[q] = fmaf(-cq.v[q], d.v[q], hx_old.v[q]);
+        stv<W>(hp, hn);
       }
     }
     if (chunk && a.f) fl.store(src, kc, [&](int i) { return ringF + ((t + i) & km) * a.csrc; });
@@ -1002,16 +1098,16 @@ __global__ void __launch_bounds__(NT, 1) k_res_fwd(const SmallArgs a) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (gy[g] < 0) continue;
-      const int y = opaque(gy[g]), c = opaque(gc[g]), ly = y - r0;
+      const int y = gco<G>(gy[g]), c = gco<G>(gc[g]), ly = y - r0;
+      V h[2 * P];
+      B.zwin<W, 2 * P, P - 1>(fHx, y, c, h);  // h[j] = Hx(y + P - 1 - j)
       float w[12];
-      xwin(sHz + ly * np, c, w);
-      F4 h[2 * P];
-      B.zwin<2 * P, P - 1>(fHx, y, c, h);  // h[j] = Hx(y + P - 1 - j)
+      xwin<W>(sHz + ly * np, c, w);
       float *ep = sE + ly * np + 4 + c;
-      const F4 e_old = lds4(ep);
-      F4 cx, cz;
+      const V e_old = ldv<W>(ep);
+      V cx, cz;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < W; ++q) {
         cx.v[q] = di<P>(w, q, a.c.cx);
         float sacc = 0.f;
 #pragma unroll
@@ -1022,41 +1118,41 @@ __global__ void __launch_bounds__(NT, 1) k_res_fwd(const SmallArgs a) {
       const int bc = xband(c, nx, a.Wx);
       if (bc >= 0) {
         float *mp = sMxe + ly * 2 * a.Wx + bc;
-        F4 mx = lds4(mp);
-        const F4 ax = lds4(bt + T.x(0) + bc), bx = lds4(bt + T.x(1) + bc);
-        const F4 rk = lds4(bt + T.x(2) + bc);
+        V mx = ldv<W>(mp);
+        const V ax = ldv<W>(bt + T.x(0) + bc), bx = ldv<W>(bt + T.x(1) + bc);
+        const V rk = ldv<W>(bt + T.x(2) + bc);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < W; ++q) {
           mx.v[q] = fmaf(bx.v[q], mx.v[q], ax.v[q] * cx.v[q]);
           cx.v[q] = fmaf(cx.v[q], rk.v[q], mx.v[q]);
         }
-        st4(mp, mx);
+        stv<W>(mp, mx);
       }
       const int zr = zband(y, ny, a.Wz);
       if (zr >= 0) {
         float *mp = sMze + ly * nx + c;
-        F4 mz = lds4(mp);
+        V mz = ldv<W>(mp);
         const float ay = bt[T.z(0) + zr], by = bt[T.z(1) + zr];
         const float rky = bt[T.z(2) + zr];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < W; ++q) {
           mz.v[q] = fmaf(by, mz.v[q], ay * cz.v[q]);
           cz.v[q] = fmaf(cz.v[q], rky, mz.v[q]);
         }
-        st4(mp, mz);
+        stv<W>(mp, mz);
       }
-      F4 curl, en;
+      V curl, en;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < W; ++q) {
         curl.v[q] = cx.v[q] - cz.v[q];
         en.v[q] = fmaf(ca[g].v[q], e_old.v[q], cb[g].v[q] * curl.v[q]);
       }
       if constexpr (STORE != kStoreNone) {
         const int64_t li = (int64_t)ly * nx + c;
-        snap_store<STORE>(stE, li, e_old);
-        snap_store<STORE>(stC, li, curl);
+        snap_store_w<STORE, W>(stE, li, e_old);
+        snap_store_w<STORE, W>(stC, li, curl);
       }
-      st4(ep, en);
+      stv<W>(ep, en);
     }
     // the sources of step t, added to the updated E of their cells
     if (a.f) {
@@ -1077,56 +1173,62 @@ __global__ void __launch_bounds__(NT, 1) k_res_fwd(const SmallArgs a) {
   res_state<false>(a.st, sm, Ly, a.bt, s, r0, Rb, ny, a.numel);
 }
 
-// Snapshot words of one float4 group as stored (fp32, bf16 or FP8), loaded a
-// step ahead and decoded at use.
-template <int SNAP>
+// Snapshot words of one group (W cells) as stored (fp32, bf16 or FP8),
+// loaded a step ahead and decoded at use.
+template <int SNAP, int W>
 struct SnapWords {
-  static constexpr int kWords = SNAP == kStoreF32 ? 4 : SNAP == kStoreBF16 ? 2 : 1;
+  static constexpr int kBytes = W * (SNAP == kStoreF32 ? 4 : SNAP == kStoreBF16 ? 2 : 1);
+  static constexpr int kWords = (kBytes + 3) / 4;
   uint32_t w[kWords];
   // elem: the group's first cell
   __device__ __forceinline__ void load(const void *base, int64_t elem) {
-    if constexpr (SNAP == kStoreF32) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4 *>(base) + elem / 4);
-      w[0] = u.x;
-      w[1] = u.y;
-      w[2] = u.z;
-      w[3] = u.w;
-    } else if constexpr (SNAP == kStoreBF16) {
-      const uint2 u = __ldg(reinterpret_cast<const uint2 *>(base) + elem / 4);
-      w[0] = u.x;
-      w[1] = u.y;
+    if constexpr (kBytes == 16) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4 *>(base) + elem / W);
+      w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
+    } else if constexpr (kBytes == 8) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2 *>(base) + elem / W);
+      w[0] = u.x, w[1] = u.y;
+    } else if constexpr (kBytes == 4) {
+      w[0] = __ldg(reinterpret_cast<const uint32_t *>(base) + elem / W);
     } else {
-      w[0] = __ldg(reinterpret_cast<const uint32_t *>(base) + elem / 4);
+      w[0] = __ldg(reinterpret_cast<const unsigned short *>(base) + elem / W);
     }
   }
-  __device__ __forceinline__ F4 get() const {
+  __device__ __forceinline__ VW<W> get() const {
+    VW<W> r;
     if constexpr (SNAP == kStoreF32) {
-      return F4{{__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
-                 __uint_as_float(w[3])}};
+#pragma unroll
+      for (int q = 0; q < W; ++q) r.v[q] = __uint_as_float(w[q]);
     } else if constexpr (SNAP == kStoreBF16) {
-      const float2 e0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0]));
-      const float2 e1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[1]));
-      return F4{{e0.x, e0.y, e1.x, e1.y}};
+#pragma unroll
+      for (int h = 0; h < W / 2; ++h) {
+        const float2 e = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[h]));
+        r.v[2 * h] = e.x, r.v[2 * h + 1] = e.y;
+      }
     } else {
-      const __half2_raw lo =
-          __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[0] & 0xffffu), __NV_E4M3);
-      const __half2_raw hi =
-          __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[0] >> 16), __NV_E4M3);
-      const float2 fa = __half22float2(__half2(lo)), fb = __half22float2(__half2(hi));
-      return F4{{fa.x, fa.y, fb.x, fb.y}};
+#pragma unroll
+      for (int h = 0; h < W / 2; ++h) {
+        const __half2_raw pr = __nv_cvt_fp8x2_to_halfraw2(
+            (__nv_fp8x2_storage_t)((w[0] >> (16 * h)) & 0xffffu), __NV_E4M3);
+        const float2 f = __half22float2(__half2(pr));
+        r.v[2 * h] = f.x, r.v[2 * h + 1] = f.y;
+      }
     }
+    return r;
   }
 };
-template <int P, int SNAP, int NT, int G>
+
+template <int P, int SNAP, int NT, int G, int W>
 __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
   constexpr int KM = res_kmax(G);
+  using V = VW<W>;
   __shared__ int s_stop;
   const cg::cluster_group cl = cg::this_cluster();
   if (res_start(cl, a.flags, &s_stop)) return;
   const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
   const int s = (int)(blockIdx.x / cs);
-  const int ny = a.ny, nx = a.nx, nx4 = nx >> 2, R = a.rows, K = a.kchunk, km = K - 1, nt = a.nt;
-  const int r0 = rank * R, r1 = min(ny, r0 + R), Rb = r1 - r0, ng = Rb * nx4;
+  const int ny = a.ny, nx = a.nx, nxw = nx / W, R = a.rows, K = a.kchunk, km = K - 1, nt = a.nt;
+  const int r0 = rank * R, r1 = min(ny, r0 + R), Rb = r1 - r0, ng = Rb * nxw;
   const ResLayout Ly{R, nx, a.Wx, a.Wz, kResFieldsAdj, K, a.csrc, a.crec, 0, 0};
   const int np = Ly.pitch();
   const RBlk B{r0, r1, R, ny, np};
@@ -1144,28 +1246,28 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
   const float cqs = a.cq_arr ? 0.f : __ldg(a.cq);
   const int64_t sb = (int64_t)s * a.numel;
   int gy[G], gc[G];
-  F4 ca[G], cb[G], gca[G], gcb[G];
-  SnapWords<SNAP> se[G], sc[G];
+  V ca[G], cb[G], gca[G], gcb[G];
+  SnapWords<SNAP, W> se[G], sc[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const int k = (int)threadIdx.x + g * NT;
     gy[g] = -1;
     gc[g] = 0;
-    ca[g] = cb[g] = gca[g] = gcb[g] = zero4();
+    ca[g] = cb[g] = gca[g] = gcb[g] = zerov<W>();
     if (k < ng) {
-      const int ly = k / nx4;
+      const int ly = k / nxw;
       gy[g] = r0 + ly;
-      gc[g] = (k - ly * nx4) * 4;
+      gc[g] = (k - ly * nxw) * W;
       const int64_t cell = sb + (int64_t)gy[g] * nx + gc[g];
       const int64_t mb = (a.batched ? sb : 0) + (int64_t)gy[g] * nx + gc[g];
-      ca[g] = ld4(a.ca + mb);
-      cb[g] = ld4(a.cb + mb);
-      gca[g] = lds4(a.gca + cell);
-      gcb[g] = lds4(a.gcb + cell);
+      ca[g] = ldgv<W>(a.ca + mb);
+      cb[g] = ldgv<W>(a.cb + mb);
+      gca[g] = ldv<W>(a.gca + cell);
+      gcb[g] = ldv<W>(a.gcb + cell);
     }
   }
   auto snap_at = [&](int t, int g) -> int64_t {
-    return (int64_t)t * a.step_elems + ((int64_t)s * ny + opaque(gy[g])) * a.snap_pitch + gc[g];
+    return (int64_t)t * a.step_elems + ((int64_t)s * ny + gco<G>(gy[g])) * a.snap_pitch + gc[g];
   };
   // step t's snapshots of the thread's groups, into registers
   auto fetch_snap = [&](int t) {
@@ -1224,44 +1326,44 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (gy[g] < 0) continue;
-      const int y = opaque(gy[g]), c = opaque(gc[g]), ly = y - r0;
-      const F4 lam = lds4(sLe + ly * np + 4 + c);
-      F4 gv;
+      const int y = gco<G>(gy[g]), c = gco<G>(gc[g]), ly = y - r0;
+      const V lam = ldv<W>(sLe + ly * np + 4 + c);
+      V gv;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) gv.v[q] = cb[g].v[q] * lam.v[q];
-      F4 pz, px = gv;
+      for (int q = 0; q < W; ++q) gv.v[q] = cb[g].v[q] * lam.v[q];
+      V pz, px = gv;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) pz.v[q] = -gv.v[q];
+      for (int q = 0; q < W; ++q) pz.v[q] = -gv.v[q];
       const int zr = zband(y, ny, a.Wz);
       if (zr >= 0) {
         float *mp = sMze + ly * nx + c;
-        F4 M = lds4(mp);
+        V M = ldv<W>(mp);
         const float ay = bt[T.z(0) + zr], by = bt[T.z(1) + zr];
         const float rky = bt[T.z(2) + zr];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < W; ++q) {
           M.v[q] -= gv.v[q];
           pz.v[q] = fmaf(ay, M.v[q], -gv.v[q] * rky);
           M.v[q] *= by;
         }
-        st4(mp, M);
+        stv<W>(mp, M);
       }
       const int bc = xband(c, nx, a.Wx);
       if (bc >= 0) {
         float *mp = sMxe + ly * 2 * a.Wx + bc;
-        F4 M = lds4(mp);
-        const F4 ax = lds4(bt + T.x(0) + bc), bx = lds4(bt + T.x(1) + bc);
-        const F4 rk = lds4(bt + T.x(2) + bc);
+        V M = ldv<W>(mp);
+        const V ax = ldv<W>(bt + T.x(0) + bc), bx = ldv<W>(bt + T.x(1) + bc);
+        const V rk = ldv<W>(bt + T.x(2) + bc);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < W; ++q) {
           M.v[q] += gv.v[q];
           px.v[q] = fmaf(ax.v[q], M.v[q], gv.v[q] * rk.v[q]);
           M.v[q] *= bx.v[q];
         }
-        st4(mp, M);
+        stv<W>(mp, M);
       }
-      st4(sPx + ly * np + 4 + c, px);
-      st4(sPz + ly * np + 4 + c, pz);
+      stv<W>(sPx + ly * np + 4 + c, px);
+      stv<W>(sPz + ly * np + 4 + c, pz);
     }
     if (chunk && a.res)
       rl.store(rec, kc, [&](int i) { return ringV + ((u + i) & km) * a.crec; });
@@ -1270,46 +1372,49 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (gy[g] < 0) continue;
-      const int y = opaque(gy[g]), c = opaque(gc[g]), ly = y - r0;
+      const int y = gco<G>(gy[g]), c = gco<G>(gc[g]), ly = y - r0;
       const int64_t mb = (a.batched ? sb : 0) + (int64_t)y * nx + c;
-      const F4 cq = a.cq_arr ? ld4(a.cq + mb) : splat4(cqs);
+      const V cq = a.cq_arr ? ldgv<W>(a.cq + mb) : splatv<W>(cqs);
+      // the z window of pz first with one group a thread (see the forward's
+      // H phase); with three, after lambda_Hz (fewer live registers)
+      V p[2 * P];  // p[j] = pz(y + P - j)
+      if constexpr (G == 1) B.zwin<W, 2 * P, P>(fPz, y, c, p);
       {
         float w[12];
-        xwin(sPx + ly * np, c, w);
+        xwin<W>(sPx + ly * np, c, w);
         float *hp = sLhz + ly * np + 4 + c;
-        const F4 lhz_old = lds4(hp);
-        F4 lhz, v;
+        const V lhz_old = ldv<W>(hp);
+        V lhz, v;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < W; ++q) {
           lhz.v[q] = lhz_old.v[q] - dh<P>(w, q, a.c.cx);
           v.v[q] = cq.v[q] * lhz.v[q];
         }
-        st4(hp, lhz);
+        stv<W>(hp, lhz);
         const int bc = xband(c, nx, a.Wx);
         if (bc >= 0) {
           float *mp = sMxh + ly * 2 * a.Wx + bc;
-          F4 M = lds4(mp);
-          const F4 ah = lds4(bt + T.x(3) + bc), bh = lds4(bt + T.x(4) + bc);
-          const F4 rk = lds4(bt + T.x(5) + bc);
+          V M = ldv<W>(mp);
+          const V ah = ldv<W>(bt + T.x(3) + bc), bh = ldv<W>(bt + T.x(4) + bc);
+          const V rk = ldv<W>(bt + T.x(5) + bc);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < W; ++q) {
             M.v[q] += v.v[q];
             const float vq = v.v[q];
             v.v[q] = fmaf(ah.v[q], M.v[q], vq * rk.v[q]);
             M.v[q] *= bh.v[q];
           }
-          st4(mp, M);
+          stv<W>(mp, M);
         }
-        st4(sQx + ly * np + 4 + c, v);
+        stv<W>(sQx + ly * np + 4 + c, v);
       }
       {
-        F4 p[2 * P];
-        B.zwin<2 * P, P>(fPz, y, c, p);  // p[j] = pz(y + P - j)
+        if constexpr (G != 1) B.zwin<W, 2 * P, P>(fPz, y, c, p);
         float *hp = sLhx + ly * np + 4 + c;
-        const F4 lhx = lds4(hp);
-        F4 lh, qz;
+        const V lhx = ldv<W>(hp);
+        V lh, qz;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < W; ++q) {
           float d = 0.f;
 #pragma unroll
           for (int k2 = 1; k2 <= P; ++k2)  // pz(y + k) - pz(y - k + 1)
@@ -1317,23 +1422,23 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
           lh.v[q] = lhx.v[q] - d;
           qz.v[q] = -cq.v[q] * lh.v[q];
         }
-        st4(hp, lh);
+        stv<W>(hp, lh);
         const int zr = zband(y, ny, a.Wz);
         if (zr >= 0) {
           float *mp = sMzh + ly * nx + c;
-          F4 M = lds4(mp);
+          V M = ldv<W>(mp);
           const float ayh = bt[T.z(3) + zr], byh = bt[T.z(4) + zr];
           const float rkyh = bt[T.z(5) + zr];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < W; ++q) {
             const float vq = qz.v[q];
             M.v[q] += vq;
             qz.v[q] = fmaf(ayh, M.v[q], vq * rkyh);
             M.v[q] *= byh;
           }
-          st4(mp, M);
+          stv<W>(mp, M);
         }
-        st4(sQz + ly * np + 4 + c, qz);
+        stv<W>(sQz + ly * np + 4 + c, qz);
       }
     }
     cluster_sync();
@@ -1341,18 +1446,18 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (gy[g] < 0) continue;
-      const int y = opaque(gy[g]), c = opaque(gc[g]), ly = y - r0;
+      const int y = gco<G>(gy[g]), c = gco<G>(gc[g]), ly = y - r0;
+      V qv[2 * P];
+      B.zwin<W, 2 * P, P - 1>(fQz, y, c, qv);  // qv[j] = qz(y + P - 1 - j)
       float w[12];
-      xwin(sQx + ly * np, c, w);
-      F4 qv[2 * P];
-      B.zwin<2 * P, P - 1>(fQz, y, c, qv);  // qv[j] = qz(y + P - 1 - j)
+      xwin<W>(sQx + ly * np, c, w);
       float *lp = sLe + ly * np + 4 + c;
-      const F4 lam = lds4(lp);
+      const V lam = ldv<W>(lp);
       {
-        const F4 ev = se[g].get(), cv = sc[g].get();
+        const V ev = se[g].get(), cv = sc[g].get();
         const bool rowmask = !a.grad_mask || (y >= a.n_pml && y < ny - a.n_pml);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < W; ++q) {
           const bool colmask = !a.grad_mask || (c + q >= a.n_pml && c + q < nx - a.n_pml);
           if (rowmask && colmask) {
             gca[g].v[q] = fmaf(ev.v[q], lam.v[q], gca[g].v[q]);
@@ -1360,9 +1465,9 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
           }
         }
       }
-      F4 en;
+      V en;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < W; ++q) {
         // Ca lam rounded on its own (never fused with the subtraction below),
         // as the stencil kernel queues it for 2P - 1 rows
         const float cla = __fmul_rn(ca[g].v[q], lam.v[q]);
@@ -1372,7 +1477,7 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
           dz = fmaf(a.c.cy[k2 - 1], qv[P - k2].v[q] - qv[P - 1 + k2].v[q], dz);
         en.v[q] = cla - di<P>(w, q, a.c.cx) - dz;
       }
-      st4(lp, en);
+      stv<W>(lp, en);
     }
     // registers: the snapshots of step t - 1 (the next cluster barrier is a
     // phase away)
@@ -1395,8 +1500,8 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
   for (int g = 0; g < G; ++g) {
     if (gy[g] < 0) continue;
     const int64_t cell = sb + (int64_t)gy[g] * nx + gc[g];
-    st4(a.gca + cell, gca[g]);
-    st4(a.gcb + cell, gcb[g]);
+    stv<W>(a.gca + cell, gca[g]);
+    stv<W>(a.gcb + cell, gcb[g]);
   }
   res_state<false>(a.st, sm, Ly, a.bt, s, r0, Rb, ny, a.numel);
 }
@@ -1461,17 +1566,17 @@ bool cluster_fits(K kern, int nt, int cs, size_t smem) {
 }
 
 // The kernel of a launch: L2 variant with NT threads, or resident with
-// (NT, G) = (128, 1), (256, 1) or (512, 3).
-template <int P, int NT, int G, bool RES>
+// (NT, G, W) = (128, 1, 4), (256, 1, 4), (512, 3, 4) or (256, 1, 2).
+template <int P, int NT, int G, bool RES, int W = 4>
 struct SmallKern {
   template <int STORE>
   static void *fwd_k() {
-    if constexpr (RES) return (void *)k_res_fwd<P, STORE, NT, G>;
+    if constexpr (RES) return (void *)k_res_fwd<P, STORE, NT, G, W>;
     else return (void *)k_small_fwd<P, STORE, NT>;
   }
   template <int SNAP>
   static void *adj_k() {
-    if constexpr (RES) return (void *)k_res_adj<P, SNAP, NT, G>;
+    if constexpr (RES) return (void *)k_res_adj<P, SNAP, NT, G, W>;
     else return (void *)k_small_adj<P, SNAP, NT>;
   }
   static void *fwd(int store) {
@@ -1496,10 +1601,12 @@ template <int P>
 void *small_kernel(const SmallPlan &pl, bool adjoint, int store) {
   using R0 = SmallKern<P, 128, 1, true>;
   using R1 = SmallKern<P, 256, 1, true>;
+  using R2 = SmallKern<P, 256, 1, true, 2>;
   using R3 = SmallKern<P, 512, 3, true>;
   using L256 = SmallKern<P, 256, 1, false>;
   using L1024 = SmallKern<P, 1024, 1, false>;
   if (pl.resident) {
+    if (pl.width == 2) return adjoint ? R2::adj(store) : R2::fwd(store);
     if (pl.block == 128) return adjoint ? R0::adj(store) : R0::fwd(store);
     if (pl.block == 256) return adjoint ? R1::adj(store) : R1::fwd(store);
     return adjoint ? R3::adj(store) : R3::fwd(store);
@@ -1530,7 +1637,8 @@ int env_int(const char *name, int dflt) {
 // thread moves its global traffic in chunks of up to 8 steps (as many as
 // shared memory holds), else one step at a time.  For tests and
 // comparisons: MW_SMALL_CLUSTER caps the blocks a shot (at most 16),
-// MW_SMALL_CHUNK the steps a chunk, and MW_SMALL_L2=1 forces the L2 variant.
+// MW_SMALL_CHUNK the steps a chunk, MW_SMALL_WIDTH=4 keeps groups of 4 cells,
+// and MW_SMALL_L2=1 forces the L2 variant.
 bool small_plan(int order, bool adjoint, int store, int ny, int nx, int Wx, int Wz, int n_src,
                 int n_rec, SmallPlan *pl) {
   const int P = order / 2;
@@ -1551,7 +1659,10 @@ bool small_plan(int order, bool adjoint, int store, int ny, int nx, int Wx, int 
       c.cluster = (ny + c.rows - 1) / c.rows;
       const int64_t groups = (int64_t)c.rows * (nx / 4);
       if (groups > 1536) break;  // fewer blocks only make it larger
-      c.block = groups <= 128 ? 128 : groups <= 256 ? 256 : 512;
+      // groups of 2 cells where a 256-thread block then takes one group a
+      // thread (more warps on a small block), else of 4
+      c.width = (int64_t)c.rows * (nx / 2) <= 256 && env_int("MW_SMALL_WIDTH", 2) != 4 ? 2 : 4;
+      c.block = c.width == 2 ? 256 : groups <= 128 ? 128 : groups <= 256 ? 256 : 512;
       const bool one = c.block <= 256;  // one group a thread
       c.csrc = std::max(0, std::min(n_src, c.block));
       c.crec = std::max(0, std::min(n_rec, c.block));
@@ -1577,6 +1688,7 @@ bool small_plan(int order, bool adjoint, int store, int ny, int nx, int Wx, int 
   }
   SmallPlan c{};
   c.resident = false;
+  c.width = 4;
   c.block = (int64_t)ny * (nx / 4) <= (int64_t)std::min(16, cap) * 256 ? 256 : 1024;
   for (int cs : {std::min(16, cap), std::min(8, cap)}) {
     c.cluster = cs;

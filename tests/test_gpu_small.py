@@ -2,9 +2,9 @@
 the adjoint, in one cooperative launch) against the step-by-step launches,
 bit for bit, in both variants: the resident one (each block's rows in shared
 memory, halo rows read from the neighbouring blocks), with the library's
-cluster and chunks of global traffic, with at most 4 blocks a shot, and with
-chunks of 2 steps, and the one whose state stays in global memory
-(MW_SMALL_L2=1).
+cluster, group width and chunks of global traffic, with at most 4 blocks a
+shot, with groups of 4 cells only, and with chunks of 2 steps, and the one
+whose state stays in global memory (MW_SMALL_L2=1).
 
 Both paths make the same floating-point operations in the same order for
 every update, source sum, receiver sample and gradient term, so records,
@@ -29,11 +29,12 @@ pytestmark = pytest.mark.gpu
 
 
 VARIANTS = {"resident": {}, "resident-4": {"MW_SMALL_CLUSTER": "4"},
+            "resident-w4": {"MW_SMALL_WIDTH": "4"},
             "resident-chunk2": {"MW_SMALL_CHUNK": "2"}, "l2": {"MW_SMALL_L2": "1"}}
 
 
 def _run(prob, f, res, state0, adj0, small, monkeypatch, variant="resident"):
-    for k in ("MW_SMALL_CLUSTER", "MW_SMALL_CHUNK", "MW_SMALL_L2"):
+    for k in ("MW_SMALL_CLUSTER", "MW_SMALL_CHUNK", "MW_SMALL_WIDTH", "MW_SMALL_L2"):
         monkeypatch.delenv(k, raising=False)
     if small:
         monkeypatch.delenv("MW_NO_SMALL", raising=False)
