@@ -8,14 +8,16 @@
 // On a few thousand to a few hundred thousand cells the marching-strip
 // kernels are bound by launch and row latency: a launch walks a handful of
 // rows per warp, each waiting for its TMA copy.  Here one launch runs every
-// step.  The state stays in place in global memory (it fits in L2); each
-// shot gets a thread-block cluster (16 blocks, or the portable 8), whose
-// threads own float4 groups of cells (row, 4 columns), and the steps' phases
-// are separated by the cluster's hardware barrier.  Reads of anything the
-// launch writes bypass L1 (ld.global.cg), since L1 is not coherent between
-// blocks.  Every update,
-// source sum and receiver sample is the stencil kernels' operation for
-// operation, so the results are bitwise those of the step-by-step launches.
+// step: each shot gets a thread-block cluster (up to 16 blocks), whose
+// threads own groups of cells (a row's 4, or 2, consecutive columns), and
+// the steps' phases are separated by the cluster's hardware barrier.  Two
+// variants: the resident one (further below), whose blocks keep their rows
+// of every field in shared memory, and, for grids too large for that, the
+// one here, whose state stays in place in global memory (it fits in L2;
+// reads of anything the launch writes bypass L1 (ld.global.cg), since L1 is
+// not coherent between blocks).  Every update, source sum and receiver
+// sample is the stencil kernels' operation for operation, so the results
+// are bitwise those of the step-by-step launches.
 //
 // Forward step t:  H phase (Hz, Hx and their band memories; the receivers of
 //   step t - 1, read from E) | E phase (snapshots of E^t and curl^t, the E
@@ -28,7 +30,8 @@
 //   pz) | H-node phase (lambda_Hz, lambda_Hx from px, pz; their transposed
 //   band terms qx, qz) | E phase (lambda_E = Ca lam - D_x qx - D_z qz, then
 //   res[t - 1] added in the receiver cells).  px, pz, qx, qz live in
-//   workspace arrays between the phases.
+//   workspace arrays (resident: shared memory) between the phases; the
+//   resident adjoint accumulates the gradients in its lambda_E phase.
 #include <cooperative_groups.h>
 #include <cuda.h>
 
