@@ -35,6 +35,10 @@
 #include <cooperative_groups.h>
 #include <cuda.h>
 
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "mw_device.cuh"
 #include "mw_internal.cuh"
 
@@ -1512,15 +1516,28 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
 // One cluster of `cs` blocks per shot, `smem` bytes of dynamic shared memory
 // per block.  A cluster of more than 8 blocks is beyond the portable limit
 // and needs the kernel's opt-in.
+// (The attributes a kernel already has on a device are remembered, so that
+// repeated launches make no further calls.)
 template <typename K>
 cudaError_t set_attrs(K kern, int cs, size_t smem) {
-  if (cs > 8) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void *>, std::pair<bool, size_t>> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto &d = done[{dev, reinterpret_cast<const void *>(kern)}];
+  if (cs > 8 && !d.first) {
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
+    d.first = true;
   }
-  if (smem > 48 * 1024)
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (smem > 48 * 1024 && smem > d.second) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    d.second = smem;
+  }
   return cudaSuccess;
 }
 template <typename K>
@@ -1642,8 +1659,38 @@ int env_int(const char *name, int dflt) {
 // comparisons: MW_SMALL_CLUSTER caps the blocks a shot (at most 16),
 // MW_SMALL_CHUNK the steps a chunk, MW_SMALL_WIDTH=4 keeps groups of 4 cells,
 // and MW_SMALL_L2=1 forces the L2 variant.
+bool small_plan_uncached(int order, bool adjoint, int store, int ny, int nx, int Wx, int Wz,
+                         int n_src, int n_rec, SmallPlan *pl);
+
+// (Plans are remembered per device, shape and test setting.)
 bool small_plan(int order, bool adjoint, int store, int ny, int nx, int Wx, int Wz, int n_src,
                 int n_rec, SmallPlan *pl) {
+  using Key = std::tuple<int, int, int, int, int, int, int, int, int, int, int, int, int, int>;
+  static std::mutex mu;
+  static std::map<Key, std::pair<bool, SmallPlan>> plans;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const Key key{dev, order, adjoint ? 1 : 0, store, ny, nx, Wx, Wz, n_src, n_rec,
+                env_int("MW_SMALL_CLUSTER", 16), env_int("MW_SMALL_CHUNK", 8),
+                env_int("MW_SMALL_WIDTH", 2) * 2 + env_int("MW_SMALL_L2", 0), 0};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = plans.find(key);
+    if (it != plans.end()) {
+      *pl = it->second.second;
+      return it->second.first;
+    }
+  }
+  SmallPlan p{};
+  const bool ok = small_plan_uncached(order, adjoint, store, ny, nx, Wx, Wz, n_src, n_rec, &p);
+  std::lock_guard<std::mutex> lk(mu);
+  plans[key] = {ok, p};
+  *pl = p;
+  return ok;
+}
+
+bool small_plan_uncached(int order, bool adjoint, int store, int ny, int nx, int Wx, int Wz,
+                         int n_src, int n_rec, SmallPlan *pl) {
   const int P = order / 2;
   const int cap = std::max(1, std::min(16, env_int("MW_SMALL_CLUSTER", 16)));
   int kcap = 8;  // a power of two
