@@ -132,17 +132,19 @@ __device__ __forceinline__ void shift_queue(F4 (&q)[N]) {
     for (int k = 0; k < NQ - 1; ++k) q[k] = q[k + M];
   }
 }
-// iterations per unrolled group of a walk: 1 at order 8, 2 for the forward
-// and the adjoint at order 6, the full 2P ring for the shorter adjoint
-// stencils (measured on B200: order 8 runs 1.3-1.6x faster with groups of
-// 2 than with the full ring of 8, and one iteration a group -- half the
-// loop's code, more queue moves -- takes its bf16-snapshot forward and
-// adjoint launches from 0.147 / 0.226 to 0.139 / 0.217 ms at 1064^2 x 16
-// shots; order 4 gains 3 % in the forward and nothing in the adjoint with
-// groups of 2)
+// iterations per unrolled group of a walk: 1 for the adjoint (but at order
+// 6, where one iteration a group spills) and for the forward at order 8,
+// else 2 (measured on B200: order 8 runs 1.3-1.6x
+// faster with groups of 2 than with the full ring of 8, and one iteration a
+// group -- half the loop's code, more queue moves -- takes its bf16-snapshot
+// forward and adjoint launches from 0.147 / 0.226 to 0.139 / 0.217 ms at
+// 1064^2 x 16 shots; the order-4 E-alone adjoint, unrolled over its full
+// ring of 4 before, from 0.308 to 0.303 ms at 2128^2 x 8 shots, with 88
+// registers instead of 123; the order-4 one-step forward gained 3 % with
+// groups of 2 over the full ring)
 template <int P, bool ADJ>
 __host__ __device__ constexpr int walk_group() {
-  return ADJ && P <= 2 ? 2 * P : (P == 4 ? 1 : 2);
+  return ADJ ? (P == 3 ? 2 : 1) : (P == 4 ? 1 : 2);
 }
 
 // ---- sources and receivers in the rows a walk computes -------------------
