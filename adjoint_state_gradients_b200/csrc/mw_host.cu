@@ -430,7 +430,7 @@ Launch plan(const mw_params *p, int kind) {
   if (two) interior_rect(g, fwd2_halo(P) + 4, 4 * P - 2);
   else interior_rect(g, 8, 2 * P - 1);
   const int64_t items = cols_items * g.n_chunks;
-  const int wpc = adjoint ? kAdjWarpsPerCta : kWarpsPerCta;
+  const int wpc = adjoint ? adj_warps_per_cta(P) : kWarpsPerCta;
   int64_t grid = (items + wpc - 1) / wpc;
   const int64_t cap = slots / wpc;
   if (grid > cap) grid = cap;

@@ -27,7 +27,10 @@ namespace mw {
 constexpr int kFwdStripCols = 120;  // forward: columns owned per warp (30 float4)
 constexpr int kAdjStripCols = 112;  // adjoint: columns owned per warp (28 float4)
 constexpr int kWarpsPerCta = 4;    // forward CTA: 4 warps
-constexpr int kAdjWarpsPerCta = 5; // adjoint CTA: 5 warps
+constexpr int kAdjWarpsPerCta = 5; // adjoint CTA: 5 warps (at most)
+// warps of an adjoint CTA: 4 at order 8, whose larger stages then fit three
+// CTAs an SM, else 5
+__host__ __device__ constexpr int adj_warps_per_cta(int P) { return P == 4 ? 4 : kAdjWarpsPerCta; }
 
 struct Geom {
   int ny, nx, S;

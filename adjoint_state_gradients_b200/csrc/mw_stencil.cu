@@ -986,7 +986,7 @@ __device__ __forceinline__ bool adj_walk(const AdjMaps &m, const StepArgs &a, co
 }
 
 template <int P, int SNAP, int L>
-__global__ void __launch_bounds__(32 * kAdjWarpsPerCta) k_adjoint(const __grid_constant__ AdjMaps m,
+__global__ void __launch_bounds__(32 * adj_warps_per_cta(P)) k_adjoint(const __grid_constant__ AdjMaps m,
                                                                   const StepArgs a,
                                                                   const int batched,
                                                                   const int cq_arr) {
@@ -1633,7 +1633,7 @@ void adj_layout_t(int Wx, bool cq_arr, StepArgs *a, size_t *smem) {
   a->stage_floats = o;
   a->warp_floats = wf;
   a->band_box_floats = 2 * Wx;
-  *smem = (size_t)(32 + kAdjWarpsPerCta * wf) * sizeof(float) + 128;
+  *smem = (size_t)(32 + adj_warps_per_cta(P) * wf) * sizeof(float) + 128;
 }
 
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per
@@ -1673,9 +1673,9 @@ cudaError_t fwd_t(const FwdMaps &m, const StepArgs &a, bool batched, bool cq_arr
 template <int P, int SNAP>
 cudaError_t adj_t(const AdjMaps &m, const StepArgs &a, bool batched, bool cq_arr, int grid,
                   cudaStream_t st) {
-  const size_t smem = (size_t)(32 + kAdjWarpsPerCta * a.warp_floats) * sizeof(float) + 128;
+  const size_t smem = (size_t)(32 + adj_warps_per_cta(P) * a.warp_floats) * sizeof(float) + 128;
   allow_big_smem(k_adjoint<P, SNAP, kAdjL>, adj_smem_flag<P, SNAP>());
-  const cudaError_t e = launch_dependent(k_adjoint<P, SNAP, kAdjL>, grid, 32 * kAdjWarpsPerCta,
+  const cudaError_t e = launch_dependent(k_adjoint<P, SNAP, kAdjL>, grid, 32 * adj_warps_per_cta(P),
                                          smem, st, m, a, batched ? 1 : 0, cq_arr ? 1 : 0);
   if (e != cudaSuccess) return e;
   count_launches(1);
@@ -1787,9 +1787,9 @@ int slots_t(bool adjoint, int Wx, bool cq_arr) {
   StepArgs a{};
   if (adjoint) {
     adj_layout_t<P>(Wx, cq_arr, &a, &smem);
-    return occupancy(k_adjoint<P, kStoreF32, kAdjL>, 32 * kAdjWarpsPerCta, smem,
+    return occupancy(k_adjoint<P, kStoreF32, kAdjL>, 32 * adj_warps_per_cta(P), smem,
                      adj_smem_flag<P, kStoreF32>()) *
-           kAdjWarpsPerCta;
+           adj_warps_per_cta(P);
   }
   fwd_layout_t<P>(Wx, cq_arr, false, &a, &smem);
   return occupancy(k_forward<P, kStoreF32, kFwdL, kStoreNone>, 32 * kWarpsPerCta, smem,
