@@ -7,6 +7,7 @@
 // record_receivers_ey, add_adjoint_sources_ey, record_adjoint_at_sources,
 // combine_grad and convert_grad_ca_cb_to_eps_sigma; the model-coefficient
 // forms are the ones whose derivatives that last kernel uses.
+#include <cooperative_groups.h>
 #include <math.h>
 
 #include "mw_internal.cuh"
@@ -314,10 +315,21 @@ __global__ void k_residual(int64_t n, const float *__restrict__ d, const float *
 
 // Misfit 1/2 sum res^2 in one block: fixed per-thread strides and a fixed
 // tree, so the value does not depend on scheduling.
-__global__ void k_misfit(int64_t n, const float *__restrict__ res, double *__restrict__ J) {
+// J = 1/2 sum res[i]^2 in double, in an order fixed whatever the timing,
+// by one cluster of kMisfitBlocks blocks: block b sums its chunk [b C,
+// b C + C) (thread t the elements t, t + 1024, ... of it, then a fixed
+// tree), and block 0 adds the blocks' sums in rank order through the
+// cluster's distributed shared memory.
+constexpr int kMisfitBlocks = 8;
+__global__ void __cluster_dims__(kMisfitBlocks, 1, 1) __launch_bounds__(1024)
+    k_misfit(int64_t n, const float *__restrict__ res, double *__restrict__ J) {
   __shared__ double part[1024];
+  cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
+  const int b = (int)cl.block_rank();
+  const int64_t C = (n + kMisfitBlocks - 1) / kMisfitBlocks;
+  const int64_t lo = (int64_t)b * C, hi = lo + C < n ? lo + C : n;
   double acc = 0.0;
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+  for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) {
     const double r = res[i];
     acc += r * r;
   }
@@ -327,7 +339,13 @@ __global__ void k_misfit(int64_t n, const float *__restrict__ res, double *__res
     if ((int)threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *J = 0.5 * part[0];
+  cl.sync();  // every block's sum is in its part[0]
+  if (b == 0 && threadIdx.x == 0) {
+    double sum = 0.0;
+    for (int k = 0; k < kMisfitBlocks; ++k) sum += *cl.map_shared_rank(&part[0], k);
+    *J = 0.5 * sum;
+  }
+  cl.sync();  // no block leaves while block 0 reads its sum
 }
 
 int grid_for(int64_t n, int block) {
@@ -471,7 +489,7 @@ cudaError_t launch_residual(int64_t n, const float *d, const float *o, float *re
   count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || J == nullptr) return e;
-  k_misfit<<<1, 1024, 0, st>>>(n, res, J);
+  k_misfit<<<kMisfitBlocks, 1024, 0, st>>>(n, res, J);
   count_launches(1);
   return cudaGetLastError();
 }
