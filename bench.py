@@ -162,6 +162,15 @@ def per_step_ms(counts, ms, classes, nt):
     return t / max(n, 1)
 
 
+def steps_per_launch(counts, classes, nt):
+    """Mean time steps one launch of a pass advances: 1, 2 (two-step
+    launches) or nt (whole-sweep launches), mixed as counted."""
+    a, b, w = classes
+    n = counts[a] + (counts[b] if b is not None else 0) + sum(counts[k] for k in w)
+    st = counts[a] + (2 * counts[b] if b is not None else 0) + nt * sum(counts[k] for k in w)
+    return st / n if n else 1.0
+
+
 TAIL_RESERVE = 12e9  # device bytes left free beside the workspace
 
 
@@ -504,12 +513,7 @@ class Sweep:
         top = "adjoint" if self.grad else "forward"   # the dominant kernel
         top_launch_ms = launch_ms[top]
 
-        def steps_per_launch(c):
-            a, b, w = c
-            n = counts[a] + (counts[b] if b is not None else 0) + sum(counts[k] for k in w)
-            st = counts[a] + (2 * counts[b] if b is not None else 0) + nt * sum(counts[k] for k in w)
-            return st / n if n else 1.0
-        spl = {k: steps_per_launch(c) for k, c in classes.items()}
+        spl = {k: steps_per_launch(counts, c, nt) for k, c in classes.items()}
         top_bytes = passes[top] * wl.ny * wl.nx * S
         achieved = top_bytes / (top_launch_ms / 1e3) / 1e9
         kname = {("adjoint", "fp32"): "kStoreF32", ("adjoint", "ckpt"): "kStoreF32",

@@ -80,6 +80,15 @@ def test_per_step_time_of_each_launch_kind():
     assert bench.N_CLASSES == 12
 
 
+def test_steps_per_launch():
+    counts = [0] * 12
+    assert bench.steps_per_launch(counts, (2, None, (8, 11)), 300) == 1.0  # nothing ran
+    counts[0], counts[4] = 2, 98   # a pass of two one-step and 98 two-step launches
+    assert bench.steps_per_launch(counts, (0, 4, ()), 4000) == pytest.approx(198 / 100)
+    counts[8] = 3                  # three whole-sweep adjoint launches
+    assert bench.steps_per_launch(counts, (2, None, (8, 11)), 300) == 300.0
+
+
 def test_oracle_sample_is_bounded():
     for n in range(1, 6):
         wl = synth.WORKLOADS[n]
