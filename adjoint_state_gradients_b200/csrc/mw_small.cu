@@ -1516,28 +1516,17 @@ __global__ void __launch_bounds__(NT, 1) k_res_adj(const SmallArgs a) {
 // One cluster of `cs` blocks per shot, `smem` bytes of dynamic shared memory
 // per block.  A cluster of more than 8 blocks is beyond the portable limit
 // and needs the kernel's opt-in.
-// (The attributes a kernel already has on a device are remembered, so that
-// repeated launches make no further calls.)
+// (Set on every launch, two calls: attributes belong to the context, which
+// a device reset replaces.)
 template <typename K>
 cudaError_t set_attrs(K kern, int cs, size_t smem) {
-  static std::mutex mu;
-  static std::map<std::pair<int, const void *>, std::pair<bool, size_t>> done;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> lk(mu);
-  auto &d = done[{dev, reinterpret_cast<const void *>(kern)}];
-  if (cs > 8 && !d.first) {
+  if (cs > 8) {
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    d.first = true;
   }
-  if (smem > 48 * 1024 && smem > d.second) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    d.second = smem;
-  }
+  if (smem > 48 * 1024)
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   return cudaSuccess;
 }
 template <typename K>
